@@ -1,0 +1,80 @@
+"""Oracle: one decode step of attention over the compressed cache.  TEST INFRASTRUCTURE ONLY.
+
+Source: KV-COBRA project page, "Efficiency" (the cache is stored as packed b-bit
+codes; dequantisation and the inverse rotation are applied when it is read) and
+"How KV-COBRA Works" (keys are rotated and truncated with H.V^T before
+quantisation, so the inverse is V.H^T).
+
+The oracle works in the ORIGINAL d-space: it dequantises every code, reconstructs
+k_hat_t = M_K^T y_hat_K,t and v_hat_t = M_V^T y_hat_V,t in fp64, then applies
+textbook softmax attention (two-pass, fp64).  It deliberately does not use the
+latent shortcut (q moved into the key basis, values accumulated in the value basis)
+that the GPU path uses, so that shortcut is checked against an independent
+formulation.
+
+Reading: the synthetic workloads have no rotary embedding, so keys are compared with
+queries exactly as stored; the softmax scale is 1/sqrt(d) with d the head dimension
+(not the retained rank).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .codec import dequantize
+
+
+def reconstruct(codes, M, delta, b):
+    """x_hat [T, d] = dequantize(codes) @ M in fp64 (M: [r, d] as stored in the plan)."""
+    y = dequantize(codes, delta, b)
+    return y @ np.asarray(M, dtype=np.float64)
+
+
+def softmax_attention(q, K, V, scale):
+    """Textbook attention for G queries over T tokens, fp64, two-pass softmax.
+
+    q: [G, d]; K, V: [T, d].  Returns o [G, d].  For T == 0 the output is zero (the
+    defined behaviour of an empty cache).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    if K.shape[0] == 0:
+        return np.zeros((q.shape[0], V.shape[1]))
+    s = (q @ K.T) * scale                       # [G, T]
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    l = p.sum(axis=1, keepdims=True)
+    return (p @ V) / l
+
+
+def decode_head(q, k_codes, v_codes, unit_k, unit_v, scale):
+    """One KV head: G query vectors against the dequantised, reconstructed cache.
+
+    unit_k / unit_v: dicts with keys M (r x d), delta, b.  k_codes [T, r_K],
+    v_codes [T, r_V].
+    """
+    K = reconstruct(k_codes, unit_k["M"], unit_k["delta"], unit_k["b"])
+    V = reconstruct(v_codes, unit_v["M"], unit_v["delta"], unit_v["b"])
+    return softmax_attention(q, K, V, scale)
+
+
+def split_merge_attention(q, K, V, scale, n_split):
+    """The same attention computed over ``n_split`` contiguous token ranges with an
+    online (max, sum, weighted-sum) state per range, merged by log-sum-exp.  Used
+    only to pin that a split-context merge equals the two-pass result."""
+    q = np.asarray(q, dtype=np.float64)
+    T = K.shape[0]
+    bounds = np.linspace(0, T, n_split + 1).astype(int)
+    parts = []
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        if b <= a:
+            continue
+        s = (q @ K[a:b].T) * scale
+        m = s.max(axis=1)
+        p = np.exp(s - m[:, None])
+        parts.append((m, p.sum(axis=1), p @ V[a:b]))
+    M = np.max(np.stack([p[0] for p in parts]), axis=0)
+    l = sum(np.exp(p[0] - M) * p[1] for p in parts)
+    z = sum(np.exp(p[0] - M)[:, None] * p[2] for p in parts)
+    return z / l[:, None]
