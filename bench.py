@@ -1,0 +1,501 @@
+#!/usr/bin/env python
+"""Benchmark of the KV-COBRA transform-coded KV cache on B200.
+
+Headline (the metric): decode-attention effective HBM GB/s (and % of the measured HBM
+peak) over a 32-layer Llama-3.1-8B-shaped cache (32 query / 8 KV heads, d = 128) of
+131072 tokens compressed at a joint 1 bit per dimension; plus encode Mtok/s for the
+28-layer Qwen2.5-7B-shaped prefill of 131072 tokens at 2 bits per dimension.
+
+One step = one decode step of the whole model: for each of the 32 layers, append the
+new token's K/V (encode: project, quantize, pack) and run decode attention over the
+131072-token cache (q into the key basis, unpack + scores, online softmax, value
+accumulation in the latent basis, split merge, back-projection).  The 32 layers are
+captured in one CUDA graph and replayed; inputs are resident in HBM.  GB/s counts the
+algorithmic bytes of a step: packed codes of every cached token plus the projection
+bases (fp32 M_K and M_V) of every KV head.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: replicas only (each rank runs the same workload on its own GPU; no data-path
+collective); timing is the max over ranks.  ``--impl reference`` times the CPU oracle
+(the plain fp64 restatement of the method) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_quantization_head_b200 import kvtc, synth  # noqa: E402
+
+DECODE_WORKLOAD = "llama8b-32L-128k-1bpd"
+ENCODE_WORKLOAD = "qwen7b-28L-128k-2bpd"
+METRIC = "decode-attn effective HBM GB/s (% of peak) at 128k ctx; encode Mtok/s"
+
+
+# ---------------------------------------------------------------------------- helpers
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu_id)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def record_external(event, stream):
+    """cudaEventRecordWithFlags(..., cudaEventRecordExternal): an event that stays a timing
+    node when recorded inside CUDA-graph capture."""
+    from cuda.bindings import runtime as rt
+    err, = rt.cudaEventRecordWithFlags(event.cuda_event, stream.cuda_stream, rt.cudaEventRecordExternal)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaEventRecordWithFlags: {err}")
+
+
+def algorithmic_bytes(plan, layers, seq_len, n_seq):
+    """Packed codes of every cached token plus the fp32 bases M_K, M_V, per KV head."""
+    H = plan.shape["n_kv_heads"]
+    per_layer = []
+    for layer in layers:
+        t = 0
+        for h in range(H):
+            for kind in (0, 1):
+                info = plan.unit((layer * H + h) * 2 + kind)
+                t += n_seq * seq_len * info["r"] * info["b"] // 8 + info["r"] * 128 * 4
+        per_layer.append(t)
+    return per_layer
+
+
+# ---------------------------------------------------------------------------- our arm
+def build_decode_setup(torch, w, rank):
+    """Calibrate, allocate the cache, prefill 131071 tokens of every layer (encode path),
+    and prepare the step's inputs.  Returns a dict of state."""
+    t0 = time.time()
+    k_cal, v_cal, q_cal = synth.calibration_set(w)
+    plan = kvtc.kvtc_calibrate(k_cal, v_cal, q_cal, n_layers=w.n_layers, n_kv_heads=w.n_kv_heads,
+                               group=w.group, bpd=w.bpd, seed=w.seed).upload()
+    t_cal = time.time() - t0
+    H, G, L, T, B = w.n_kv_heads, w.group, w.n_layers, w.seq_len, w.batch
+    pages = (T + 127) // 128
+    rng = np.random.default_rng(1234 + rank)
+    bt = torch.from_numpy(rng.permutation(B * pages).astype(np.int32).reshape(B, pages))
+    cache = kvtc.Cache(plan, B * pages, bt)
+    dev = torch.device("cuda")
+    specs = {(l, h, kd): synth.unit_spec(w, l, h, kd) for l in range(L) for h in range(H) for kd in (0, 1)}
+    prefix = T - 1
+    for layer in range(L):
+        for s in range(B):
+            k, v = synth.layer_kv_torch(w, layer, prefix, dev, seq=s, specs=specs)
+            try:
+                kvtc.kvtc_encode_prefill(plan, cache, layer, k, v, s, 0)
+            except kvtc.KvtcError:
+                cu = torch.tensor([0, prefix], dtype=torch.int32, device=dev)
+                pos = torch.tensor([0], dtype=torch.int32, device=dev)
+                # one sequence per call: cu_seqlens / pos_start describe only sequence s
+                sub = kvtc.Cache.__new__(kvtc.Cache)
+                sub.__dict__.update(cache.__dict__)
+                sub.desc = kvtc.CacheDesc(cache.pool.data_ptr(), cache.pages_per_unit,
+                                          cache.block_table[s:s + 1].data_ptr(), 1, pages,
+                                          cache.status.data_ptr())
+                kvtc.kvtc_encode_append(plan, sub, layer, k, v, cu, pos)
+            del k, v
+    torch.cuda.synchronize()
+    # step inputs: one new token per sequence and layer, and the decode queries
+    dt = torch.bfloat16
+    k_new = torch.empty((L, B, H, 128), dtype=dt, device=dev)
+    v_new = torch.empty((L, B, H, 128), dtype=dt, device=dev)
+    q = torch.empty((L, B, H * G, 128), dtype=dt, device=dev)
+    for layer in range(L):
+        for s in range(B):
+            k1, v1 = synth.layer_kv_torch(w, layer, 1, dev, seq=10_000 + s, specs=specs)
+            k_new[layer, s] = k1[0]
+            v_new[layer, s] = v1[0]
+            q[layer, s] = torch.from_numpy(synth.decode_queries(w, layer, s)).to(dev, dt)
+    out = torch.empty((L, B, H * G, 128), dtype=dt, device=dev)
+    cu = torch.arange(B + 1, dtype=torch.int32, device=dev)
+    pos = torch.full((B,), prefix, dtype=torch.int32, device=dev)
+    seq_lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+    ws = torch.empty(kvtc.kvtc_decode_workspace_bytes(plan, B, T), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    return dict(plan=plan, cache=cache, k_new=k_new, v_new=v_new, q=q, out=out, cu=cu, pos=pos,
+                seq_lens=seq_lens, ws=ws, t_cal=t_cal, t_setup=time.time() - t0)
+
+
+def decode_step(st, w, events=None, stream=None):
+    plan, cache = st["plan"], st["cache"]
+    for layer in range(w.n_layers):
+        kvtc.kvtc_encode_append(plan, cache, layer, st["k_new"][layer], st["v_new"][layer], st["cu"], st["pos"],
+                                stream=stream)
+        if events is not None:
+            record_external(events[layer][0], stream)
+        kvtc.kvtc_decode_attention(plan, cache, layer, st["q"][layer], st["seq_lens"], w.seq_len,
+                                   st["out"][layer], st["ws"], stream=stream)
+        if events is not None:
+            record_external(events[layer][1], stream)
+
+
+def kernels_per_step(plan, w):
+    n = 0
+    H = plan.shape["n_kv_heads"]
+    for layer in range(w.n_layers):
+        groups = {(plan.unit((layer * H + h) * 2)["b"], plan.unit((layer * H + h) * 2 + 1)["b"]) for h in range(H)}
+        n += 1 + len(groups) + 1          # append, split kernel(s), combine
+    return n
+
+
+def cpu_baseline_decode(torch, st, w, budget_s=12.0):
+    """The oracle (as it stands) on a bounded sample: KV heads of layer 0 over the full
+    131072-token cache, fp64 d-space attention over the GPU-written pages."""
+    from oracle import attention as oatt
+    from oracle import codec as ocodec
+    plan, cache = st["plan"], st["cache"]
+    H, G, T = w.n_kv_heads, w.group, w.seq_len
+    pages = (T + 127) // 128
+    q = st["q"][0, 0].float().cpu().numpy().astype(np.float64)
+    bt = cache.block_table.cpu().numpy()[0]
+    done_bytes, t_used, heads = 0, 0.0, 0
+    for h in range(H):
+        uK, uV = h * 2, h * 2 + 1
+        infos = [plan.unit(uK), plan.unit(uV)]
+        pools = [cache.unit_pool(u).cpu().numpy() for u in (uK, uV)]
+        units = [dict(M=plan.matrix(u), delta=i["delta"], b=i["b"]) for u, i in zip((uK, uV), infos)]
+        t0 = time.perf_counter()
+        codes = []
+        for kind, (pool, info) in enumerate(zip(pools, infos)):
+            pb = info["page_bytes"]
+            pg = [pool[int(bt[p]) * pb:(int(bt[p]) + 1) * pb] for p in range(pages)]
+            codes.append(ocodec.unpack_sequence(pg, kind, info["r"], info["b"], T))
+        oatt.decode_head(q[h * G:(h + 1) * G], codes[0], codes[1], units[0], units[1], 1 / math.sqrt(128))
+        t_used += time.perf_counter() - t0
+        done_bytes += sum(T * i["r"] * i["b"] // 8 + i["r"] * 128 * 4 for i in infos)
+        heads += 1
+        if t_used >= budget_s:
+            break
+    return done_bytes, t_used, heads
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def encode_bench(torch, w, steps, warmup, rank):
+    """Encode Mtok/s: every layer's K and V of 131072 tokens, resident in HBM."""
+    dev = torch.device("cuda")
+    k_cal, v_cal, q_cal = synth.calibration_set(w)
+    plan = kvtc.kvtc_calibrate(k_cal, v_cal, q_cal, n_layers=w.n_layers, n_kv_heads=w.n_kv_heads,
+                               group=w.group, bpd=w.bpd, seed=w.seed).upload()
+    T = w.seq_len
+    pages = T // 128
+    bt = torch.arange(pages, dtype=torch.int32).reshape(1, pages)
+    cache = kvtc.Cache(plan, pages, bt)
+    specs = {(l, h, kd): synth.unit_spec(w, l, h, kd) for l in range(w.n_layers) for h in range(w.n_kv_heads)
+             for kd in (0, 1)}
+    kv = [synth.layer_kv_torch(w, l, T, dev, specs=specs) for l in range(w.n_layers)]
+    cu = torch.tensor([0, T], dtype=torch.int32, device=dev)
+    pos = torch.tensor([0], dtype=torch.int32, device=dev)
+    use_prefill = True
+    try:
+        kvtc.kvtc_encode_prefill(plan, cache, 0, kv[0][0], kv[0][1], 0, 0)
+    except kvtc.KvtcError:
+        use_prefill = False
+
+    def one_pass():
+        for l in range(w.n_layers):
+            if use_prefill:
+                kvtc.kvtc_encode_prefill(plan, cache, l, kv[l][0], kv[l][1], 0, 0)
+            else:
+                kvtc.kvtc_encode_append(plan, cache, l, kv[l][0], kv[l][1], cu, pos)
+
+    for _ in range(max(1, warmup)):
+        one_pass()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one_pass()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    in_bytes = w.n_layers * T * w.n_kv_heads * 128 * 2 * 2
+    code_bytes = sum(T * plan.unit(u)["r"] * plan.unit(u)["b"] // 8 for u in range(plan.shape["n_units"]))
+    flops = sum(2 * 128 * plan.unit(u)["r"] for u in range(plan.shape["n_units"])) * T
+    return {"workload": w.name, "path": "prefill (tensor cores)" if use_prefill else "append (CUDA cores)",
+            "ms_per_pass": ms, "mtok_s": T / ms / 1e3, "gb_s": (in_bytes + code_bytes) / ms / 1e6,
+            "bytes_per_pass": in_bytes + code_bytes, "tflop_s": flops / ms / 1e9, "layers": w.n_layers}
+
+
+def run_ours(args, torch, dist, rank, world):
+    w = synth.WORKLOADS[args.workload]
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+    st = build_decode_setup(torch, w, rank)
+    plan = st["plan"]
+    stream = torch.cuda.Stream()
+    L = w.n_layers
+    per_layer_bytes = algorithmic_bytes(plan, range(L), w.seq_len, w.batch)
+    step_bytes = sum(per_layer_bytes)
+
+    # warm the kernels (sets function attributes) before capture
+    with torch.cuda.stream(stream):
+        decode_step(st, w, stream=stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        decode_step(st, w, stream=stream)
+    # a second graph with timing events around every layer's decode call
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+    for ea, eb in events:            # torch creates the CUDA events lazily, on first record
+        ea.record(stream)
+        eb.record(stream)
+    torch.cuda.synchronize()
+    g_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_ev, stream=stream):
+        decode_step(st, w, events=events, stream=stream)
+    torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    gpu_id = torch.cuda.get_device_properties(torch.cuda.current_device()).uuid
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(f"GPU-{gpu_id}") as clk:
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+
+    # per-launch duration of the dominant kernel (decode call of one layer)
+    durs = []
+    for _ in range(max(1, min(args.steps, 10))):
+        g_ev.replay()
+        torch.cuda.synchronize()
+        durs.extend(events[l][0].elapsed_time(events[l][1]) for l in range(L))
+    dec_ms = statistics.mean(durs)
+    hbm_peak, tf_peak, peak_kind = measured_peaks()
+    achieved = (step_bytes / L) / (dec_ms * 1e-3) / 1e9
+
+    # end to end: H2D of the step's inputs from pinned memory, the graph, D2H of outputs
+    q_h = st["q"].cpu().pin_memory()
+    kn_h = st["k_new"].cpu().pin_memory()
+    vn_h = st["v_new"].cpu().pin_memory()
+    out_h = torch.empty_like(st["out"], device="cpu").pin_memory()
+    h2d = q_h.numel() * 2 + kn_h.numel() * 2 + vn_h.numel() * 2
+    d2h = out_h.numel() * 2
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            st["q"].copy_(q_h, non_blocking=True)
+            g.replay()
+            out_h.copy_(st["out"], non_blocking=True)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for _ in range(args.steps):
+            st["q"].copy_(q_h, non_blocking=True)
+            st["k_new"].copy_(kn_h, non_blocking=True)
+            st["v_new"].copy_(vn_h, non_blocking=True)
+            g.replay()
+            out_h.copy_(st["out"], non_blocking=True)
+        f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / args.steps
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    value = world * step_bytes / (ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "layers": L, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+                   "head_dim": 128, "batch": w.batch, "seq_len": w.seq_len, "bpd": w.bpd,
+                   "parallelism": f"replicas x{world}",
+                   "step": "per layer: append 1 token + decode attention; 32 layers in one CUDA graph",
+                   "l2": f"inputs larger than L2: {step_bytes / 1e9:.3f} GB of codes+bases per step vs 126 MB",
+                   "compute": "fp16 tensor-core operands (codes exact, q split hi+lo), fp32 accumulation"},
+        "pct_of_peak": round(100 * value / world / hbm_peak, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                     "kernel": "decode (split kernel + combine) of one layer", "peak_kind": peak_kind,
+                     "bytes_per_launch": step_bytes // L, "launch_ms": round(dec_ms, 5)},
+        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": kernels_per_step(plan, w) * args.steps,
+        "clocks": clk.summary(),
+        "setup_s": {"calibrate": round(st["t_cal"], 1), "total": round(st["t_setup"], 1)},
+    }
+    if not args.no_encode:
+        res["encode"] = encode_bench(torch, synth.WORKLOADS[ENCODE_WORKLOAD], max(1, min(args.steps, 5)),
+                                     args.warmup, rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        b, t, heads = cpu_baseline_decode(torch, st, w)
+        res["cpu_baseline"] = {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
+                               "kind": "oracle",
+                               "sample": f"{heads} KV head(s) of layer 0 (G={w.group} queries each) over the "
+                                         f"{w.seq_len}-token cache: unpack + fp64 d-space attention"}
+    return res
+
+
+# ---------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The CPU oracle as it stands on a bounded sample of the decode workload: one KV head
+    of the 32-layer 1-bpd model over a 131072-token cache that the oracle itself encodes
+    (setup, untimed); each step is one oracle decode of that head."""
+    from oracle import attention as oatt
+    from oracle import calibration as ocal
+    from oracle import codec as ocodec
+    w = synth.WORKLOADS[args.workload]
+    k_cal, v_cal, q_cal = synth.calibration_set(w, layers=[0])
+    units = ocal.calibrate(k_cal, v_cal, q_cal, 1, w.n_kv_heads, bpd=w.bpd, seed=w.seed)
+    T = w.seq_len
+    uK, uV = units[0], units[1]
+    codes = []
+    for kind, u in ((0, uK), (1, uV)):
+        x = synth.cache_tokens(w, 0, 0, kind, T)
+        codes.append(ocodec.encode_tokens(x, ocodec.to_bf16(u["M"].astype(np.float32)), u["inv_delta"], u["b"]))
+    pages = [ocodec.pack_sequence(c, kind, u["b"]) for kind, (c, u) in enumerate(zip(codes, (uK, uV)))]
+    q = synth.decode_queries(w, 0)[:w.group].astype(np.float64)
+    M = [dict(M=u["M"].astype(np.float32), delta=np.float32(u["delta"]), b=u["b"]) for u in (uK, uV)]
+
+    def step():
+        ck = ocodec.unpack_sequence(pages[0], 0, uK["r"], uK["b"], T)
+        cv = ocodec.unpack_sequence(pages[1], 1, uV["r"], uV["b"], T)
+        return oatt.decode_head(q, ck, cv, M[0], M[1], 1 / math.sqrt(128))
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    b = sum(T * u["r"] * u["b"] // 8 + u["r"] * 128 * 4 for u in (uK, uV))
+    value = b / dt / 1e9
+    cores = blas_threads()
+    sample = (f"1 KV head (G={w.group} queries) of layer 0 over a {T}-token cache encoded by the oracle; "
+              "unpack + fp64 d-space attention per step")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "seq_len": T, "sample": sample},
+            "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DECODE_WORKLOAD)
+    ap.add_argument("--no-encode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as td
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+        dist = td
+    res = run_ours(args, torch, dist, rank, world)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,166 @@
+// kvtc_encode_append: canonical-order per-token encode on CUDA cores.
+//
+// KV-COBRA project page, "How KV-COBRA Works" (Inference): each key (and value) is
+// rotated and truncated with H.V^T and quantized with the unit's b-bit quantizer.  One
+// thread computes one latent coordinate y_j of one token of one unit as the fp32 chain
+// acc = fma(x_k, M_jk, acc), k = 0..127 in order (the canonical arithmetic the oracle
+// reproduces bit for bit), quantizes it and merges its bits into the page word.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kvtc_internal.h"
+#include "layout.cuh"
+
+namespace kvtc {
+
+struct AppendArgs {
+  const UnitDesc* units;  // device, all units of the plan
+  int unit0;              // first unit of the layer
+  int n_units;            // units in the layer (2 * H)
+  int H;
+  const void* k;
+  const void* v;
+  int bf16;
+  const int32_t* cu_seqlens;
+  const int32_t* pos_start;
+  int n_seq;
+  int n_tok;
+  int coords_per_token;   // sum over the layer's units of r
+  char* pool;
+  uint64_t pages_per_unit;
+  const int32_t* block_table;
+  int max_pages;
+  int32_t* status;
+};
+
+__device__ __forceinline__ uint8_t quantize_code(float y, float inv_delta, int b) {
+  const float t = __fmul_rn(y, inv_delta);
+  const float u = __fadd_rn(t, static_cast<float>(1 << (b - 1)));
+  float f = floorf(u);
+  f = fmaxf(f, 0.0f);                                   // NaN -> 0
+  f = fminf(f, static_cast<float>((1 << b) - 1));
+  return static_cast<uint8_t>(f);
+}
+
+// Overwrites the b-bit code (t, j) of a page: clears its bits, then sets them.
+__device__ __forceinline__ void store_code(uint32_t* page, int kind, int r, int b, int t, int j, uint32_t c) {
+  const int np = code_nparts(b);
+  for (int i = 0; i < np; ++i) {
+    int lo, w;
+    code_part(b, i, lo, w);
+    const FieldPos f = field_pos(kind, r, lo, w, t, j);
+    const uint32_t mask = ((1u << w) - 1u) << f.bit;
+    const uint32_t bits = ((c >> lo) & ((1u << w) - 1u)) << f.bit;
+    atomicAnd(page + f.word, ~mask);
+    if (bits) atomicOr(page + f.word, bits);
+  }
+}
+
+__global__ void __launch_bounds__(128) encode_append_kernel(AppendArgs a) {
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long total = static_cast<long long>(a.n_tok) * a.coords_per_token;
+  if (gid >= total) return;
+  const int tok = static_cast<int>(gid / a.coords_per_token);
+  int c = static_cast<int>(gid % a.coords_per_token);
+  int ul = 0;
+  while (ul < a.n_units - 1 && c >= a.units[a.unit0 + ul].r) {
+    c -= a.units[a.unit0 + ul].r;
+    ++ul;
+  }
+  const int u = a.unit0 + ul;
+  const UnitDesc ud = a.units[u];
+  const int kind = ul & 1;
+  const int head = ul >> 1;
+  const int j = c;
+
+  // canonical projection
+  float acc = 0.0f;
+  const size_t xoff = (static_cast<size_t>(tok) * a.H + head) * kD;
+  if (a.bf16) {
+    const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(kind ? a.v : a.k) + xoff;
+    const uint16_t* m = ud.Mbf + static_cast<size_t>(j) * kD;
+#pragma unroll 8
+    for (int k = 0; k < kD; ++k) {
+      const float xv = __bfloat162float(x[k]);
+      const float mv = __uint_as_float(static_cast<uint32_t>(m[k]) << 16);
+      acc = __fmaf_rn(xv, mv, acc);
+    }
+  } else {
+    const float* x = static_cast<const float*>(kind ? a.v : a.k) + xoff;
+    const float* m = ud.M + static_cast<size_t>(j) * kD;
+#pragma unroll 8
+    for (int k = 0; k < kD; ++k) acc = __fmaf_rn(x[k], m[k], acc);
+  }
+  const uint32_t code = quantize_code(acc, ud.inv_delta, ud.b);
+
+  // token -> (sequence, position) -> page
+  int lo = 0, hi = a.n_seq - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.cu_seqlens[mid] <= tok)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  const int s = lo;
+  const long long pos = static_cast<long long>(a.pos_start[s]) + (tok - a.cu_seqlens[s]);
+  if (pos < 0 || pos >= static_cast<long long>(a.max_pages) * kPage) {
+    if (a.status) atomicOr(a.status, KVTC_STATUS_BAD_POS);
+    return;
+  }
+  const int lp = static_cast<int>(pos / kPage);
+  const int slot = static_cast<int>(pos % kPage);
+  const int32_t pid = a.block_table[static_cast<size_t>(s) * a.max_pages + lp];
+  if (pid < 0 || static_cast<uint64_t>(pid) >= a.pages_per_unit) {
+    if (a.status) atomicOr(a.status, KVTC_STATUS_BAD_PAGE);
+    return;
+  }
+  uint32_t* page = reinterpret_cast<uint32_t*>(a.pool + a.pages_per_unit * ud.prefix +
+                                               static_cast<uint64_t>(pid) * ud.page_bytes);
+  store_code(page, kind, ud.r, ud.b, slot, j, code);
+}
+
+}  // namespace kvtc
+
+using namespace kvtc;
+
+extern "C" kvtc_status kvtc_encode_append(const kvtc_plan* plan, const kvtc_cache* cache, int layer,
+                                          const void* k, const void* v, kvtc_dtype dtype,
+                                          const int32_t* cu_seqlens, const int32_t* pos_start, int n_tok,
+                                          void* stream) {
+  kvtc_status st = check_uploaded(plan);
+  if (st != KVTC_OK) return st;
+  if (!cache || !cache->pool || !cache->block_table) return fail(KVTC_EINVAL, "cache is incomplete");
+  if (layer < 0 || layer >= plan->L) return fail(KVTC_EINVAL, "layer out of range");
+  if (dtype != KVTC_F32 && dtype != KVTC_BF16) return fail(KVTC_EINVAL, "dtype must be F32 or BF16");
+  if (n_tok < 0 || cache->n_seq < 1 || cache->max_pages < 1) return fail(KVTC_EINVAL, "bad sizes");
+  if (n_tok == 0) return KVTC_OK;
+  if (!k || !v || !cu_seqlens || !pos_start) return fail(KVTC_EINVAL, "null device pointer");
+  if (reinterpret_cast<uintptr_t>(cache->pool) & 15) return fail(KVTC_EINVAL, "pool must be 16-byte aligned");
+  AppendArgs a;
+  a.units = plan->d_units;
+  a.unit0 = layer * plan->H * 2;
+  a.n_units = plan->H * 2;
+  a.H = plan->H;
+  a.k = k;
+  a.v = v;
+  a.bf16 = dtype == KVTC_BF16;
+  a.cu_seqlens = cu_seqlens;
+  a.pos_start = pos_start;
+  a.n_seq = cache->n_seq;
+  a.n_tok = n_tok;
+  a.coords_per_token = 0;
+  for (int ul = 0; ul < a.n_units; ++ul) a.coords_per_token += plan->r[a.unit0 + ul];
+  a.pool = static_cast<char*>(cache->pool);
+  a.pages_per_unit = cache->pages_per_unit;
+  a.block_table = cache->block_table;
+  a.max_pages = cache->max_pages;
+  a.status = cache->status;
+  const long long total = static_cast<long long>(n_tok) * a.coords_per_token;
+  const long long blocks = (total + 127) / 128;
+  if (blocks > 0x7FFFFFFFll) return fail(KVTC_EINVAL, "too many tokens for one call");
+  encode_append_kernel<<<static_cast<unsigned>(blocks), 128, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "encode_append launch");
+  return KVTC_OK;
+}

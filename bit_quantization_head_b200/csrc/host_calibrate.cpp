@@ -1,0 +1,419 @@
+// kvtc_calibrate: per-unit eigenbasis, attention-KL weights, C1 + C2 allocation, folded
+// random-sign Walsh-Hadamard projection and Gaussian quantizer step.
+//
+// Source: KV-COBRA project page, "How KV-COBRA Works" (distortion D(r,b), calibration),
+// "C1, per head", "C2, across heads", "Hadamard rotation", "Attention-KL reordering";
+// joint K+V pool per the KV-COBRA abstract.  The eigen-solver here is cyclic Jacobi
+// (a different algorithm from the LAPACK routine the oracle uses), run on host threads
+// over units.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <memory>
+#include <thread>
+#include <vector>
+
+#include "kvtc_internal.h"
+
+namespace kvtc {
+namespace {
+
+// ------------------------------------------------------------------ eigen-solver
+// Cyclic Jacobi on a symmetric n x n matrix A (row-major, destroyed).  On return lam
+// holds the eigenvalues in descending order and V (row-major, column i = eigenvector
+// i) the eigenvectors, each with its largest-magnitude component positive (ties: the
+// lowest index).
+void jacobi_eig(std::vector<double>& A, int n, std::vector<double>& lam, std::vector<double>& V) {
+  V.assign(static_cast<size_t>(n) * n, 0.0);
+  for (int i = 0; i < n; ++i) V[i * n + i] = 1.0;
+  double fro = 0.0;
+  for (double x : A) fro += x * x;
+  fro = std::sqrt(fro);
+  for (int sweep = 0; sweep < 60; ++sweep) {
+    double off = 0.0;
+    for (int p = 0; p < n; ++p)
+      for (int q = p + 1; q < n; ++q) off += A[p * n + q] * A[p * n + q];
+    if (std::sqrt(2.0 * off) <= 1e-17 * fro || off == 0.0) break;
+    for (int p = 0; p < n - 1; ++p) {
+      for (int q = p + 1; q < n; ++q) {
+        double apq = A[p * n + q];
+        if (apq == 0.0) continue;
+        double app = A[p * n + p], aqq = A[q * n + q];
+        double theta = (aqq - app) / (2.0 * apq);
+        double t = (theta >= 0 ? 1.0 : -1.0) / (std::fabs(theta) + std::sqrt(theta * theta + 1.0));
+        double c = 1.0 / std::sqrt(t * t + 1.0), s = t * c;
+        // A <- J^T A J with J the rotation in the (p, q) plane.
+        for (int k = 0; k < n; ++k) {
+          double akp = A[k * n + p], akq = A[k * n + q];
+          A[k * n + p] = c * akp - s * akq;
+          A[k * n + q] = s * akp + c * akq;
+        }
+        for (int k = 0; k < n; ++k) {
+          double apk = A[p * n + k], aqk = A[q * n + k];
+          A[p * n + k] = c * apk - s * aqk;
+          A[q * n + k] = s * apk + c * aqk;
+        }
+        A[p * n + q] = A[q * n + p] = 0.0;
+        for (int k = 0; k < n; ++k) {
+          double vkp = V[k * n + p], vkq = V[k * n + q];
+          V[k * n + p] = c * vkp - s * vkq;
+          V[k * n + q] = s * vkp + c * vkq;
+        }
+      }
+    }
+  }
+  std::vector<int> idx(n);
+  for (int i = 0; i < n; ++i) idx[i] = i;
+  std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return A[a * n + a] > A[b * n + b]; });
+  lam.resize(n);
+  std::vector<double> W(static_cast<size_t>(n) * n);
+  for (int j = 0; j < n; ++j) {
+    int src = idx[j];
+    lam[j] = A[src * n + src];
+    int kmax = 0;
+    for (int k = 1; k < n; ++k)
+      if (std::fabs(V[k * n + src]) > std::fabs(V[kmax * n + src])) kmax = k;
+    double sgn = V[kmax * n + src] < 0 ? -1.0 : 1.0;
+    for (int k = 0; k < n; ++k) W[k * n + j] = sgn * V[k * n + src];
+  }
+  V.swap(W);
+}
+
+// ------------------------------------------------------------------ model pieces
+double q_of_b(int b) { return std::ldexp(1.0, -2 * b) / 12.0; }
+
+// D(r,b) = sum_{i>r} w_i + q(b) sum_{i<=r} w_i (w sorted descending).
+double distortion(const std::vector<double>& w, int r, int b) {
+  double tail = 0.0, head = 0.0;
+  for (int i = r; i < static_cast<int>(w.size()); ++i) tail += w[i];
+  for (int i = 0; i < r; ++i) head += w[i];
+  return tail + q_of_b(b) * head;
+}
+
+// C1: b = min(8, floor(B/r)), feasible iff b >= 2; min D, ties -> fewer bits, smaller r.
+bool c1(const std::vector<double>& w, int B, int& r_out, int& b_out) {
+  bool found = false;
+  double bestD = 0.0;
+  int bestBits = 0, bestR = 0, bestB = 0;
+  int d = static_cast<int>(w.size());
+  for (int r = 2; r <= d; r += 2) {
+    int b = std::min(8, B / r);
+    if (b < 2) continue;
+    double D = distortion(w, r, b);
+    bool better = !found || D < bestD || (D == bestD && (r * b < bestBits || (r * b == bestBits && r < bestR)));
+    if (better) {
+      found = true;
+      bestD = D;
+      bestBits = r * b;
+      bestR = r;
+      bestB = b;
+    }
+  }
+  r_out = bestR;
+  b_out = bestB;
+  return found;
+}
+
+struct Cand {
+  int r, b, bits;
+};
+
+// Candidates (r even in [2,d], b in [2,8]) ordered by (bits, r).
+std::vector<Cand> candidates(int d) {
+  std::vector<Cand> c;
+  for (int r = 2; r <= d; r += 2)
+    for (int b = 2; b <= 8; ++b) c.push_back({r, b, r * b});
+  std::stable_sort(c.begin(), c.end(), [](const Cand& x, const Cand& y) {
+    return x.bits != y.bits ? x.bits < y.bits : x.r < y.r;
+  });
+  return c;
+}
+
+// C2 in Lagrangian form: bisect mu so that sum_u bits(argmin D_u + mu*bits) fits the
+// budget, spend the leftover greedily on the best distortion drop per bit, and give each
+// unit C1 at its resulting budget.
+bool c2(const std::vector<std::vector<double>>& ws, long long total_bits, std::vector<int>& r_out,
+        std::vector<int>& b_out, double& mu_out) {
+  const int U = static_cast<int>(ws.size());
+  const int d = static_cast<int>(ws[0].size());
+  const std::vector<Cand> cand = candidates(d);
+  const int n = static_cast<int>(cand.size());
+  std::vector<double> D(static_cast<size_t>(U) * n);
+  for (int u = 0; u < U; ++u)
+    for (int c = 0; c < n; ++c) D[static_cast<size_t>(u) * n + c] = distortion(ws[u], cand[c].r, cand[c].b);
+  auto pick = [&](int u, double mu) {
+    int best = 0;
+    double bv = D[static_cast<size_t>(u) * n] + mu * static_cast<double>(cand[0].bits);
+    for (int c = 1; c < n; ++c) {
+      double v = D[static_cast<size_t>(u) * n + c] + mu * static_cast<double>(cand[c].bits);
+      if (v < bv) {
+        bv = v;
+        best = c;
+      }
+    }
+    return best;
+  };
+  auto bits_at = [&](double mu) {
+    long long t = 0;
+    for (int u = 0; u < U; ++u) t += cand[pick(u, mu)].bits;
+    return t;
+  };
+  double lo = 0.0, hi = 1.0;
+  while (bits_at(hi) > total_bits) {
+    hi *= 2.0;
+    if (hi > 1e300) return false;
+  }
+  if (bits_at(lo) <= total_bits) {
+    hi = lo;
+  } else {
+    for (int it = 0; it < 200; ++it) {
+      double mid = 0.5 * (lo + hi);
+      if (bits_at(mid) <= total_bits)
+        hi = mid;
+      else
+        lo = mid;
+    }
+  }
+  std::vector<int> sel(U);
+  long long used = 0;
+  for (int u = 0; u < U; ++u) {
+    sel[u] = pick(u, hi);
+    used += cand[sel[u]].bits;
+  }
+  long long left = total_bits - used;
+  for (;;) {
+    int bu = -1, bc = -1;
+    double bg = 0.0;
+    for (int u = 0; u < U; ++u) {
+      const int b0 = cand[sel[u]].bits;
+      const double D0 = D[static_cast<size_t>(u) * n + sel[u]];
+      for (int c = 0; c < n; ++c) {
+        const int extra = cand[c].bits - b0;
+        const double Dc = D[static_cast<size_t>(u) * n + c];
+        if (extra <= 0 || extra > left || !(Dc < D0)) continue;
+        const double g = (D0 - Dc) / extra;
+        if (bu < 0 || g > bg) {
+          bu = u;
+          bc = c;
+          bg = g;
+        }
+      }
+    }
+    if (bu < 0) break;
+    left -= cand[bc].bits - cand[sel[bu]].bits;
+    sel[bu] = bc;
+  }
+  r_out.resize(U);
+  b_out.resize(U);
+  for (int u = 0; u < U; ++u)
+    if (!c1(ws[u], cand[sel[u]].bits, r_out[u], b_out[u])) return false;
+  mu_out = hi;
+  return true;
+}
+
+// ------------------------------------------------------------------ quantizer step
+double phi(double x) { return std::isfinite(x) ? std::exp(-0.5 * x * x) / std::sqrt(2.0 * M_PI) : 0.0; }
+double Phi(double x) {
+  if (x == INFINITY) return 1.0;
+  if (x == -INFINITY) return 0.0;
+  return 0.5 * std::erfc(-x / std::sqrt(2.0));
+}
+
+// Slope of the MSE of the 2^b-level mid-rise uniform quantizer on N(0,1) w.r.t. its step.
+double mse_slope(double step, int b) {
+  const int L = 1 << b;
+  double t = 0.0;
+  for (int k = 0; k < L; ++k) {
+    double lo = k == 0 ? -INFINITY : (k - L / 2.0) * step;
+    double hi = k == L - 1 ? INFINITY : (k + 1 - L / 2.0) * step;
+    double ck = k - (L - 1) / 2.0;
+    t += ck * (phi(lo) - phi(hi) - ck * step * (Phi(hi) - Phi(lo)));
+  }
+  return -2.0 * t;
+}
+
+// g(b): root of the slope by bisection.
+double gaussian_step(int b) {
+  double lo = 1e-3, hi = 4.0;
+  for (int it = 0; it < 200; ++it) {
+    double mid = 0.5 * (lo + hi);
+    if (mse_slope(mid, b) < 0.0)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+// ------------------------------------------------------------------ Hadamard
+uint64_t splitmix64_at(uint64_t seed, uint64_t n) {
+  uint64_t z = seed + (n + 1) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Entry (i, j) of the orthonormal block Walsh-Hadamard of order r (blocks: powers of two
+// of r's binary expansion, largest first; Sylvester entry sign = (-1)^popcount(i & j)).
+double block_hadamard_entry(int r, int i, int j) {
+  int off = 0;
+  for (int bit = 30; bit >= 0; --bit) {
+    int n = 1 << bit;
+    if (!(r & n)) continue;
+    if (i >= off && i < off + n) {
+      if (j < off || j >= off + n) return 0.0;
+      int a = i - off, c = j - off;
+      return (__builtin_popcount(a & c) & 1 ? -1.0 : 1.0) / std::sqrt(static_cast<double>(n));
+    }
+    off += n;
+  }
+  return 0.0;
+}
+
+struct UnitWork {
+  std::vector<double> w, lam, Vs;  // Vs: d x d row-major, column i = i-th sorted vector
+};
+
+}  // namespace
+}  // namespace kvtc
+
+using namespace kvtc;
+
+extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* k_cal, const float* v_cal,
+                                      const float* q_cal, kvtc_plan** out) {
+  if (!desc || !k_cal || !v_cal || !out) return fail(KVTC_EINVAL, "null argument");
+  *out = nullptr;
+  const int L = desc->n_layers, H = desc->n_kv_heads, G = desc->group, d = desc->head_dim, N = desc->n_cal;
+  if (L < 1 || H < 1 || G < 1 || N < 2) return fail(KVTC_EINVAL, "bad calibration shape");
+  if (d != kD) return fail(KVTC_EINVAL, "head_dim must be 128");
+  const bool kl = desc->weight_mode == KVTC_WEIGHTS_KL;
+  if (!kl && desc->weight_mode != KVTC_WEIGHTS_MSE) return fail(KVTC_EINVAL, "bad weight_mode");
+  if (kl && !q_cal) return fail(KVTC_EINVAL, "KL weights need calibration queries");
+  const bool fixed = desc->fixed_r > 0 || desc->fixed_b > 0;
+  if (fixed && (desc->fixed_r < 2 || desc->fixed_r > d || (desc->fixed_r & 1) || desc->fixed_b < 2 ||
+                desc->fixed_b > 8))
+    return fail(KVTC_EINVAL, "fixed_r must be even in [2,128] and fixed_b in [2,8]");
+  const int U = 2 * L * H;
+  if (!fixed && !(desc->bpd > 0.0)) return fail(KVTC_EINVAL, "bpd must be > 0");
+
+  std::vector<UnitWork> work(U);
+  std::atomic<int> next(0);
+  auto worker = [&]() {
+    std::vector<double> C(static_cast<size_t>(d) * d), lam, V;
+    for (;;) {
+      int u = next.fetch_add(1);
+      if (u >= U) break;
+      const int kind = u & 1, head = (u >> 1) % H, layer = (u >> 1) / H;
+      const float* X = (kind == 0 ? k_cal : v_cal) + (static_cast<size_t>(layer) * H + head) * N * d;
+      std::fill(C.begin(), C.end(), 0.0);
+      for (int t = 0; t < N; ++t) {
+        const float* x = X + static_cast<size_t>(t) * d;
+        for (int i = 0; i < d; ++i) {
+          const double xi = x[i];
+          double* row = &C[static_cast<size_t>(i) * d];
+          for (int j = i; j < d; ++j) row[j] += xi * static_cast<double>(x[j]);
+        }
+      }
+      for (int i = 0; i < d; ++i)
+        for (int j = i; j < d; ++j) {
+          C[i * d + j] /= N;
+          C[j * d + i] = C[i * d + j];
+        }
+      jacobi_eig(C, d, lam, V);
+      std::vector<double> wraw(lam);
+      if (kind == 0 && kl) {
+        const float* Q = q_cal + (static_cast<size_t>(layer) * H + head) * G * N * d;
+        std::vector<double> sq(d, 0.0), proj(d);
+        const size_t nq = static_cast<size_t>(G) * N;
+        for (size_t t = 0; t < nq; ++t) {
+          const float* q = Q + t * d;
+          std::fill(proj.begin(), proj.end(), 0.0);
+          for (int k = 0; k < d; ++k) {
+            const double qk = q[k];
+            const double* vr = &V[static_cast<size_t>(k) * d];
+            for (int i = 0; i < d; ++i) proj[i] += qk * vr[i];
+          }
+          for (int i = 0; i < d; ++i) sq[i] += proj[i] * proj[i];
+        }
+        for (int i = 0; i < d; ++i) wraw[i] = (sq[i] / nq) * lam[i];
+      }
+      std::vector<int> ord(d);
+      for (int i = 0; i < d; ++i) ord[i] = i;
+      std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return wraw[a] > wraw[b]; });
+      UnitWork& wk = work[u];
+      wk.w.resize(d);
+      wk.lam.resize(d);
+      wk.Vs.resize(static_cast<size_t>(d) * d);
+      for (int i = 0; i < d; ++i) {
+        wk.w[i] = wraw[ord[i]];
+        wk.lam[i] = lam[ord[i]];
+        for (int k = 0; k < d; ++k) wk.Vs[static_cast<size_t>(k) * d + i] = V[static_cast<size_t>(k) * d + ord[i]];
+      }
+    }
+  };
+  unsigned nth = std::max(1u, std::min(std::thread::hardware_concurrency(), 64u));
+  nth = std::min<unsigned>(nth, static_cast<unsigned>(U));
+  {
+    std::vector<std::thread> pool;
+    for (unsigned i = 1; i < nth; ++i) pool.emplace_back(worker);
+    worker();
+    for (auto& t : pool) t.join();
+  }
+
+  std::vector<int> R(U), B(U);
+  double mu = 0.0;
+  if (fixed) {
+    std::fill(R.begin(), R.end(), desc->fixed_r);
+    std::fill(B.begin(), B.end(), desc->fixed_b);
+  } else {
+    const long long total = std::llround(desc->bpd * d * U);
+    if (4ll * U > total) return fail(KVTC_EINFEASIBLE, "budget below 4 bits per unit");
+    std::vector<std::vector<double>> ws(U);
+    for (int u = 0; u < U; ++u) ws[u] = work[u].w;
+    if (!c2(ws, total, R, B, mu)) return fail(KVTC_EINFEASIBLE, "no allocation meets the budget");
+  }
+
+  std::unique_ptr<kvtc_plan> p(new (std::nothrow) kvtc_plan());
+  if (!p) return fail(KVTC_ENOMEM, "out of host memory");
+  p->L = L;
+  p->H = H;
+  p->G = G;
+  p->d = d;
+  p->U = U;
+  p->mu = mu;
+  double gstep[9] = {0};
+  for (int b = 2; b <= 8; ++b) gstep[b] = gaussian_step(b);
+  for (int u = 0; u < U; ++u) {
+    const int r = R[u], b = B[u];
+    const UnitWork& wk = work[u];
+    double mean = 0.0;
+    for (int i = 0; i < r; ++i) mean += wk.lam[i];
+    mean /= r;
+    const double sigma = std::sqrt(mean);
+    const double delta = gstep[b] * sigma;
+    std::vector<double> eps(r);
+    for (int i = 0; i < r; ++i) eps[i] = (splitmix64_at(desc->seed, static_cast<uint64_t>(u) * 256 + i) >> 63) ? -1.0 : 1.0;
+    std::vector<float> M(static_cast<size_t>(r) * d);
+    for (int i = 0; i < r; ++i)
+      for (int k = 0; k < d; ++k) {
+        double acc = 0.0;
+        for (int j = 0; j < r; ++j) {
+          const double h = block_hadamard_entry(r, i, j);
+          if (h != 0.0) acc += h * eps[j] * wk.Vs[static_cast<size_t>(k) * d + j];
+        }
+        M[static_cast<size_t>(i) * d + k] = static_cast<float>(acc);
+      }
+    p->r.push_back(r);
+    p->b.push_back(b);
+    p->delta.push_back(delta);
+    p->inv_delta.push_back(static_cast<float>(1.0 / delta));
+    p->sigma.push_back(sigma);
+    p->D.push_back(distortion(wk.w, r, b));
+    p->M.push_back(std::move(M));
+    p->w.push_back(wk.w);
+    p->lam.push_back(wk.lam);
+  }
+  *out = p.release();
+  return KVTC_OK;
+}

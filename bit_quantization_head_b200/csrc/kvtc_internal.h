@@ -1,0 +1,53 @@
+// Internal declarations shared by the host side and the CUDA kernels of libkvtc.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "../../include/kvtc.h"
+
+namespace kvtc {
+
+constexpr int kPage = KVTC_PAGE_TOKENS;
+constexpr int kD = KVTC_HEAD_DIM;
+
+// Per-unit parameters as the kernels read them (device array, one per unit).
+struct UnitDesc {
+  int r;               // retained coordinates (even, 2..128)
+  int b;               // bits per code (2..8)
+  float delta;         // quantizer step
+  float inv_delta;     // fp32(1/delta)
+  uint64_t page_bytes; // 16 * r * b
+  uint64_t prefix;     // sum of page_bytes over the units before this one
+  const float* M;      // device fp32 [r][d]
+  const uint16_t* Mbf; // device bf16 bits [r][d] (round-to-nearest-even of M)
+  float mnorm;         // largest row 2-norm of the bf16 M (rounded up)
+};
+
+// Sets the thread-local error message and returns the status.
+kvtc_status fail(kvtc_status s, const std::string& msg);
+kvtc_status cuda_fail(int err, const char* what);
+
+}  // namespace kvtc
+
+struct kvtc_plan {
+  int L = 0, H = 0, G = 0, d = 0, U = 0;
+  std::vector<int> r, b;
+  std::vector<double> delta, sigma, D;
+  std::vector<float> inv_delta;
+  std::vector<std::vector<float>> M;       // [U][r*d]
+  std::vector<std::vector<double>> w, lam; // [U][d] (empty for imported plans)
+  double mu = 0.0;
+  // device copy (kvtc_plan_upload)
+  int device = -1;
+  kvtc::UnitDesc* d_units = nullptr;
+  float* d_M = nullptr;
+  uint16_t* d_Mbf = nullptr;
+  std::vector<kvtc::UnitDesc> h_units;      // descriptors with device pointers
+};
+
+namespace kvtc {
+// Validates that the plan is uploaded to the current device.
+kvtc_status check_uploaded(const kvtc_plan* plan);
+}  // namespace kvtc

@@ -5,7 +5,7 @@ Bit-Rank Allocation"), sections "How KV-COBRA Works" (distortion model, calibrat
 inference), "C1, per head", "C2, across heads", "Hadamard rotation" and
 "Attention-KL reordering"; joint K+V allocation from the KV-COBRA abstract.
 
-Readings taken where the page is silent (each is listed in the design doc):
+Readings taken where the page is silent:
   * the "SVD of prefill keys" is the eigen-decomposition of the uncentered second
     moment C = X^T X / N (its eigenvectors are the right singular vectors of X);
   * for a value unit the weights are the eigenvalues (MSE weights), since the page

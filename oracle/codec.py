@@ -5,7 +5,7 @@ and truncated with H.V^T and quantized with its head's b*-bit quantizer) and
 "Efficiency" (the cache is stored as packed b-bit codes), and the "0 per-token
 overhead" figure (only per-unit static parameters exist).
 
-Readings (listed in DESIGN.md):
+Readings taken where the page is silent:
   * Projection arithmetic is fp32, the exact canonical order: for each output
     coordinate j, acc <- fma(x_k, M_jk, acc) for k = 0..d-1 ascending, acc starts at
     0, each fma rounded once (round to nearest even).  Operands: the input values
