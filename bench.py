@@ -250,9 +250,11 @@ def blas_threads():
         return 1
 
 
-def encode_bench(torch, w, steps, warmup, rank):
+def encode_bench(torch, w, steps, warmup, rank, n_layers=None):
     """Encode Mtok/s: every layer's K and V of 131072 tokens, resident in HBM."""
     dev = torch.device("cuda")
+    if n_layers:
+        w = synth.scaled(w, n_layers=n_layers)
     k_cal, v_cal, q_cal = synth.calibration_set(w)
     plan = kvtc.kvtc_calibrate(k_cal, v_cal, q_cal, n_layers=w.n_layers, n_kv_heads=w.n_kv_heads,
                                group=w.group, bpd=w.bpd, seed=w.seed).upload()
@@ -281,6 +283,7 @@ def encode_bench(torch, w, steps, warmup, rank):
     for _ in range(max(1, warmup)):
         one_pass()
     torch.cuda.synchronize()
+    fix = kvtc.kvtc_plan_prefill_stats(plan, reset=True) if use_prefill else (0, 0)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(steps):
@@ -292,13 +295,19 @@ def encode_bench(torch, w, steps, warmup, rank):
     code_bytes = sum(T * plan.unit(u)["r"] * plan.unit(u)["b"] // 8 for u in range(plan.shape["n_units"]))
     flops = sum(2 * 128 * plan.unit(u)["r"] for u in range(plan.shape["n_units"])) * T
     return {"workload": w.name, "path": "prefill (tensor cores)" if use_prefill else "append (CUDA cores)",
+            "recomputed_fraction": (fix[1] / fix[0]) if fix[0] else None,
             "ms_per_pass": ms, "mtok_s": T / ms / 1e3, "gb_s": (in_bytes + code_bytes) / ms / 1e6,
             "bytes_per_pass": in_bytes + code_bytes, "tflop_s": flops / ms / 1e9, "layers": w.n_layers}
 
 
 def run_ours(args, torch, dist, rank, world):
     w = synth.WORKLOADS[args.workload]
+    if args.layers:
+        w = synth.scaled(w, n_layers=args.layers)
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+    if args.no_decode:
+        return {"encode": encode_bench(torch, synth.WORKLOADS[ENCODE_WORKLOAD], max(1, min(args.steps, 5)),
+                                       args.warmup, rank, args.encode_layers)}
     st = build_decode_setup(torch, w, rank)
     plan = st["plan"]
     stream = torch.cuda.Stream()
@@ -324,14 +333,15 @@ def run_ours(args, torch, dist, rank, world):
         decode_step(st, w, events=events, stream=stream)
     torch.cuda.synchronize()
 
-    for _ in range(max(3, args.warmup)):
-        g.replay()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            g.replay()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     gpu_id = torch.cuda.get_device_properties(torch.cuda.current_device()).uuid
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(f"GPU-{gpu_id}") as clk:
+    with ClockSampler(f"GPU-{gpu_id}") as clk, torch.cuda.stream(stream):
         torch.cuda.synchronize()
         e0.record(stream)
         for _ in range(args.steps):
@@ -348,7 +358,8 @@ def run_ours(args, torch, dist, rank, world):
     # per-launch duration of the dominant kernel (decode call of one layer)
     durs = []
     for _ in range(max(1, min(args.steps, 10))):
-        g_ev.replay()
+        with torch.cuda.stream(stream):
+            g_ev.replay()
         torch.cuda.synchronize()
         durs.extend(events[l][0].elapsed_time(events[l][1]) for l in range(L))
     dec_ms = statistics.mean(durs)
@@ -409,7 +420,7 @@ def run_ours(args, torch, dist, rank, world):
     }
     if not args.no_encode:
         res["encode"] = encode_bench(torch, synth.WORKLOADS[ENCODE_WORKLOAD], max(1, min(args.steps, 5)),
-                                     args.warmup, rank)
+                                     args.warmup, rank, args.encode_layers)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         b, t, heads = cpu_baseline_decode(torch, st, w)
         res["cpu_baseline"] = {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
@@ -473,6 +484,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DECODE_WORKLOAD)
     ap.add_argument("--no-encode", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="encode measurement only (profiling)")
+    ap.add_argument("--encode-layers", type=int, default=0, help="limit the encode workload's layers")
+    ap.add_argument("--layers", type=int, default=0, help="limit the decode workload's layers (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -1,4 +1,23 @@
-// Decode kernels (templates).  Included by decode.cu and the per-b_K instantiation units.
+// Decode split kernel (templates).  Included by decode.cu and the per-variant
+// instantiation units decode_v*.cu.
+//
+// CTA = (context split, KV head [, head group of 8], sequence); four warps, each streaming
+// its own pages through a ring of cp.async.bulk + mbarrier stages.  Per 16-token block a
+// warp
+//   * scores its G (<= 8) query heads with m16n8k16 MMAs whose A operand comes straight
+//     from the packed words: one AND leaves each code in the low mantissa bits of an fp16
+//     half, the exact subnormal c * 2^(e-24), e the field's bit offset (undone in fp32);
+//     q~ is split into fp16 hi + lo, and for G <= 4 the lo half rides in the four unused
+//     columns of the same MMA;
+//   * runs an online softmax whose rescale is lazy: it happens only when a score exceeds
+//     the running max by more than 2^8 (a warp vote), so the common block costs one FFMA
+//     and one ex2 per score;
+//   * stores P in fp16 scaled by 2^(7-e) so that P * A = p * c * 2^-17 for any e, moves it
+//     into the B fragment with movmatrix, and accumulates the value latents with MMAs
+//     whose A operand again comes straight from the packed value words.  One extra A row
+//     of ones (when r_V is not a multiple of 16) accumulates l = sum p with the same
+//     rounded P, so z - m_V * l cancels consistently.
+// Each warp writes (m, l, z) partials; decode.cu merges them and back-projects.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -14,16 +33,19 @@ namespace dec {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kPartStride = 132;     // floats per partial: m, l, z[128], pad
-constexpr int kTargetCtas = 2 * 148; // two CTAs per SM on a B200
+constexpr int kPartStride = 132;      // floats per partial: m, l, 2 pad, z[128]
+constexpr int kTargetCtas = 3 * 148;  // three CTAs per SM on a B200
 constexpr int kMaxHeadsPerLaunch = 64;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLazy = 8.0f;         // log2 of the growth allowed before a rescale
 
 struct DecodeArgs {
   const UnitDesc* units;
   int layer, H, G, n_hg;
-  int heads[kMaxHeadsPerLaunch];  // KV heads handled by this launch
+  int heads[kMaxHeadsPerLaunch];        // KV heads handled by this launch
+  int split_prefix[kMaxHeadsPerLaunch + 1];  // CTAs of head i: [prefix[i], prefix[i+1])
   int n_heads;
+  int part_stride;                       // partial slots per query head in the workspace
   const void* q;
   int q_bf16;
   const int32_t* seq_lens;
@@ -34,73 +56,77 @@ struct DecodeArgs {
   int max_pages;
   int32_t* status;
   float scale;
-  int n_split, pages_per_split, n_stage;
+  int n_stage;
   uint32_t stage_bytes;
   float* ws;  // partials [n_seq][Hq][n_split * kWarps][kPartStride]
 };
 
-// Compile-time description of a b-bit code's parts (widths 8/4/2/1, lowest bits first).
+// ------------------------------------------------------------------ code extraction
+// B in {2, 4, 8}: a single part of width B.  B == 0: any width, parts at run time.
+__host__ __device__ constexpr int pair_offset(int w, int blk, int eta) { return ((2 * blk + eta) % (16 / w)) * w; }
+
+// bit offset e of the code inside each fp16 half after extraction
 template <int B>
-struct CodeParts {
-  static constexpr int n = (B & 8 ? 1 : 0) + (B & 4 ? 1 : 0) + (B & 2 ? 1 : 0) + (B & 1);
-  __host__ __device__ static constexpr int width(int i) {
-    int k = 0;
-    for (int w = 8; w >= 1; w >>= 1)
-      if (B & w) {
-        if (k == i) return w;
-        ++k;
-      }
-    return 0;
-  }
-  __host__ __device__ static constexpr int low(int i) {
-    int k = 0, lo = 0;
-    for (int w = 8; w >= 1; w >>= 1)
-      if (B & w) {
-        if (k == i) return lo;
-        lo += w;
-        ++k;
-      }
-    return 0;
-  }
-  static constexpr bool fast = (B == 2 || B == 4 || B == 8);
-  // bit offset e of the code inside each fp16 half after extraction (fast path only)
-  __host__ __device__ static constexpr int e(int blk, int eta) {
-    return B == 2 ? 4 * (blk & 1) + 2 * eta : (B == 4 ? 4 * eta : 0);
-  }
-};
-
-// Bit offset of the (blk, eta) pair inside a part word of width w.
-__host__ __device__ constexpr int pair_offset(int w, int blk, int eta) {
-  return ((2 * blk + eta) % (16 / w)) * w;
+__host__ __device__ constexpr int e_of(int blk, int eta) {
+  return B == 2 ? 4 * (blk & 1) + 2 * eta : (B == 4 ? 4 * eta : 0);
+}
+template <int B>
+__host__ __device__ constexpr int n_e() {
+  return B == 2 ? 4 : (B == 4 ? 2 : 1);
+}
+template <int B>
+__host__ __device__ constexpr int e_idx(int blk, int eta) {
+  return B == 2 ? 2 * (blk & 1) + eta : (B == 4 ? eta : 0);
 }
 
-// The pair of codes of (blk, eta) from the part words W[p] (one per part), as an fp16x2
-// whose halves are the subnormals c * 2^(e - 24).
 template <int B, int BLK, int ETA>
-__device__ __forceinline__ uint32_t extract_pair(const uint32_t (&W)[CodeParts<B>::n]) {
-  using P = CodeParts<B>;
-  if constexpr (P::fast) {
-    constexpr int off = pair_offset(B, BLK, ETA);
-    constexpr uint32_t m = (1u << B) - 1u;
-    if constexpr (off >= 8) {
-      return (W[0] >> 8) & ((m << (off - 8)) | (m << (off + 8)));
-    } else {
-      return W[0] & ((m << off) | (m << (off + 16)));
-    }
+__device__ __forceinline__ uint32_t fast_pair(uint32_t W) {
+  constexpr int off = pair_offset(B, BLK, ETA);
+  constexpr uint32_t m = (1u << B) - 1u;
+  if constexpr (off >= 8) {
+    return (W >> 8) & ((m << (off - 8)) | (m << (off + 8)));
   } else {
-    uint32_t v = 0;
-#pragma unroll
-    for (int p = 0; p < P::n; ++p) {
-      const int w = P::width(p), lo = P::low(p);
-      const int off = pair_offset(w, BLK, ETA);
-      const uint32_t m = (1u << w) - 1u;
-      v |= ((W[p] >> off) & (m | (m << 16))) << lo;
-    }
-    return v;
+    return W & ((m << off) | (m << (off + 16)));
   }
 }
 
-// Shared-memory layout of one CTA.
+// Run-time part description of a b-bit code, indexed by log2 of the width (8/4/2/1):
+// has[lw] says whether the width-2^lw part exists, lo[lw] its lowest code bit.
+struct Parts {
+  bool has[4];
+  int lo[4];
+};
+__device__ __forceinline__ Parts parts_of(int b) {
+  Parts P;
+  int lo = 0;
+#pragma unroll
+  for (int lw = 3; lw >= 0; --lw) {
+    P.has[lw] = (b >> lw) & 1;
+    P.lo[lw] = lo;
+    if (P.has[lw]) lo += 1 << lw;
+  }
+  return P;
+}
+
+// Generic pair extraction: the code assembled at bits [0, b) of each half (e = 0).
+// W[lw] is the word of the width-2^lw part.
+template <int BLK, int ETA>
+__device__ __forceinline__ uint32_t gen_pair(const uint32_t (&W)[4], const Parts& P) {
+  uint32_t v = 0;
+#pragma unroll
+  for (int lw = 3; lw >= 0; --lw) {
+    if (P.has[lw]) {
+      constexpr int dummy = 0;
+      (void)dummy;
+      const int off = ((2 * BLK + ETA) & ((16 >> lw) - 1)) << lw;
+      const uint32_t m = (1u << (1 << lw)) - 1u;
+      v |= ((W[lw] >> off) & (m | (m << 16))) << P.lo[lw];
+    }
+  }
+  return v;
+}
+
+// ------------------------------------------------------------------ shared memory
 struct SmemHead {
   float q[8][128];   // the launch's query heads (zero beyond G)
   float qt[8][128];  // q~ = M_K q
@@ -108,122 +134,246 @@ struct SmemHead {
   int E[8];          // power-of-two normalisation of q~ for fp16
 };
 
-// Per-warp running state (kept in registers; every index below is compile-time).
-struct WarpState {
+// ------------------------------------------------------------------ per-warp state
+template <int BK, int BV, bool PACK, int NT>
+struct WS {
   const uint32_t* pk;  // K page in shared memory
   const uint32_t* pv;  // V page in shared memory
-  int tok0, seq_len, rK, rV, nks, nmt, g, tq;
-  float alpha[2], beta[2];
-  uint32_t bh[8][2], bl[8][2];
-  float z[8][4];
-  float m_run[2], l_run[2];
+  int tok0, seq_len;
+  int rK, rV, nks, nmt, g, tq;
+  Parts partsK, partsV;
+  int ones_mt, ones_lr;  // m-tile / local row of the ones row (ones_mt < 0: none)
+  // B fragments of q^: PACK -> bq[ks] (hi for g < 4, lo for g >= 4); else bh, bl
+  uint32_t bh[NT][2];
+  uint32_t bl[PACK ? 1 : NT][2];
+  float alpha[2], beta[2], m_run[2];
+  float al[2][n_e<BK == 0 ? 8 : BK>()], nb[2][n_e<BV == 0 ? 8 : BV>()];
+  float z[NT][4];
+  float lcvt[2];  // l accumulated from the fp16 P when there is no ones row
+  uint32_t kw[NT][2], vw[NT][2];  // current words of the fast paths
 };
 
-// One 16-token block of a page: scores, online softmax, value accumulation.
-template <int BK, int BV, int BLK>
-__device__ __forceinline__ void do_block(WarpState& w) {
-  using PK = CodeParts<BK>;
-  using PV = CodeParts<BV>;
-  // ---- scores: S[tok][head] = sum_j codeK[tok][j] * q^[head][j]
-  float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+// Score argument constants: x = al * acc + nb, with e undone in al (key side) and the P
+// scale 2^(7 - e_V) folded into nb (value side).
+template <int BK, int BV, bool PACK, int NT>
+__device__ __forceinline__ void refresh_constants(WS<BK, BV, PACK, NT>& w) {
+  constexpr int NEK = n_e<BK == 0 ? 8 : BK>();
+  constexpr int NEV = n_e<BV == 0 ? 8 : BV>();
 #pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
-    if (ks < w.nks) {
-      uint32_t W0[PK::n], W1[PK::n];
-      const int rho0 = 8 * ks + w.tq, rho1 = rho0 + 4;
+  for (int c = 0; c < 2; ++c) {
 #pragma unroll
-      for (int pp = 0; pp < PK::n; ++pp) {
-        const int wd = PK::width(pp), lo = PK::low(pp);
-        const uint32_t* plane = w.pk + 4 * w.rK * lo;
-        const int wsel = w.g * wd + (BLK * wd) / 8;
-        W0[pp] = 2 * rho0 < w.rK ? plane[rho0 * 8 * wd + wsel] : 0u;
-        W1[pp] = 2 * rho1 < w.rK ? plane[rho1 * 8 * wd + wsel] : 0u;
-      }
-      const uint32_t A0 = extract_pair<BK, BLK, 0>(W0), A1 = extract_pair<BK, BLK, 1>(W0);
-      const uint32_t A2 = extract_pair<BK, BLK, 0>(W1), A3 = extract_pair<BK, BLK, 1>(W1);
-      mma_16816(sc, A0, A1, A2, A3, w.bh[ks][0], w.bh[ks][1]);
-      mma_16816(sc, A0, A1, A2, A3, w.bl[ks][0], w.bl[ks][1]);
+    for (int i = 0; i < NEK; ++i) {
+      const int e = BK == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (BK == 4 ? 4 * i : 0);
+      w.al[c][i] = w.alpha[c] * (1.0f / static_cast<float>(1 << e));
+    }
+    const float base = -(w.beta[c] + (w.m_run[c] == -INFINITY ? 0.0f : w.m_run[c])) + 7.0f;
+#pragma unroll
+    for (int i = 0; i < NEV; ++i) {
+      const int e = BV == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (BV == 4 ? 4 * i : 0);
+      w.nb[c][i] = base - static_cast<float>(e);
     }
   }
-  // rows: sc[0..1] token tok0 + 16*BLK + g (eta 0), sc[2..3] that + 8 (eta 1)
-  constexpr int eK0 = PK::fast ? PK::e(BLK, 0) : 0;
-  constexpr int eK1 = PK::fast ? PK::e(BLK, 1) : 0;
+}
+
+// Loads the words this lane needs for block BLK (fast paths reload when the word changes).
+template <int BK, int BV, bool PACK, int NT, int BLK>
+__device__ __forceinline__ void load_words(WS<BK, BV, PACK, NT>& w) {
+  if constexpr (BK != 0 && (BLK * BK) % 8 == 0) {
+    const int wsel = w.g * BK + (BLK * BK) / 8;
+#pragma unroll
+    for (int ks = 0; ks < NT; ++ks) {
+      if (ks < w.nks) {
+        const int r0 = 8 * ks + w.tq, r1 = r0 + 4;
+        w.kw[ks][0] = 2 * r0 < w.rK ? w.pk[r0 * 8 * BK + wsel] : 0u;
+        w.kw[ks][1] = 2 * r1 < w.rK ? w.pk[r1 * 8 * BK + wsel] : 0u;
+      }
+    }
+  }
+  if constexpr (BV != 0 && (BLK * BV) % 8 == 0) {
+    const int wsel = w.tq * BV + (BLK * BV) / 8;
+#pragma unroll
+    for (int mt = 0; mt < NT; ++mt) {
+      if (mt < w.nmt) {
+        const int j0 = 16 * mt + w.g, j1 = j0 + 8;
+        w.vw[mt][0] = j0 < w.rV ? w.pv[j0 * 4 * BV + wsel] : 0u;
+        w.vw[mt][1] = j1 < w.rV ? w.pv[j1 * 4 * BV + wsel] : 0u;
+      }
+    }
+  }
+}
+
+// Generic words of a K row (or V row) for block BLK: one word per part.
+template <int BLK>
+__device__ __forceinline__ void gen_words(const uint32_t* page, int r, int row, bool ok, int owner, bool is_k,
+                                          const Parts& P, uint32_t (&W)[4]) {
+#pragma unroll
+  for (int lw = 3; lw >= 0; --lw) {
+    W[lw] = 0u;
+    if (P.has[lw] && ok) {
+      const int wd = 1 << lw;
+      const uint32_t* plane = page + 4 * r * P.lo[lw];
+      const int row_words = (is_k ? 8 : 4) * wd;
+      W[lw] = plane[row * row_words + owner * wd + ((BLK * wd) >> 3)];
+    }
+  }
+}
+
+// One 16-token block: scores, lazy online softmax, value accumulation.
+template <int BK, int BV, bool PACK, int NT, int BLK>
+__device__ __forceinline__ void do_block(WS<BK, BV, PACK, NT>& w) {
+  load_words<BK, BV, PACK, NT, BLK>(w);
+  // ---- scores S[tok][head] = sum_j codeK[tok][j] * q^[head][j]
+  float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  float sd[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // second accumulator (lo MMAs) when not packed
+#pragma unroll
+  for (int ks = 0; ks < NT; ++ks) {
+    if (ks < w.nks) {
+      uint32_t A0, A1, A2, A3;
+      if constexpr (BK != 0) {
+        A0 = fast_pair<BK, BLK, 0>(w.kw[ks][0]);
+        A1 = fast_pair<BK, BLK, 1>(w.kw[ks][0]);
+        A2 = fast_pair<BK, BLK, 0>(w.kw[ks][1]);
+        A3 = fast_pair<BK, BLK, 1>(w.kw[ks][1]);
+      } else {
+        uint32_t W0[4], W1[4];
+        const int r0 = 8 * ks + w.tq, r1 = r0 + 4;
+        gen_words<BLK>(w.pk, w.rK, r0, 2 * r0 < w.rK, w.g, true, w.partsK, W0);
+        gen_words<BLK>(w.pk, w.rK, r1, 2 * r1 < w.rK, w.g, true, w.partsK, W1);
+        A0 = gen_pair<BLK, 0>(W0, w.partsK);
+        A1 = gen_pair<BLK, 1>(W0, w.partsK);
+        A2 = gen_pair<BLK, 0>(W1, w.partsK);
+        A3 = gen_pair<BLK, 1>(W1, w.partsK);
+      }
+      if constexpr (PACK) {
+        // alternate two accumulators so consecutive k-steps do not chain
+        if (ks & 1)
+          mma_16816(sd, A0, A1, A2, A3, w.bh[ks][0], w.bh[ks][1]);
+        else
+          mma_16816(sc, A0, A1, A2, A3, w.bh[ks][0], w.bh[ks][1]);
+      } else {
+        mma_16816(sc, A0, A1, A2, A3, w.bh[ks][0], w.bh[ks][1]);
+        mma_16816(sd, A0, A1, A2, A3, w.bl[ks][0], w.bl[ks][1]);
+      }
+    }
+  }
+  float full[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (PACK) {
+      const float t = sc[i] + sd[i];
+      full[i] = t + __shfl_xor_sync(0xffffffffu, t, 2);  // hi (t' < 2) + lo (t' >= 2)
+    } else {
+      full[i] = sc[i] + sd[i];
+    }
+  }
+  // rows: full[0..1] token tok0 + 16*BLK + g (eta 0), full[2..3] that + 8 (eta 1)
+  constexpr int ik0 = e_idx<BK == 0 ? 8 : BK>(BLK, 0), ik1 = e_idx<BK == 0 ? 8 : BK>(BLK, 1);
+  constexpr int iv0 = e_idx<BV == 0 ? 8 : BV>(BLK, 0), iv1 = e_idx<BV == 0 ? 8 : BV>(BLK, 1);
+  constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
   const int t0 = w.tok0 + 16 * BLK + w.g, t1 = t0 + 8;
-  float s2[4];
+  const bool live0 = t0 < w.seq_len, live1 = t1 < w.seq_len;
+  float x[4];
+  x[0] = live0 ? fmaf(w.al[0][ik0], full[0], w.nb[0][iv0]) : -INFINITY;
+  x[1] = live0 ? fmaf(w.al[1][ik0], full[1], w.nb[1][iv0]) : -INFINITY;
+  x[2] = live1 ? fmaf(w.al[0][ik1], full[2], w.nb[0][iv1]) : -INFINITY;
+  x[3] = live1 ? fmaf(w.al[1][ik1], full[3], w.nb[1][iv1]) : -INFINITY;
+  // ---- lazy online softmax: x = s - m_run + 7 - e_V; rescale only past 2^kLazy
+  constexpr float lim0 = kLazy + 7.0f - ev0, lim1 = kLazy + 7.0f - ev1;
+  // grow also on the first live block (the running max starts undefined)
+  const bool grow = x[0] > lim0 || x[1] > lim0 || x[2] > lim1 || x[3] > lim1 ||
+                    ((w.m_run[0] == -INFINITY || w.m_run[1] == -INFINITY) && (live0 || live1));
+  if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    s2[c] = t0 < w.seq_len ? fmaf(w.alpha[c] * (1.0f / (1 << eK0)), sc[c], -w.beta[c]) : -INFINITY;
-    s2[2 + c] = t1 < w.seq_len ? fmaf(w.alpha[c] * (1.0f / (1 << eK1)), sc[2 + c], -w.beta[c]) : -INFINITY;
-  }
-  // ---- online softmax (log2 domain); block max over the 16 tokens of each head
-  float resc[2];
+    for (int c = 0; c < 2; ++c) {
+      // block max of the true scores s = x - nb + beta... in the m_run frame: s - m_run
+      float v = fmaxf(x[c] - (7.0f - ev0), x[2 + c] - (7.0f - ev1));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+      // v = block max of (s - m_run); the new running max is m_run + max(v, 0)
+      const float old = w.m_run[c];
+      float shift = 0.0f;
+      if (v == -INFINITY) {
+        // no live token of this head in the block: nothing to do
+      } else if (old == -INFINITY) {
+        // first scores of this warp: x was computed with m_run taken as 0
+        w.m_run[c] = v;  // v is the true block max here
+        shift = v;
+      } else if (v > 0.0f) {
+        w.m_run[c] = old + v;
+        shift = v;
+        const float resc = ex2(-v);
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    float v = fmaxf(s2[c], s2[2 + c]);
-    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-    const float mn = fmaxf(w.m_run[c], v);
-    resc[c] = mn == -INFINITY ? 1.0f : ex2(w.m_run[c] - mn);
-    w.m_run[c] = mn;
-    w.l_run[c] *= resc[c];
+        for (int mt = 0; mt < NT; ++mt) {
+          w.z[mt][c] *= resc;
+          w.z[mt][2 + c] *= resc;
+        }
+        w.lcvt[c] *= resc;
+      }
+      x[c] -= shift;
+      x[2 + c] -= shift;
+    }
+    refresh_constants(w);
   }
+  float p[4];
 #pragma unroll
-  for (int mt = 0; mt < 8; ++mt) {
-    w.z[mt][0] *= resc[0];
-    w.z[mt][1] *= resc[1];
-    w.z[mt][2] *= resc[0];
-    w.z[mt][3] *= resc[1];
+  for (int i = 0; i < 4; ++i) p[i] = ex2(x[i]);
+  if constexpr (PACK) {
+    if (w.tq >= 2) p[0] = p[1] = p[2] = p[3] = 0.0f;  // columns 4..7 are the lo MMA
   }
-  // probabilities, stored scaled by 2^(7 - e_V(row)) for the value MMA
-  constexpr int eV0 = PV::fast ? PV::e(BLK, 0) : 0;
-  constexpr int eV1 = PV::fast ? PV::e(BLK, 1) : 0;
-  float pr[4];
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    const float mm = w.m_run[c] == -INFINITY ? 0.0f : w.m_run[c];
-    pr[c] = ex2(s2[c] - mm);
-    pr[2 + c] = ex2(s2[2 + c] - mm);
-  }
-  constexpr float sv0 = static_cast<float>(1 << (7 - eV0)), sv1 = static_cast<float>(1 << (7 - eV1));
-  const uint32_t P0 = pack_half2(pr[0] * sv0, pr[1] * sv0);
-  const uint32_t P1 = pack_half2(pr[2] * sv1, pr[3] * sv1);
-  // l from the same fp16-rounded weights the value MMA uses, so that the centering
-  // z - m_V * l cancels consistently
-  {
+  const uint32_t P0 = pack_half2(p[0], p[1]);
+  const uint32_t P1 = pack_half2(p[2], p[3]);
+  if (w.ones_mt < 0) {
+    // l from the same fp16-rounded weights (no ones row available)
     const float2 f0 = half2_to_float2(P0), f1 = half2_to_float2(P1);
-    w.l_run[0] += fmaf(f0.x, 1.0f / sv0, f1.x * (1.0f / sv1));
-    w.l_run[1] += fmaf(f0.y, 1.0f / sv0, f1.y * (1.0f / sv1));
+    constexpr float u0 = 1.0f / static_cast<float>(1 << (7 - ev0)), u1 = 1.0f / static_cast<float>(1 << (7 - ev1));
+    w.lcvt[0] += fmaf(f0.x, u0, f1.x * u1);
+    w.lcvt[1] += fmaf(f0.y, u0, f1.y * u1);
   }
   const uint32_t b0 = movmatrix_trans(P0), b1 = movmatrix_trans(P1);
   // ---- values: Z^T[j][head] += sum_tok codeV[tok][j] * P[tok][head]
+  constexpr uint32_t one0 = (1u << ev0) | (1u << (ev0 + 16)), one1 = (1u << ev1) | (1u << (ev1 + 16));
 #pragma unroll
-  for (int mt = 0; mt < 8; ++mt) {
+  for (int mt = 0; mt < NT; ++mt) {
     if (mt < w.nmt) {
-      uint32_t W0[PV::n], W1[PV::n];
-      const int j0 = 16 * mt + w.g, j1 = j0 + 8;
-#pragma unroll
-      for (int pp = 0; pp < PV::n; ++pp) {
-        const int wd = PV::width(pp), lo = PV::low(pp);
-        const uint32_t* plane = w.pv + 4 * w.rV * lo;
-        const int wsel = w.tq * wd + (BLK * wd) / 8;
-        W0[pp] = j0 < w.rV ? plane[j0 * 4 * wd + wsel] : 0u;
-        W1[pp] = j1 < w.rV ? plane[j1 * 4 * wd + wsel] : 0u;
+      uint32_t A0, A1, A2, A3;
+      if constexpr (BV != 0) {
+        A0 = fast_pair<BV, BLK, 0>(w.vw[mt][0]);
+        A1 = fast_pair<BV, BLK, 0>(w.vw[mt][1]);
+        A2 = fast_pair<BV, BLK, 1>(w.vw[mt][0]);
+        A3 = fast_pair<BV, BLK, 1>(w.vw[mt][1]);
+      } else {
+        uint32_t W0[4], W1[4];
+        const int j0 = 16 * mt + w.g, j1 = j0 + 8;
+        gen_words<BLK>(w.pv, w.rV, j0, j0 < w.rV, w.tq, false, w.partsV, W0);
+        gen_words<BLK>(w.pv, w.rV, j1, j1 < w.rV, w.tq, false, w.partsV, W1);
+        A0 = gen_pair<BLK, 0>(W0, w.partsV);
+        A1 = gen_pair<BLK, 0>(W1, w.partsV);
+        A2 = gen_pair<BLK, 1>(W0, w.partsV);
+        A3 = gen_pair<BLK, 1>(W1, w.partsV);
       }
-      const uint32_t A0 = extract_pair<BV, BLK, 0>(W0), A1 = extract_pair<BV, BLK, 0>(W1);
-      const uint32_t A2 = extract_pair<BV, BLK, 1>(W0), A3 = extract_pair<BV, BLK, 1>(W1);
+      if (mt == w.ones_mt) {  // the ones row (row r_V) accumulates l
+        if (w.ones_lr == w.g) {
+          A0 = one0;
+          A2 = one1;
+        }
+        if (w.ones_lr == w.g + 8) {
+          A1 = one0;
+          A3 = one1;
+        }
+      }
       mma_16816(w.z[mt], A0, A1, A2, A3, b0, b1);
     }
   }
 }
 
-template <int BK, int BV, int... BLK>
-__device__ __forceinline__ void do_page(WarpState& w, std::integer_sequence<int, BLK...>) {
-  (do_block<BK, BV, BLK>(w), ...);
+template <int BK, int BV, bool PACK, int NT, int... BLK>
+__device__ __forceinline__ void do_page(WS<BK, BV, PACK, NT>& w, std::integer_sequence<int, BLK...>) {
+  (do_block<BK, BV, PACK, NT, BLK>(w), ...);
 }
 
-template <int BK, int BV>
-__global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const DecodeArgs a) {
+template <int BK, int BV, bool PACK, int NT>
+__global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   SmemHead& sh = *reinterpret_cast<SmemHead*>(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sizeof(SmemHead));
@@ -231,8 +381,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const DecodeA
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
-  const int split = blockIdx.x;
-  const int hi = blockIdx.y / a.n_hg, hg = blockIdx.y % a.n_hg;
+  // CTA -> (KV head, context split): heads get splits in proportion to their bytes
+  int hi = 0;
+  while (hi + 1 < a.n_heads && static_cast<int>(blockIdx.x) >= a.split_prefix[hi + 1]) ++hi;
+  const int split = blockIdx.x - a.split_prefix[hi];
+  const int n_split = a.split_prefix[hi + 1] - a.split_prefix[hi];
+  const int hg = blockIdx.y;
   const int s = blockIdx.z;
   const int h = a.heads[hi];
   const int uK = (a.layer * a.H + h) * 2, uV = uK + 1;
@@ -247,13 +401,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const DecodeA
     seq_len = seq_len < 0 ? 0 : a.max_pages * kPage;
   }
   const int n_pages = (seq_len + kPage - 1) / kPage;
-  const int p_begin = split * a.pages_per_split;
-  const int p_end = min(p_begin + a.pages_per_split, n_pages);
+  const int pages_per_split = (n_pages + n_split - 1) / n_split;
+  const int p_begin = split * pages_per_split;
+  const int p_end = min(p_begin + pages_per_split, n_pages);
   const int n_my = p_end > p_begin + warp ? (p_end - p_begin - warp + kWarps - 1) / kWarps : 0;
 
   // ---- prologue: barriers, query, first copies, q~ = M_K q ----
   if (lane == 0)
     for (int i = 0; i < a.n_stage; ++i) mbar_init(&bars[warp * 8 + i], 1);
+  // Programmatic dependent launch: the preceding kernel (e.g. the append that wrote the
+  // newest token) must be complete before pages are read; the next kernel may launch.
+  griddep_wait();
+  griddep_launch_dependents();
   for (int i = tid; i < 8 * 128; i += kThreads) {
     const int gg = i >> 7, k = i & 127;
     float v = 0.0f;
@@ -274,9 +433,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const DecodeA
   auto stage_ptr = [&](int i) {
     return stages + (static_cast<size_t>(warp) * a.n_stage + (i % a.n_stage)) * a.stage_bytes;
   };
-  // Fill the stage of this warp's i-th page (lane 0).  Every use of a stage completes
-  // its barrier phase exactly once: with the copies' bytes, or by a plain arrival when
-  // the page id is invalid.
+  // Fill the stage of this warp's i-th page (lane 0).  Every use of a stage completes its
+  // barrier phase exactly once: with the copies' bytes, or by a plain arrival when the
+  // page id is invalid.
   auto issue = [&](int i) {
     const int p = p_begin + warp + i * kWarps;
     const int32_t pid = bt[p];
@@ -294,28 +453,49 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const DecodeA
   if (lane == 0)
     for (int i = 0; i < n_first; ++i) issue(i);
 
-  for (int i = tid; i < 8 * 128; i += kThreads) {
-    const int gg = i >> 7, j = i & 127;
-    float acc = 0.0f;
-    if (gg < ng && j < rK) {
-      const float* m = dK.M + static_cast<size_t>(j) * kD;
-      for (int k = 0; k < kD; ++k) acc = __fmaf_rn(m[k], sh.q[gg][k], acc);
+  // q~[gg][j] = sum_k M_K[j][k] q[gg][k]: thread j reads row j of M once (float4, each
+  // 128-byte line reused by the same thread) and forms all ng dot products.
+  for (int j = tid; j < 128; j += kThreads) {
+    float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    if (j < rK) {
+      const float4* m4 = reinterpret_cast<const float4*>(dK.M + static_cast<size_t>(j) * kD);
+#pragma unroll 4
+      for (int k = 0; k < 32; ++k) {
+        const float4 m = m4[k];
+#pragma unroll
+        for (int gg = 0; gg < 8; ++gg) {
+          if (gg < ng) {
+            const float4 qv = reinterpret_cast<const float4*>(sh.q[gg])[k];
+            acc[gg] = fmaf(m.x, qv.x, fmaf(m.y, qv.y, fmaf(m.z, qv.z, fmaf(m.w, qv.w, acc[gg]))));
+          }
+        }
+      }
     }
-    sh.qt[gg][j] = acc;
+#pragma unroll
+    for (int gg = 0; gg < 8; ++gg) sh.qt[gg][j] = (gg < ng && j < rK) ? acc[gg] : 0.0f;
   }
   __syncthreads();
-  if (tid < 8) {
-    float S = 0.0f, amax = 0.0f;
-    for (int j = 0; j < rK; ++j) {
-      S += sh.qt[tid][j];
-      amax = fmaxf(amax, fabsf(sh.qt[tid][j]));
+  if (warp == 0) {
+    // per head: S = sum_j q~_j and the fp16 normalisation exponent
+#pragma unroll
+    for (int gg = 0; gg < 8; ++gg) {
+      float S = sh.qt[gg][lane] + sh.qt[gg][lane + 32] + sh.qt[gg][lane + 64] + sh.qt[gg][lane + 96];
+      float amax = fmaxf(fmaxf(fabsf(sh.qt[gg][lane]), fabsf(sh.qt[gg][lane + 32])),
+                         fmaxf(fabsf(sh.qt[gg][lane + 64]), fabsf(sh.qt[gg][lane + 96])));
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        S += __shfl_xor_sync(0xffffffffu, S, o);
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      }
+      if (lane == 0) {
+        sh.S[gg] = S;
+        sh.E[gg] = amax > 0.0f ? ilogbf(amax) - 14 : 0;
+      }
     }
-    sh.S[tid] = S;
-    sh.E[tid] = amax > 0.0f ? ilogbf(amax) - 14 : 0;
   }
   __syncthreads();
 
-  WarpState w;
+  WS<BK, BV, PACK, NT> w;
   w.rK = rK;
   w.rV = rV;
   w.nks = (rK + 15) >> 4;
@@ -323,38 +503,50 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const DecodeA
   w.g = g;
   w.tq = tq;
   w.seq_len = seq_len;
-  // B fragments of q^ = q~ * 2^-E (hi and lo fp16 parts) for head n = g.
+  w.partsK = parts_of(dK.b);
+  w.partsV = parts_of(dV.b);
+  w.ones_mt = (rV & 15) ? (rV >> 4) : -1;
+  w.ones_lr = rV & 15;
+  // B fragments of q^ = q~ * 2^-E.  Packed (G <= 4): column n < 4 holds the hi part of
+  // head n, column n >= 4 the lo part of head n - 4.
   {
-    const float scl = ldexpf(1.0f, -sh.E[g]);
+    const int hsrc = PACK ? (g & 3) : g;
+    const float scl = ldexpf(1.0f, -sh.E[hsrc]);
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
+    for (int ks = 0; ks < NT; ++ks) {
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int k0 = 16 * ks + 8 * half + 2 * tq;
-        const float x0 = sh.qt[g][k0] * scl, x1 = sh.qt[g][k0 + 1] * scl;
+        const float x0 = sh.qt[hsrc][k0] * scl, x1 = sh.qt[hsrc][k0 + 1] * scl;
         const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
         const __half l0 = __float2half_rn(x0 - __half2float(h0)), l1 = __float2half_rn(x1 - __half2float(h1));
-        w.bh[ks][half] = static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
-        w.bl[ks][half] = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
+        const uint32_t hw = static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
+        const uint32_t lw = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
+        if constexpr (PACK) {
+          w.bh[ks][half] = g < 4 ? hw : lw;
+        } else {
+          w.bh[ks][half] = hw;
+          w.bl[ks][half] = lw;
+        }
       }
     }
   }
-  // Score constants (log2 domain) for this lane's heads n = 2tq, 2tq + 1:
-  // s2 = alpha_n * 2^-e * acc - beta_n.
+  // Score constants (log2 domain) for this lane's heads.
   {
-    const float mK = 0.5f * static_cast<float>((1 << BK) - 1);
+    const float mK = 0.5f * static_cast<float>((1 << dK.b) - 1);
     const float base = a.scale * dK.delta * kLog2e;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      const int n = 2 * tq + c;
+      const int n = PACK ? 2 * (tq & 1) + c : 2 * tq + c;
       w.alpha[c] = n < ng ? base * ldexpf(1.0f, sh.E[n] + 24) : 0.0f;
       w.beta[c] = n < ng ? base * mK * sh.S[n] : 0.0f;
       w.m_run[c] = -INFINITY;
-      w.l_run[c] = 0.0f;
+      w.lcvt[c] = 0.0f;
     }
+    refresh_constants(w);
   }
 #pragma unroll
-  for (int mt = 0; mt < 8; ++mt) w.z[mt][0] = w.z[mt][1] = w.z[mt][2] = w.z[mt][3] = 0.0f;
+  for (int mt = 0; mt < NT; ++mt) w.z[mt][0] = w.z[mt][1] = w.z[mt][2] = w.z[mt][3] = 0.0f;
 
   // ---- main loop over this warp's pages ----
   bool dead = false;
@@ -366,7 +558,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const DecodeA
     if (!mbar_wait_bounded_warp(&bars[warp * 8 + (i % a.n_stage)], (i / a.n_stage) & 1)) {
       if (lane == 0 && a.status) atomicOr(a.status, KVTC_STATUS_TIMEOUT);
       dead = true;
-      // drain (bounded) the copies issued after this page
       for (int i2 = i + 1; i2 < next_issue; ++i2)
         (void)mbar_wait_bounded_warp(&bars[warp * 8 + (i2 % a.n_stage)], (i2 / a.n_stage) & 1);
       break;
@@ -376,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const DecodeA
       w.pk = reinterpret_cast<const uint32_t*>(st);
       w.pv = reinterpret_cast<const uint32_t*>(st + bytesK);
       w.tok0 = p * kPage;
-      do_page<BK, BV>(w, std::make_integer_sequence<int, 8>{});
+      do_page<BK, BV, PACK, NT>(w, std::make_integer_sequence<int, 8>{});
     } else if (lane == 0 && a.status) {
       atomicOr(a.status, KVTC_STATUS_BAD_PAGE);
     }
@@ -389,44 +580,61 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const DecodeA
     __syncwarp();
   }
 
-  // ---- write this warp's partials: (m, l, z) per query head ----
+  // ---- l: from the ones row, or the per-lane sums ----
+  float l_out[2];
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
-    float l = w.l_run[c];
-    l += __shfl_xor_sync(0xffffffffu, l, 4);
-    l += __shfl_xor_sync(0xffffffffu, l, 8);
-    l += __shfl_xor_sync(0xffffffffu, l, 16);
-    w.l_run[c] = l;
+    if (w.ones_mt >= 0) {
+      // select z[ones_mt][row] with a masked sum (a select here would be turned into a
+      // run-time index and push the fragments to local memory)
+      float v = 0.0f;
+      const float lo_row = w.ones_lr < 8 ? 1.0f : 0.0f, hi_row = 1.0f - lo_row;
+#pragma unroll
+      for (int mt = 0; mt < NT; ++mt) {
+        const float on = mt == w.ones_mt ? 1.0f : 0.0f;
+        v = fmaf(on * lo_row, w.z[mt][c], fmaf(on * hi_row, w.z[mt][2 + c], v));
+      }
+      // the value sits in lanes with g == ones_lr % 8 (same tq); z holds l * 2^-17
+      const int src = ((w.ones_lr & 7) << 2) | tq;
+      l_out[c] = ldexpf(__shfl_sync(0xffffffffu, v, src), 17);
+    } else {
+      float l = w.lcvt[c];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      l_out[c] = l;
+    }
   }
+
+  // ---- write this warp's partials: (m, l, z) per query head ----
   const int part = split * kWarps + warp;
-  const int n_part = a.n_split * kWarps;
+  const int n_part = a.part_stride;
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
-    const int n = 2 * tq + c;
-    if (n < ng) {
+    const int n = PACK ? 2 * tq + c : 2 * tq + c;  // column of the z fragment
+    const bool real = PACK ? (tq < 2 && n < ng) : n < ng;
+    if (real) {
       float* dst = a.ws + ((static_cast<size_t>(s) * Hq + h * a.G + g0 + n) * n_part + part) * kPartStride;
       if (g == 0) {
         dst[0] = dead ? -INFINITY : w.m_run[c];
-        dst[1] = dead ? 0.0f : w.l_run[c];
+        dst[1] = dead ? 0.0f : l_out[c];
       }
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
+      for (int mt = 0; mt < NT; ++mt) {
         if (mt < w.nmt) {
           const int j0 = 16 * mt + g, j1 = j0 + 8;
-          if (j0 < rV) dst[2 + j0] = dead ? 0.0f : w.z[mt][c];
-          if (j1 < rV) dst[2 + j1] = dead ? 0.0f : w.z[mt][2 + c];
+          if (j0 < rV) dst[4 + j0] = dead ? 0.0f : w.z[mt][c];
+          if (j1 < rV) dst[4 + j1] = dead ? 0.0f : w.z[mt][2 + c];
         }
       }
     }
   }
 }
 
-}  // namespace dec
-}  // namespace kvtc
-
-namespace kvtc {
-namespace dec {
 using SplitFn = void (*)(const DecodeArgs);
-template <int BK> SplitFn split_fn_bk(int bV);
+// Kernel for (code width variants, packed, rank class); widths: 2, 4, 8 or 0 (any).
+template <int BK>
+SplitFn split_fn_bk(int bV, bool pack, bool small);
+
 }  // namespace dec
 }  // namespace kvtc

@@ -1,0 +1,27 @@
+// Instantiations of the decode split kernel for key code width class 2 (0 = any width).
+#include "decode_kernel.cuh"
+
+namespace kvtc {
+namespace dec {
+template <>
+SplitFn split_fn_bk<2>(int bV, bool pack, bool small) {
+    if (bV == 2 && pack == true && small == true) return decode_split_kernel<2, 2, true, 4>;
+    if (bV == 2 && pack == true && small == false) return decode_split_kernel<2, 2, true, 8>;
+    if (bV == 2 && pack == false && small == true) return decode_split_kernel<2, 2, false, 4>;
+    if (bV == 2 && pack == false && small == false) return decode_split_kernel<2, 2, false, 8>;
+    if (bV == 4 && pack == true && small == true) return decode_split_kernel<2, 4, true, 4>;
+    if (bV == 4 && pack == true && small == false) return decode_split_kernel<2, 4, true, 8>;
+    if (bV == 4 && pack == false && small == true) return decode_split_kernel<2, 4, false, 4>;
+    if (bV == 4 && pack == false && small == false) return decode_split_kernel<2, 4, false, 8>;
+    if (bV == 8 && pack == true && small == true) return decode_split_kernel<2, 8, true, 4>;
+    if (bV == 8 && pack == true && small == false) return decode_split_kernel<2, 8, true, 8>;
+    if (bV == 8 && pack == false && small == true) return decode_split_kernel<2, 8, false, 4>;
+    if (bV == 8 && pack == false && small == false) return decode_split_kernel<2, 8, false, 8>;
+    if (bV == 0 && pack == true && small == true) return decode_split_kernel<2, 0, true, 4>;
+    if (bV == 0 && pack == true && small == false) return decode_split_kernel<2, 0, true, 8>;
+    if (bV == 0 && pack == false && small == true) return decode_split_kernel<2, 0, false, 4>;
+    if (bV == 0 && pack == false && small == false) return decode_split_kernel<2, 0, false, 8>;
+    return nullptr;
+}
+}  // namespace dec
+}  // namespace kvtc

@@ -10,6 +10,7 @@
 
 #include "kvtc_internal.h"
 #include "layout.cuh"
+#include "ptx.cuh"
 
 namespace kvtc {
 
@@ -56,7 +57,11 @@ __device__ __forceinline__ void store_code(uint32_t* page, int kind, int r, int 
   }
 }
 
-__global__ void __launch_bounds__(128) encode_append_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constant__ AppendArgs a) {
+  // Programmatic dependent launch: wait for the producer of k/v, then let the next kernel
+  // (typically the decode of this layer) start its prologue.
+  griddep_wait();
+  griddep_launch_dependents();
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long total = static_cast<long long>(a.n_tok) * a.coords_per_token;
   if (gid >= total) return;
@@ -159,8 +164,17 @@ extern "C" kvtc_status kvtc_encode_append(const kvtc_plan* plan, const kvtc_cach
   const long long total = static_cast<long long>(n_tok) * a.coords_per_token;
   const long long blocks = (total + 127) / 128;
   if (blocks > 0x7FFFFFFFll) return fail(KVTC_EINVAL, "too many tokens for one call");
-  encode_append_kernel<<<static_cast<unsigned>(blocks), 128, 0, static_cast<cudaStream_t>(stream)>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(128);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, encode_append_kernel, a);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "encode_append launch");
   return KVTC_OK;
 }

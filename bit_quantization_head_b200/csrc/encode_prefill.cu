@@ -44,6 +44,7 @@ struct PrefillArgs {
   const int32_t* block_table;
   int max_pages;
   int32_t* status;
+  uint64_t* stats;  // [0] codes produced, [1] codes recomputed in canonical order
 };
 
 // Byte offset of element (row, col) (bf16) in the core-matrix layout.
@@ -144,9 +145,15 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const PrefillArgs a) 
   // While the MMA runs: this thread's token norm ||x||_2 (for the error bound).
   const int tok = tid;
   float nx = 0.0f;
-  for (int k = 0; k < kD; ++k) {
-    const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sA + core_off(tok, k)));
-    nx = fmaf(x, x, nx);
+#pragma unroll 4
+  for (int ch = 0; ch < 16; ++ch) {
+    const uint4 xv = *reinterpret_cast<const uint4*>(sA + core_off(tok, ch * 8));
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float x0 = __uint_as_float(xw[q] << 16), x1 = __uint_as_float(xw[q] & 0xFFFF0000u);
+      nx = fmaf(x1, x1, fmaf(x0, x0, nx));
+    }
   }
   const float beta = ldexpf(sqrtf(nx) * 1.001f, -14) * ud.mnorm;
 
@@ -156,6 +163,7 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const PrefillArgs a) 
 
   // ---- epilogue: TMEM lane = token; quantize r latents ----
   const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  uint32_t n_fix = 0;
   for (int c0 = 0; c0 < rpad; c0 += 16) {
     uint32_t v[16];
     __syncwarp();  // tcgen05.ld is .sync.aligned: reconverge after the fixup branches
@@ -176,16 +184,28 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const PrefillArgs a) 
         if (qlo != qhi || !ok) {
           // canonical chain (the arithmetic of kvtc_encode_append)
           float acc = 0.0f;
-          for (int k = 0; k < kD; ++k) {
-            const float xv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sA + core_off(tok, k)));
-            const float mv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sB + core_off(j, k)));
-            acc = __fmaf_rn(xv, mv, acc);
+          for (int ch = 0; ch < 16; ++ch) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(sA + core_off(tok, ch * 8));
+            const uint4 mv = *reinterpret_cast<const uint4*>(sB + core_off(j, ch * 8));
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, mw[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {  // k = 8ch + 2q, then 8ch + 2q + 1: ascending
+              acc = __fmaf_rn(__uint_as_float(xw[q] << 16), __uint_as_float(mw[q] << 16), acc);
+              acc = __fmaf_rn(__uint_as_float(xw[q] & 0xFFFF0000u), __uint_as_float(mw[q] & 0xFFFF0000u), acc);
+            }
           }
           code = quant(acc, ud.inv_delta, b);
+          ++n_fix;
         }
         sC[tok * r + j] = code;
       }
     }
+  }
+  if (a.stats) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) n_fix += __shfl_xor_sync(0xffffffffu, n_fix, o);
+    if ((tid & 31) == 0 && n_fix) atomicAdd(reinterpret_cast<unsigned long long*>(a.stats + 1), n_fix);
+    if (tid == 0) atomicAdd(reinterpret_cast<unsigned long long*>(a.stats), static_cast<unsigned long long>(kPage) * r);
   }
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
@@ -298,6 +318,7 @@ extern "C" kvtc_status kvtc_encode_prefill(const kvtc_plan* plan, const kvtc_cac
   a.block_table = cache->block_table;
   a.max_pages = cache->max_pages;
   a.status = cache->status;
+  a.stats = plan->d_stats;
   const size_t smem = 65536 + 16384 + 64;
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -306,5 +327,21 @@ extern "C" kvtc_status kvtc_encode_prefill(const kvtc_plan* plan, const kvtc_cac
   prefill_kernel<<<grid, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return KVTC_OK;
+}
+
+extern "C" kvtc_status kvtc_plan_prefill_stats(const kvtc_plan* plan, uint64_t* codes, uint64_t* recomputed,
+                                               int reset) {
+  kvtc_status st = check_uploaded(plan);
+  if (st != KVTC_OK) return st;
+  uint64_t h[2] = {0, 0};
+  cudaError_t e = cudaMemcpy(h, plan->d_stats, sizeof(h), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill stats copy");
+  if (codes) *codes = h[0];
+  if (recomputed) *recomputed = h[1];
+  if (reset) {
+    e = cudaMemset(plan->d_stats, 0, sizeof(h));
+    if (e != cudaSuccess) return cuda_fail(e, "prefill stats reset");
+  }
   return KVTC_OK;
 }

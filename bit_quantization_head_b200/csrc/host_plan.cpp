@@ -47,6 +47,8 @@ static void free_device(kvtc_plan* p) {
   if (p->d_units) cudaFree(p->d_units);
   if (p->d_M) cudaFree(p->d_M);
   if (p->d_Mbf) cudaFree(p->d_Mbf);
+  if (p->d_stats) cudaFree(p->d_stats);
+  p->d_stats = nullptr;
   p->d_units = nullptr;
   p->d_M = nullptr;
   p->d_Mbf = nullptr;
@@ -270,7 +272,9 @@ kvtc_status kvtc_plan_upload(kvtc_plan* plan, void* stream) {
     }
   if ((e = cudaMalloc(&plan->d_M, total * sizeof(float))) != cudaSuccess ||
       (e = cudaMalloc(&plan->d_Mbf, total * sizeof(uint16_t))) != cudaSuccess ||
-      (e = cudaMalloc(&plan->d_units, plan->U * sizeof(UnitDesc))) != cudaSuccess) {
+      (e = cudaMalloc(&plan->d_units, plan->U * sizeof(UnitDesc))) != cudaSuccess ||
+      (e = cudaMalloc(&plan->d_stats, 2 * sizeof(uint64_t))) != cudaSuccess ||
+      (e = cudaMemsetAsync(plan->d_stats, 0, 2 * sizeof(uint64_t), st)) != cudaSuccess) {
     free_device(plan);
     return cuda_fail(e, "cudaMalloc (plan upload)");
   }

@@ -44,6 +44,7 @@ struct kvtc_plan {
   kvtc::UnitDesc* d_units = nullptr;
   float* d_M = nullptr;
   uint16_t* d_Mbf = nullptr;
+  uint64_t* d_stats = nullptr;               // prefill counters (codes, recomputed)
   std::vector<kvtc::UnitDesc> h_units;      // descriptors with device pointers
 };
 

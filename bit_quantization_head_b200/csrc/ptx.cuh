@@ -51,6 +51,12 @@ __device__ __forceinline__ bool mbar_wait_bounded_warp(uint64_t* bar, uint32_t p
   return __all_sync(0xffffffffu, ok);
 }
 
+// ---- programmatic dependent launch (no-ops when the launch is not programmatic) -------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // ---- warp-level tensor core + fragment transpose --------------------------------------
 // D += A * B, m16n8k16, A/B fp16, D fp32.
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,

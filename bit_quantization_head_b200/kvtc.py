@@ -82,6 +82,7 @@ def lib():
         "kvtc_unit_pool_offset": (C.c_uint64, [_P, C.c_int, C.c_uint64]),
         "kvtc_encode_append": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, _P, C.c_int, _P, _P, C.c_int, _P]),
         "kvtc_encode_prefill": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, _P, C.c_int, C.c_int, C.c_int, _P]),
+        "kvtc_plan_prefill_stats": (st, [_P, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64), C.c_int]),
         "kvtc_decode_workspace_bytes": (C.c_uint64, [_P, C.c_int, C.c_int]),
         "kvtc_decode_attention": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, C.c_int, _P, C.c_int, C.c_float,
                                        _P, C.c_int, _P, C.c_uint64, _P]),
@@ -263,6 +264,13 @@ def kvtc_encode_append(plan, cache, layer, k, v, cu_seqlens, pos_start, stream=N
 def kvtc_encode_prefill(plan, cache, layer, k, v, seq, pos_start, stream=None):
     _check(lib().kvtc_encode_prefill(plan.handle, C.byref(cache.desc), layer, _dev_ptr(k), _dev_ptr(v), seq,
                                      pos_start, k.shape[0], _stream(stream)))
+
+
+def kvtc_plan_prefill_stats(plan, reset=False):
+    """(codes produced, codes recomputed in canonical order) by kvtc_encode_prefill."""
+    a, b = C.c_uint64(), C.c_uint64()
+    _check(lib().kvtc_plan_prefill_stats(plan.handle, C.byref(a), C.byref(b), int(reset)))
+    return a.value, b.value
 
 
 def kvtc_decode_workspace_bytes(plan, n_seq, max_seq_len):

@@ -229,6 +229,14 @@ kvtc_status kvtc_encode_prefill(const kvtc_plan* plan, const kvtc_cache* cache, 
                                 const void* k, const void* v, int seq, int pos_start, int n_tok,
                                 void* stream);
 
+/*
+ * kvtc_plan_prefill_stats -- diagnostics of kvtc_encode_prefill since the plan was
+ * uploaded (or last reset): codes produced and codes whose tensor-core sum fell within
+ * the error bound of a quantizer threshold and were recomputed in canonical order.
+ * Synchronous (copies two counters to the host); reset != 0 zeroes them.
+ */
+kvtc_status kvtc_plan_prefill_stats(const kvtc_plan* plan, uint64_t* codes, uint64_t* recomputed, int reset);
+
 /* ------------------------------------------------------------------ decode ------- */
 
 /* Workspace bytes kvtc_decode_attention needs for n_seq sequences of at most
