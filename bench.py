@@ -404,7 +404,7 @@ def run_ours(args, torch, dist, rank, world):
         "config": {"workload": w.name, "layers": L, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
                    "head_dim": 128, "batch": w.batch, "seq_len": w.seq_len, "bpd": w.bpd,
                    "parallelism": f"replicas x{world}",
-                   "step": "per layer: append 1 token + decode attention; 32 layers in one CUDA graph",
+                   "step": f"per layer: append 1 token + decode attention; {L} layers in one CUDA graph",
                    "l2": f"inputs larger than L2: {step_bytes / 1e9:.3f} GB of codes+bases per step vs 126 MB",
                    "compute": "fp16 tensor-core operands (codes exact, q split hi+lo), fp32 accumulation"},
         "pct_of_peak": round(100 * value / world / hbm_peak, 2),

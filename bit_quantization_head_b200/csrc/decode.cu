@@ -6,23 +6,29 @@
 // same algebra as NOVA-KV's query-side fold on the pith.science review page) and values
 // are accumulated in their latent basis, back-projected once per query head.
 //
-// Kernel 1 (decode_split_kernel<BK, BV>): CTA = (context split, KV head, sequence), four
-// warps, each streaming its own pages through a ring of cp.async.bulk + mbarrier stages.
-// Per 16-token block a warp computes the G (<= 8) query heads' scores with m16n8k16
-// tensor-core MMAs whose A operand is taken directly from the packed words: one AND
-// leaves each code c in the low mantissa bits of an fp16 half, i.e. the subnormal
-// c * 2^(e-24) (exact), with e the field's bit offset; e is undone per row in fp32.
-// q~ is split into fp16 hi + lo (about 22 bits).  Online softmax per block; P goes to
-// fp16 (scaled by 2^(7-e) so P * A = p * c * 2^-17 whatever e is), is transposed into
+// Kernel 0 (decode_prep_kernel): q~ = M_K q for every query head, once per call.
+// Kernel 1 (decode_split_kernel<BK, BV, PACK, NT>): CTA = (context split, KV head [, head
+// group of 8], sequence), four warps, each streaming its own pages through a ring of
+// cp.async.bulk + mbarrier stages.  Per 16-token block a warp computes the G (<= 8) query
+// heads' scores with m16n8k16 tensor-core MMAs whose A operand is taken directly from the
+// packed words: one AND leaves each code c in the low mantissa bits of an fp16 half, i.e.
+// the subnormal c * 2^(e-24) (exact), with e the field's bit offset; e is undone per row in
+// fp32.  q~ is split into fp16 hi + lo (about 22 bits).  Online softmax per block; P goes
+// to fp16 (scaled by 2^(7-e) so P * A = p * c * 2^-17 whatever e is), is transposed into
 // the B fragment with movmatrix, and multiplies the value codes (A = V codes, rows =
-// latent coordinates) into fp32 accumulators.  Each warp writes (m, l, z) partials.
+// latent coordinates) into fp32 accumulators.  Each CTA writes one (m, l, z) partial per
+// query head.
 // Kernel 2 (decode_combine_kernel): log-sum-exp merge of the partials, centering
 // (z - m_V * l), dequantization (delta_V) and the back-projection o = M_V^T y.
+// All launches use programmatic dependent launch, so each kernel's set-up overlaps the
+// tail of the one before it.
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <cmath>
 #include <map>
+#include <mutex>
+#include <set>
 #include <utility>
 #include <vector>
 
@@ -32,9 +38,91 @@ namespace kvtc {
 namespace dec {
 namespace {
 
-// o[s][qh][:] from the partials of every split and warp.  Each warp folds a quarter of
-// the partials (lane l holds latent coordinates 4l..4l+3), the warps' sums meet in shared
-// memory, then every thread back-projects one output coordinate.
+// ---- kernel 0: q~ = M_K q for every query head (the split kernels read it) -------------
+struct PrepArgs {
+  const UnitDesc* units;
+  int layer, H, G, n_hg;
+  const void* q;
+  int q_bf16;
+  float* qt;  // [n_seq][Hq][128]
+};
+
+// Sum over the 32 lanes of eight per-lane values v[0..7] with nine shuffles (each step
+// halves the values a lane keeps); lane l ends with the total of value (l >> 2) & 7.
+__device__ __forceinline__ float warp_sum8(const float (&v)[8], int lane) {
+  float a4[4], a2[2];
+  const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float send = u16 ? v[i] : v[i + 4], keep = u16 ? v[i + 4] : v[i];
+    a4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float send = u8 ? a4[i] : a4[i + 2], keep = u8 ? a4[i + 2] : a4[i];
+    a2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  float a1 = (u4 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, u4 ? a2[0] : a2[1], 4);
+  a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+  a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+  return a1;
+}
+
+// CTA = (16 rows of M_K, KV head x head group of 8, sequence); warp w forms rows
+// 16 * chunk + 4w .. +3 for the group's query heads: lane l holds columns 4l..4l+3 of the
+// row (one coalesced 512-byte load per row) and the partial dot products are summed
+// across lanes with warp_sum8.
+__global__ void __launch_bounds__(128) decode_prep_kernel(const __grid_constant__ PrepArgs a) {
+  // The split kernels that follow may start now (they wait for this grid to complete).
+  griddep_launch_dependents();
+  const int chunk = blockIdx.x, h = blockIdx.y / a.n_hg, hg = blockIdx.y % a.n_hg, s = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const UnitDesc dK = a.units[(a.layer * a.H + h) * 2];
+  const int rK = dK.r;
+  const int j0 = 16 * chunk + 4 * warp;
+  float4 m[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    m[i] = j0 + i < rK ? reinterpret_cast<const float4*>(dK.M + static_cast<size_t>(j0 + i) * kD)[lane]
+                       : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  // q is the predecessor's output: wait for it (this also makes the completion of this
+  // grid imply the completion of the one before it, which the split kernels rely on).
+  griddep_wait();
+  if (16 * chunk >= rK) return;
+  const int Hq = a.H * a.G, g0 = hg * 8, ng = min(8, a.G - g0);
+  float4 qv[8];
+#pragma unroll
+  for (int gg = 0; gg < 8; ++gg) {
+    qv[gg] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (gg < ng) {
+      const size_t off = (static_cast<size_t>(s) * Hq + h * a.G + g0 + gg) * kD + 4 * lane;
+      if (a.q_bf16) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.q) + off);
+        qv[gg] = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                             __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u));
+      } else {
+        qv[gg] = *reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + off);
+      }
+    }
+  }
+  const int head = (lane >> 2) & 7;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float v[8];
+#pragma unroll
+    for (int gg = 0; gg < 8; ++gg)
+      v[gg] = fmaf(m[i].x, qv[gg].x, fmaf(m[i].y, qv[gg].y, fmaf(m[i].z, qv[gg].z, m[i].w * qv[gg].w)));
+    const float t = warp_sum8(v, lane);
+    if ((lane & 3) == 0 && head < ng && j0 + i < rK)
+      a.qt[(static_cast<size_t>(s) * Hq + h * a.G + g0 + head) * kD + j0 + i] = t;
+  }
+}
+
+// ---- kernel 2: merge the partials, centre, dequantise, back-project --------------------
+// CTA = (query head, sequence), 256 threads.  M_V (r_V rows of 512 bytes) is copied into
+// shared memory by one bulk copy issued before the wait for the split kernels, so the
+// back-projection reads it from shared memory; warps fold the partials (lane l holds
+// latent coordinates 4l..4l+3) and meet in shared memory.
 struct CombineArgs {
   const UnitDesc* units;
   int layer, H, G;
@@ -43,37 +131,47 @@ struct CombineArgs {
   const float* ws;
   void* out;
   int out_bf16;
+  int32_t* status;
 };
+constexpr int kCombThreads = 256;
+constexpr int kCombWarps = kCombThreads / 32;
 
-__global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ CombineArgs ca) {
-  griddep_wait();
-  griddep_launch_dependents();
-  const UnitDesc* units = ca.units;
-  const int layer = ca.layer, H = ca.H, G = ca.G;
-  const float* ws = ca.ws;
-  void* out = ca.out;
-  const int out_bf16 = ca.out_bf16;
-  __shared__ float zsh[4][128];
-  __shared__ float lsh[4];
-  __shared__ float mxsh[4];
+__global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(const __grid_constant__ CombineArgs ca) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  float* Ms = reinterpret_cast<float*>(smem);  // [r_V][128]
+  __shared__ __align__(16) float zsh[kCombWarps][128];  // written as float4
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ float lsh[kCombWarps];
+  __shared__ float mxsh[kCombWarps];
   __shared__ float y[128];
   const int qh = blockIdx.x, s = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int Hq = H * G, h = qh / G;
-  const UnitDesc dV = units[(layer * H + h) * 2 + 1];
+  const int Hq = ca.H * ca.G, h = qh / ca.G;
+  const UnitDesc dV = ca.units[(ca.layer * ca.H + h) * 2 + 1];
+  const int rV = dV.r;
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(rV) * kD * 4u);
+    bulk_copy_g2s(Ms, dV.M, static_cast<uint32_t>(rV) * kD * 4u, &bar);
+  }
+  griddep_wait();
+  griddep_launch_dependents();
   const int n_part = ca.nparts[h];
-  const float* base = ws + (static_cast<size_t>(s) * Hq + qh) * ca.part_stride * kPartStride;
+  const float* base = ca.ws + (static_cast<size_t>(s) * Hq + qh) * ca.part_stride * kPartStride;
   // global max of the partial maxima (log2 domain)
   float mx = -INFINITY;
-  for (int i = tid; i < n_part; i += 128) mx = fmaxf(mx, base[static_cast<size_t>(i) * kPartStride]);
+  for (int i = tid; i < n_part; i += kCombThreads) mx = fmaxf(mx, base[static_cast<size_t>(i) * kPartStride]);
+#pragma unroll
   for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if (lane == 0) mxsh[warp] = mx;
   __syncthreads();
-  mx = fmaxf(fmaxf(mxsh[0], mxsh[1]), fmaxf(mxsh[2], mxsh[3]));
-  const int rV = dV.r;
+  mx = mxsh[0];
+#pragma unroll
+  for (int w = 1; w < kCombWarps; ++w) mx = fmaxf(mx, mxsh[w]);
   float4 zacc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   float lacc = 0.0f;
 #pragma unroll 4
-  for (int i = warp; i < n_part; i += 4) {
+  for (int i = warp; i < n_part; i += kCombWarps) {
     const float* pp = base + static_cast<size_t>(i) * kPartStride;
     const float mi = pp[0];
     const float wi = mi == -INFINITY ? 0.0f : exp2f(mi - mx);
@@ -87,29 +185,49 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   reinterpret_cast<float4*>(zsh[warp])[lane] = zacc;
   if (lane == 0) lsh[warp] = lacc;
   __syncthreads();
-  const float L = lsh[0] + lsh[1] + lsh[2] + lsh[3];
+  float L = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kCombWarps; ++w) L += lsh[w];
   const float mV = 0.5f * static_cast<float>((1 << dV.b) - 1);
   if (tid < rV) {
-    const float zs = zsh[0][tid] + zsh[1][tid] + zsh[2][tid] + zsh[3][tid];
+    float zs = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kCombWarps; ++w) zs += zsh[w][tid];
     // z holds sum p*c*2^-17 (uncentered codes); center and dequantize
     y[tid] = L > 0.0f ? dV.delta * (ldexpf(zs, 17) - mV * L) / L : 0.0f;
   }
-  __syncthreads();
-  float o0 = 0.0f, o1 = 0.0f, o2 = 0.0f, o3 = 0.0f;
-  int j = 0;
-  for (; j + 4 <= rV; j += 4) {
-    o0 = fmaf(dV.M[static_cast<size_t>(j) * kD + tid], y[j], o0);
-    o1 = fmaf(dV.M[static_cast<size_t>(j + 1) * kD + tid], y[j + 1], o1);
-    o2 = fmaf(dV.M[static_cast<size_t>(j + 2) * kD + tid], y[j + 2], o2);
-    o3 = fmaf(dV.M[static_cast<size_t>(j + 3) * kD + tid], y[j + 3], o3);
+  // M_V in shared memory (bounded wait; on a time-out the output is zero and the status
+  // word says so)
+  bool ok = false;
+  for (uint32_t it = 0; it < (1u << 20) && !ok; ++it) ok = mbar_try_wait(&bar, 0);
+  ok = __syncthreads_and(ok);
+  if (!ok) {
+    if (tid == 0 && ca.status) atomicOr(ca.status, KVTC_STATUS_TIMEOUT);
+    bool done = false;
+    for (uint32_t it = 0; it < (1u << 20) && !done; ++it) done = mbar_try_wait(&bar, 0);
   }
-  for (; j < rV; ++j) o0 = fmaf(dV.M[static_cast<size_t>(j) * kD + tid], y[j], o0);
-  const float o = (o0 + o1) + (o2 + o3);
-  const size_t off = (static_cast<size_t>(s) * Hq + qh) * kD + tid;
-  if (out_bf16)
-    static_cast<__nv_bfloat16*>(out)[off] = __float2bfloat16_rn(o);
-  else
-    static_cast<float*>(out)[off] = o;
+  // o[k] = sum_j M_V[j][k] y[j]: threads k and k + 128 take the even and odd j
+  const int k = tid & 127, par = tid >> 7;
+  float o0 = 0.0f, o1 = 0.0f;
+  if (ok) {
+    int j = par;
+    for (; j + 2 < rV; j += 4) {
+      o0 = fmaf(Ms[j * kD + k], y[j], o0);
+      o1 = fmaf(Ms[(j + 2) * kD + k], y[j + 2], o1);
+    }
+    if (j < rV) o0 = fmaf(Ms[j * kD + k], y[j], o0);
+  }
+  __syncthreads();
+  if (par) zsh[0][k] = o0 + o1;
+  __syncthreads();
+  if (!par) {
+    const float o = (o0 + o1) + zsh[0][k];
+    const size_t off = (static_cast<size_t>(s) * Hq + qh) * kD + k;
+    if (ca.out_bf16)
+      static_cast<__nv_bfloat16*>(ca.out)[off] = __float2bfloat16_rn(o);
+    else
+      static_cast<float*>(ca.out)[off] = o;
+  }
 }
 
 // Width class of a code: 2, 4 and 8 have specialised extraction; others share the
@@ -143,7 +261,9 @@ int sm_count() {
 
 // Resident CTAs per SM of a kernel variant at a given dynamic shared-memory size (cached).
 int occupancy(SplitFn fn, size_t smem) {
+  static std::mutex mu;
   static std::map<std::pair<const void*, size_t>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
   auto key = std::make_pair(reinterpret_cast<const void*>(fn), smem);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
@@ -177,10 +297,11 @@ cudaError_t launch_pdl(void (*fn)(KArgs...), dim3 grid, dim3 block, size_t smem,
 using namespace kvtc;
 using namespace kvtc::dec;
 
+// Workspace: the partials [n_seq][Hq][cap][kPartStride] floats, then q~ [n_seq][Hq][128].
 extern "C" uint64_t kvtc_decode_workspace_bytes(const kvtc_plan* plan, int n_seq, int max_seq_len) {
   if (!plan || n_seq < 1 || max_seq_len < 0) return 0;
-  return static_cast<uint64_t>(n_seq) * plan->H * plan->G * split_cap(max_seq_len) * kWarps * kPartStride *
-         sizeof(float);
+  const uint64_t heads = static_cast<uint64_t>(n_seq) * plan->H * plan->G;
+  return heads * (static_cast<uint64_t>(split_cap(max_seq_len)) * kPartStride + kD) * sizeof(float);
 }
 
 extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_cache* cache, int layer,
@@ -200,6 +321,8 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
   if (max_seq_len > cache->max_pages * kPage) return fail(KVTC_EINVAL, "max_seq_len exceeds the block table");
   if (reinterpret_cast<uintptr_t>(cache->pool) & 15) return fail(KVTC_EINVAL, "pool must be 16-byte aligned");
   if (reinterpret_cast<uintptr_t>(workspace) & 15) return fail(KVTC_EINVAL, "workspace must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(q) & 15) return fail(KVTC_EINVAL, "q must be 16-byte aligned");
+  if (plan->H > kMaxHeadsPerLaunch) return fail(KVTC_EINVAL, "at most 64 KV heads per layer");
   const int n_seq = cache->n_seq;
   const uint64_t need = kvtc_decode_workspace_bytes(plan, n_seq, max_seq_len);
   if (workspace_bytes < need) return fail(KVTC_ECAPACITY, "decode workspace too small");
@@ -207,18 +330,41 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int n_hg = (plan->G + 7) / 8;
   const int cap = split_cap(max_seq_len);
-  const int part_stride = cap * kWarps;
+  const int part_stride = cap;
+  const int Hq = plan->H * plan->G;
+  float* parts = static_cast<float*>(workspace);
+  float* qt = parts + static_cast<size_t>(n_seq) * Hq * cap * kPartStride;
 
-  // Group the layer's KV heads by kernel variant: width classes of b_K and b_V, and the
-  // rank class (both ranks <= 64 use the 4-tile variant).  One launch per group, sized to
-  // one wave of resident CTAs; within a group each head gets context splits in proportion
-  // to its bytes per page.
+  // ---- kernel 0: q~ = M_K q
+  {
+    PrepArgs pa;
+    pa.units = plan->d_units;
+    pa.layer = layer;
+    pa.H = plan->H;
+    pa.G = plan->G;
+    pa.n_hg = n_hg;
+    pa.q = q;
+    pa.q_bf16 = q_dtype == KVTC_BF16;
+    pa.qt = qt;
+    cudaError_t e = launch_pdl(decode_prep_kernel, dim3(kD / 16, plan->H * n_hg, n_seq), dim3(128), 0, cs, pa);
+    if (e != cudaSuccess) return cuda_fail(e, "decode prep launch");
+  }
+
+  // ---- kernel 1: split kernels.  The layer's KV heads are grouped by kernel variant
+  // (width classes of b_K and b_V, and the rank class: both ranks <= 64 use the 4-tile
+  // variant).  One launch per group; the launches run side by side, so each gets the
+  // share of a wave of resident CTAs that its bytes are of the layer's, and within a group
+  // each head gets context splits in proportion to its bytes per page.
   const bool pack = plan->G <= 4;
   std::map<int, std::vector<int>> groups;
+  std::vector<double> head_bytes_pp(plan->H);
+  double layer_bytes = 0.0;
   for (int h = 0; h < plan->H; ++h) {
     const int uK = (layer * plan->H + h) * 2;
     const bool small = plan->r[uK] <= 64 && plan->r[uK + 1] <= 64;
     groups[(width_class(plan->b[uK]) * 16 + width_class(plan->b[uK + 1])) * 2 + (small ? 1 : 0)].push_back(h);
+    head_bytes_pp[h] = 16.0 * (plan->r[uK] * plan->b[uK] + plan->r[uK + 1] * plan->b[uK + 1]);
+    layer_bytes += head_bytes_pp[h];
   }
   CombineArgs ca;
   ca.units = plan->d_units;
@@ -226,26 +372,23 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
   ca.H = plan->H;
   ca.G = plan->G;
   ca.part_stride = part_stride;
-  ca.ws = static_cast<const float*>(workspace);
+  ca.ws = parts;
   ca.out = out;
   ca.out_bf16 = out_dtype == KVTC_BF16;
+  ca.status = cache->status;
   for (int h = 0; h < kMaxHeadsPerLaunch; ++h) ca.nparts[h] = 0;
-  if (plan->H > kMaxHeadsPerLaunch) return fail(KVTC_EINVAL, "at most 64 KV heads per layer");
 
   const size_t head_bytes = ((sizeof(SmemHead) + 8 * kWarps * 8 + 127) / 128) * 128;
+  bool first = true;
   for (auto& kv : groups) {
     const bool small = kv.first & 1;
     const int wk = (kv.first >> 1) >> 4, wv = (kv.first >> 1) & 15;
     const std::vector<int>& hs = kv.second;
     uint32_t stage_bytes = 0;
-    std::vector<double> bytes(hs.size());
-    double total_bytes = 0.0;
-    for (size_t i = 0; i < hs.size(); ++i) {
-      const int uK = (layer * plan->H + hs[i]) * 2;
-      const uint32_t sb = static_cast<uint32_t>(16 * (plan->r[uK] * plan->b[uK] + plan->r[uK + 1] * plan->b[uK + 1]));
-      stage_bytes = std::max(stage_bytes, (sb + 127u) / 128u * 128u);
-      bytes[i] = sb;
-      total_bytes += sb;
+    double group_bytes = 0.0;
+    for (int h : hs) {
+      stage_bytes = std::max(stage_bytes, (static_cast<uint32_t>(head_bytes_pp[h]) + 127u) / 128u * 128u);
+      group_bytes += head_bytes_pp[h];
     }
     // shared memory for three CTAs per SM where the pages allow it
     const size_t budget = 74 * 1024;
@@ -255,12 +398,15 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     n_stage = std::max(1, std::min(n_stage, 6));
     if (n_stage < 2) n_stage = std::min<int>(2, static_cast<int>((220 * 1024 - head_bytes) / (kWarps * stage_bytes)));
     n_stage = std::max(1, n_stage);
-    const size_t smem = head_bytes + static_cast<size_t>(kWarps) * n_stage * stage_bytes;
+    // the stage region also holds the end-of-kernel merge of the four warps' partials
+    const size_t merge_bytes = static_cast<size_t>(kWarps) * 8 * kPartStride * sizeof(float);
+    const size_t smem = head_bytes + std::max<size_t>(static_cast<size_t>(kWarps) * n_stage * stage_bytes, merge_bytes);
     SplitFn fn = split_fn(wk == 0 ? 3 : wk, wv == 0 ? 3 : wv, pack, small);
     if (!fn) return fail(KVTC_EINVAL, "no decode kernel for this code width");
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (decode)");
-    const int wave = occupancy(fn, smem) * sm_count();
+    const double share = group_bytes / layer_bytes;
+    const int wave = static_cast<int>(occupancy(fn, smem) * sm_count() * share);
     const int columns = std::max(static_cast<int>(hs.size()), wave / std::max(1, n_hg * n_seq));
     DecodeArgs a;
     a.units = plan->d_units;
@@ -273,13 +419,13 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     a.split_prefix[0] = 0;
     for (size_t i = 0; i < hs.size(); ++i) {
       a.heads[i] = hs[i];
-      int ns = static_cast<int>(std::floor(columns * bytes[i] / total_bytes));
+      int ns = static_cast<int>(std::floor(columns * head_bytes_pp[hs[i]] / group_bytes));
       ns = std::max(1, std::min(ns, cap));
       a.split_prefix[i + 1] = a.split_prefix[i] + ns;
-      ca.nparts[hs[i]] = ns * kWarps;
+      ca.nparts[hs[i]] = ns;
     }
-    a.q = q;
-    a.q_bf16 = q_dtype == KVTC_BF16;
+    a.qt = qt;
+    a.wait_first = first ? 1 : 0;
     a.seq_lens = seq_lens;
     a.n_seq = n_seq;
     a.pool = static_cast<const char*>(cache->pool);
@@ -290,17 +436,37 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     a.scale = scale;
     a.n_stage = n_stage;
     a.stage_bytes = stage_bytes;
-    a.ws = static_cast<float*>(workspace);
+    a.ws = parts;
     dim3 grid(a.split_prefix[hs.size()], n_hg, n_seq);
     e = launch_pdl(fn, grid, dim3(kThreads), smem, cs, a);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    first = false;
   }
-  dim3 cgrid(plan->H * plan->G, n_seq);
+
+  // ---- kernel 2: combine (M_V staged in shared memory)
   {
-    cudaError_t e = launch_pdl(decode_combine_kernel, cgrid, dim3(128), 0, cs, ca);
+    int rv_max = 2;
+    for (int h = 0; h < plan->H; ++h) rv_max = std::max(rv_max, plan->r[(layer * plan->H + h) * 2 + 1]);
+    const size_t smem = static_cast<size_t>(rv_max) * kD * sizeof(float);
+    // the largest size (r_V = 128) is set once per device
+    static std::mutex mu;
+    static std::set<int> devices_set;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      if (!devices_set.count(dev)) {
+        e = cudaFuncSetAttribute(decode_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kD * kD * sizeof(float)));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (combine)");
+        devices_set.insert(dev);
+      }
+    }
+    e = launch_pdl(decode_combine_kernel, dim3(Hq, n_seq), dim3(kCombThreads), smem, cs, ca);
     if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
   }
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVTC_OK;
 }

@@ -17,7 +17,9 @@
 //     whose A operand again comes straight from the packed value words.  One extra A row
 //     of ones (when r_V is not a multiple of 16) accumulates l = sum p with the same
 //     rounded P, so z - m_V * l cancels consistently.
-// Each warp writes (m, l, z) partials; decode.cu merges them and back-projects.
+// The four warps' (m, l, z) partials meet in shared memory and each CTA writes one partial
+// per query head; decode.cu's combine kernel merges those and back-projects.  q~ = M_K q
+// comes from decode.cu's prep kernel through the workspace.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -46,8 +48,8 @@ struct DecodeArgs {
   int split_prefix[kMaxHeadsPerLaunch + 1];  // CTAs of head i: [prefix[i], prefix[i+1])
   int n_heads;
   int part_stride;                       // partial slots per query head in the workspace
-  const void* q;
-  int q_bf16;
+  const float* qt;    // q~ = M_K q per query head [n_seq][Hq][128] (the prep kernel's output)
+  int wait_first;     // 1: wait for the preceding grid before reading; 0: at exit (see decode.cu)
   const int32_t* seq_lens;
   int n_seq;
   const char* pool;
@@ -58,7 +60,7 @@ struct DecodeArgs {
   float scale;
   int n_stage;
   uint32_t stage_bytes;
-  float* ws;  // partials [n_seq][Hq][n_split * kWarps][kPartStride]
+  float* ws;  // partials [n_seq][Hq][part_stride][kPartStride]
 };
 
 // ------------------------------------------------------------------ code extraction
@@ -128,8 +130,7 @@ __device__ __forceinline__ uint32_t gen_pair(const uint32_t (&W)[4], const Parts
 
 // ------------------------------------------------------------------ shared memory
 struct SmemHead {
-  float q[8][128];   // the launch's query heads (zero beyond G)
-  float qt[8][128];  // q~ = M_K q
+  float qt[8][128];  // q~ = M_K q (zero beyond the head group and beyond r_K)
   float S[8];        // sum_j q~_j
   int E[8];          // power-of-two normalisation of q~ for fp16
 };
@@ -143,6 +144,7 @@ struct WS {
   int rK, rV, nks, nmt, g, tq;
   Parts partsK, partsV;
   int ones_mt, ones_lr;  // m-tile / local row of the ones row (ones_mt < 0: none)
+  uint32_t ones_m0, ones_m1;  // lane masks: this lane's A rows g / g+8 are the ones row
   // B fragments of q^: PACK -> bq[ks] (hi for g < 4, lo for g >= 4); else bh, bl
   uint32_t bh[NT][2];
   uint32_t bl[PACK ? 1 : NT][2];
@@ -150,7 +152,6 @@ struct WS {
   float al[2][n_e<BK == 0 ? 8 : BK>()], nb[2][n_e<BV == 0 ? 8 : BV>()];
   float z[NT][4];
   float lcvt[2];  // l accumulated from the fp16 P when there is no ones row
-  uint32_t kw[NT][2], vw[NT][2];  // current words of the fast paths
 };
 
 // Score argument constants: x = al * acc + nb, with e undone in al (key side) and the P
@@ -175,33 +176,6 @@ __device__ __forceinline__ void refresh_constants(WS<BK, BV, PACK, NT>& w) {
   }
 }
 
-// Loads the words this lane needs for block BLK (fast paths reload when the word changes).
-template <int BK, int BV, bool PACK, int NT, int BLK>
-__device__ __forceinline__ void load_words(WS<BK, BV, PACK, NT>& w) {
-  if constexpr (BK != 0 && (BLK * BK) % 8 == 0) {
-    const int wsel = w.g * BK + (BLK * BK) / 8;
-#pragma unroll
-    for (int ks = 0; ks < NT; ++ks) {
-      if (ks < w.nks) {
-        const int r0 = 8 * ks + w.tq, r1 = r0 + 4;
-        w.kw[ks][0] = 2 * r0 < w.rK ? w.pk[r0 * 8 * BK + wsel] : 0u;
-        w.kw[ks][1] = 2 * r1 < w.rK ? w.pk[r1 * 8 * BK + wsel] : 0u;
-      }
-    }
-  }
-  if constexpr (BV != 0 && (BLK * BV) % 8 == 0) {
-    const int wsel = w.tq * BV + (BLK * BV) / 8;
-#pragma unroll
-    for (int mt = 0; mt < NT; ++mt) {
-      if (mt < w.nmt) {
-        const int j0 = 16 * mt + w.g, j1 = j0 + 8;
-        w.vw[mt][0] = j0 < w.rV ? w.pv[j0 * 4 * BV + wsel] : 0u;
-        w.vw[mt][1] = j1 < w.rV ? w.pv[j1 * 4 * BV + wsel] : 0u;
-      }
-    }
-  }
-}
-
 // Generic words of a K row (or V row) for block BLK: one word per part.
 template <int BLK>
 __device__ __forceinline__ void gen_words(const uint32_t* page, int r, int row, bool ok, int owner, bool is_k,
@@ -218,50 +192,46 @@ __device__ __forceinline__ void gen_words(const uint32_t* page, int r, int row, 
   }
 }
 
-// One 16-token block: scores, lazy online softmax, value accumulation.
+// ---- the work is done per half page (4 blocks of 16 tokens): the loop over k-steps
+// (or m-tiles) is outside the loop over blocks, so a rank guard costs once per half page
+// and the four blocks' MMA chains interleave.
+
+// Score MMA(s) of one block for k-step (rows r0, r1 of this lane).
 template <int BK, int BV, bool PACK, int NT, int BLK>
-__device__ __forceinline__ void do_block(WS<BK, BV, PACK, NT>& w) {
-  load_words<BK, BV, PACK, NT, BLK>(w);
-  // ---- scores S[tok][head] = sum_j codeK[tok][j] * q^[head][j]
-  float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  float sd[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // second accumulator (lo MMAs) when not packed
-#pragma unroll
-  for (int ks = 0; ks < NT; ++ks) {
-    if (ks < w.nks) {
-      uint32_t A0, A1, A2, A3;
-      if constexpr (BK != 0) {
-        A0 = fast_pair<BK, BLK, 0>(w.kw[ks][0]);
-        A1 = fast_pair<BK, BLK, 1>(w.kw[ks][0]);
-        A2 = fast_pair<BK, BLK, 0>(w.kw[ks][1]);
-        A3 = fast_pair<BK, BLK, 1>(w.kw[ks][1]);
-      } else {
-        uint32_t W0[4], W1[4];
-        const int r0 = 8 * ks + w.tq, r1 = r0 + 4;
-        gen_words<BLK>(w.pk, w.rK, r0, 2 * r0 < w.rK, w.g, true, w.partsK, W0);
-        gen_words<BLK>(w.pk, w.rK, r1, 2 * r1 < w.rK, w.g, true, w.partsK, W1);
-        A0 = gen_pair<BLK, 0>(W0, w.partsK);
-        A1 = gen_pair<BLK, 1>(W0, w.partsK);
-        A2 = gen_pair<BLK, 0>(W1, w.partsK);
-        A3 = gen_pair<BLK, 1>(W1, w.partsK);
-      }
-      if constexpr (PACK) {
-        // alternate two accumulators so consecutive k-steps do not chain
-        if (ks & 1)
-          mma_16816(sd, A0, A1, A2, A3, w.bh[ks][0], w.bh[ks][1]);
-        else
-          mma_16816(sc, A0, A1, A2, A3, w.bh[ks][0], w.bh[ks][1]);
-      } else {
-        mma_16816(sc, A0, A1, A2, A3, w.bh[ks][0], w.bh[ks][1]);
-        mma_16816(sd, A0, A1, A2, A3, w.bl[ks][0], w.bl[ks][1]);
-      }
-    }
+__device__ __forceinline__ void k_block(const WS<BK, BV, PACK, NT>& w, int ks, int r0, int r1, bool ok0, bool ok1,
+                                        float (&sc)[4], float (&sd)[4]) {
+  uint32_t A0, A1, A2, A3;
+  if constexpr (BK != 0) {
+    const int wsel = w.g * BK + (BLK * BK) / 8;
+    const uint32_t W0 = ok0 ? w.pk[r0 * 8 * BK + wsel] : 0u;
+    const uint32_t W1 = ok1 ? w.pk[r1 * 8 * BK + wsel] : 0u;
+    A0 = fast_pair<BK, BLK, 0>(W0);
+    A1 = fast_pair<BK, BLK, 1>(W0);
+    A2 = fast_pair<BK, BLK, 0>(W1);
+    A3 = fast_pair<BK, BLK, 1>(W1);
+  } else {
+    uint32_t W0[4], W1[4];
+    gen_words<BLK>(w.pk, w.rK, r0, ok0, w.g, true, w.partsK, W0);
+    gen_words<BLK>(w.pk, w.rK, r1, ok1, w.g, true, w.partsK, W1);
+    A0 = gen_pair<BLK, 0>(W0, w.partsK);
+    A1 = gen_pair<BLK, 1>(W0, w.partsK);
+    A2 = gen_pair<BLK, 0>(W1, w.partsK);
+    A3 = gen_pair<BLK, 1>(W1, w.partsK);
   }
+  mma_16816(sc, A0, A1, A2, A3, w.bh[ks][0], w.bh[ks][1]);
+  if constexpr (!PACK) mma_16816(sd, A0, A1, A2, A3, w.bl[ks][0], w.bl[ks][1]);
+}
+
+// Score arguments of one block: x = s - m_run + 7 - e_V (log2 domain), -inf if masked.
+// Returns whether the block asks for a rescale (a score past the running max by 2^kLazy).
+template <int BK, int BV, bool PACK, int NT, bool FULL, int BLK>
+__device__ __forceinline__ bool x_block(const WS<BK, BV, PACK, NT>& w, const float (&sc)[4], const float (&sd)[4],
+                                        float (&x)[4]) {
   float full[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     if constexpr (PACK) {
-      const float t = sc[i] + sd[i];
-      full[i] = t + __shfl_xor_sync(0xffffffffu, t, 2);  // hi (t' < 2) + lo (t' >= 2)
+      full[i] = sc[i] + __shfl_xor_sync(0xffffffffu, sc[i], 2);  // hi (t' < 2) + lo (t' >= 2)
     } else {
       full[i] = sc[i] + sd[i];
     }
@@ -270,34 +240,114 @@ __device__ __forceinline__ void do_block(WS<BK, BV, PACK, NT>& w) {
   constexpr int ik0 = e_idx<BK == 0 ? 8 : BK>(BLK, 0), ik1 = e_idx<BK == 0 ? 8 : BK>(BLK, 1);
   constexpr int iv0 = e_idx<BV == 0 ? 8 : BV>(BLK, 0), iv1 = e_idx<BV == 0 ? 8 : BV>(BLK, 1);
   constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
-  const int t0 = w.tok0 + 16 * BLK + w.g, t1 = t0 + 8;
-  const bool live0 = t0 < w.seq_len, live1 = t1 < w.seq_len;
-  float x[4];
-  x[0] = live0 ? fmaf(w.al[0][ik0], full[0], w.nb[0][iv0]) : -INFINITY;
-  x[1] = live0 ? fmaf(w.al[1][ik0], full[1], w.nb[1][iv0]) : -INFINITY;
-  x[2] = live1 ? fmaf(w.al[0][ik1], full[2], w.nb[0][iv1]) : -INFINITY;
-  x[3] = live1 ? fmaf(w.al[1][ik1], full[3], w.nb[1][iv1]) : -INFINITY;
-  // ---- lazy online softmax: x = s - m_run + 7 - e_V; rescale only past 2^kLazy
+  x[0] = fmaf(w.al[0][ik0], full[0], w.nb[0][iv0]);
+  x[1] = fmaf(w.al[1][ik0], full[1], w.nb[1][iv0]);
+  x[2] = fmaf(w.al[0][ik1], full[2], w.nb[0][iv1]);
+  x[3] = fmaf(w.al[1][ik1], full[3], w.nb[1][iv1]);
+  if constexpr (!FULL) {
+    const int t0 = w.tok0 + 16 * BLK + w.g, t1 = t0 + 8;
+    if (t0 >= w.seq_len) x[0] = x[1] = -INFINITY;
+    if (t1 >= w.seq_len) x[2] = x[3] = -INFINITY;
+  }
   constexpr float lim0 = kLazy + 7.0f - ev0, lim1 = kLazy + 7.0f - ev1;
-  // grow also on the first live block (the running max starts undefined)
-  const bool grow = x[0] > lim0 || x[1] > lim0 || x[2] > lim1 || x[3] > lim1 ||
-                    ((w.m_run[0] == -INFINITY || w.m_run[1] == -INFINITY) && (live0 || live1));
+  return fmaxf(x[0], x[1]) > lim0 || fmaxf(x[2], x[3]) > lim1;
+}
+
+// Block maximum of s - m_run for head column c of one block (x with the e_V offset removed).
+template <int BV, int BLK>
+__device__ __forceinline__ float xmax_block(const float (&x)[4], int c) {
+  constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
+  return fmaxf(x[c] - (7.0f - ev0), x[2 + c] - (7.0f - ev1));
+}
+
+// P of one block in fp16 (already scaled by 2^(7 - e_V) through x), transposed into the
+// B fragment of the value MMA; l from the rounded P when there is no ones row.
+template <int BK, int BV, bool PACK, int NT, int BLK>
+__device__ __forceinline__ void p_block(WS<BK, BV, PACK, NT>& w, const float (&x)[4], uint32_t (&bp)[2]) {
+  const uint32_t P0 = pack_half2(ex2(x[0]), ex2(x[1]));
+  const uint32_t P1 = pack_half2(ex2(x[2]), ex2(x[3]));
+  if (w.ones_mt < 0) {
+    constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
+    const float2 f0 = half2_to_float2(P0), f1 = half2_to_float2(P1);
+    constexpr float u0 = 1.0f / static_cast<float>(1 << (7 - ev0)), u1 = 1.0f / static_cast<float>(1 << (7 - ev1));
+    w.lcvt[0] += fmaf(f0.x, u0, f1.x * u1);
+    w.lcvt[1] += fmaf(f0.y, u0, f1.y * u1);
+  }
+  bp[0] = movmatrix_trans(P0);
+  bp[1] = movmatrix_trans(P1);
+}
+
+// Value MMA of one block for m-tile mt (rows j0, j1 of this lane).
+template <int BK, int BV, bool PACK, int NT, int BLK>
+__device__ __forceinline__ void v_block(const WS<BK, BV, PACK, NT>& w, int j0, int j1, bool ok0, bool ok1,
+                                        bool ones, const uint32_t (&bp)[2], float (&z)[4]) {
+  uint32_t A0, A1, A2, A3;
+  if constexpr (BV != 0) {
+    const int wsel = w.tq * BV + (BLK * BV) / 8;
+    const uint32_t W0 = ok0 ? w.pv[j0 * 4 * BV + wsel] : 0u;
+    const uint32_t W1 = ok1 ? w.pv[j1 * 4 * BV + wsel] : 0u;
+    A0 = fast_pair<BV, BLK, 0>(W0);
+    A1 = fast_pair<BV, BLK, 0>(W1);
+    A2 = fast_pair<BV, BLK, 1>(W0);
+    A3 = fast_pair<BV, BLK, 1>(W1);
+  } else {
+    uint32_t W0[4], W1[4];
+    gen_words<BLK>(w.pv, w.rV, j0, ok0, w.tq, false, w.partsV, W0);
+    gen_words<BLK>(w.pv, w.rV, j1, ok1, w.tq, false, w.partsV, W1);
+    A0 = gen_pair<BLK, 0>(W0, w.partsV);
+    A1 = gen_pair<BLK, 0>(W1, w.partsV);
+    A2 = gen_pair<BLK, 1>(W0, w.partsV);
+    A3 = gen_pair<BLK, 1>(W1, w.partsV);
+  }
+  if (ones) {  // the ones row (row r_V, zero so far) accumulates l
+    constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
+    constexpr uint32_t one0 = (1u << ev0) | (1u << (ev0 + 16)), one1 = (1u << ev1) | (1u << (ev1 + 16));
+    A0 |= one0 & w.ones_m0;
+    A2 |= one1 & w.ones_m0;
+    A1 |= one0 & w.ones_m1;
+    A3 |= one1 & w.ones_m1;
+  }
+  mma_16816(z, A0, A1, A2, A3, bp[0], bp[1]);
+}
+
+// Half page H2 (blocks 4*H2 .. 4*H2+3): scores, lazy online softmax, value accumulation.
+template <int BK, int BV, bool PACK, int NT, bool FULL, int H2, int... BB>
+__device__ __forceinline__ void do_half(WS<BK, BV, PACK, NT>& w, std::integer_sequence<int, BB...>) {
+  float sc[4][4], sd[4][4];
+#pragma unroll
+  for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sc[bb][i] = sd[bb][i] = 0.0f;
+  // ---- scores S[tok][head] = sum_j codeK[tok][j] * q^[head][j]
+#pragma unroll
+  for (int ks = 0; ks < NT; ++ks) {
+    if (ks < w.nks) {
+      const int r0 = 8 * ks + w.tq, r1 = r0 + 4;
+      const bool ok0 = 2 * r0 < w.rK, ok1 = 2 * r1 < w.rK;
+      (k_block<BK, BV, PACK, NT, 4 * H2 + BB>(w, ks, r0, r1, ok0, ok1, sc[BB], sd[BB]), ...);
+    }
+  }
+  float x[4][4];
+  bool grow = false;
+  ((grow |= x_block<BK, BV, PACK, NT, FULL, 4 * H2 + BB>(w, sc[BB], sd[BB], x[BB])), ...);
+  // grow also while the running max is undefined (the first live half page)
+  grow |= w.m_run[0] == -INFINITY || w.m_run[1] == -INFINITY;
+  // ---- lazy online softmax: rescale only when a score passes the running max by 2^kLazy
   if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      // block max of the true scores s = x - nb + beta... in the m_run frame: s - m_run
-      float v = fmaxf(x[c] - (7.0f - ev0), x[2 + c] - (7.0f - ev1));
+      float v = -INFINITY;
+      ((v = fmaxf(v, xmax_block<BV, 4 * H2 + BB>(x[BB], c))), ...);
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-      // v = block max of (s - m_run); the new running max is m_run + max(v, 0)
+      // v = max over the half page of s - m_run (m_run taken as 0 while undefined)
       const float old = w.m_run[c];
       float shift = 0.0f;
       if (v == -INFINITY) {
-        // no live token of this head in the block: nothing to do
+        // no live token of this head here: nothing to do
       } else if (old == -INFINITY) {
-        // first scores of this warp: x was computed with m_run taken as 0
-        w.m_run[c] = v;  // v is the true block max here
+        w.m_run[c] = v;
         shift = v;
       } else if (v > 0.0f) {
         w.m_run[c] = old + v;
@@ -310,66 +360,33 @@ __device__ __forceinline__ void do_block(WS<BK, BV, PACK, NT>& w) {
         }
         w.lcvt[c] *= resc;
       }
-      x[c] -= shift;
-      x[2 + c] -= shift;
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        x[bb][c] -= shift;
+        x[bb][2 + c] -= shift;
+      }
     }
     refresh_constants(w);
   }
-  float p[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) p[i] = ex2(x[i]);
-  if constexpr (PACK) {
-    if (w.tq >= 2) p[0] = p[1] = p[2] = p[3] = 0.0f;  // columns 4..7 are the lo MMA
-  }
-  const uint32_t P0 = pack_half2(p[0], p[1]);
-  const uint32_t P1 = pack_half2(p[2], p[3]);
-  if (w.ones_mt < 0) {
-    // l from the same fp16-rounded weights (no ones row available)
-    const float2 f0 = half2_to_float2(P0), f1 = half2_to_float2(P1);
-    constexpr float u0 = 1.0f / static_cast<float>(1 << (7 - ev0)), u1 = 1.0f / static_cast<float>(1 << (7 - ev1));
-    w.lcvt[0] += fmaf(f0.x, u0, f1.x * u1);
-    w.lcvt[1] += fmaf(f0.y, u0, f1.y * u1);
-  }
-  const uint32_t b0 = movmatrix_trans(P0), b1 = movmatrix_trans(P1);
+  // ---- probabilities -> B fragments
+  uint32_t bp[4][2];
+  (p_block<BK, BV, PACK, NT, 4 * H2 + BB>(w, x[BB], bp[BB]), ...);
   // ---- values: Z^T[j][head] += sum_tok codeV[tok][j] * P[tok][head]
-  constexpr uint32_t one0 = (1u << ev0) | (1u << (ev0 + 16)), one1 = (1u << ev1) | (1u << (ev1 + 16));
 #pragma unroll
   for (int mt = 0; mt < NT; ++mt) {
     if (mt < w.nmt) {
-      uint32_t A0, A1, A2, A3;
-      if constexpr (BV != 0) {
-        A0 = fast_pair<BV, BLK, 0>(w.vw[mt][0]);
-        A1 = fast_pair<BV, BLK, 0>(w.vw[mt][1]);
-        A2 = fast_pair<BV, BLK, 1>(w.vw[mt][0]);
-        A3 = fast_pair<BV, BLK, 1>(w.vw[mt][1]);
-      } else {
-        uint32_t W0[4], W1[4];
-        const int j0 = 16 * mt + w.g, j1 = j0 + 8;
-        gen_words<BLK>(w.pv, w.rV, j0, j0 < w.rV, w.tq, false, w.partsV, W0);
-        gen_words<BLK>(w.pv, w.rV, j1, j1 < w.rV, w.tq, false, w.partsV, W1);
-        A0 = gen_pair<BLK, 0>(W0, w.partsV);
-        A1 = gen_pair<BLK, 0>(W1, w.partsV);
-        A2 = gen_pair<BLK, 1>(W0, w.partsV);
-        A3 = gen_pair<BLK, 1>(W1, w.partsV);
-      }
-      if (mt == w.ones_mt) {  // the ones row (row r_V) accumulates l
-        if (w.ones_lr == w.g) {
-          A0 = one0;
-          A2 = one1;
-        }
-        if (w.ones_lr == w.g + 8) {
-          A1 = one0;
-          A3 = one1;
-        }
-      }
-      mma_16816(w.z[mt], A0, A1, A2, A3, b0, b1);
+      const int j0 = 16 * mt + w.g, j1 = j0 + 8;
+      const bool ok0 = j0 < w.rV, ok1 = j1 < w.rV;
+      const bool ones = mt == w.ones_mt;
+      (v_block<BK, BV, PACK, NT, 4 * H2 + BB>(w, j0, j1, ok0, ok1, ones, bp[BB], w.z[mt]), ...);
     }
   }
 }
 
-template <int BK, int BV, bool PACK, int NT, int... BLK>
-__device__ __forceinline__ void do_page(WS<BK, BV, PACK, NT>& w, std::integer_sequence<int, BLK...>) {
-  (do_block<BK, BV, PACK, NT, BLK>(w), ...);
+template <int BK, int BV, bool PACK, int NT, bool FULL>
+__device__ __forceinline__ void do_page(WS<BK, BV, PACK, NT>& w) {
+  do_half<BK, BV, PACK, NT, FULL, 0>(w, std::make_integer_sequence<int, 4>{});
+  do_half<BK, BV, PACK, NT, FULL, 1>(w, std::make_integer_sequence<int, 4>{});
 }
 
 template <int BK, int BV, bool PACK, int NT>
@@ -379,6 +396,13 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sizeof(SmemHead));
   unsigned char* stages = smem + ((sizeof(SmemHead) + 8 * kWarps * 8 + 127) / 128) * 128;
 
+  // Programmatic dependent launch.  The first split launch of a call waits here for the
+  // preceding grid (the q~ prep kernel, which completes only after its own predecessor,
+  // e.g. the append that wrote the newest token).  A later split launch of the same call
+  // starts only once every CTA of the one before it is past this point, so it reads at
+  // once and waits at exit instead, which keeps completion ordered for the combine.
+  if (a.wait_first) griddep_wait();
+  griddep_launch_dependents();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
   // CTA -> (KV head, context split): heads get splits in proportion to their bytes
@@ -406,22 +430,17 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
   const int p_end = min(p_begin + pages_per_split, n_pages);
   const int n_my = p_end > p_begin + warp ? (p_end - p_begin - warp + kWarps - 1) / kWarps : 0;
 
-  // ---- prologue: barriers, query, first copies, q~ = M_K q ----
+  // ---- prologue: barriers, q~, first copies ----
   if (lane == 0)
     for (int i = 0; i < a.n_stage; ++i) mbar_init(&bars[warp * 8 + i], 1);
-  // Programmatic dependent launch: the preceding kernel (e.g. the append that wrote the
-  // newest token) must be complete before pages are read; the next kernel may launch.
-  griddep_wait();
-  griddep_launch_dependents();
-  for (int i = tid; i < 8 * 128; i += kThreads) {
-    const int gg = i >> 7, k = i & 127;
-    float v = 0.0f;
-    if (gg < ng) {
-      const size_t off = (static_cast<size_t>(s) * Hq + h * a.G + g0 + gg) * kD + k;
-      v = a.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[off])
-                   : static_cast<const float*>(a.q)[off];
+  for (int i = tid; i < 8 * 32; i += kThreads) {
+    const int gg = i >> 5, k4 = i & 31;
+    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (gg < ng && 4 * k4 < rK) {
+      v = reinterpret_cast<const float4*>(a.qt + (static_cast<size_t>(s) * Hq + h * a.G + g0 + gg) * kD)[k4];
+      if (4 * k4 + 2 >= rK) v.z = v.w = 0.0f;  // r_K is even: only the upper pair can be past it
     }
-    sh.q[gg][k] = v;
+    reinterpret_cast<float4*>(sh.qt[gg])[k4] = v;
   }
   fence_mbar_init();
   __syncthreads();
@@ -453,27 +472,6 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
   if (lane == 0)
     for (int i = 0; i < n_first; ++i) issue(i);
 
-  // q~[gg][j] = sum_k M_K[j][k] q[gg][k]: thread j reads row j of M once (float4, each
-  // 128-byte line reused by the same thread) and forms all ng dot products.
-  for (int j = tid; j < 128; j += kThreads) {
-    float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
-    if (j < rK) {
-      const float4* m4 = reinterpret_cast<const float4*>(dK.M + static_cast<size_t>(j) * kD);
-#pragma unroll 4
-      for (int k = 0; k < 32; ++k) {
-        const float4 m = m4[k];
-#pragma unroll
-        for (int gg = 0; gg < 8; ++gg) {
-          if (gg < ng) {
-            const float4 qv = reinterpret_cast<const float4*>(sh.q[gg])[k];
-            acc[gg] = fmaf(m.x, qv.x, fmaf(m.y, qv.y, fmaf(m.z, qv.z, fmaf(m.w, qv.w, acc[gg]))));
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int gg = 0; gg < 8; ++gg) sh.qt[gg][j] = (gg < ng && j < rK) ? acc[gg] : 0.0f;
-  }
   __syncthreads();
   if (warp == 0) {
     // per head: S = sum_j q~_j and the fp16 normalisation exponent
@@ -507,6 +505,8 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
   w.partsV = parts_of(dV.b);
   w.ones_mt = (rV & 15) ? (rV >> 4) : -1;
   w.ones_lr = rV & 15;
+  w.ones_m0 = (w.ones_mt >= 0 && w.ones_lr == g) ? 0xFFFFFFFFu : 0u;
+  w.ones_m1 = (w.ones_mt >= 0 && w.ones_lr == g + 8) ? 0xFFFFFFFFu : 0u;
   // B fragments of q^ = q~ * 2^-E.  Packed (G <= 4): column n < 4 holds the hi part of
   // head n, column n >= 4 the lo part of head n - 4.
   {
@@ -567,7 +567,10 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
       w.pk = reinterpret_cast<const uint32_t*>(st);
       w.pv = reinterpret_cast<const uint32_t*>(st + bytesK);
       w.tok0 = p * kPage;
-      do_page<BK, BV, PACK, NT>(w, std::make_integer_sequence<int, 8>{});
+      if (w.tok0 + kPage <= w.seq_len)
+        do_page<BK, BV, PACK, NT, true>(w);
+      else
+        do_page<BK, BV, PACK, NT, false>(w);
     } else if (lane == 0 && a.status) {
       atomicOr(a.status, KVTC_STATUS_BAD_PAGE);
     }
@@ -606,15 +609,17 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
     }
   }
 
-  // ---- write this warp's partials: (m, l, z) per query head ----
-  const int part = split * kWarps + warp;
-  const int n_part = a.part_stride;
+  // ---- merge the four warps' (m, l, z) per query head in shared memory (the stage
+  // buffers are free: every copy issued has been waited for), then write one partial per
+  // CTA and query head ----
+  float* mb = reinterpret_cast<float*>(stages);  // [kWarps][8][kPartStride]
+  __syncthreads();
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
-    const int n = PACK ? 2 * tq + c : 2 * tq + c;  // column of the z fragment
+    const int n = 2 * tq + c;  // column of the z fragment (a query head, or a copy in packed mode)
     const bool real = PACK ? (tq < 2 && n < ng) : n < ng;
     if (real) {
-      float* dst = a.ws + ((static_cast<size_t>(s) * Hq + h * a.G + g0 + n) * n_part + part) * kPartStride;
+      float* dst = mb + (warp * 8 + n) * kPartStride;
       if (g == 0) {
         dst[0] = dead ? -INFINITY : w.m_run[c];
         dst[1] = dead ? 0.0f : l_out[c];
@@ -629,6 +634,33 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
       }
     }
   }
+  __syncthreads();
+  for (int idx = tid; idx < ng * (rV + 2); idx += kThreads) {
+    const int n = idx / (rV + 2), e = idx - n * (rV + 2);
+    float mw[kWarps], M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < kWarps; ++q) {
+      mw[q] = mb[(q * 8 + n) * kPartStride];
+      M = fmaxf(M, mw[q]);
+    }
+    float acc = 0.0f;
+    if (M != -INFINITY) {
+      const int src = e == 0 ? 1 : 4 + (e - 1);  // e == 0: l; e >= 1: z[e - 1]
+      if (e <= rV) {
+#pragma unroll
+        for (int q = 0; q < kWarps; ++q)
+          if (mw[q] != -INFINITY) acc = fmaf(ex2(mw[q] - M), mb[(q * 8 + n) * kPartStride + src], acc);
+      }
+    }
+    float* dst = a.ws + ((static_cast<size_t>(s) * Hq + h * a.G + g0 + n) * a.part_stride + split) * kPartStride;
+    if (e == 0) {
+      dst[0] = M;
+      dst[1] = acc;
+    } else if (e <= rV) {
+      dst[4 + (e - 1)] = acc;
+    }
+  }
+  if (!a.wait_first) griddep_wait();
 }
 
 using SplitFn = void (*)(const DecodeArgs);

@@ -26,7 +26,6 @@ struct AppendArgs {
   const int32_t* pos_start;
   int n_seq;
   int n_tok;
-  int coords_per_token;   // sum over the layer's units of r
   char* pool;
   uint64_t pages_per_unit;
   const int32_t* block_table;
@@ -57,44 +56,54 @@ __device__ __forceinline__ void store_code(uint32_t* page, int kind, int r, int 
   }
 }
 
+// CTA = (token, unit of the layer); thread j computes coordinate j.  The token's row is
+// staged in shared memory once; each thread holds its row of M in registers; the fma
+// chain then runs in the canonical k order from registers and broadcast reads.
 __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constant__ AppendArgs a) {
   // Programmatic dependent launch: wait for the producer of k/v, then let the next kernel
   // (typically the decode of this layer) start its prologue.
   griddep_wait();
   griddep_launch_dependents();
-  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long long total = static_cast<long long>(a.n_tok) * a.coords_per_token;
-  if (gid >= total) return;
-  const int tok = static_cast<int>(gid / a.coords_per_token);
-  int c = static_cast<int>(gid % a.coords_per_token);
-  int ul = 0;
-  while (ul < a.n_units - 1 && c >= a.units[a.unit0 + ul].r) {
-    c -= a.units[a.unit0 + ul].r;
-    ++ul;
-  }
+  __shared__ float xs[kD];
+  const int tok = blockIdx.x, ul = blockIdx.y, j = threadIdx.x;
   const int u = a.unit0 + ul;
   const UnitDesc ud = a.units[u];
   const int kind = ul & 1;
   const int head = ul >> 1;
-  const int j = c;
-
-  // canonical projection
-  float acc = 0.0f;
   const size_t xoff = (static_cast<size_t>(tok) * a.H + head) * kD;
+  if (a.bf16)
+    xs[j] = __bfloat162float((static_cast<const __nv_bfloat16*>(kind ? a.v : a.k) + xoff)[j]);
+  else
+    xs[j] = (static_cast<const float*>(kind ? a.v : a.k) + xoff)[j];
+  __syncthreads();
+  if (j >= ud.r) return;
+
+  // canonical projection: acc = fma(x_k, M_jk, acc) for k = 0..127 in order
+  float acc = 0.0f;
   if (a.bf16) {
-    const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(kind ? a.v : a.k) + xoff;
-    const uint16_t* m = ud.Mbf + static_cast<size_t>(j) * kD;
-#pragma unroll 8
-    for (int k = 0; k < kD; ++k) {
-      const float xv = __bfloat162float(x[k]);
-      const float mv = __uint_as_float(static_cast<uint32_t>(m[k]) << 16);
-      acc = __fmaf_rn(xv, mv, acc);
+    const uint4* m4 = reinterpret_cast<const uint4*>(ud.Mbf + static_cast<size_t>(j) * kD);
+    uint4 mr[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) mr[c] = m4[c];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const uint32_t w[4] = {mr[c].x, mr[c].y, mr[c].z, mr[c].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc = __fmaf_rn(xs[8 * c + 2 * q], __uint_as_float(w[q] << 16), acc);
+        acc = __fmaf_rn(xs[8 * c + 2 * q + 1], __uint_as_float(w[q] & 0xFFFF0000u), acc);
+      }
     }
   } else {
-    const float* x = static_cast<const float*>(kind ? a.v : a.k) + xoff;
-    const float* m = ud.M + static_cast<size_t>(j) * kD;
-#pragma unroll 8
-    for (int k = 0; k < kD; ++k) acc = __fmaf_rn(x[k], m[k], acc);
+    const float4* m4 = reinterpret_cast<const float4*>(ud.M + static_cast<size_t>(j) * kD);
+#pragma unroll 4
+    for (int c = 0; c < 32; ++c) {
+      const float4 m = m4[c];
+      acc = __fmaf_rn(xs[4 * c], m.x, acc);
+      acc = __fmaf_rn(xs[4 * c + 1], m.y, acc);
+      acc = __fmaf_rn(xs[4 * c + 2], m.z, acc);
+      acc = __fmaf_rn(xs[4 * c + 3], m.w, acc);
+    }
   }
   const uint32_t code = quantize_code(acc, ud.inv_delta, ud.b);
 
@@ -154,18 +163,13 @@ extern "C" kvtc_status kvtc_encode_append(const kvtc_plan* plan, const kvtc_cach
   a.pos_start = pos_start;
   a.n_seq = cache->n_seq;
   a.n_tok = n_tok;
-  a.coords_per_token = 0;
-  for (int ul = 0; ul < a.n_units; ++ul) a.coords_per_token += plan->r[a.unit0 + ul];
   a.pool = static_cast<char*>(cache->pool);
   a.pages_per_unit = cache->pages_per_unit;
   a.block_table = cache->block_table;
   a.max_pages = cache->max_pages;
   a.status = cache->status;
-  const long long total = static_cast<long long>(n_tok) * a.coords_per_token;
-  const long long blocks = (total + 127) / 128;
-  if (blocks > 0x7FFFFFFFll) return fail(KVTC_EINVAL, "too many tokens for one call");
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.gridDim = dim3(static_cast<unsigned>(n_tok), static_cast<unsigned>(a.n_units));
   cfg.blockDim = dim3(128);
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
