@@ -86,6 +86,8 @@ def lib():
         "kvtc_decode_workspace_bytes": (C.c_uint64, [_P, C.c_int, C.c_int]),
         "kvtc_decode_attention": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, C.c_int, _P, C.c_int, C.c_float,
                                        _P, C.c_int, _P, C.c_uint64, _P]),
+        "kvtc_decode_attention_noalloc": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, C.c_int, _P, C.c_int,
+                                               C.c_float, _P, C.c_int, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -283,3 +285,11 @@ def kvtc_decode_attention(plan, cache, layer, q, seq_lens, max_seq_len, out, wor
                                        _dev_ptr(seq_lens), max_seq_len, scale, _dev_ptr(out), _dtype_code(out),
                                        _dev_ptr(workspace), workspace.numel() * workspace.element_size(),
                                        _stream(stream)))
+
+
+def kvtc_decode_attention_noalloc(plan, cache, layer, q, seq_lens, max_seq_len, out, scale=0.0, stream=None):
+    """Decode attention using the library's own fixed scratch array (no workspace
+    argument), for callers that cannot allocate device memory."""
+    _check(lib().kvtc_decode_attention_noalloc(plan.handle, C.byref(cache.desc), layer, _dev_ptr(q),
+                                               _dtype_code(q), _dev_ptr(seq_lens), max_seq_len, scale,
+                                               _dev_ptr(out), _dtype_code(out), _stream(stream)))

@@ -265,6 +265,28 @@ kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_cache* cache
                                   kvtc_dtype out_dtype, void* workspace, uint64_t workspace_bytes,
                                   void* stream);
 
+/*
+ * kvtc_decode_attention_noalloc -- kvtc_decode_attention without a caller workspace.
+ * The KV-COBRA pages have no counterpart to this call; it exists for callers that cannot
+ * allocate device memory (a host runtime that owns every allocation through its own
+ * pool, a plugin limited to the buffers it is handed, code running while allocation is
+ * not permitted).  Its split-K scratch is a fixed 16 MiB array inside the library
+ * (a file-scope __device__ array: every GPU that loads the library holds it until the
+ * process exits); nothing is allocated per call.
+ *   - The first call on a device looks up the array's device address (once per device,
+ *     with that device current).  Make that first call before any stream capture.
+ *   - Calls whose kvtc_decode_workspace_bytes(plan, n_seq, max_seq_len) exceeds 16 MiB
+ *     return KVTC_ECAPACITY; use kvtc_decode_attention with a workspace for those.
+ *   - Every call shares the one array and leaves its contents behind.  No part of it has
+ *     to start at zero (each call writes every slot it later reads), but two calls that
+ *     run at the same time on the GPU (different streams, or overlapping graphs) race.
+ * Arguments, results and error codes otherwise as kvtc_decode_attention.
+ */
+kvtc_status kvtc_decode_attention_noalloc(const kvtc_plan* plan, const kvtc_cache* cache, int layer,
+                                          const void* q, kvtc_dtype q_dtype, const int32_t* seq_lens,
+                                          int max_seq_len, float softmax_scale, void* out,
+                                          kvtc_dtype out_dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
