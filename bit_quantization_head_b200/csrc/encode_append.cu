@@ -2,9 +2,10 @@
 //
 // KV-COBRA project page, "How KV-COBRA Works" (Inference): each key (and value) is
 // rotated and truncated with H.V^T and quantized with the unit's b-bit quantizer.  One
-// thread computes one latent coordinate y_j of one token of one unit as the fp32 chain
-// acc = fma(x_k, M_jk, acc), k = 0..127 in order (the canonical arithmetic the oracle
-// reproduces bit for bit), quantizes it and merges its bits into the page word.
+// thread computes one latent coordinate y_j of one token of one unit in the canonical
+// fp32 order (eight fma chains over k mod 8, then a fixed pairwise sum: the arithmetic
+// the oracle reproduces bit for bit), quantizes it and merges its bits into the page
+// word.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -58,7 +59,7 @@ __device__ __forceinline__ void store_code(uint32_t* page, int kind, int r, int 
 
 // CTA = (token, unit of the layer); thread j computes coordinate j.  The token's row is
 // staged in shared memory once; each thread holds its row of M in registers; the fma
-// chain then runs in the canonical k order from registers and broadcast reads.
+// chains then run in the canonical order from registers and broadcast reads.
 __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constant__ AppendArgs a) {
   // Programmatic dependent launch: wait for the producer of k/v, then let the next kernel
   // (typically the decode of this layer) start its prologue.
@@ -78,8 +79,9 @@ __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constan
   __syncthreads();
   if (j >= ud.r) return;
 
-  // canonical projection: acc = fma(x_k, M_jk, acc) for k = 0..127 in order
-  float acc = 0.0f;
+  // canonical projection: eight chains a_e = fma(x_k, M_jk, a_e) over k = e (mod 8)
+  // ascending, then ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7))
+  float ch[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
   if (a.bf16) {
     const uint4* m4 = reinterpret_cast<const uint4*>(ud.Mbf + static_cast<size_t>(j) * kD);
     uint4 mr[16];
@@ -90,21 +92,27 @@ __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constan
       const uint32_t w[4] = {mr[c].x, mr[c].y, mr[c].z, mr[c].w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        acc = __fmaf_rn(xs[8 * c + 2 * q], __uint_as_float(w[q] << 16), acc);
-        acc = __fmaf_rn(xs[8 * c + 2 * q + 1], __uint_as_float(w[q] & 0xFFFF0000u), acc);
+        ch[2 * q] = __fmaf_rn(xs[8 * c + 2 * q], __uint_as_float(w[q] << 16), ch[2 * q]);
+        ch[2 * q + 1] = __fmaf_rn(xs[8 * c + 2 * q + 1], __uint_as_float(w[q] & 0xFFFF0000u), ch[2 * q + 1]);
       }
     }
   } else {
     const float4* m4 = reinterpret_cast<const float4*>(ud.M + static_cast<size_t>(j) * kD);
 #pragma unroll 4
-    for (int c = 0; c < 32; ++c) {
-      const float4 m = m4[c];
-      acc = __fmaf_rn(xs[4 * c], m.x, acc);
-      acc = __fmaf_rn(xs[4 * c + 1], m.y, acc);
-      acc = __fmaf_rn(xs[4 * c + 2], m.z, acc);
-      acc = __fmaf_rn(xs[4 * c + 3], m.w, acc);
+    for (int c = 0; c < 16; ++c) {
+      const float4 m0 = m4[2 * c], m1 = m4[2 * c + 1];
+      ch[0] = __fmaf_rn(xs[8 * c], m0.x, ch[0]);
+      ch[1] = __fmaf_rn(xs[8 * c + 1], m0.y, ch[1]);
+      ch[2] = __fmaf_rn(xs[8 * c + 2], m0.z, ch[2]);
+      ch[3] = __fmaf_rn(xs[8 * c + 3], m0.w, ch[3]);
+      ch[4] = __fmaf_rn(xs[8 * c + 4], m1.x, ch[4]);
+      ch[5] = __fmaf_rn(xs[8 * c + 5], m1.y, ch[5]);
+      ch[6] = __fmaf_rn(xs[8 * c + 6], m1.z, ch[6]);
+      ch[7] = __fmaf_rn(xs[8 * c + 7], m1.w, ch[7]);
     }
   }
+  const float acc = __fadd_rn(__fadd_rn(__fadd_rn(ch[0], ch[1]), __fadd_rn(ch[2], ch[3])),
+                              __fadd_rn(__fadd_rn(ch[4], ch[5]), __fadd_rn(ch[6], ch[7])));
   const uint32_t code = quantize_code(acc, ud.inv_delta, ud.b);
 
   // token -> (sequence, position) -> page

@@ -197,8 +197,10 @@ uint64_t kvtc_unit_pool_offset(const kvtc_plan* plan, int unit, uint64_t pages_p
  * kvtc_encode_append -- "Inference": each new key/value is rotated and truncated with
  * M_u = H.V_r^T and quantized with the unit's b-bit uniform quantizer, then written into
  * its page slot.  Canonical arithmetic (bit-exact with the oracle): for each retained
- * coordinate j, y_j = the fp32 chain acc = fma(x_k, M_jk, acc), k = 0..d-1 in order,
- * with M in the input's precision (bf16-rounded M for bf16 input, fp32 M for fp32);
+ * coordinate j, eight fp32 chains a_e = fma(x_k, M_jk, a_e) over k = e, e+8, ... in
+ * ascending order (e = 0..7, each from 0), then y_j = ((a_0 + a_1) + (a_2 + a_3)) +
+ * ((a_4 + a_5) + (a_6 + a_7)); M in the input's precision (bf16-rounded M for bf16
+ * input, fp32 M for fp32);
  * code = min(max(floor(fl(fl(y * inv_delta) + 2^(b-1))), 0), 2^b - 1) (NaN -> 0).
  *
  * k, v: device [n_tok][H_kv][d] of dtype.  cu_seqlens: device int32 [n_seq + 1], the new

@@ -6,9 +6,11 @@ and truncated with H.V^T and quantized with its head's b*-bit quantizer) and
 overhead" figure (only per-unit static parameters exist).
 
 Readings taken where the page is silent:
-  * Projection arithmetic is fp32, the exact canonical order: for each output
-    coordinate j, acc <- fma(x_k, M_jk, acc) for k = 0..d-1 ascending, acc starts at
-    0, each fma rounded once (round to nearest even).  Operands: the input values
+  * Projection arithmetic is fp32 in one fixed order (the pages fix none): for each
+    output coordinate j, eight interleaved chains a_e <- fma(x_k, M_jk, a_e) over
+    k = e, e+8, ..., e+d-8 ascending (e = 0..7), each starting at 0, each fma rounded
+    once (round to nearest even); then y_j = ((a_0 + a_1) + (a_2 + a_3)) +
+    ((a_4 + a_5) + (a_6 + a_7)), each add rounded once.  Operands: the input values
     exactly as stored; M in the input's precision (bf16-rounded M for bf16 inputs,
     fp32 M for fp32 inputs).
   * Quantizer (mid-rise, 2^b levels, no zero level): t = fl32(y * inv_delta),
@@ -70,28 +72,33 @@ def to_bf16(x):
 
 
 def project_canonical(x, M):
-    """y[n, j] = the canonical fp32 fma chain of x[n, :] against M[j, :].
+    """y[n, j] = the canonical fp32 projection of x[n, :] against M[j, :] (module
+    docstring: eight interleaved fma chains over k mod 8, then a fixed pairwise sum).
 
     x: [n, d] float32 (values exactly as the device reads them); M: [r, d] float32
-    operand matrix.  Returns [n, r] float32.  When every product x_k * M_jk is exact
-    in fp32 (both operands bf16-representable) the fma reduces to an fp32 add of the
-    exact product; otherwise the fp64 emulation ``fmaf32`` is used.
+    operand matrix, d a multiple of 8.  Returns [n, r] float32.  When every product
+    x_k * M_jk is exact in fp32 (both operands bf16-representable) the fma reduces to
+    an fp32 add of the exact product; otherwise the fp64 emulation ``fmaf32`` is used.
     """
     x = np.asarray(x, dtype=np.float32)
     M = np.asarray(M, dtype=np.float32)
     n, d = x.shape
     r = M.shape[0]
-    acc = np.zeros((n, r), dtype=np.float32)
+    assert d % 8 == 0
+    chains = np.zeros((n, r, 8), dtype=np.float32)
     exact_products = (np.array_equal(to_bf16(x), x, equal_nan=True)
                       and np.array_equal(to_bf16(M), M))
-    for k in range(d):
-        xk = x[:, k:k + 1]
-        mk = M[None, :, k]
+    for k0 in range(0, d, 8):
+        xk = x[:, None, k0:k0 + 8]          # [n, 1, 8]: element e feeds chain e
+        mk = M[None, :, k0:k0 + 8]          # [1, r, 8]
         if exact_products:
-            acc = (acc + xk * mk).astype(np.float32)
+            with np.errstate(invalid="ignore", over="ignore"):
+                chains = (chains + xk * mk).astype(np.float32)
         else:
-            acc = fmaf32(np.broadcast_to(xk, acc.shape), np.broadcast_to(mk, acc.shape), acc)
-    return acc
+            chains = fmaf32(np.broadcast_to(xk, chains.shape), np.broadcast_to(mk, chains.shape), chains)
+    a = [chains[:, :, e] for e in range(8)]
+    with np.errstate(invalid="ignore", over="ignore"):
+        return (((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]))).astype(np.float32)
 
 
 def quantize(y, inv_delta, b):

@@ -39,16 +39,56 @@ def test_fmaf_emulation_matches_c_library_fmaf():
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
+def _chains_by_emulated_fma(x, M):
+    """The canonical order written out with the fp64-emulated fma: chain e takes
+    k = e, e+8, ... ascending; then the fixed pairwise sum."""
+    n, r = x.shape[0], M.shape[0]
+    a = [np.zeros((n, r), np.float32) for _ in range(8)]
+    for k in range(x.shape[1]):
+        e = k % 8
+        a[e] = codec.fmaf32(np.broadcast_to(x[:, k:k + 1], (n, r)), np.broadcast_to(M[None, :, k], (n, r)), a[e])
+    return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]))
+
+
 def test_canonical_projection_fast_path_equals_emulated_fma_on_bf16_operands():
     rng = np.random.default_rng(1)
     x = codec.to_bf16(rng.standard_normal((40, 128)).astype(np.float32))
     M = codec.to_bf16(rng.standard_normal((12, 128)).astype(np.float32) / 8)
     fast = codec.project_canonical(x, M)
-    acc = np.zeros((40, 12), np.float32)
-    for k in range(128):
-        acc = codec.fmaf32(np.broadcast_to(x[:, k:k + 1], acc.shape),
-                           np.broadcast_to(M[None, :, k], acc.shape), acc)
-    assert np.array_equal(fast.view(np.uint32), acc.view(np.uint32))
+    ref = _chains_by_emulated_fma(x, M)
+    assert np.array_equal(fast.view(np.uint32), ref.view(np.uint32))
+
+
+def test_canonical_projection_equals_exact_rational_evaluation_of_its_order():
+    # Each fma and each add of the stated order evaluated exactly and rounded once to
+    # fp32 with rational arithmetic: independent of numpy's float32 and of fmaf32.
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((3, 32)) * 10.0 ** rng.integers(-2, 3, (3, 32))).astype(np.float32)
+    M = (rng.standard_normal((2, 32)) * 10.0 ** rng.integers(-2, 3, (2, 32))).astype(np.float32)
+    got = codec.project_canonical(x, M)
+    for i in range(3):
+        for j in range(2):
+            a = [Fraction(0)] * 8
+            for k in range(32):
+                a[k % 8] = _rn32(Fraction(float(x[i, k])) * Fraction(float(M[j, k])) + a[k % 8])
+            s01, s23 = _rn32(a[0] + a[1]), _rn32(a[2] + a[3])
+            s45, s67 = _rn32(a[4] + a[5]), _rn32(a[6] + a[7])
+            y = _rn32(_rn32(s01 + s23) + _rn32(s45 + s67))
+            assert Fraction(float(got[i, j])) == y
+
+
+def test_canonical_projection_order_is_not_the_sequential_chain():
+    # The order is part of the definition: on cancelling inputs the sequential fma
+    # chain and the eight-chain order give different fp32 results.
+    x = np.zeros((1, 16), np.float32)
+    M = np.zeros((1, 16), np.float32)
+    x[0, 0], x[0, 1], x[0, 8] = 1.0, 2.0 ** -30, -1.0
+    M[0, 0] = M[0, 1] = M[0, 8] = 1.0
+    y = codec.project_canonical(x, M)[0, 0]
+    seq = np.float32(0.0)
+    for k in range(16):
+        seq = codec.fmaf32(x[0, k], M[0, k], seq)
+    assert y == np.float32(2.0 ** -30) and seq == np.float32(0.0)
 
 
 def test_canonical_projection_within_fp32_accumulation_bound():
