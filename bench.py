@@ -300,6 +300,23 @@ def encode_bench(torch, w, steps, warmup, rank, n_layers=None):
             "bytes_per_pass": in_bytes + code_bytes, "tflop_s": flops / ms / 1e9, "layers": w.n_layers}
 
 
+def max_over_ranks(torch, dist, x):
+    """The largest value of x over the ranks (every rank gets it); x itself when alone.
+    The reduction runs on the backend's device (CUDA for NCCL, host for gloo)."""
+    if not dist:
+        return x
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(world, step_bytes, ms):
+    """Whole-job GB/s: every rank streams step_bytes per step (replicas, weak scaling);
+    the step time is the slowest rank's."""
+    return world * step_bytes / (ms * 1e-3) / 1e9
+
+
 def run_ours(args, torch, dist, rank, world):
     w = synth.WORKLOADS[args.workload]
     if args.layers:
@@ -348,11 +365,8 @@ def run_ours(args, torch, dist, rank, world):
             g.replay()
         e1.record(stream)
         torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(torch, dist, e0.elapsed_time(e1) / args.steps)
     if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
 
     # per-launch duration of the dominant kernel (decode call of one layer)
@@ -390,13 +404,9 @@ def run_ours(args, torch, dist, rank, world):
             out_h.copy_(st["out"], non_blocking=True)
         f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / args.steps
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(torch, dist, f0.elapsed_time(f1) / args.steps)
 
-    value = world * step_bytes / (ms * 1e-3) / 1e9
+    value = aggregate_value(world, step_bytes, ms)
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
@@ -412,7 +422,7 @@ def run_ours(args, torch, dist, rank, world):
                      "frac": round(achieved / hbm_peak, 4), "traffic": None,
                      "kernel": "decode (split kernel + combine) of one layer", "peak_kind": peak_kind,
                      "bytes_per_launch": step_bytes // L, "launch_ms": round(dec_ms, 5)},
-        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(aggregate_value(world, step_bytes, e2e_ms), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": kernels_per_step(plan, w) * args.steps,
         "clocks": clk.summary(),
@@ -501,7 +511,7 @@ def main():
         import datetime
         import torch.distributed as td
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
-        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = td
     res = run_ours(args, torch, dist, rank, world)
     if rank == 0:
