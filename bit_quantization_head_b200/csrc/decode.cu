@@ -199,12 +199,12 @@ __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(const __gr
   // M_V in shared memory (bounded wait; on a time-out the output is zero and the status
   // word says so)
   bool ok = false;
-  for (uint32_t it = 0; it < (1u << 20) && !ok; ++it) ok = mbar_try_wait(&bar, 0);
+  for (uint32_t it = 0; it < (1u << 16) && !ok; ++it) ok = mbar_try_wait_sleep(&bar, 0, 20000u);
   ok = __syncthreads_and(ok);
   if (!ok) {
     if (tid == 0 && ca.status) atomicOr(ca.status, KVTC_STATUS_TIMEOUT);
     bool done = false;
-    for (uint32_t it = 0; it < (1u << 20) && !done; ++it) done = mbar_try_wait(&bar, 0);
+    for (uint32_t it = 0; it < (1u << 16) && !done; ++it) done = mbar_try_wait_sleep(&bar, 0, 20000u);
   }
   // o[k] = sum_j M_V[j][k] y[j]: threads k and k + 128 take the even and odd j
   const int k = tid & 127, par = tid >> 7;
@@ -234,12 +234,18 @@ __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(const __gr
 // run-time path (class 0).
 int width_class(int b) { return (b == 2 || b == 4 || b == 8) ? b : 0; }
 
-SplitFn split_fn(int bK, int bV, bool pack, bool small) {
+// Cost model of one page for the split allocation (warp instructions per page and warp:
+// softmax, bookkeeping and the per-16-coordinate MMA rows).
+constexpr double kPageCost = 320.0;
+constexpr size_t kReadSlack = 2048;
+constexpr double kTileCost = 56.0;
+
+SplitFn split_fn(int bK, int bV, bool pack) {
   switch (width_class(bK)) {
-    case 2: return split_fn_bk<2>(width_class(bV), pack, small);
-    case 4: return split_fn_bk<4>(width_class(bV), pack, small);
-    case 8: return split_fn_bk<8>(width_class(bV), pack, small);
-    default: return split_fn_bk<0>(width_class(bV), pack, small);
+    case 2: return split_fn_bk<2>(width_class(bV), pack);
+    case 4: return split_fn_bk<4>(width_class(bV), pack);
+    case 8: return split_fn_bk<8>(width_class(bV), pack);
+    default: return split_fn_bk<0>(width_class(bV), pack);
   }
 }
 
@@ -351,20 +357,23 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
   }
 
   // ---- kernel 1: split kernels.  The layer's KV heads are grouped by kernel variant
-  // (width classes of b_K and b_V, and the rank class: both ranks <= 64 use the 4-tile
-  // variant).  One launch per group; the launches run side by side, so each gets the
-  // share of a wave of resident CTAs that its bytes are of the layer's, and within a group
-  // each head gets context splits in proportion to its bytes per page.
+  // (width classes of b_K and b_V).  One launch per group; the launches run side by side,
+  // so each gets the share of a wave of resident CTAs that its work is of the layer's,
+  // and within a group each head gets context splits in proportion to its work per page.
+  // The work of a page is mostly instruction issue, not bytes: the online softmax costs
+  // the same for every head, and each 16 coordinates of K or V add one MMA row of work
+  // per block, so a page's cost is modelled as kPageCost + kTileCost * (k-steps + m-tiles)
+  // (warp instructions, from the kernel's instruction mix).
   const bool pack = plan->G <= 4;
   std::map<int, std::vector<int>> groups;
-  std::vector<double> head_bytes_pp(plan->H);
-  double layer_bytes = 0.0;
+  std::vector<double> head_bytes_pp(plan->H), head_cost(plan->H);
+  double layer_cost = 0.0;
   for (int h = 0; h < plan->H; ++h) {
     const int uK = (layer * plan->H + h) * 2;
-    const bool small = plan->r[uK] <= 64 && plan->r[uK + 1] <= 64;
-    groups[(width_class(plan->b[uK]) * 16 + width_class(plan->b[uK + 1])) * 2 + (small ? 1 : 0)].push_back(h);
+    groups[width_class(plan->b[uK]) * 16 + width_class(plan->b[uK + 1])].push_back(h);
     head_bytes_pp[h] = 16.0 * (plan->r[uK] * plan->b[uK] + plan->r[uK + 1] * plan->b[uK + 1]);
-    layer_bytes += head_bytes_pp[h];
+    head_cost[h] = kPageCost + kTileCost * ((plan->r[uK] + 15) / 16 + (plan->r[uK + 1] + 15) / 16);
+    layer_cost += head_cost[h];
   }
   CombineArgs ca;
   ca.units = plan->d_units;
@@ -381,17 +390,17 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
   const size_t head_bytes = ((sizeof(SmemHead) + 8 * kWarps * 8 + 127) / 128) * 128;
   bool first = true;
   for (auto& kv : groups) {
-    const bool small = kv.first & 1;
-    const int wk = (kv.first >> 1) >> 4, wv = (kv.first >> 1) & 15;
+    const int wk = kv.first >> 4, wv = kv.first & 15;
     const std::vector<int>& hs = kv.second;
     uint32_t stage_bytes = 0;
-    double group_bytes = 0.0;
+    double group_cost = 0.0;
     for (int h : hs) {
       stage_bytes = std::max(stage_bytes, (static_cast<uint32_t>(head_bytes_pp[h]) + 127u) / 128u * 128u);
-      group_bytes += head_bytes_pp[h];
+      group_cost += head_cost[h];
     }
-    // shared memory for three CTAs per SM where the pages allow it
-    const size_t budget = 74 * 1024;
+    // shared memory for kMinBlocks CTAs per SM where the pages allow it (228 KB per SM,
+    // 1 KB of it reserved per CTA)
+    const size_t budget = 233472 / kMinBlocks - 1024 - kReadSlack;
     int n_stage = budget > head_bytes
                       ? static_cast<int>((budget - head_bytes) / (static_cast<size_t>(kWarps) * stage_bytes))
                       : 0;
@@ -400,12 +409,14 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     n_stage = std::max(1, n_stage);
     // the stage region also holds the end-of-kernel merge of the four warps' partials
     const size_t merge_bytes = static_cast<size_t>(kWarps) * 8 * kPartStride * sizeof(float);
-    const size_t smem = head_bytes + std::max<size_t>(static_cast<size_t>(kWarps) * n_stage * stage_bytes, merge_bytes);
-    SplitFn fn = split_fn(wk == 0 ? 3 : wk, wv == 0 ? 3 : wv, pack, small);
+    // + slack: the kernel reads whole 16-row tiles, up to 2 KB past a page's last row
+    const size_t smem = head_bytes + std::max<size_t>(static_cast<size_t>(kWarps) * n_stage * stage_bytes, merge_bytes) +
+                        kReadSlack;
+    SplitFn fn = split_fn(wk == 0 ? 3 : wk, wv == 0 ? 3 : wv, pack);
     if (!fn) return fail(KVTC_EINVAL, "no decode kernel for this code width");
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (decode)");
-    const double share = group_bytes / layer_bytes;
+    const double share = group_cost / layer_cost;
     const int wave = static_cast<int>(occupancy(fn, smem) * sm_count() * share);
     const int columns = std::max(static_cast<int>(hs.size()), wave / std::max(1, n_hg * n_seq));
     DecodeArgs a;
@@ -419,7 +430,7 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     a.split_prefix[0] = 0;
     for (size_t i = 0; i < hs.size(); ++i) {
       a.heads[i] = hs[i];
-      int ns = static_cast<int>(std::floor(columns * head_bytes_pp[hs[i]] / group_bytes));
+      int ns = static_cast<int>(std::floor(columns * head_cost[hs[i]] / group_cost));
       ns = std::max(1, std::min(ns, cap));
       a.split_prefix[i + 1] = a.split_prefix[i] + ns;
       ca.nparts[hs[i]] = ns;

@@ -17,9 +17,10 @@
 //     whose A operand again comes straight from the packed value words.  One extra A row
 //     of ones (when r_V is not a multiple of 16) accumulates l = sum p with the same
 //     rounded P, so z - m_V * l cancels consistently.
-// The four warps' (m, l, z) partials meet in shared memory and each CTA writes one partial
-// per query head; decode.cu's combine kernel merges those and back-projects.  q~ = M_K q
-// comes from decode.cu's prep kernel through the workspace.
+// IL blocks are processed together (their MMA chains interleave).  The four warps'
+// (m, l, z) partials meet in shared memory and each CTA writes one partial per query
+// head; decode.cu's combine kernel merges those and back-projects.  q~ = M_K q comes from
+// decode.cu's prep kernel through the workspace.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -30,13 +31,19 @@
 #include "kvtc_internal.h"
 #include "ptx.cuh"
 
+#ifndef KVTC_DECODE_IL
+#define KVTC_DECODE_IL 4
+#endif
+
 namespace kvtc {
 namespace dec {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
+constexpr int kNT = 8;                // 16-row tiles of a rank (r <= 128)
+constexpr int kIL = KVTC_DECODE_IL;   // blocks processed together
+constexpr int kMinBlocks = kIL >= 4 ? 2 : (kIL == 2 ? 3 : 4);  // resident CTAs per SM aimed for
 constexpr int kPartStride = 132;      // floats per partial: m, l, 2 pad, z[128]
-constexpr int kTargetCtas = 3 * 148;  // three CTAs per SM on a B200
 constexpr int kMaxHeadsPerLaunch = 64;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;         // log2 of the growth allowed before a rescale
@@ -81,12 +88,14 @@ __host__ __device__ constexpr int e_idx(int blk, int eta) {
   return B == 2 ? 2 * (blk & 1) + eta : (B == 4 ? eta : 0);
 }
 
+// A-fragment pair of block BLK (eta = 0: the lane's first row, 1: its second) from word
+// W, or from Wh = W >> 8 when the field sits at bit 8 or above.
 template <int B, int BLK, int ETA>
-__device__ __forceinline__ uint32_t fast_pair(uint32_t W) {
+__device__ __forceinline__ uint32_t fast_pair(uint32_t W, uint32_t Wh) {
   constexpr int off = pair_offset(B, BLK, ETA);
   constexpr uint32_t m = (1u << B) - 1u;
   if constexpr (off >= 8) {
-    return (W >> 8) & ((m << (off - 8)) | (m << (off + 8)));
+    return Wh & ((m << (off - 8)) | (m << (off + 8)));
   } else {
     return W & ((m << off) | (m << (off + 16)));
   }
@@ -118,62 +127,12 @@ __device__ __forceinline__ uint32_t gen_pair(const uint32_t (&W)[4], const Parts
 #pragma unroll
   for (int lw = 3; lw >= 0; --lw) {
     if (P.has[lw]) {
-      constexpr int dummy = 0;
-      (void)dummy;
       const int off = ((2 * BLK + ETA) & ((16 >> lw) - 1)) << lw;
       const uint32_t m = (1u << (1 << lw)) - 1u;
       v |= ((W[lw] >> off) & (m | (m << 16))) << P.lo[lw];
     }
   }
   return v;
-}
-
-// ------------------------------------------------------------------ shared memory
-struct SmemHead {
-  float qt[8][128];  // q~ = M_K q (zero beyond the head group and beyond r_K)
-  float S[8];        // sum_j q~_j
-  int E[8];          // power-of-two normalisation of q~ for fp16
-};
-
-// ------------------------------------------------------------------ per-warp state
-template <int BK, int BV, bool PACK, int NT>
-struct WS {
-  const uint32_t* pk;  // K page in shared memory
-  const uint32_t* pv;  // V page in shared memory
-  int tok0, seq_len;
-  int rK, rV, nks, nmt, g, tq;
-  Parts partsK, partsV;
-  int ones_mt, ones_lr;  // m-tile / local row of the ones row (ones_mt < 0: none)
-  uint32_t ones_m0, ones_m1;  // lane masks: this lane's A rows g / g+8 are the ones row
-  // B fragments of q^: PACK -> bq[ks] (hi for g < 4, lo for g >= 4); else bh, bl
-  uint32_t bh[NT][2];
-  uint32_t bl[PACK ? 1 : NT][2];
-  float alpha[2], beta[2], m_run[2];
-  float al[2][n_e<BK == 0 ? 8 : BK>()], nb[2][n_e<BV == 0 ? 8 : BV>()];
-  float z[NT][4];
-  float lcvt[2];  // l accumulated from the fp16 P when there is no ones row
-};
-
-// Score argument constants: x = al * acc + nb, with e undone in al (key side) and the P
-// scale 2^(7 - e_V) folded into nb (value side).
-template <int BK, int BV, bool PACK, int NT>
-__device__ __forceinline__ void refresh_constants(WS<BK, BV, PACK, NT>& w) {
-  constexpr int NEK = n_e<BK == 0 ? 8 : BK>();
-  constexpr int NEV = n_e<BV == 0 ? 8 : BV>();
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-#pragma unroll
-    for (int i = 0; i < NEK; ++i) {
-      const int e = BK == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (BK == 4 ? 4 * i : 0);
-      w.al[c][i] = w.alpha[c] * (1.0f / static_cast<float>(1 << e));
-    }
-    const float base = -(w.beta[c] + (w.m_run[c] == -INFINITY ? 0.0f : w.m_run[c])) + 7.0f;
-#pragma unroll
-    for (int i = 0; i < NEV; ++i) {
-      const int e = BV == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (BV == 4 ? 4 * i : 0);
-      w.nb[c][i] = base - static_cast<float>(e);
-    }
-  }
 }
 
 // Generic words of a K row (or V row) for block BLK: one word per part.
@@ -192,31 +151,75 @@ __device__ __forceinline__ void gen_words(const uint32_t* page, int r, int row, 
   }
 }
 
-// ---- the work is done per half page (4 blocks of 16 tokens): the loop over k-steps
-// (or m-tiles) is outside the loop over blocks, so a rank guard costs once per half page
-// and the four blocks' MMA chains interleave.
+// ------------------------------------------------------------------ shared memory
+struct SmemHead {
+  float qt[8][128];  // q~ = M_K q (zero beyond the head group and beyond r_K)
+  float S[8];        // sum_j q~_j
+  int E[8];          // power-of-two normalisation of q~ for fp16
+};
 
-// Score MMA(s) of one block for k-step (rows r0, r1 of this lane).
-template <int BK, int BV, bool PACK, int NT, int BLK>
-__device__ __forceinline__ void k_block(const WS<BK, BV, PACK, NT>& w, int ks, int r0, int r1, bool ok0, bool ok1,
-                                        float (&sc)[4], float (&sd)[4]) {
+// ------------------------------------------------------------------ per-warp state
+template <int BK, int BV, bool PACK>
+struct WS {
+  const uint32_t* pk;  // K page in shared memory
+  const uint32_t* pv;  // V page in shared memory
+  int tok0, seq_len;
+  bool partial;        // the page holds positions at or beyond seq_len
+  int rK, rV, nks, nmt, g, tq;
+  Parts partsK, partsV;
+  int ones_mt, ones_lr;  // m-tile / local row of the ones row (ones_mt < 0: none)
+  uint32_t ones_m0, ones_m1;  // lane masks: this lane's A rows g / g+8 are the ones row
+  // B fragments of q^: PACK -> bh[ks] (hi for g < 4, lo for g >= 4); else bh, bl
+  uint32_t bh[kNT][2];
+  uint32_t bl[PACK ? 1 : kNT][2];
+  float alpha[2], beta[2], m_run[2];
+  float al[2][n_e<BK == 0 ? 8 : BK>()], nb[2][n_e<BV == 0 ? 8 : BV>()];
+  float z[kNT][4];
+  float lcvt[2];  // l accumulated from the fp16 P when there is no ones row
+};
+
+// Score argument constants: x = al * acc + nb, with e undone in al (key side) and the P
+// scale 2^(7 - e_V) folded into nb (value side).
+template <int BK, int BV, bool PACK>
+__device__ __forceinline__ void refresh_constants(WS<BK, BV, PACK>& w) {
+  constexpr int NEK = n_e<BK == 0 ? 8 : BK>();
+  constexpr int NEV = n_e<BV == 0 ? 8 : BV>();
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+#pragma unroll
+    for (int i = 0; i < NEK; ++i) {
+      const int e = BK == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (BK == 4 ? 4 * i : 0);
+      w.al[c][i] = w.alpha[c] * (1.0f / static_cast<float>(1 << e));
+    }
+    const float base = -(w.beta[c] + (w.m_run[c] == -INFINITY ? 0.0f : w.m_run[c])) + 7.0f;
+#pragma unroll
+    for (int i = 0; i < NEV; ++i) {
+      const int e = BV == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (BV == 4 ? 4 * i : 0);
+      w.nb[c][i] = base - static_cast<float>(e);
+    }
+  }
+}
+
+// Score MMA(s) of one block for k-step ks.  Fast widths: W0, W1 are the words of rows
+// r0, r1 of this lane that hold the block's fields (Wh = W >> 8).  Generic widths: the
+// words are read here (rows r0, r1).
+template <int BK, int BV, bool PACK, int BLK>
+__device__ __forceinline__ void k_block(const WS<BK, BV, PACK>& w, int ks, uint32_t W0, uint32_t W0h, uint32_t W1,
+                                        uint32_t W1h, int r0, int r1, float (&sc)[4], float (&sd)[4]) {
   uint32_t A0, A1, A2, A3;
   if constexpr (BK != 0) {
-    const int wsel = w.g * BK + (BLK * BK) / 8;
-    const uint32_t W0 = ok0 ? w.pk[r0 * 8 * BK + wsel] : 0u;
-    const uint32_t W1 = ok1 ? w.pk[r1 * 8 * BK + wsel] : 0u;
-    A0 = fast_pair<BK, BLK, 0>(W0);
-    A1 = fast_pair<BK, BLK, 1>(W0);
-    A2 = fast_pair<BK, BLK, 0>(W1);
-    A3 = fast_pair<BK, BLK, 1>(W1);
+    A0 = fast_pair<BK, BLK, 0>(W0, W0h);
+    A1 = fast_pair<BK, BLK, 1>(W0, W0h);
+    A2 = fast_pair<BK, BLK, 0>(W1, W1h);
+    A3 = fast_pair<BK, BLK, 1>(W1, W1h);
   } else {
-    uint32_t W0[4], W1[4];
-    gen_words<BLK>(w.pk, w.rK, r0, ok0, w.g, true, w.partsK, W0);
-    gen_words<BLK>(w.pk, w.rK, r1, ok1, w.g, true, w.partsK, W1);
-    A0 = gen_pair<BLK, 0>(W0, w.partsK);
-    A1 = gen_pair<BLK, 1>(W0, w.partsK);
-    A2 = gen_pair<BLK, 0>(W1, w.partsK);
-    A3 = gen_pair<BLK, 1>(W1, w.partsK);
+    uint32_t G0[4], G1[4];
+    gen_words<BLK>(w.pk, w.rK, r0, true, w.g, true, w.partsK, G0);
+    gen_words<BLK>(w.pk, w.rK, r1, true, w.g, true, w.partsK, G1);
+    A0 = gen_pair<BLK, 0>(G0, w.partsK);
+    A1 = gen_pair<BLK, 1>(G0, w.partsK);
+    A2 = gen_pair<BLK, 0>(G1, w.partsK);
+    A3 = gen_pair<BLK, 1>(G1, w.partsK);
   }
   mma_16816(sc, A0, A1, A2, A3, w.bh[ks][0], w.bh[ks][1]);
   if constexpr (!PACK) mma_16816(sd, A0, A1, A2, A3, w.bl[ks][0], w.bl[ks][1]);
@@ -224,8 +227,8 @@ __device__ __forceinline__ void k_block(const WS<BK, BV, PACK, NT>& w, int ks, i
 
 // Score arguments of one block: x = s - m_run + 7 - e_V (log2 domain), -inf if masked.
 // Returns whether the block asks for a rescale (a score past the running max by 2^kLazy).
-template <int BK, int BV, bool PACK, int NT, bool FULL, int BLK>
-__device__ __forceinline__ bool x_block(const WS<BK, BV, PACK, NT>& w, const float (&sc)[4], const float (&sd)[4],
+template <int BK, int BV, bool PACK, int BLK>
+__device__ __forceinline__ bool x_block(const WS<BK, BV, PACK>& w, const float (&sc)[4], const float (&sd)[4],
                                         float (&x)[4]) {
   float full[4];
 #pragma unroll
@@ -244,7 +247,7 @@ __device__ __forceinline__ bool x_block(const WS<BK, BV, PACK, NT>& w, const flo
   x[1] = fmaf(w.al[1][ik0], full[1], w.nb[1][iv0]);
   x[2] = fmaf(w.al[0][ik1], full[2], w.nb[0][iv1]);
   x[3] = fmaf(w.al[1][ik1], full[3], w.nb[1][iv1]);
-  if constexpr (!FULL) {
+  if (w.partial) {  // warp-uniform: only the last page of a sequence
     const int t0 = w.tok0 + 16 * BLK + w.g, t1 = t0 + 8;
     if (t0 >= w.seq_len) x[0] = x[1] = -INFINITY;
     if (t1 >= w.seq_len) x[2] = x[3] = -INFINITY;
@@ -262,8 +265,8 @@ __device__ __forceinline__ float xmax_block(const float (&x)[4], int c) {
 
 // P of one block in fp16 (already scaled by 2^(7 - e_V) through x), transposed into the
 // B fragment of the value MMA; l from the rounded P when there is no ones row.
-template <int BK, int BV, bool PACK, int NT, int BLK>
-__device__ __forceinline__ void p_block(WS<BK, BV, PACK, NT>& w, const float (&x)[4], uint32_t (&bp)[2]) {
+template <int BK, int BV, bool PACK, int BLK>
+__device__ __forceinline__ void p_block(WS<BK, BV, PACK>& w, const float (&x)[4], uint32_t (&bp)[2]) {
   const uint32_t P0 = pack_half2(ex2(x[0]), ex2(x[1]));
   const uint32_t P1 = pack_half2(ex2(x[2]), ex2(x[3]));
   if (w.ones_mt < 0) {
@@ -277,71 +280,90 @@ __device__ __forceinline__ void p_block(WS<BK, BV, PACK, NT>& w, const float (&x
   bp[1] = movmatrix_trans(P1);
 }
 
-// Value MMA of one block for m-tile mt (rows j0, j1 of this lane).
-template <int BK, int BV, bool PACK, int NT, int BLK>
-__device__ __forceinline__ void v_block(const WS<BK, BV, PACK, NT>& w, int j0, int j1, bool ok0, bool ok1,
-                                        bool ones, const uint32_t (&bp)[2], float (&z)[4]) {
+// Value MMA of one block for m-tile mt (words as in k_block; rows j0, j1).  Rows past
+// r_V hold whatever follows the page in shared memory: their z rows are never read,
+// except the ones row, whose A value is replaced whole.
+template <int BK, int BV, bool PACK, int BLK>
+__device__ __forceinline__ void v_block(const WS<BK, BV, PACK>& w, uint32_t W0, uint32_t W0h, uint32_t W1,
+                                        uint32_t W1h, int j0, int j1, bool ones, const uint32_t (&bp)[2],
+                                        float (&z)[4]) {
   uint32_t A0, A1, A2, A3;
   if constexpr (BV != 0) {
-    const int wsel = w.tq * BV + (BLK * BV) / 8;
-    const uint32_t W0 = ok0 ? w.pv[j0 * 4 * BV + wsel] : 0u;
-    const uint32_t W1 = ok1 ? w.pv[j1 * 4 * BV + wsel] : 0u;
-    A0 = fast_pair<BV, BLK, 0>(W0);
-    A1 = fast_pair<BV, BLK, 0>(W1);
-    A2 = fast_pair<BV, BLK, 1>(W0);
-    A3 = fast_pair<BV, BLK, 1>(W1);
+    A0 = fast_pair<BV, BLK, 0>(W0, W0h);
+    A1 = fast_pair<BV, BLK, 0>(W1, W1h);
+    A2 = fast_pair<BV, BLK, 1>(W0, W0h);
+    A3 = fast_pair<BV, BLK, 1>(W1, W1h);
   } else {
-    uint32_t W0[4], W1[4];
-    gen_words<BLK>(w.pv, w.rV, j0, ok0, w.tq, false, w.partsV, W0);
-    gen_words<BLK>(w.pv, w.rV, j1, ok1, w.tq, false, w.partsV, W1);
-    A0 = gen_pair<BLK, 0>(W0, w.partsV);
-    A1 = gen_pair<BLK, 0>(W1, w.partsV);
-    A2 = gen_pair<BLK, 1>(W0, w.partsV);
-    A3 = gen_pair<BLK, 1>(W1, w.partsV);
+    uint32_t G0[4], G1[4];
+    gen_words<BLK>(w.pv, w.rV, j0, true, w.tq, false, w.partsV, G0);
+    gen_words<BLK>(w.pv, w.rV, j1, true, w.tq, false, w.partsV, G1);
+    A0 = gen_pair<BLK, 0>(G0, w.partsV);
+    A1 = gen_pair<BLK, 0>(G1, w.partsV);
+    A2 = gen_pair<BLK, 1>(G0, w.partsV);
+    A3 = gen_pair<BLK, 1>(G1, w.partsV);
   }
-  if (ones) {  // the ones row (row r_V, zero so far) accumulates l
+  if (ones) {  // the ones row (row r_V) accumulates l: its A value is all ones
     constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
     constexpr uint32_t one0 = (1u << ev0) | (1u << (ev0 + 16)), one1 = (1u << ev1) | (1u << (ev1 + 16));
-    A0 |= one0 & w.ones_m0;
-    A2 |= one1 & w.ones_m0;
-    A1 |= one0 & w.ones_m1;
-    A3 |= one1 & w.ones_m1;
+    A0 = (A0 & ~w.ones_m0) | (one0 & w.ones_m0);
+    A2 = (A2 & ~w.ones_m0) | (one1 & w.ones_m0);
+    A1 = (A1 & ~w.ones_m1) | (one0 & w.ones_m1);
+    A3 = (A3 & ~w.ones_m1) | (one1 & w.ones_m1);
   }
   mma_16816(z, A0, A1, A2, A3, bp[0], bp[1]);
 }
 
-// Half page H2 (blocks 4*H2 .. 4*H2+3): scores, lazy online softmax, value accumulation.
-template <int BK, int BV, bool PACK, int NT, bool FULL, int H2, int... BB>
-__device__ __forceinline__ void do_half(WS<BK, BV, PACK, NT>& w, std::integer_sequence<int, BB...>) {
-  float sc[4][4], sd[4][4];
+// Blocks B0 .. B0 + IL - 1 of the page: scores, lazy online softmax, value accumulation.
+template <int BK, int BV, bool PACK, int B0, int... BB>
+__device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_sequence<int, BB...>) {
+  constexpr int IL = sizeof...(BB);
+  float sc[IL][4], sd[IL][4];
 #pragma unroll
-  for (int bb = 0; bb < 4; ++bb)
+  for (int bb = 0; bb < IL; ++bb)
 #pragma unroll
     for (int i = 0; i < 4; ++i) sc[bb][i] = sd[bb][i] = 0.0f;
   // ---- scores S[tok][head] = sum_j codeK[tok][j] * q^[head][j]
 #pragma unroll
-  for (int ks = 0; ks < NT; ++ks) {
+  for (int ks = 0; ks < kNT; ++ks) {
     if (ks < w.nks) {
+      // rows past r_K meet zero q^ coefficients (q~ is zero there), so they are read
+      // unmasked; the shared-memory allocation has slack for the over-read
       const int r0 = 8 * ks + w.tq, r1 = r0 + 4;
-      const bool ok0 = 2 * r0 < w.rK, ok1 = 2 * r1 < w.rK;
-      (k_block<BK, BV, PACK, NT, 4 * H2 + BB>(w, ks, r0, r1, ok0, ok1, sc[BB], sd[BB]), ...);
+      constexpr int KB = BK == 0 ? 1 : BK;
+      constexpr int KW0 = (B0 * KB) / 8, KWN = ((B0 + IL - 1) * KB) / 8 - KW0 + 1;
+      uint32_t W0[KWN], W1[KWN], W0h[KWN], W1h[KWN];
+#pragma unroll
+      for (int q = 0; q < KWN; ++q) {
+        if constexpr (BK != 0) {
+          W0[q] = w.pk[r0 * 8 * BK + w.g * BK + KW0 + q];
+          W1[q] = w.pk[r1 * 8 * BK + w.g * BK + KW0 + q];
+        } else {
+          W0[q] = W1[q] = 0u;
+        }
+        W0h[q] = W0[q] >> 8;
+        W1h[q] = W1[q] >> 8;
+      }
+      (k_block<BK, BV, PACK, B0 + BB>(w, ks, W0[((B0 + BB) * KB) / 8 - KW0], W0h[((B0 + BB) * KB) / 8 - KW0],
+                                      W1[((B0 + BB) * KB) / 8 - KW0], W1h[((B0 + BB) * KB) / 8 - KW0], r0, r1,
+                                      sc[BB], sd[BB]),
+       ...);
     }
   }
-  float x[4][4];
+  float x[IL][4];
   bool grow = false;
-  ((grow |= x_block<BK, BV, PACK, NT, FULL, 4 * H2 + BB>(w, sc[BB], sd[BB], x[BB])), ...);
-  // grow also while the running max is undefined (the first live half page)
+  ((grow |= x_block<BK, BV, PACK, B0 + BB>(w, sc[BB], sd[BB], x[BB])), ...);
+  // grow also while the running max is undefined (the first live block)
   grow |= w.m_run[0] == -INFINITY || w.m_run[1] == -INFINITY;
   // ---- lazy online softmax: rescale only when a score passes the running max by 2^kLazy
   if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       float v = -INFINITY;
-      ((v = fmaxf(v, xmax_block<BV, 4 * H2 + BB>(x[BB], c))), ...);
+      ((v = fmaxf(v, xmax_block<BV, B0 + BB>(x[BB], c))), ...);
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-      // v = max over the half page of s - m_run (m_run taken as 0 while undefined)
+      // v = max over the group of s - m_run (m_run taken as 0 while undefined)
       const float old = w.m_run[c];
       float shift = 0.0f;
       if (v == -INFINITY) {
@@ -354,14 +376,14 @@ __device__ __forceinline__ void do_half(WS<BK, BV, PACK, NT>& w, std::integer_se
         shift = v;
         const float resc = ex2(-v);
 #pragma unroll
-        for (int mt = 0; mt < NT; ++mt) {
+        for (int mt = 0; mt < kNT; ++mt) {
           w.z[mt][c] *= resc;
           w.z[mt][2 + c] *= resc;
         }
         w.lcvt[c] *= resc;
       }
 #pragma unroll
-      for (int bb = 0; bb < 4; ++bb) {
+      for (int bb = 0; bb < IL; ++bb) {
         x[bb][c] -= shift;
         x[bb][2 + c] -= shift;
       }
@@ -369,33 +391,48 @@ __device__ __forceinline__ void do_half(WS<BK, BV, PACK, NT>& w, std::integer_se
     refresh_constants(w);
   }
   // ---- probabilities -> B fragments
-  uint32_t bp[4][2];
-  (p_block<BK, BV, PACK, NT, 4 * H2 + BB>(w, x[BB], bp[BB]), ...);
+  uint32_t bp[IL][2];
+  (p_block<BK, BV, PACK, B0 + BB>(w, x[BB], bp[BB]), ...);
   // ---- values: Z^T[j][head] += sum_tok codeV[tok][j] * P[tok][head]
 #pragma unroll
-  for (int mt = 0; mt < NT; ++mt) {
+  for (int mt = 0; mt < kNT; ++mt) {
     if (mt < w.nmt) {
       const int j0 = 16 * mt + w.g, j1 = j0 + 8;
-      const bool ok0 = j0 < w.rV, ok1 = j1 < w.rV;
       const bool ones = mt == w.ones_mt;
-      (v_block<BK, BV, PACK, NT, 4 * H2 + BB>(w, j0, j1, ok0, ok1, ones, bp[BB], w.z[mt]), ...);
+      constexpr int VB = BV == 0 ? 1 : BV;
+      constexpr int VW0 = (B0 * VB) / 8, VWN = ((B0 + IL - 1) * VB) / 8 - VW0 + 1;
+      uint32_t W0[VWN], W1[VWN], W0h[VWN], W1h[VWN];
+#pragma unroll
+      for (int q = 0; q < VWN; ++q) {
+        if constexpr (BV != 0) {
+          W0[q] = w.pv[j0 * 4 * BV + w.tq * BV + VW0 + q];
+          W1[q] = w.pv[j1 * 4 * BV + w.tq * BV + VW0 + q];
+        } else {
+          W0[q] = W1[q] = 0u;
+        }
+        W0h[q] = W0[q] >> 8;
+        W1h[q] = W1[q] >> 8;
+      }
+      (v_block<BK, BV, PACK, B0 + BB>(w, W0[((B0 + BB) * VB) / 8 - VW0], W0h[((B0 + BB) * VB) / 8 - VW0],
+                                      W1[((B0 + BB) * VB) / 8 - VW0], W1h[((B0 + BB) * VB) / 8 - VW0], j0, j1,
+                                      ones, bp[BB], w.z[mt]),
+       ...);
     }
   }
 }
 
-template <int BK, int BV, bool PACK, int NT, bool FULL>
-__device__ __forceinline__ void do_page(WS<BK, BV, PACK, NT>& w) {
-  do_half<BK, BV, PACK, NT, FULL, 0>(w, std::make_integer_sequence<int, 4>{});
-  do_half<BK, BV, PACK, NT, FULL, 1>(w, std::make_integer_sequence<int, 4>{});
+template <int BK, int BV, bool PACK, int... GG>
+__device__ __forceinline__ void do_page_groups(WS<BK, BV, PACK>& w, std::integer_sequence<int, GG...>) {
+  (do_group<BK, BV, PACK, GG * kIL>(w, std::make_integer_sequence<int, kIL>{}), ...);
 }
 
-template <int BK, int BV, bool PACK, int NT>
-__global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  SmemHead& sh = *reinterpret_cast<SmemHead*>(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sizeof(SmemHead));
-  unsigned char* stages = smem + ((sizeof(SmemHead) + 8 * kWarps * 8 + 127) / 128) * 128;
+template <int BK, int BV, bool PACK>
+__device__ __forceinline__ void do_page(WS<BK, BV, PACK>& w) {
+  do_page_groups<BK, BV, PACK>(w, std::make_integer_sequence<int, 8 / kIL>{});
+}
 
+template <int BK, int BV, bool PACK>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
   // Programmatic dependent launch.  The first split launch of a call waits here for the
   // preceding grid (the q~ prep kernel, which completes only after its own predecessor,
   // e.g. the append that wrote the newest token).  A later split launch of the same call
@@ -403,6 +440,11 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
   // once and waits at exit instead, which keeps completion ordered for the combine.
   if (a.wait_first) griddep_wait();
   griddep_launch_dependents();
+  extern __shared__ __align__(128) unsigned char smem[];
+  SmemHead& sh = *reinterpret_cast<SmemHead*>(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sizeof(SmemHead));
+  unsigned char* stages = smem + ((sizeof(SmemHead) + 8 * kWarps * 8 + 127) / 128) * 128;
+
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
   // CTA -> (KV head, context split): heads get splits in proportion to their bytes
@@ -429,8 +471,9 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
   const int p_begin = split * pages_per_split;
   const int p_end = min(p_begin + pages_per_split, n_pages);
   const int n_my = p_end > p_begin + warp ? (p_end - p_begin - warp + kWarps - 1) / kWarps : 0;
+  const int32_t* bt = a.block_table + static_cast<size_t>(s) * a.max_pages;
 
-  // ---- prologue: barriers, q~, first copies ----
+  // ---- prologue: barriers, q~, page ids, first copies ----
   if (lane == 0)
     for (int i = 0; i < a.n_stage; ++i) mbar_init(&bars[warp * 8 + i], 1);
   for (int i = tid; i < 8 * 32; i += kThreads) {
@@ -448,52 +491,66 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
   const uint32_t bytesK = static_cast<uint32_t>(dK.page_bytes), bytesV = static_cast<uint32_t>(dV.page_bytes);
   const char* poolK = a.pool + a.pages_per_unit * dK.prefix;
   const char* poolV = a.pool + a.pages_per_unit * dV.prefix;
-  const int32_t* bt = a.block_table + static_cast<size_t>(s) * a.max_pages;
   auto stage_ptr = [&](int i) {
     return stages + (static_cast<size_t>(warp) * a.n_stage + (i % a.n_stage)) * a.stage_bytes;
   };
-  // Fill the stage of this warp's i-th page (lane 0).  Every use of a stage completes its
-  // barrier phase exactly once: with the copies' bytes, or by a plain arrival when the
-  // page id is invalid.
-  auto issue = [&](int i) {
-    const int p = p_begin + warp + i * kWarps;
-    const int32_t pid = bt[p];
-    uint64_t* bar = &bars[warp * 8 + (i % a.n_stage)];
+  // Page ids of this warp's pages, 32 at a time: lane l holds the id of page base + l of
+  // the current window (-1 past the end), so no dependent global load is left in the loop.
+  int pid_win = -1;
+  int pid_base = -1;
+  auto pid_of = [&](int i) {  // warp-uniform i
+    const int base = i & ~31;
+    if (base != pid_base) {
+      const int ii = base + lane;
+      pid_win = ii < n_my ? bt[p_begin + warp + ii * kWarps] : -1;
+      pid_base = base;
+    }
+    return __shfl_sync(0xffffffffu, pid_win, i & 31);
+  };
+  // Fill the stage of this warp's i-th page.  Every use of a stage completes its barrier
+  // phase exactly once: with the copies' bytes, or by a plain arrival when the page id
+  // is invalid.  vmask (lane 0) has bit i % n_stage set when the stage holds a page.
+  uint32_t vmask = 0;
+  auto issue = [&](int i, int pid) {  // lane 0
+    const int slot = i % a.n_stage;
+    uint64_t* bar = &bars[warp * 8 + slot];
     if (pid < 0 || static_cast<uint64_t>(pid) >= a.pages_per_unit) {
+      vmask &= ~(1u << slot);
       mbar_arrive(bar);
       return;
     }
+    vmask |= 1u << slot;
     unsigned char* st = stage_ptr(i);
     mbar_arrive_expect_tx(bar, bytesK + bytesV);
     bulk_copy_g2s(st, poolK + static_cast<uint64_t>(pid) * bytesK, bytesK, bar);
     bulk_copy_g2s(st + bytesK, poolV + static_cast<uint64_t>(pid) * bytesV, bytesV, bar);
   };
   const int n_first = min(a.n_stage, n_my);
-  if (lane == 0)
-    for (int i = 0; i < n_first; ++i) issue(i);
+  for (int i = 0; i < n_first; ++i) {
+    const int pid = pid_of(i);
+    if (lane == 0) issue(i, pid);
+  }
 
-  __syncthreads();
-  if (warp == 0) {
-    // per head: S = sum_j q~_j and the fp16 normalisation exponent
+  // per head: S = sum_j q~_j and the fp16 normalisation exponent (warp w: heads 2w, 2w+1)
 #pragma unroll
-    for (int gg = 0; gg < 8; ++gg) {
-      float S = sh.qt[gg][lane] + sh.qt[gg][lane + 32] + sh.qt[gg][lane + 64] + sh.qt[gg][lane + 96];
-      float amax = fmaxf(fmaxf(fabsf(sh.qt[gg][lane]), fabsf(sh.qt[gg][lane + 32])),
-                         fmaxf(fabsf(sh.qt[gg][lane + 64]), fabsf(sh.qt[gg][lane + 96])));
+  for (int hh = 0; hh < 2; ++hh) {
+    const int gg = 2 * warp + hh;
+    float S = sh.qt[gg][lane] + sh.qt[gg][lane + 32] + sh.qt[gg][lane + 64] + sh.qt[gg][lane + 96];
+    float amax = fmaxf(fmaxf(fabsf(sh.qt[gg][lane]), fabsf(sh.qt[gg][lane + 32])),
+                       fmaxf(fabsf(sh.qt[gg][lane + 64]), fabsf(sh.qt[gg][lane + 96])));
 #pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        S += __shfl_xor_sync(0xffffffffu, S, o);
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      }
-      if (lane == 0) {
-        sh.S[gg] = S;
-        sh.E[gg] = amax > 0.0f ? ilogbf(amax) - 14 : 0;
-      }
+    for (int o = 16; o; o >>= 1) {
+      S += __shfl_xor_sync(0xffffffffu, S, o);
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    }
+    if (lane == 0) {
+      sh.S[gg] = S;
+      sh.E[gg] = amax > 0.0f ? ilogbf(amax) - 14 : 0;
     }
   }
   __syncthreads();
 
-  WS<BK, BV, PACK, NT> w;
+  WS<BK, BV, PACK> w;
   w.rK = rK;
   w.rV = rV;
   w.nks = (rK + 15) >> 4;
@@ -501,6 +558,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
   w.g = g;
   w.tq = tq;
   w.seq_len = seq_len;
+  w.partial = false;
   w.partsK = parts_of(dK.b);
   w.partsV = parts_of(dV.b);
   w.ones_mt = (rV & 15) ? (rV >> 4) : -1;
@@ -513,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
     const int hsrc = PACK ? (g & 3) : g;
     const float scl = ldexpf(1.0f, -sh.E[hsrc]);
 #pragma unroll
-    for (int ks = 0; ks < NT; ++ks) {
+    for (int ks = 0; ks < kNT; ++ks) {
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int k0 = 16 * ks + 8 * half + 2 * tq;
@@ -546,15 +604,14 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
     refresh_constants(w);
   }
 #pragma unroll
-  for (int mt = 0; mt < NT; ++mt) w.z[mt][0] = w.z[mt][1] = w.z[mt][2] = w.z[mt][3] = 0.0f;
+  for (int mt = 0; mt < kNT; ++mt) w.z[mt][0] = w.z[mt][1] = w.z[mt][2] = w.z[mt][3] = 0.0f;
 
   // ---- main loop over this warp's pages ----
   bool dead = false;
   int next_issue = n_first;
   for (int i = 0; i < n_my; ++i) {
     const int p = p_begin + warp + i * kWarps;
-    const int32_t pid = bt[p];
-    const bool valid = pid >= 0 && static_cast<uint64_t>(pid) < a.pages_per_unit;
+    const bool valid = (__shfl_sync(0xffffffffu, vmask, 0) >> (i % a.n_stage)) & 1u;
     if (!mbar_wait_bounded_warp(&bars[warp * 8 + (i % a.n_stage)], (i / a.n_stage) & 1)) {
       if (lane == 0 && a.status) atomicOr(a.status, KVTC_STATUS_TIMEOUT);
       dead = true;
@@ -567,17 +624,16 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
       w.pk = reinterpret_cast<const uint32_t*>(st);
       w.pv = reinterpret_cast<const uint32_t*>(st + bytesK);
       w.tok0 = p * kPage;
-      if (w.tok0 + kPage <= w.seq_len)
-        do_page<BK, BV, PACK, NT, true>(w);
-      else
-        do_page<BK, BV, PACK, NT, false>(w);
+      w.partial = w.tok0 + kPage > w.seq_len;
+      do_page<BK, BV, PACK>(w);
     } else if (lane == 0 && a.status) {
       atomicOr(a.status, KVTC_STATUS_BAD_PAGE);
     }
     // release the stage: every lane is done reading it, then refill it
     __syncwarp();
     if (next_issue < n_my && next_issue == i + a.n_stage) {
-      if (lane == 0) issue(next_issue);
+      const int npid = pid_of(next_issue);
+      if (lane == 0) issue(next_issue, npid);
       ++next_issue;
     }
     __syncwarp();
@@ -593,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
       float v = 0.0f;
       const float lo_row = w.ones_lr < 8 ? 1.0f : 0.0f, hi_row = 1.0f - lo_row;
 #pragma unroll
-      for (int mt = 0; mt < NT; ++mt) {
+      for (int mt = 0; mt < kNT; ++mt) {
         const float on = mt == w.ones_mt ? 1.0f : 0.0f;
         v = fmaf(on * lo_row, w.z[mt][c], fmaf(on * hi_row, w.z[mt][2 + c], v));
       }
@@ -625,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
         dst[1] = dead ? 0.0f : l_out[c];
       }
 #pragma unroll
-      for (int mt = 0; mt < NT; ++mt) {
+      for (int mt = 0; mt < kNT; ++mt) {
         if (mt < w.nmt) {
           const int j0 = 16 * mt + g, j1 = j0 + 8;
           if (j0 < rV) dst[4 + j0] = dead ? 0.0f : w.z[mt][c];
@@ -664,9 +720,9 @@ __global__ void __launch_bounds__(kThreads, NT == 4 ? 3 : 2) decode_split_kernel
 }
 
 using SplitFn = void (*)(const DecodeArgs);
-// Kernel for (code width variants, packed, rank class); widths: 2, 4, 8 or 0 (any).
+// Kernel for (code width variants, packed); widths: 2, 4, 8 or 0 (any).
 template <int BK>
-SplitFn split_fn_bk(int bV, bool pack, bool small);
+SplitFn split_fn_bk(int bV, bool pack);
 
 }  // namespace dec
 }  // namespace kvtc

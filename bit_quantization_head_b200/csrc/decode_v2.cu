@@ -4,24 +4,16 @@
 namespace kvtc {
 namespace dec {
 template <>
-SplitFn split_fn_bk<2>(int bV, bool pack, bool small) {
-    if (bV == 2 && pack == true && small == true) return decode_split_kernel<2, 2, true, 4>;
-    if (bV == 2 && pack == true && small == false) return decode_split_kernel<2, 2, true, 8>;
-    if (bV == 2 && pack == false && small == true) return decode_split_kernel<2, 2, false, 4>;
-    if (bV == 2 && pack == false && small == false) return decode_split_kernel<2, 2, false, 8>;
-    if (bV == 4 && pack == true && small == true) return decode_split_kernel<2, 4, true, 4>;
-    if (bV == 4 && pack == true && small == false) return decode_split_kernel<2, 4, true, 8>;
-    if (bV == 4 && pack == false && small == true) return decode_split_kernel<2, 4, false, 4>;
-    if (bV == 4 && pack == false && small == false) return decode_split_kernel<2, 4, false, 8>;
-    if (bV == 8 && pack == true && small == true) return decode_split_kernel<2, 8, true, 4>;
-    if (bV == 8 && pack == true && small == false) return decode_split_kernel<2, 8, true, 8>;
-    if (bV == 8 && pack == false && small == true) return decode_split_kernel<2, 8, false, 4>;
-    if (bV == 8 && pack == false && small == false) return decode_split_kernel<2, 8, false, 8>;
-    if (bV == 0 && pack == true && small == true) return decode_split_kernel<2, 0, true, 4>;
-    if (bV == 0 && pack == true && small == false) return decode_split_kernel<2, 0, true, 8>;
-    if (bV == 0 && pack == false && small == true) return decode_split_kernel<2, 0, false, 4>;
-    if (bV == 0 && pack == false && small == false) return decode_split_kernel<2, 0, false, 8>;
-    return nullptr;
+SplitFn split_fn_bk<2>(int bV, bool pack) {
+  if (bV == 2 && pack == true) return decode_split_kernel<2, 2, true>;
+  if (bV == 2 && pack == false) return decode_split_kernel<2, 2, false>;
+  if (bV == 4 && pack == true) return decode_split_kernel<2, 4, true>;
+  if (bV == 4 && pack == false) return decode_split_kernel<2, 4, false>;
+  if (bV == 8 && pack == true) return decode_split_kernel<2, 8, true>;
+  if (bV == 8 && pack == false) return decode_split_kernel<2, 8, false>;
+  if (bV == 0 && pack == true) return decode_split_kernel<2, 0, true>;
+  if (bV == 0 && pack == false) return decode_split_kernel<2, 0, false>;
+  return nullptr;
 }
 }  // namespace dec
 }  // namespace kvtc

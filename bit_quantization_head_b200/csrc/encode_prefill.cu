@@ -50,7 +50,7 @@ constexpr uint32_t kHalfBytes = 128 * 128;     // one 64-column half of a 128-ro
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;  // 128 rows x 128 bf16
 constexpr int kQueueCap = 2048;
 constexpr int kTmemCols = 512;                  // two stages x (D_K, D_V) x 128 columns
-constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint32_t kWaitLimit = 1u << 16;      // sleeps of up to 20 us per wait
 
 struct PrefillArgs {
   const UnitDesc* units;
@@ -118,9 +118,10 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
 // Bounded wait on an mbarrier phase.  Returns false after the limit, or at once when the
 // CTA has given up (dead), so that no role can wait forever on another.
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t phase, volatile int* dead) {
+  if (mbar_try_wait(bar, phase)) return true;
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if (mbar_try_wait(bar, phase)) return true;
-    if ((i & 255) == 255 && *dead) return false;
+    if (mbar_try_wait_sleep(bar, phase, 20000u)) return true;  // sleeps up to 20 us
+    if (*dead) return false;
   }
   return false;
 }

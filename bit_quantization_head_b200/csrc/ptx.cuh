@@ -43,11 +43,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
       : "memory");
   return ok != 0;
 }
+// try_wait with a suspend-time hint: the thread sleeps until the phase completes or
+// about ns nanoseconds pass, instead of returning at once (so waiting warps leave their
+// issue slots to the others).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t phase, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(phase), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait by every lane of a warp: returns false (the same value in every lane)
-// if the phase did not complete within the limit on some lane.
+// if the phase did not complete within the limit on some lane (at most 2^16 sleeps of
+// up to 20 us each).
 __device__ __forceinline__ bool mbar_wait_bounded_warp(uint64_t* bar, uint32_t phase) {
-  bool ok = false;
-  for (uint32_t i = 0; i < (1u << 20) && !ok; ++i) ok = mbar_try_wait(bar, phase);
+  bool ok = mbar_try_wait(bar, phase);
+  for (uint32_t i = 0; i < (1u << 16) && !ok; ++i) ok = mbar_try_wait_sleep(bar, phase, 20000u);
   return __all_sync(0xffffffffu, ok);
 }
 
