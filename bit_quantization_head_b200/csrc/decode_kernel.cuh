@@ -174,6 +174,10 @@ struct WS {
   uint32_t bl[PACK ? 1 : kNT][2];
   float alpha[2], beta[2], m_run[2];
   float al[2][n_e<BK == 0 ? 8 : BK>()], nb[2][n_e<BV == 0 ? 8 : BV>()];
+  // PACK: after the hi/lo exchange a lane keeps one token row (lo: row g + 8, else g);
+  // its constants by block parity p
+  bool lo;
+  float alL[2][2], nbL[2][2], limL[2], offL[2], uL[2];
   float z[kNT][4];
   float lcvt[2];  // l accumulated from the fp16 P when there is no ones row
 };
@@ -196,6 +200,21 @@ __device__ __forceinline__ void refresh_constants(WS<BK, BV, PACK>& w) {
     for (int i = 0; i < NEV; ++i) {
       const int e = BV == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (BV == 4 ? 4 * i : 0);
       w.nb[c][i] = base - static_cast<float>(e);
+    }
+    if constexpr (PACK) {
+      // the lane's row eta = lo: e_K(p, eta), e_V(p, eta) for block parity p
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const float ek = BK == 2 ? 4.0f * p + (w.lo ? 2.0f : 0.0f) : (BK == 4 ? (w.lo ? 4.0f : 0.0f) : 0.0f);
+        const float ev = BV == 2 ? 4.0f * p + (w.lo ? 2.0f : 0.0f) : (BV == 4 ? (w.lo ? 4.0f : 0.0f) : 0.0f);
+        w.alL[c][p] = w.alpha[c] * exp2f(-ek);
+        w.nbL[c][p] = base - ev;
+        if (c == 0) {
+          w.limL[p] = kLazy + 7.0f - ev;
+          w.offL[p] = 7.0f - ev;
+          w.uL[p] = exp2f(ev - 7.0f);
+        }
+      }
     }
   }
 }
@@ -230,15 +249,25 @@ __device__ __forceinline__ void k_block(const WS<BK, BV, PACK>& w, int ks, uint3
 template <int BK, int BV, bool PACK, int BLK>
 __device__ __forceinline__ bool x_block(const WS<BK, BV, PACK>& w, const float (&sc)[4], const float (&sd)[4],
                                         float (&x)[4]) {
+  if constexpr (PACK) {
+    // hi lanes (t' < 2) keep row g and receive its lo part; lo lanes keep row g + 8 and
+    // receive its hi part: each (row, head) score is formed once
+    constexpr int p = BLK & 1;
+    const float k0 = w.lo ? sc[2] : sc[0], k1 = w.lo ? sc[3] : sc[1];
+    const float s0 = w.lo ? sc[0] : sc[2], s1 = w.lo ? sc[1] : sc[3];
+    const float f0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 2);
+    const float f1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 2);
+    x[0] = fmaf(w.alL[0][p], f0, w.nbL[0][p]);
+    x[1] = fmaf(w.alL[1][p], f1, w.nbL[1][p]);
+    if (w.partial) {  // warp-uniform: only the last page of a sequence
+      const int t = w.tok0 + 16 * BLK + w.g + (w.lo ? 8 : 0);
+      if (t >= w.seq_len) x[0] = x[1] = -INFINITY;
+    }
+    return fmaxf(x[0], x[1]) > w.limL[p];
+  }
   float full[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if constexpr (PACK) {
-      full[i] = sc[i] + __shfl_xor_sync(0xffffffffu, sc[i], 2);  // hi (t' < 2) + lo (t' >= 2)
-    } else {
-      full[i] = sc[i] + sd[i];
-    }
-  }
+  for (int i = 0; i < 4; ++i) full[i] = sc[i] + sd[i];
   // rows: full[0..1] token tok0 + 16*BLK + g (eta 0), full[2..3] that + 8 (eta 1)
   constexpr int ik0 = e_idx<BK == 0 ? 8 : BK>(BLK, 0), ik1 = e_idx<BK == 0 ? 8 : BK>(BLK, 1);
   constexpr int iv0 = e_idx<BV == 0 ? 8 : BV>(BLK, 0), iv1 = e_idx<BV == 0 ? 8 : BV>(BLK, 1);
@@ -257,8 +286,9 @@ __device__ __forceinline__ bool x_block(const WS<BK, BV, PACK>& w, const float (
 }
 
 // Block maximum of s - m_run for head column c of one block (x with the e_V offset removed).
-template <int BV, int BLK>
-__device__ __forceinline__ float xmax_block(const float (&x)[4], int c) {
+template <int BK, int BV, bool PACK, int BLK>
+__device__ __forceinline__ float xmax_block(const WS<BK, BV, PACK>& w, const float (&x)[4], int c) {
+  if constexpr (PACK) return x[c] - w.offL[BLK & 1];
   constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
   return fmaxf(x[c] - (7.0f - ev0), x[2 + c] - (7.0f - ev1));
 }
@@ -267,6 +297,20 @@ __device__ __forceinline__ float xmax_block(const float (&x)[4], int c) {
 // B fragment of the value MMA; l from the rounded P when there is no ones row.
 template <int BK, int BV, bool PACK, int BLK>
 __device__ __forceinline__ void p_block(WS<BK, BV, PACK>& w, const float (&x)[4], uint32_t (&bp)[2]) {
+  if constexpr (PACK) {
+    // this lane's row, its two heads; hi lanes also take row g + 8 from their lo partner,
+    // lo lanes (columns 4..7 of the value MMA's B) carry zeros
+    const uint32_t Pm = pack_half2(ex2(x[0]), ex2(x[1]));
+    const uint32_t Po = __shfl_xor_sync(0xffffffffu, Pm, 2);
+    if (w.ones_mt < 0) {
+      const float2 f = half2_to_float2(Pm);
+      w.lcvt[0] = fmaf(f.x, w.uL[BLK & 1], w.lcvt[0]);
+      w.lcvt[1] = fmaf(f.y, w.uL[BLK & 1], w.lcvt[1]);
+    }
+    bp[0] = movmatrix_trans(w.lo ? 0u : Pm);
+    bp[1] = movmatrix_trans(w.lo ? 0u : Po);
+    return;
+  }
   const uint32_t P0 = pack_half2(ex2(x[0]), ex2(x[1]));
   const uint32_t P1 = pack_half2(ex2(x[2]), ex2(x[3]));
   if (w.ones_mt < 0) {
@@ -359,7 +403,8 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       float v = -INFINITY;
-      ((v = fmaxf(v, xmax_block<BV, B0 + BB>(x[BB], c))), ...);
+      ((v = fmaxf(v, xmax_block<BK, BV, PACK, B0 + BB>(w, x[BB], c))), ...);
+      if constexpr (PACK) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));  // the other row
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
@@ -559,6 +604,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   w.tq = tq;
   w.seq_len = seq_len;
   w.partial = false;
+  w.lo = PACK && tq >= 2;
   w.partsK = parts_of(dK.b);
   w.partsV = parts_of(dV.b);
   w.ones_mt = (rV & 15) ? (rV >> 4) : -1;
@@ -658,6 +704,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       l_out[c] = ldexpf(__shfl_sync(0xffffffffu, v, src), 17);
     } else {
       float l = w.lcvt[c];
+      if constexpr (PACK) l += __shfl_xor_sync(0xffffffffu, l, 2);  // rows g and g + 8
       l += __shfl_xor_sync(0xffffffffu, l, 4);
       l += __shfl_xor_sync(0xffffffffu, l, 8);
       l += __shfl_xor_sync(0xffffffffu, l, 16);
