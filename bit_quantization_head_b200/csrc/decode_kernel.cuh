@@ -26,6 +26,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
 #include <utility>
 
 #include "kvtc_internal.h"
@@ -86,6 +87,13 @@ __host__ __device__ constexpr int n_e() {
 template <int B>
 __host__ __device__ constexpr int e_idx(int blk, int eta) {
   return B == 2 ? 2 * (blk & 1) + eta : (B == 4 ? eta : 0);
+}
+
+// W >> 8 as mul.hi (the FMA pipe), leaving the ALU pipe to the field extraction.
+__device__ __forceinline__ uint32_t shr8(uint32_t w) {
+  uint32_t r;
+  asm("mul.hi.u32 %0, %1, 16777216;\n" : "=r"(r) : "r"(w));
+  return r;
 }
 
 // A-fragment pair of block BLK (eta = 0: the lane's first row, 1: its second) from word
@@ -264,25 +272,26 @@ __device__ __forceinline__ bool x_block(const WS<BK, BV, PACK>& w, const float (
       if (t >= w.seq_len) x[0] = x[1] = -INFINITY;
     }
     return fmaxf(x[0], x[1]) > w.limL[p];
-  }
-  float full[4];
+  } else {
+    float full[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) full[i] = sc[i] + sd[i];
-  // rows: full[0..1] token tok0 + 16*BLK + g (eta 0), full[2..3] that + 8 (eta 1)
-  constexpr int ik0 = e_idx<BK == 0 ? 8 : BK>(BLK, 0), ik1 = e_idx<BK == 0 ? 8 : BK>(BLK, 1);
-  constexpr int iv0 = e_idx<BV == 0 ? 8 : BV>(BLK, 0), iv1 = e_idx<BV == 0 ? 8 : BV>(BLK, 1);
-  constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
-  x[0] = fmaf(w.al[0][ik0], full[0], w.nb[0][iv0]);
-  x[1] = fmaf(w.al[1][ik0], full[1], w.nb[1][iv0]);
-  x[2] = fmaf(w.al[0][ik1], full[2], w.nb[0][iv1]);
-  x[3] = fmaf(w.al[1][ik1], full[3], w.nb[1][iv1]);
-  if (w.partial) {  // warp-uniform: only the last page of a sequence
-    const int t0 = w.tok0 + 16 * BLK + w.g, t1 = t0 + 8;
-    if (t0 >= w.seq_len) x[0] = x[1] = -INFINITY;
-    if (t1 >= w.seq_len) x[2] = x[3] = -INFINITY;
+    for (int i = 0; i < 4; ++i) full[i] = sc[i] + sd[i];
+    // rows: full[0..1] token tok0 + 16*BLK + g (eta 0), full[2..3] that + 8 (eta 1)
+    constexpr int ik0 = e_idx<BK == 0 ? 8 : BK>(BLK, 0), ik1 = e_idx<BK == 0 ? 8 : BK>(BLK, 1);
+    constexpr int iv0 = e_idx<BV == 0 ? 8 : BV>(BLK, 0), iv1 = e_idx<BV == 0 ? 8 : BV>(BLK, 1);
+    constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
+    x[0] = fmaf(w.al[0][ik0], full[0], w.nb[0][iv0]);
+    x[1] = fmaf(w.al[1][ik0], full[1], w.nb[1][iv0]);
+    x[2] = fmaf(w.al[0][ik1], full[2], w.nb[0][iv1]);
+    x[3] = fmaf(w.al[1][ik1], full[3], w.nb[1][iv1]);
+    if (w.partial) {  // warp-uniform: only the last page of a sequence
+      const int t0 = w.tok0 + 16 * BLK + w.g, t1 = t0 + 8;
+      if (t0 >= w.seq_len) x[0] = x[1] = -INFINITY;
+      if (t1 >= w.seq_len) x[2] = x[3] = -INFINITY;
+    }
+    constexpr float lim0 = kLazy + 7.0f - ev0, lim1 = kLazy + 7.0f - ev1;
+    return fmaxf(x[0], x[1]) > lim0 || fmaxf(x[2], x[3]) > lim1;
   }
-  constexpr float lim0 = kLazy + 7.0f - ev0, lim1 = kLazy + 7.0f - ev1;
-  return fmaxf(x[0], x[1]) > lim0 || fmaxf(x[2], x[3]) > lim1;
 }
 
 // Block maximum of s - m_run for head column c of one block (x with the e_V offset removed).
@@ -366,32 +375,41 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
   for (int bb = 0; bb < IL; ++bb)
 #pragma unroll
     for (int i = 0; i < 4; ++i) sc[bb][i] = sd[bb][i] = 0.0f;
-  // ---- scores S[tok][head] = sum_j codeK[tok][j] * q^[head][j]
+  // ---- scores S[tok][head] = sum_j codeK[tok][j] * q^[head][j]; the k-steps run from
+  // a jump into the unrolled sequence (no per-step test)
+  auto kstep = [&](auto KSC) {
+    constexpr int ks = decltype(KSC)::value;
+    // rows past r_K meet zero q^ coefficients (q~ is zero there), so they are read
+    // unmasked; the shared-memory allocation has slack for the over-read
+    const int r0 = 8 * ks + w.tq, r1 = r0 + 4;
+    constexpr int KB = BK == 0 ? 1 : BK;
+    constexpr int KW0 = (B0 * KB) / 8, KWN = ((B0 + IL - 1) * KB) / 8 - KW0 + 1;
+    uint32_t W0[KWN], W1[KWN], W0h[KWN], W1h[KWN];
 #pragma unroll
-  for (int ks = 0; ks < kNT; ++ks) {
-    if (ks < w.nks) {
-      // rows past r_K meet zero q^ coefficients (q~ is zero there), so they are read
-      // unmasked; the shared-memory allocation has slack for the over-read
-      const int r0 = 8 * ks + w.tq, r1 = r0 + 4;
-      constexpr int KB = BK == 0 ? 1 : BK;
-      constexpr int KW0 = (B0 * KB) / 8, KWN = ((B0 + IL - 1) * KB) / 8 - KW0 + 1;
-      uint32_t W0[KWN], W1[KWN], W0h[KWN], W1h[KWN];
-#pragma unroll
-      for (int q = 0; q < KWN; ++q) {
-        if constexpr (BK != 0) {
-          W0[q] = w.pk[r0 * 8 * BK + w.g * BK + KW0 + q];
-          W1[q] = w.pk[r1 * 8 * BK + w.g * BK + KW0 + q];
-        } else {
-          W0[q] = W1[q] = 0u;
-        }
-        W0h[q] = W0[q] >> 8;
-        W1h[q] = W1[q] >> 8;
+    for (int q = 0; q < KWN; ++q) {
+      if constexpr (BK != 0) {
+        W0[q] = w.pk[r0 * 8 * BK + w.g * BK + KW0 + q];
+        W1[q] = w.pk[r1 * 8 * BK + w.g * BK + KW0 + q];
+      } else {
+        W0[q] = W1[q] = 0u;
       }
-      (k_block<BK, BV, PACK, B0 + BB>(w, ks, W0[((B0 + BB) * KB) / 8 - KW0], W0h[((B0 + BB) * KB) / 8 - KW0],
-                                      W1[((B0 + BB) * KB) / 8 - KW0], W1h[((B0 + BB) * KB) / 8 - KW0], r0, r1,
-                                      sc[BB], sd[BB]),
-       ...);
+      W0h[q] = shr8(W0[q]);
+      W1h[q] = shr8(W1[q]);
     }
+    (k_block<BK, BV, PACK, B0 + BB>(w, ks, W0[((B0 + BB) * KB) / 8 - KW0], W0h[((B0 + BB) * KB) / 8 - KW0],
+                                    W1[((B0 + BB) * KB) / 8 - KW0], W1h[((B0 + BB) * KB) / 8 - KW0], r0, r1,
+                                    sc[BB], sd[BB]),
+     ...);
+  };
+  switch (w.nks) {
+    default: kstep(std::integral_constant<int, 7>{}); [[fallthrough]];
+    case 7: kstep(std::integral_constant<int, 6>{}); [[fallthrough]];
+    case 6: kstep(std::integral_constant<int, 5>{}); [[fallthrough]];
+    case 5: kstep(std::integral_constant<int, 4>{}); [[fallthrough]];
+    case 4: kstep(std::integral_constant<int, 3>{}); [[fallthrough]];
+    case 3: kstep(std::integral_constant<int, 2>{}); [[fallthrough]];
+    case 2: kstep(std::integral_constant<int, 1>{}); [[fallthrough]];
+    case 1: kstep(std::integral_constant<int, 0>{});
   }
   float x[IL][4];
   bool grow = false;
@@ -438,31 +456,40 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
   // ---- probabilities -> B fragments
   uint32_t bp[IL][2];
   (p_block<BK, BV, PACK, B0 + BB>(w, x[BB], bp[BB]), ...);
-  // ---- values: Z^T[j][head] += sum_tok codeV[tok][j] * P[tok][head]
+  // ---- values: Z^T[j][head] += sum_tok codeV[tok][j] * P[tok][head] (m-tiles likewise
+  // entered by a jump)
+  auto vtile = [&](auto MTC) {
+    constexpr int mt = decltype(MTC)::value;
+    const int j0 = 16 * mt + w.g, j1 = j0 + 8;
+    const bool ones = mt == w.ones_mt;
+    constexpr int VB = BV == 0 ? 1 : BV;
+    constexpr int VW0 = (B0 * VB) / 8, VWN = ((B0 + IL - 1) * VB) / 8 - VW0 + 1;
+    uint32_t W0[VWN], W1[VWN], W0h[VWN], W1h[VWN];
 #pragma unroll
-  for (int mt = 0; mt < kNT; ++mt) {
-    if (mt < w.nmt) {
-      const int j0 = 16 * mt + w.g, j1 = j0 + 8;
-      const bool ones = mt == w.ones_mt;
-      constexpr int VB = BV == 0 ? 1 : BV;
-      constexpr int VW0 = (B0 * VB) / 8, VWN = ((B0 + IL - 1) * VB) / 8 - VW0 + 1;
-      uint32_t W0[VWN], W1[VWN], W0h[VWN], W1h[VWN];
-#pragma unroll
-      for (int q = 0; q < VWN; ++q) {
-        if constexpr (BV != 0) {
-          W0[q] = w.pv[j0 * 4 * BV + w.tq * BV + VW0 + q];
-          W1[q] = w.pv[j1 * 4 * BV + w.tq * BV + VW0 + q];
-        } else {
-          W0[q] = W1[q] = 0u;
-        }
-        W0h[q] = W0[q] >> 8;
-        W1h[q] = W1[q] >> 8;
+    for (int q = 0; q < VWN; ++q) {
+      if constexpr (BV != 0) {
+        W0[q] = w.pv[j0 * 4 * BV + w.tq * BV + VW0 + q];
+        W1[q] = w.pv[j1 * 4 * BV + w.tq * BV + VW0 + q];
+      } else {
+        W0[q] = W1[q] = 0u;
       }
-      (v_block<BK, BV, PACK, B0 + BB>(w, W0[((B0 + BB) * VB) / 8 - VW0], W0h[((B0 + BB) * VB) / 8 - VW0],
-                                      W1[((B0 + BB) * VB) / 8 - VW0], W1h[((B0 + BB) * VB) / 8 - VW0], j0, j1,
-                                      ones, bp[BB], w.z[mt]),
-       ...);
+      W0h[q] = shr8(W0[q]);
+      W1h[q] = shr8(W1[q]);
     }
+    (v_block<BK, BV, PACK, B0 + BB>(w, W0[((B0 + BB) * VB) / 8 - VW0], W0h[((B0 + BB) * VB) / 8 - VW0],
+                                    W1[((B0 + BB) * VB) / 8 - VW0], W1h[((B0 + BB) * VB) / 8 - VW0], j0, j1, ones,
+                                    bp[BB], w.z[mt]),
+     ...);
+  };
+  switch (w.nmt) {
+    default: vtile(std::integral_constant<int, 7>{}); [[fallthrough]];
+    case 7: vtile(std::integral_constant<int, 6>{}); [[fallthrough]];
+    case 6: vtile(std::integral_constant<int, 5>{}); [[fallthrough]];
+    case 5: vtile(std::integral_constant<int, 4>{}); [[fallthrough]];
+    case 4: vtile(std::integral_constant<int, 3>{}); [[fallthrough]];
+    case 3: vtile(std::integral_constant<int, 2>{}); [[fallthrough]];
+    case 2: vtile(std::integral_constant<int, 1>{}); [[fallthrough]];
+    case 1: vtile(std::integral_constant<int, 0>{});
   }
 }
 
@@ -536,9 +563,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const uint32_t bytesK = static_cast<uint32_t>(dK.page_bytes), bytesV = static_cast<uint32_t>(dV.page_bytes);
   const char* poolK = a.pool + a.pages_per_unit * dK.prefix;
   const char* poolV = a.pool + a.pages_per_unit * dV.prefix;
-  auto stage_ptr = [&](int i) {
-    return stages + (static_cast<size_t>(warp) * a.n_stage + (i % a.n_stage)) * a.stage_bytes;
-  };
+  unsigned char* const warp_stages = stages + static_cast<size_t>(warp) * a.n_stage * a.stage_bytes;
+  auto stage_ptr = [&](int slot) { return warp_stages + static_cast<size_t>(slot) * a.stage_bytes; };
   // Page ids of this warp's pages, 32 at a time: lane l holds the id of page base + l of
   // the current window (-1 past the end), so no dependent global load is left in the loop.
   int pid_win = -1;
@@ -554,10 +580,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   };
   // Fill the stage of this warp's i-th page.  Every use of a stage completes its barrier
   // phase exactly once: with the copies' bytes, or by a plain arrival when the page id
-  // is invalid.  vmask (lane 0) has bit i % n_stage set when the stage holds a page.
+  // is invalid.  vmask (lane 0) has bit slot set when the stage holds a page.
   uint32_t vmask = 0;
-  auto issue = [&](int i, int pid) {  // lane 0
-    const int slot = i % a.n_stage;
+  auto issue = [&](int slot, int pid) {  // lane 0
     uint64_t* bar = &bars[warp * 8 + slot];
     if (pid < 0 || static_cast<uint64_t>(pid) >= a.pages_per_unit) {
       vmask &= ~(1u << slot);
@@ -565,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       return;
     }
     vmask |= 1u << slot;
-    unsigned char* st = stage_ptr(i);
+    unsigned char* st = stage_ptr(slot);
     mbar_arrive_expect_tx(bar, bytesK + bytesV);
     bulk_copy_g2s(st, poolK + static_cast<uint64_t>(pid) * bytesK, bytesK, bar);
     bulk_copy_g2s(st + bytesK, poolV + static_cast<uint64_t>(pid) * bytesV, bytesV, bar);
@@ -573,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const int n_first = min(a.n_stage, n_my);
   for (int i = 0; i < n_first; ++i) {
     const int pid = pid_of(i);
-    if (lane == 0) issue(i, pid);
+    if (lane == 0) issue(i, pid);  // page i < n_stage uses slot i
   }
 
   // per head: S = sum_j q~_j and the fp16 normalisation exponent (warp w: heads 2w, 2w+1)
@@ -655,18 +680,28 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   // ---- main loop over this warp's pages ----
   bool dead = false;
   int next_issue = n_first;
+  int slot = 0;        // stage of page i (i mod n_stage), kept incrementally
+  uint32_t phase = 0;  // barrier phase of that use of the stage ((i / n_stage) & 1)
   for (int i = 0; i < n_my; ++i) {
     const int p = p_begin + warp + i * kWarps;
-    const bool valid = (__shfl_sync(0xffffffffu, vmask, 0) >> (i % a.n_stage)) & 1u;
-    if (!mbar_wait_bounded_warp(&bars[warp * 8 + (i % a.n_stage)], (i / a.n_stage) & 1)) {
+    const bool valid = (__shfl_sync(0xffffffffu, vmask, 0) >> slot) & 1u;
+    if (!mbar_wait_bounded_warp(&bars[warp * 8 + slot], phase)) {
       if (lane == 0 && a.status) atomicOr(a.status, KVTC_STATUS_TIMEOUT);
       dead = true;
-      for (int i2 = i + 1; i2 < next_issue; ++i2)
-        (void)mbar_wait_bounded_warp(&bars[warp * 8 + (i2 % a.n_stage)], (i2 / a.n_stage) & 1);
+      // wait (bounded) for the copies still in flight before leaving
+      int s2 = slot;
+      uint32_t ph2 = phase;
+      for (int i2 = i + 1; i2 < next_issue; ++i2) {
+        if (++s2 == a.n_stage) {
+          s2 = 0;
+          ph2 ^= 1u;
+        }
+        (void)mbar_wait_bounded_warp(&bars[warp * 8 + s2], ph2);
+      }
       break;
     }
     if (valid) {
-      const unsigned char* st = stage_ptr(i);
+      const unsigned char* st = stage_ptr(slot);
       w.pk = reinterpret_cast<const uint32_t*>(st);
       w.pv = reinterpret_cast<const uint32_t*>(st + bytesK);
       w.tok0 = p * kPage;
@@ -679,10 +714,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     __syncwarp();
     if (next_issue < n_my && next_issue == i + a.n_stage) {
       const int npid = pid_of(next_issue);
-      if (lane == 0) issue(next_issue, npid);
+      if (lane == 0) issue(slot, npid);  // page i + n_stage reuses page i's stage
       ++next_issue;
     }
     __syncwarp();
+    if (++slot == a.n_stage) {
+      slot = 0;
+      phase ^= 1u;
+    }
   }
 
   // ---- l: from the ones row, or the per-lane sums ----
