@@ -28,7 +28,6 @@
 #include <cmath>
 #include <map>
 #include <mutex>
-#include <set>
 #include <utility>
 #include <vector>
 
@@ -119,10 +118,12 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(const __grid_constant_
 }
 
 // ---- kernel 2: merge the partials, centre, dequantise, back-project --------------------
-// CTA = (query head, sequence), 256 threads.  M_V (r_V rows of 512 bytes) is copied into
-// shared memory by one bulk copy issued before the wait for the split kernels, so the
-// back-projection reads it from shared memory; warps fold the partials (lane l holds
-// latent coordinates 4l..4l+3) and meet in shared memory.
+// CTA = (query head, sequence, block of 32 output columns), 128 threads.  The CTA's slice
+// M_V[:, 32c .. 32c + 31] is loaded into shared memory before the wait for the split
+// kernels; then the four warps fold the partials (lane l holds latent coordinates
+// 4l..4l+3), meet in shared memory, and back-project the slice (each warp a quarter of
+// the latent rows).  The merge is repeated by the four column blocks of a query head: it
+// reads (4 + r_V) floats per partial, from L2.
 struct CombineArgs {
   const UnitDesc* units;
   int layer, H, G;
@@ -133,26 +134,27 @@ struct CombineArgs {
   int out_bf16;
   int32_t* status;
 };
-constexpr int kCombThreads = 256;
+constexpr int kCombThreads = 128;
 constexpr int kCombWarps = kCombThreads / 32;
+constexpr int kCombCols = 32;  // output columns per CTA
 
 __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(const __grid_constant__ CombineArgs ca) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  float* Ms = reinterpret_cast<float*>(smem);  // [r_V][128]
-  __shared__ __align__(16) float zsh[kCombWarps][128];  // written as float4
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(16) float Ms[kD][kCombCols];       // M_V rows, this CTA's columns
+  __shared__ __align__(16) float zsh[kCombWarps][kD];     // written as float4
   __shared__ float lsh[kCombWarps];
   __shared__ float mxsh[kCombWarps];
-  __shared__ float y[128];
-  const int qh = blockIdx.x, s = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ float y[kD];
+  __shared__ float osh[kCombWarps][kCombCols];
+  const int qh = blockIdx.x, s = blockIdx.y, cb = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Hq = ca.H * ca.G, h = qh / ca.G;
   const UnitDesc dV = ca.units[(ca.layer * ca.H + h) * 2 + 1];
   const int rV = dV.r;
-  if (tid == 0) {
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-    mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(rV) * kD * 4u);
-    bulk_copy_g2s(Ms, dV.M, static_cast<uint32_t>(rV) * kD * 4u, &bar);
+  // the plan's M_V is not written by the preceding kernels: load it before the wait
+  for (int i = tid; i < rV * (kCombCols / 4); i += kCombThreads) {
+    const int j = i / (kCombCols / 4), c4 = i % (kCombCols / 4);
+    reinterpret_cast<float4*>(Ms[j])[c4] =
+        reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD + cb * kCombCols)[c4];
   }
   griddep_wait();
   griddep_launch_dependents();
@@ -189,44 +191,26 @@ __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(const __gr
 #pragma unroll
   for (int w = 0; w < kCombWarps; ++w) L += lsh[w];
   const float mV = 0.5f * static_cast<float>((1 << dV.b) - 1);
-  if (tid < rV) {
+  for (int j = tid; j < rV; j += kCombThreads) {
     float zs = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kCombWarps; ++w) zs += zsh[w][tid];
+    for (int w = 0; w < kCombWarps; ++w) zs += zsh[w][j];
     // z holds sum p*c*2^-17 (uncentered codes); center and dequantize
-    y[tid] = L > 0.0f ? dV.delta * (ldexpf(zs, 17) - mV * L) / L : 0.0f;
-  }
-  // M_V in shared memory (bounded wait; on a time-out the output is zero and the status
-  // word says so)
-  bool ok = false;
-  for (uint32_t it = 0; it < (1u << 16) && !ok; ++it) ok = mbar_try_wait_sleep(&bar, 0, 20000u);
-  ok = __syncthreads_and(ok);
-  if (!ok) {
-    if (tid == 0 && ca.status) atomicOr(ca.status, KVTC_STATUS_TIMEOUT);
-    bool done = false;
-    for (uint32_t it = 0; it < (1u << 16) && !done; ++it) done = mbar_try_wait_sleep(&bar, 0, 20000u);
-  }
-  // o[k] = sum_j M_V[j][k] y[j]: threads k and k + 128 take the even and odd j
-  const int k = tid & 127, par = tid >> 7;
-  float o0 = 0.0f, o1 = 0.0f;
-  if (ok) {
-    int j = par;
-    for (; j + 2 < rV; j += 4) {
-      o0 = fmaf(Ms[j * kD + k], y[j], o0);
-      o1 = fmaf(Ms[(j + 2) * kD + k], y[j + 2], o1);
-    }
-    if (j < rV) o0 = fmaf(Ms[j * kD + k], y[j], o0);
+    y[j] = L > 0.0f ? dV.delta * (ldexpf(zs, 17) - mV * L) / L : 0.0f;
   }
   __syncthreads();
-  if (par) zsh[0][k] = o0 + o1;
+  // o[k] = sum_j M_V[j][k] y[j] for this CTA's 32 columns: warp w takes j = w, w + 4, ...
+  float o = 0.0f;
+  for (int j = warp; j < rV; j += kCombWarps) o = fmaf(Ms[j][lane], y[j], o);
+  osh[warp][lane] = o;
   __syncthreads();
-  if (!par) {
-    const float o = (o0 + o1) + zsh[0][k];
-    const size_t off = (static_cast<size_t>(s) * Hq + qh) * kD + k;
+  if (warp == 0) {
+    const float v = (osh[0][lane] + osh[1][lane]) + (osh[2][lane] + osh[3][lane]);
+    const size_t off = (static_cast<size_t>(s) * Hq + qh) * kD + cb * kCombCols + lane;
     if (ca.out_bf16)
-      static_cast<__nv_bfloat16*>(ca.out)[off] = __float2bfloat16_rn(o);
+      static_cast<__nv_bfloat16*>(ca.out)[off] = __float2bfloat16_rn(v);
     else
-      static_cast<float*>(ca.out)[off] = o;
+      static_cast<float*>(ca.out)[off] = v;
   }
 }
 
@@ -454,27 +438,9 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     first = false;
   }
 
-  // ---- kernel 2: combine (M_V staged in shared memory)
+  // ---- kernel 2: combine
   {
-    int rv_max = 2;
-    for (int h = 0; h < plan->H; ++h) rv_max = std::max(rv_max, plan->r[(layer * plan->H + h) * 2 + 1]);
-    const size_t smem = static_cast<size_t>(rv_max) * kD * sizeof(float);
-    // the largest size (r_V = 128) is set once per device
-    static std::mutex mu;
-    static std::set<int> devices_set;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-    {
-      std::lock_guard<std::mutex> lock(mu);
-      if (!devices_set.count(dev)) {
-        e = cudaFuncSetAttribute(decode_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kD * kD * sizeof(float)));
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (combine)");
-        devices_set.insert(dev);
-      }
-    }
-    e = launch_pdl(decode_combine_kernel, dim3(Hq, n_seq), dim3(kCombThreads), smem, cs, ca);
+    cudaError_t e = launch_pdl(decode_combine_kernel, dim3(Hq, n_seq, kD / kCombCols), dim3(kCombThreads), 0, cs, ca);
     if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
   }
   cudaError_t e = cudaGetLastError();

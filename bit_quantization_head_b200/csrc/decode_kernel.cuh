@@ -43,7 +43,10 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kNT = 8;                // 16-row tiles of a rank (r <= 128)
 constexpr int kIL = KVTC_DECODE_IL;   // blocks processed together
-constexpr int kMinBlocks = kIL >= 4 ? 2 : (kIL == 2 ? 3 : 4);  // resident CTAs per SM aimed for
+#ifndef KVTC_DECODE_MINB
+#define KVTC_DECODE_MINB 2
+#endif
+constexpr int kMinBlocks = KVTC_DECODE_MINB;  // resident CTAs per SM aimed for (registers, stages)
 constexpr int kPartStride = 132;      // floats per partial: m, l, 2 pad, z[128]
 constexpr int kMaxHeadsPerLaunch = 64;
 constexpr float kLog2e = 1.4426950408889634f;
