@@ -130,6 +130,58 @@ std::vector<Cand> candidates(int d) {
   return c;
 }
 
+// C2 in the pages' iterative form ("C2, across heads": with C1 as the oracle, budget moves
+// between heads until their marginal distortions equalize; a damped update converges in
+// five rounds).  Step rule (the pages give none): start at equal real-valued budgets;
+// each round m_u = (D*_u(B_u - 8) - D*_u(B_u + 8)) / 16 with D*_u(B) the distortion of
+// C1's pick at floor(B) (sum w when no rank fits); B_u <- B_u (1 + (m_u - m) / (2 m)) with
+// m the mean marginal; clip to [4, 8d] and rescale the unclipped units to the total.
+// After five rounds each unit gets C1 at floor(B_u).  Only + - * / and sequential sums,
+// in the oracle's order.
+void c2_damped(const std::vector<std::vector<double>>& ws, long long total_bits, std::vector<int>& r_out,
+               std::vector<int>& b_out) {
+  const int U = static_cast<int>(ws.size());
+  const int d = static_cast<int>(ws[0].size());
+  const double lo_b = 4.0, hi_b = 8.0 * d, step = 8.0, damping = 0.5;
+  auto dstar = [&](int u, double Bv) {
+    const int Bi = static_cast<int>(std::floor(std::min(std::max(Bv, 0.0), hi_b)));
+    int r = 0, b = 0;
+    if (!c1(ws[u], Bi, r, b)) {
+      double tot = 0.0;
+      for (double x : ws[u]) tot += x;
+      return tot;
+    }
+    return distortion(ws[u], r, b);
+  };
+  std::vector<double> bud(U, static_cast<double>(total_bits) / U), m(U);
+  for (int round = 0; round < 5; ++round) {
+    for (int u = 0; u < U; ++u) m[u] = (dstar(u, bud[u] - step) - dstar(u, bud[u] + step)) / (2.0 * step);
+    double msum = 0.0;
+    for (int u = 0; u < U; ++u) msum += m[u];
+    const double mbar = msum / U;
+    if (!(mbar > 0.0)) break;
+    for (int u = 0; u < U; ++u) bud[u] = bud[u] * (1.0 + damping * (m[u] - mbar) / mbar);
+    for (int it = 0; it < 8; ++it) {
+      for (int u = 0; u < U; ++u) bud[u] = std::min(std::max(bud[u], lo_b), hi_b);
+      double fixed = 0.0, free = 0.0;
+      for (int u = 0; u < U; ++u) {
+        if (bud[u] <= lo_b || bud[u] >= hi_b)
+          fixed += bud[u];
+        else
+          free += bud[u];
+      }
+      if (free <= 0.0) break;
+      const double scale = (static_cast<double>(total_bits) - fixed) / free;
+      for (int u = 0; u < U; ++u)
+        if (!(bud[u] <= lo_b || bud[u] >= hi_b)) bud[u] = bud[u] * scale;
+    }
+  }
+  r_out.assign(U, 0);
+  b_out.assign(U, 0);
+  for (int u = 0; u < U; ++u)
+    c1(ws[u], static_cast<int>(std::floor(std::min(std::max(bud[u], lo_b), hi_b))), r_out[u], b_out[u]);
+}
+
 // C2 in Lagrangian form: bisect mu so that sum_u bits(argmin D_u + mu*bits) fits the
 // budget, spend the leftover greedily on the best distortion drop per bit, and give each
 // unit C1 at its resulting budget.
@@ -363,6 +415,8 @@ extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* 
 
   std::vector<int> R(U), B(U);
   double mu = 0.0;
+  if (desc->c2_mode != KVTC_C2_LAGRANGE && desc->c2_mode != KVTC_C2_DAMPED)
+    return fail(KVTC_EINVAL, "c2_mode must be KVTC_C2_LAGRANGE or KVTC_C2_DAMPED");
   if (fixed) {
     std::fill(R.begin(), R.end(), desc->fixed_r);
     std::fill(B.begin(), B.end(), desc->fixed_b);
@@ -371,7 +425,11 @@ extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* 
     if (4ll * U > total) return fail(KVTC_EINFEASIBLE, "budget below 4 bits per unit");
     std::vector<std::vector<double>> ws(U);
     for (int u = 0; u < U; ++u) ws[u] = work[u].w;
-    if (!c2(ws, total, R, B, mu)) return fail(KVTC_EINFEASIBLE, "no allocation meets the budget");
+    if (desc->c2_mode == KVTC_C2_DAMPED) {
+      c2_damped(ws, total, R, B);
+    } else if (!c2(ws, total, R, B, mu)) {
+      return fail(KVTC_EINFEASIBLE, "no allocation meets the budget");
+    }
   }
 
   std::unique_ptr<kvtc_plan> p(new (std::nothrow) kvtc_plan());

@@ -55,6 +55,10 @@ typedef enum {
 typedef enum { KVTC_F32 = 0, KVTC_BF16 = 1 } kvtc_dtype;
 typedef enum { KVTC_KIND_K = 0, KVTC_KIND_V = 1 } kvtc_kind;
 typedef enum { KVTC_WEIGHTS_KL = 0, KVTC_WEIGHTS_MSE = 1 } kvtc_weight_mode;
+/* C2 solver: the Lagrangian water-filling (exact on the convex hull), or the pages'
+ * iterative form (budget moved toward the larger marginal distortion, damped, five
+ * rounds; "C2, across heads"). */
+typedef enum { KVTC_C2_LAGRANGE = 0, KVTC_C2_DAMPED = 1 } kvtc_c2_mode;
 
 /* Bits of the device status word. */
 #define KVTC_STATUS_BAD_PAGE 1u      /* block table entry outside [0, pages_per_unit)  */
@@ -82,6 +86,7 @@ typedef struct {
   int fixed_r;         /* fixed_r > 0 and fixed_b > 0: every unit gets (fixed_r,       */
   int fixed_b;         /*   fixed_b) and no allocation runs                           */
   uint64_t seed;       /* seed of the random Hadamard signs (splitmix64)              */
+  int c2_mode;         /* KVTC_C2_LAGRANGE (default) or KVTC_C2_DAMPED                */
 } kvtc_calib_desc;
 
 /*

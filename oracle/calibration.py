@@ -216,6 +216,68 @@ def c2(weights, total_bits, iters=200):
     return out, hi
 
 
+def c2_damped(weights, total_bits, rounds=5, step=8, damping=0.5):
+    """C2, across heads, in the pages' iterative form ("C2, across heads": with C1 as the
+    oracle, budget moves between heads until their marginal distortions equalize; a
+    damped update converges in five rounds).  The pages give no step rule; the one
+    taken here:
+      * every unit starts at B_u = total_bits / U (real-valued budgets);
+      * a round measures each unit's marginal distortion with C1 as the oracle,
+        m_u = (D*_u(B_u - step) - D*_u(B_u + step)) / (2 step), where D*_u(B) is the
+        distortion of C1's pick at floor(B) (all-truncated sum(w) when no rank fits);
+      * and moves budget toward the units above the mean marginal m = mean_u m_u:
+        B_u <- B_u * (1 + damping * (m_u - m) / m), then clips to [4, 8 d] and rescales
+        the unclipped units so that the budgets add up to total_bits again;
+      * after ``rounds`` rounds each unit gets C1 at floor(B_u).
+    Only +, -, *, / and sequential sums are used, so a C++ restatement reproduces the
+    budgets bit for bit.  Returns the list of (r, b).  Raises ValueError if even 4 bits
+    per unit exceed the budget.
+    Pinned: identical units stay at equal budgets; the result fits the budget; its total
+    D lies between the Lagrangian optimum and the equal-budget start.
+    """
+    U = len(weights)
+    if 4 * U > total_bits:
+        raise ValueError("budget below 4 bits per unit")
+    d = len(weights[0])
+    lo_b, hi_b = 4.0, float(8 * d)
+
+    def dstar(u, B):
+        w = weights[u]
+        Bi = int(np.floor(min(max(B, 0.0), hi_b)))
+        rb = c1(w, Bi, d)
+        if rb is None:
+            tot = 0.0
+            for x in w:
+                tot += float(x)
+            return tot
+        return distortion(w, rb[0], rb[1])
+
+    budgets = [float(total_bits) / U] * U
+    for _ in range(rounds):
+        m = [(dstar(u, budgets[u] - step) - dstar(u, budgets[u] + step)) / (2.0 * step) for u in range(U)]
+        msum = 0.0
+        for x in m:
+            msum += x
+        mbar = msum / U
+        if not mbar > 0.0:
+            break
+        budgets = [budgets[u] * (1.0 + damping * (m[u] - mbar) / mbar) for u in range(U)]
+        for _ in range(8):  # clip, then rescale the free units to the total
+            budgets = [min(max(x, lo_b), hi_b) for x in budgets]
+            fixed = 0.0
+            free = 0.0
+            for x in budgets:
+                if x <= lo_b or x >= hi_b:
+                    fixed += x
+                else:
+                    free += x
+            if free <= 0.0:
+                break
+            scale = (float(total_bits) - fixed) / free
+            budgets = [x if (x <= lo_b or x >= hi_b) else x * scale for x in budgets]
+    return [c1(weights[u], int(np.floor(min(max(budgets[u], lo_b), hi_b))), d) for u in range(U)]
+
+
 # ---------------------------------------------------------------- Hadamard + signs
 _GAMMA = 0x9E3779B97F4A7C15
 _MASK64 = (1 << 64) - 1
@@ -339,7 +401,7 @@ def gaussian_step(b, lo=1e-3, hi=4.0, iters=200):
 
 # ---------------------------------------------------------------- whole calibration
 def calibrate(k_cal, v_cal, q_cal, n_layers, n_kv_heads, bpd, seed, *,
-              weight_mode="kl", fixed_r=0, fixed_b=0, c2_iters=200):
+              weight_mode="kl", fixed_r=0, fixed_b=0, c2_iters=200, c2_mode="lagrange"):
     """Calibrate every unit (layer, KV head, K|V) and allocate (r, b).
 
     k_cal, v_cal: [L, H_kv, N, d]; q_cal: [L, H_kv, G, N, d] (float arrays).
@@ -367,7 +429,10 @@ def calibrate(k_cal, v_cal, q_cal, n_layers, n_kv_heads, bpd, seed, *,
         mu = None
     else:
         total = int(round(bpd * d * len(units)))
-        rb, mu = c2([u["w"] for u in units], total, iters=c2_iters)
+        if c2_mode == "damped":
+            rb, mu = c2_damped([u["w"] for u in units], total), 0.0
+        else:
+            rb, mu = c2([u["w"] for u in units], total, iters=c2_iters)
     steps = {b: gaussian_step(b) for b in range(B_MIN, B_MAX + 1)}
     for idx, (u, (r, b)) in enumerate(zip(units, rb)):
         signs = hadamard_signs(seed, idx, r)

@@ -67,6 +67,25 @@ def test_calibrate_matches_oracle_multilayer_1bpd(mode):
     _compare_plans(plan, units)
 
 
+def test_calibrate_damped_c2_matches_oracle_and_sits_between_bounds():
+    # the pages' iterative C2 ("C2, across heads": damped update, five rounds) against
+    # the oracle's restatement, on the two-layer 1-bpd pool
+    w = synth.scaled(synth.WORKLOADS["llama8b-32L-128k-1bpd"], n_layers=2, n_cal=256)
+    k, v, q = synth.calibration_set(w)
+    plan = kvtc.kvtc_calibrate(k, v, q, n_layers=2, n_kv_heads=8, group=4, bpd=1.0, seed=w.seed,
+                               c2_mode=kvtc.C2_DAMPED)
+    units = ocal.calibrate(k, v, q, 2, 8, bpd=1.0, seed=w.seed, c2_mode="damped")
+    _compare_plans(plan, units)
+    lag = ocal.calibrate(k, v, q, 2, 8, bpd=1.0, seed=w.seed)
+    total = 1.0 * 128 * 32
+    assert sum(u["r"] * u["b"] for u in units) <= total
+    D_damped = sum(u["D"] for u in units)
+    D_lagrange = sum(u["D"] for u in lag)
+    per_unit = int(total) // 32
+    D_equal = sum(ocal.distortion(u["w"], *ocal.c1(u["w"], per_unit)) for u in lag)
+    assert D_lagrange <= D_damped <= D_equal
+
+
 def test_plan_save_load_round_trip(tmp_path):
     w = synth.WORKLOADS["head1-fp32-1k"]
     k, v, q = synth.calibration_set(w)

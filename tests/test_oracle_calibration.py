@@ -304,3 +304,32 @@ def test_calibrate_small_model_meets_budget_and_is_deterministic():
     for a, b in zip(units, again):
         assert (a["r"], a["b"]) == (b["r"], b["b"])
         assert np.array_equal(a["M"], b["M"])
+
+
+# ---------------------------------------------------------------- C2, damped form
+def test_c2_damped_keeps_identical_units_at_equal_budgets():
+    w = np.sort(np.random.default_rng(3).exponential(1.0, 128))[::-1]
+    picks = cal.c2_damped([w] * 6, 6 * 96)
+    assert len(set(picks)) == 1 and picks[0][0] * picks[0][1] <= 96
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_c2_damped_fits_the_budget_and_lies_between_optimum_and_equal_split(seed):
+    rng = np.random.default_rng(seed)
+    ws = [np.sort(rng.exponential(1.0, 128) * np.arange(1, 129) ** -rng.uniform(0.5, 2.0))[::-1]
+          for _ in range(12)]
+    total = 12 * 128
+    picks = cal.c2_damped(ws, total)
+    assert sum(r * b for r, b in picks) <= total
+    D = sum(cal.distortion(w, r, b) for w, (r, b) in zip(ws, picks))
+    lag, _ = cal.c2(ws, total)
+    D_opt = sum(cal.distortion(w, r, b) for w, (r, b) in zip(ws, lag))
+    D_eq = sum(cal.distortion(w, *cal.c1(w, total // 12)) for w in ws)
+    assert D_opt <= D <= D_eq
+
+
+def test_c2_damped_moves_budget_toward_the_larger_marginal():
+    # two units, one with ten times the weight: it must end with more bits
+    w = np.sort(np.random.default_rng(4).exponential(1.0, 128))[::-1]
+    picks = cal.c2_damped([w, 10.0 * w], 2 * 128)
+    assert picks[1][0] * picks[1][1] > picks[0][0] * picks[0][1]
