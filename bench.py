@@ -202,11 +202,17 @@ def decode_step(st, w, events=None, stream=None):
 
 
 def kernels_per_step(plan, w):
+    """Launches of the library's kernels per step: per layer the append, the q~ prep, one
+    split kernel per code-width class pair of the layer's KV heads (2, 4 and 8 have their
+    own kernels, other widths share one) and the combine."""
+    def cls(b):
+        return b if b in (2, 4, 8) else 0
     n = 0
     H = plan.shape["n_kv_heads"]
     for layer in range(w.n_layers):
-        groups = {(plan.unit((layer * H + h) * 2)["b"], plan.unit((layer * H + h) * 2 + 1)["b"]) for h in range(H)}
-        n += 1 + len(groups) + 1          # append, split kernel(s), combine
+        groups = {(cls(plan.unit((layer * H + h) * 2)["b"]), cls(plan.unit((layer * H + h) * 2 + 1)["b"]))
+                  for h in range(H)}
+        n += 3 + len(groups)
     return n
 
 
@@ -420,7 +426,7 @@ def run_ours(args, torch, dist, rank, world):
         "pct_of_peak": round(100 * value / world / hbm_peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": None,
-                     "kernel": "decode (split kernel + combine) of one layer", "peak_kind": peak_kind,
+                     "kernel": "decode call of one layer (q~ prep + split kernel + combine)", "peak_kind": peak_kind,
                      "bytes_per_launch": step_bytes // L, "launch_ms": round(dec_ms, 5)},
         "e2e": {"value": round(aggregate_value(world, step_bytes, e2e_ms), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
@@ -428,6 +434,8 @@ def run_ours(args, torch, dist, rank, world):
         "clocks": clk.summary(),
         "setup_s": {"calibrate": round(st["t_cal"], 1), "total": round(st["t_setup"], 1)},
     }
+    if not args.no_sdpa:
+        res["sdpa_context"] = sdpa_context(torch, w, dec_ms)
     if not args.no_encode:
         res["encode"] = encode_bench(torch, synth.WORKLOADS[ENCODE_WORKLOAD], max(1, min(args.steps, 5)),
                                      args.warmup, rank, args.encode_layers)
@@ -438,6 +446,35 @@ def run_ours(args, torch, dist, rank, world):
                                "sample": f"{heads} KV head(s) of layer 0 (G={w.group} queries each) over the "
                                          f"{w.seq_len}-token cache: unpack + fp64 d-space attention"}
     return res
+
+
+def sdpa_context(torch, w, dec_ms, reps=20):
+    """Context for the pages' speed claim against FP16 SDPA (KV-COBRA project page,
+    "Efficiency"): torch's fp16 scaled_dot_product_attention for one decode query over an
+    uncompressed cache of the same shape (G query heads per KV head), timed per layer.
+    Not part of the product path; the cache is 2 * H_kv * T * 256 bytes > L2."""
+    import torch.nn.functional as F
+    T, H, Hq = w.seq_len, w.n_kv_heads, w.n_q_heads
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    k = torch.randn((w.batch, H, T, 128), generator=gen, device="cuda", dtype=torch.float16)
+    v = torch.randn((w.batch, H, T, 128), generator=gen, device="cuda", dtype=torch.float16)
+    q = torch.randn((w.batch, Hq, 1, 128), generator=gen, device="cuda", dtype=torch.float16)
+    for _ in range(3):
+        F.scaled_dot_product_attention(q, k, v, enable_gqa=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        F.scaled_dot_product_attention(q, k, v, enable_gqa=True)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    kv_bytes = 2 * w.batch * H * T * 128 * 2
+    del k, v, q
+    torch.cuda.empty_cache()
+    return {"fp16_sdpa_ms_per_layer": round(ms, 5), "fp16_sdpa_gb_s": round(kv_bytes / (ms * 1e-3) / 1e9, 1),
+            "compressed_decode_ms_per_layer": round(dec_ms, 5), "speedup": round(ms / dec_ms, 3),
+            "shape": f"batch {w.batch}, {Hq} q / {H} kv heads, {T} tokens, d 128"}
 
 
 # ---------------------------------------------------------------------------- reference arm
@@ -498,6 +535,7 @@ def main():
     ap.add_argument("--encode-layers", type=int, default=0, help="limit the encode workload's layers")
     ap.add_argument("--layers", type=int, default=0, help="limit the decode workload's layers (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sdpa", action="store_true", help="skip the fp16 SDPA context timing")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
