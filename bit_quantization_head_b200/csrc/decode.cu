@@ -320,6 +320,7 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int n_hg = (plan->G + 7) / 8;
   const int cap = split_cap(max_seq_len);
+  const int max_pages_seq = std::max(1, (max_seq_len + kPage - 1) / kPage);
   const int part_stride = cap;
   const int Hq = plan->H * plan->G;
   float* parts = static_cast<float*>(workspace);
@@ -411,13 +412,26 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     a.n_hg = n_hg;
     a.n_heads = static_cast<int>(hs.size());
     a.part_stride = part_stride;
+    // Splits per head: greedy on the modelled finishing time.  A head with s splits
+    // gives each of its 4 s warps at most ceil(P / 4 s) pages, so it ends after about
+    // ceil(P / 4 s) * cost; the column goes to the head that ends last, while columns
+    // remain (and the head has at least 8 pages per split).
+    std::vector<int> ns(hs.size(), 1);
+    auto ends = [&](size_t i) {
+      return std::ceil(static_cast<double>(max_pages_seq) / (kWarps * ns[i])) * head_cost[hs[i]];
+    };
+    for (int used = static_cast<int>(hs.size()); used < columns; ++used) {
+      size_t best = hs.size();
+      for (size_t i = 0; i < hs.size(); ++i)
+        if (ns[i] < cap && (best == hs.size() || ends(i) > ends(best))) best = i;
+      if (best == hs.size()) break;
+      ++ns[best];
+    }
     a.split_prefix[0] = 0;
     for (size_t i = 0; i < hs.size(); ++i) {
       a.heads[i] = hs[i];
-      int ns = static_cast<int>(std::floor(columns * head_cost[hs[i]] / group_cost));
-      ns = std::max(1, std::min(ns, cap));
-      a.split_prefix[i + 1] = a.split_prefix[i] + ns;
-      ca.nparts[hs[i]] = ns;
+      a.split_prefix[i + 1] = a.split_prefix[i] + ns[i];
+      ca.nparts[hs[i]] = ns[i];
     }
     a.qt = qt;
     a.wait_first = first ? 1 : 0;

@@ -7,16 +7,18 @@
 //   * scores its G (<= 8) query heads with m16n8k16 MMAs whose A operand comes straight
 //     from the packed words: one AND leaves each code in the low mantissa bits of an fp16
 //     half, the exact subnormal c * 2^(e-24), e the field's bit offset (undone in fp32);
-//     q~ is split into fp16 hi + lo, and for G <= 4 the lo half rides in the four unused
-//     columns of the same MMA;
+//     q~ is split into fp16 hi + lo; for G <= 4 (packed mode) head n's hi and lo parts sit
+//     in columns 2n and 2n + 1 of one MMA, so each lane adds its own two columns and
+//     holds one head's scores for two token rows;
 //   * runs an online softmax whose rescale is lazy: it happens only when a score exceeds
 //     the running max by more than 2^8 (a warp vote), so the common block costs one FFMA
 //     and one ex2 per score;
 //   * stores P in fp16 scaled by 2^(7-e) so that P * A = p * c * 2^-17 for any e, moves it
 //     into the B fragment with movmatrix, and accumulates the value latents with MMAs
-//     whose A operand again comes straight from the packed value words.  One extra A row
-//     of ones (when r_V is not a multiple of 16) accumulates l = sum p with the same
-//     rounded P, so z - m_V * l cancels consistently.
+//     whose A operand again comes straight from the packed value words.  l = sum p is
+//     accumulated from the same rounded P, so z - m_V * l cancels consistently: in packed
+//     mode by one more MMA whose A operand is a constant row of ones, otherwise by one
+//     extra A row of ones (when r_V is not a multiple of 16) or per-lane sums.
 // IL blocks are processed together (their MMA chains interleave).  The four warps'
 // (m, l, z) partials meet in shared memory and each CTA writes one partial per query
 // head; decode.cu's combine kernel merges those and back-projects.  q~ = M_K q comes from
@@ -180,15 +182,16 @@ struct WS {
   Parts partsK, partsV;
   int ones_mt, ones_lr;  // m-tile / local row of the ones row (ones_mt < 0: none)
   uint32_t ones_m0, ones_m1;  // lane masks: this lane's A rows g / g+8 are the ones row
-  // B fragments of q^: PACK -> bh[ks] (hi for g < 4, lo for g >= 4); else bh, bl
+  // B fragments of q^: PACK -> bh[ks] (column g: head g / 2, hi for even g, lo for odd);
+  // else bh (hi), bl (lo), column g: head g
   uint32_t bh[kNT][2];
   uint32_t bl[PACK ? 1 : kNT][2];
   float alpha[2], beta[2], m_run[2];
   float al[2][n_e<BK == 0 ? 8 : BK>()], nb[2][n_e<BV == 0 ? 8 : BV>()];
-  // PACK: after the hi/lo exchange a lane keeps one token row (lo: row g + 8, else g);
-  // its constants by block parity p
-  bool lo;
-  float alL[2][2], nbL[2][2], limL[2], offL[2], uL[2];
+  // PACK: l accumulator (row 0, column 2n: l of head n, times 2^-17) and the constant A
+  // fragments of its ones row by block parity (a0, a2; nonzero in lanes g == 0 only)
+  float zl[4];
+  uint32_t onesA[2][2];
   float z[kNT][4];
   float lcvt[2];  // l accumulated from the fp16 P when there is no ones row
 };
@@ -211,21 +214,6 @@ __device__ __forceinline__ void refresh_constants(WS<BK, BV, PACK>& w) {
     for (int i = 0; i < NEV; ++i) {
       const int e = BV == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (BV == 4 ? 4 * i : 0);
       w.nb[c][i] = base - static_cast<float>(e);
-    }
-    if constexpr (PACK) {
-      // the lane's row eta = lo: e_K(p, eta), e_V(p, eta) for block parity p
-#pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        const float ek = BK == 2 ? 4.0f * p + (w.lo ? 2.0f : 0.0f) : (BK == 4 ? (w.lo ? 4.0f : 0.0f) : 0.0f);
-        const float ev = BV == 2 ? 4.0f * p + (w.lo ? 2.0f : 0.0f) : (BV == 4 ? (w.lo ? 4.0f : 0.0f) : 0.0f);
-        w.alL[c][p] = w.alpha[c] * exp2f(-ek);
-        w.nbL[c][p] = base - ev;
-        if (c == 0) {
-          w.limL[p] = kLazy + 7.0f - ev;
-          w.offL[p] = 7.0f - ev;
-          w.uL[p] = exp2f(ev - 7.0f);
-        }
-      }
     }
   }
 }
@@ -260,29 +248,25 @@ __device__ __forceinline__ void k_block(const WS<BK, BV, PACK>& w, int ks, uint3
 template <int BK, int BV, bool PACK, int BLK>
 __device__ __forceinline__ bool x_block(const WS<BK, BV, PACK>& w, const float (&sc)[4], const float (&sd)[4],
                                         float (&x)[4]) {
+  constexpr int ik0 = e_idx<BK == 0 ? 8 : BK>(BLK, 0), ik1 = e_idx<BK == 0 ? 8 : BK>(BLK, 1);
+  constexpr int iv0 = e_idx<BV == 0 ? 8 : BV>(BLK, 0), iv1 = e_idx<BV == 0 ? 8 : BV>(BLK, 1);
+  constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
+  constexpr float lim0 = kLazy + 7.0f - ev0, lim1 = kLazy + 7.0f - ev1;
   if constexpr (PACK) {
-    // hi lanes (t' < 2) keep row g and receive its lo part; lo lanes keep row g + 8 and
-    // receive its hi part: each (row, head) score is formed once
-    constexpr int p = BLK & 1;
-    const float k0 = w.lo ? sc[2] : sc[0], k1 = w.lo ? sc[3] : sc[1];
-    const float s0 = w.lo ? sc[0] : sc[2], s1 = w.lo ? sc[1] : sc[3];
-    const float f0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 2);
-    const float f1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 2);
-    x[0] = fmaf(w.alL[0][p], f0, w.nbL[0][p]);
-    x[1] = fmaf(w.alL[1][p], f1, w.nbL[1][p]);
+    // columns 2 tq (hi) and 2 tq + 1 (lo) of head tq: x[0] row g, x[1] row g + 8
+    x[0] = fmaf(w.al[0][ik0], sc[0] + sc[1], w.nb[0][iv0]);
+    x[1] = fmaf(w.al[0][ik1], sc[2] + sc[3], w.nb[0][iv1]);
     if (w.partial) {  // warp-uniform: only the last page of a sequence
-      const int t = w.tok0 + 16 * BLK + w.g + (w.lo ? 8 : 0);
-      if (t >= w.seq_len) x[0] = x[1] = -INFINITY;
+      const int t0 = w.tok0 + 16 * BLK + w.g;
+      if (t0 >= w.seq_len) x[0] = -INFINITY;
+      if (t0 + 8 >= w.seq_len) x[1] = -INFINITY;
     }
-    return fmaxf(x[0], x[1]) > w.limL[p];
+    return x[0] > lim0 || x[1] > lim1;
   } else {
     float full[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) full[i] = sc[i] + sd[i];
     // rows: full[0..1] token tok0 + 16*BLK + g (eta 0), full[2..3] that + 8 (eta 1)
-    constexpr int ik0 = e_idx<BK == 0 ? 8 : BK>(BLK, 0), ik1 = e_idx<BK == 0 ? 8 : BK>(BLK, 1);
-    constexpr int iv0 = e_idx<BV == 0 ? 8 : BV>(BLK, 0), iv1 = e_idx<BV == 0 ? 8 : BV>(BLK, 1);
-    constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
     x[0] = fmaf(w.al[0][ik0], full[0], w.nb[0][iv0]);
     x[1] = fmaf(w.al[1][ik0], full[1], w.nb[1][iv0]);
     x[2] = fmaf(w.al[0][ik1], full[2], w.nb[0][iv1]);
@@ -292,7 +276,6 @@ __device__ __forceinline__ bool x_block(const WS<BK, BV, PACK>& w, const float (
       if (t0 >= w.seq_len) x[0] = x[1] = -INFINITY;
       if (t1 >= w.seq_len) x[2] = x[3] = -INFINITY;
     }
-    constexpr float lim0 = kLazy + 7.0f - ev0, lim1 = kLazy + 7.0f - ev1;
     return fmaxf(x[0], x[1]) > lim0 || fmaxf(x[2], x[3]) > lim1;
   }
 }
@@ -300,8 +283,8 @@ __device__ __forceinline__ bool x_block(const WS<BK, BV, PACK>& w, const float (
 // Block maximum of s - m_run for head column c of one block (x with the e_V offset removed).
 template <int BK, int BV, bool PACK, int BLK>
 __device__ __forceinline__ float xmax_block(const WS<BK, BV, PACK>& w, const float (&x)[4], int c) {
-  if constexpr (PACK) return x[c] - w.offL[BLK & 1];
   constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
+  if constexpr (PACK) return fmaxf(x[0] - (7.0f - ev0), x[1] - (7.0f - ev1));
   return fmaxf(x[c] - (7.0f - ev0), x[2 + c] - (7.0f - ev1));
 }
 
@@ -310,17 +293,12 @@ __device__ __forceinline__ float xmax_block(const WS<BK, BV, PACK>& w, const flo
 template <int BK, int BV, bool PACK, int BLK>
 __device__ __forceinline__ void p_block(WS<BK, BV, PACK>& w, const float (&x)[4], uint32_t (&bp)[2]) {
   if constexpr (PACK) {
-    // this lane's row, its two heads; hi lanes also take row g + 8 from their lo partner,
-    // lo lanes (columns 4..7 of the value MMA's B) carry zeros
-    const uint32_t Pm = pack_half2(ex2(x[0]), ex2(x[1]));
-    const uint32_t Po = __shfl_xor_sync(0xffffffffu, Pm, 2);
-    if (w.ones_mt < 0) {
-      const float2 f = half2_to_float2(Pm);
-      w.lcvt[0] = fmaf(f.x, w.uL[BLK & 1], w.lcvt[0]);
-      w.lcvt[1] = fmaf(f.y, w.uL[BLK & 1], w.lcvt[1]);
-    }
-    bp[0] = movmatrix_trans(w.lo ? 0u : Pm);
-    bp[1] = movmatrix_trans(w.lo ? 0u : Po);
+    // 8x8 tile X[row g][column 2 tq] = P(token g (+8), head tq), odd columns 0; its
+    // transpose is the B fragment with head n in column 2n (odd columns zero)
+    bp[0] = movmatrix_trans(pack_half2(ex2(x[0]), 0.0f));
+    bp[1] = movmatrix_trans(pack_half2(ex2(x[1]), 0.0f));
+    // l: the ones row times the same rounded P
+    mma_16816(w.zl, w.onesA[BLK & 1][0], 0u, w.onesA[BLK & 1][1], 0u, bp[0], bp[1]);
     return;
   }
   const uint32_t P0 = pack_half2(ex2(x[0]), ex2(x[1]));
@@ -418,14 +396,13 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
   bool grow = false;
   ((grow |= x_block<BK, BV, PACK, B0 + BB>(w, sc[BB], sd[BB], x[BB])), ...);
   // grow also while the running max is undefined (the first live block)
-  grow |= w.m_run[0] == -INFINITY || w.m_run[1] == -INFINITY;
+  grow |= w.m_run[0] == -INFINITY || (!PACK && w.m_run[1] == -INFINITY);
   // ---- lazy online softmax: rescale only when a score passes the running max by 2^kLazy
   if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < (PACK ? 1 : 2); ++c) {
       float v = -INFINITY;
       ((v = fmaxf(v, xmax_block<BK, BV, PACK, B0 + BB>(w, x[BB], c))), ...);
-      if constexpr (PACK) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));  // the other row
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
@@ -446,12 +423,20 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
           w.z[mt][c] *= resc;
           w.z[mt][2 + c] *= resc;
         }
-        w.lcvt[c] *= resc;
+        if constexpr (PACK)
+          w.zl[0] *= resc;
+        else
+          w.lcvt[c] *= resc;
       }
 #pragma unroll
       for (int bb = 0; bb < IL; ++bb) {
-        x[bb][c] -= shift;
-        x[bb][2 + c] -= shift;
+        if constexpr (PACK) {
+          x[bb][0] -= shift;
+          x[bb][1] -= shift;
+        } else {
+          x[bb][c] -= shift;
+          x[bb][2 + c] -= shift;
+        }
       }
     }
     refresh_constants(w);
@@ -464,7 +449,7 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
   auto vtile = [&](auto MTC) {
     constexpr int mt = decltype(MTC)::value;
     const int j0 = 16 * mt + w.g, j1 = j0 + 8;
-    const bool ones = mt == w.ones_mt;
+    const bool ones = !PACK && mt == w.ones_mt;
     constexpr int VB = BV == 0 ? 1 : BV;
     constexpr int VW0 = (B0 * VB) / 8, VWN = ((B0 + IL - 1) * VB) / 8 - VW0 + 1;
     uint32_t W0[VWN], W1[VWN], W0h[VWN], W1h[VWN];
@@ -542,10 +527,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     seq_len = seq_len < 0 ? 0 : a.max_pages * kPage;
   }
   const int n_pages = (seq_len + kPage - 1) / kPage;
-  const int pages_per_split = (n_pages + n_split - 1) / n_split;
-  const int p_begin = split * pages_per_split;
-  const int p_end = min(p_begin + pages_per_split, n_pages);
-  const int n_my = p_end > p_begin + warp ? (p_end - p_begin - warp + kWarps - 1) / kWarps : 0;
+  // The head's pages are cut into n_split * kWarps contiguous runs whose lengths differ
+  // by at most one page; warp w of split c takes run c * kWarps + w.
+  const int n_workers = n_split * kWarps;
+  const int worker = split * kWarps + warp;
+  const int p_begin = static_cast<int>(static_cast<long long>(worker) * n_pages / n_workers);
+  const int n_my = static_cast<int>(static_cast<long long>(worker + 1) * n_pages / n_workers) - p_begin;
   const int32_t* bt = a.block_table + static_cast<size_t>(s) * a.max_pages;
 
   // ---- prologue: barriers, q~, page ids, first copies ----
@@ -576,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     const int base = i & ~31;
     if (base != pid_base) {
       const int ii = base + lane;
-      pid_win = ii < n_my ? bt[p_begin + warp + ii * kWarps] : -1;
+      pid_win = ii < n_my ? bt[p_begin + ii] : -1;
       pid_base = base;
     }
     return __shfl_sync(0xffffffffu, pid_win, i & 31);
@@ -632,17 +619,16 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   w.tq = tq;
   w.seq_len = seq_len;
   w.partial = false;
-  w.lo = PACK && tq >= 2;
   w.partsK = parts_of(dK.b);
   w.partsV = parts_of(dV.b);
-  w.ones_mt = (rV & 15) ? (rV >> 4) : -1;
+  w.ones_mt = (!PACK && (rV & 15)) ? (rV >> 4) : -1;
   w.ones_lr = rV & 15;
   w.ones_m0 = (w.ones_mt >= 0 && w.ones_lr == g) ? 0xFFFFFFFFu : 0u;
   w.ones_m1 = (w.ones_mt >= 0 && w.ones_lr == g + 8) ? 0xFFFFFFFFu : 0u;
-  // B fragments of q^ = q~ * 2^-E.  Packed (G <= 4): column n < 4 holds the hi part of
-  // head n, column n >= 4 the lo part of head n - 4.
+  // B fragments of q^ = q~ * 2^-E.  Packed (G <= 4): column n holds head n / 2, its hi
+  // part for even n and its lo part for odd n.
   {
-    const int hsrc = PACK ? (g & 3) : g;
+    const int hsrc = PACK ? (g >> 1) : g;
     const float scl = ldexpf(1.0f, -sh.E[hsrc]);
 #pragma unroll
     for (int ks = 0; ks < kNT; ++ks) {
@@ -655,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
         const uint32_t hw = static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
         const uint32_t lw = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
         if constexpr (PACK) {
-          w.bh[ks][half] = g < 4 ? hw : lw;
+          w.bh[ks][half] = (g & 1) ? lw : hw;
         } else {
           w.bh[ks][half] = hw;
           w.bl[ks][half] = lw;
@@ -669,13 +655,23 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     const float base = a.scale * dK.delta * kLog2e;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      const int n = PACK ? 2 * (tq & 1) + c : 2 * tq + c;
+      const int n = PACK ? tq : 2 * tq + c;  // packed: one head per lane
       w.alpha[c] = n < ng ? base * ldexpf(1.0f, sh.E[n] + 24) : 0.0f;
       w.beta[c] = n < ng ? base * mK * sh.S[n] : 0.0f;
       w.m_run[c] = -INFINITY;
       w.lcvt[c] = 0.0f;
     }
     refresh_constants(w);
+    // ones row of the l MMA: fp16 subnormals 2^(e_V - 24), e_V of the block parity
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+#pragma unroll
+      for (int eta = 0; eta < 2; ++eta) {
+        const int e = BV == 2 ? 4 * p + 2 * eta : (BV == 4 ? 4 * eta : 0);
+        w.onesA[p][eta] = g == 0 ? ((1u << e) | (1u << (e + 16))) : 0u;
+      }
+    }
+    w.zl[0] = w.zl[1] = w.zl[2] = w.zl[3] = 0.0f;
   }
 #pragma unroll
   for (int mt = 0; mt < kNT; ++mt) w.z[mt][0] = w.z[mt][1] = w.z[mt][2] = w.z[mt][3] = 0.0f;
@@ -686,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   int slot = 0;        // stage of page i (i mod n_stage), kept incrementally
   uint32_t phase = 0;  // barrier phase of that use of the stage ((i / n_stage) & 1)
   for (int i = 0; i < n_my; ++i) {
-    const int p = p_begin + warp + i * kWarps;
+    const int p = p_begin + i;
     const bool valid = (__shfl_sync(0xffffffffu, vmask, 0) >> slot) & 1u;
     if (!mbar_wait_bounded_warp(&bars[warp * 8 + slot], phase)) {
       if (lane == 0 && a.status) atomicOr(a.status, KVTC_STATUS_TIMEOUT);
@@ -731,7 +727,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   float l_out[2];
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
-    if (w.ones_mt >= 0) {
+    if (PACK) {
+      // row 0 of the l MMA: lane tq (g == 0) holds head tq's l * 2^-17
+      l_out[c] = ldexpf(__shfl_sync(0xffffffffu, w.zl[0], tq), 17);
+    } else if (w.ones_mt >= 0) {
       // select z[ones_mt][row] with a masked sum (a select here would be turned into a
       // run-time index and push the fragments to local memory)
       float v = 0.0f;
@@ -746,7 +745,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       l_out[c] = ldexpf(__shfl_sync(0xffffffffu, v, src), 17);
     } else {
       float l = w.lcvt[c];
-      if constexpr (PACK) l += __shfl_xor_sync(0xffffffffu, l, 2);  // rows g and g + 8
       l += __shfl_xor_sync(0xffffffffu, l, 4);
       l += __shfl_xor_sync(0xffffffffu, l, 8);
       l += __shfl_xor_sync(0xffffffffu, l, 16);
@@ -761,8 +759,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   __syncthreads();
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
-    const int n = 2 * tq + c;  // column of the z fragment (a query head, or a copy in packed mode)
-    const bool real = PACK ? (tq < 2 && n < ng) : n < ng;
+    // head of z column 2 tq + c: packed mode keeps head tq in column 2 tq (odd columns 0)
+    const int n = PACK ? tq : 2 * tq + c;
+    const bool real = PACK ? (c == 0 && n < ng) : n < ng;
     if (real) {
       float* dst = mb + (warp * 8 + n) * kPartStride;
       if (g == 0) {
