@@ -41,6 +41,12 @@ from bit_quantization_head_b200 import kvtc, synth  # noqa: E402
 
 DECODE_WORKLOAD = "llama8b-32L-128k-1bpd"
 ENCODE_WORKLOAD = "qwen7b-28L-128k-2bpd"
+
+# DRAM bytes (read + write) of one decode call (prep + split + combine) per layer, from an
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the current decode kernels
+# on layers 0-3 of the workload; reported as roofline.traffic beside the algorithmic
+# bytes.  Set to None whenever a decode kernel changes, until it is captured again.
+DECODE_TRAFFIC = {"llama8b-32L-128k-1bpd": 34415360}
 METRIC = "decode-attn effective HBM GB/s (% of peak) at 128k ctx; encode Mtok/s"
 
 
@@ -425,7 +431,7 @@ def run_ours(args, torch, dist, rank, world):
                    "compute": "fp16 tensor-core operands (codes exact, q split hi+lo), fp32 accumulation"},
         "pct_of_peak": round(100 * value / world / hbm_peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                     "frac": round(achieved / hbm_peak, 4), "traffic": DECODE_TRAFFIC.get(w.name),
                      "kernel": "decode call of one layer (q~ prep + split kernel + combine)", "peak_kind": peak_kind,
                      "bytes_per_launch": step_bytes // L, "launch_ms": round(dec_ms, 5)},
         "e2e": {"value": round(aggregate_value(world, step_bytes, e2e_ms), 2), "unit": "GB/s",
