@@ -35,7 +35,7 @@
 #include "ptx.cuh"
 
 #ifndef KVTC_DECODE_IL
-#define KVTC_DECODE_IL 4
+#define KVTC_DECODE_IL 8
 #endif
 
 namespace kvtc {
@@ -45,6 +45,17 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kNT = 8;                // 16-row tiles of a rank (r <= 128)
 constexpr int kIL = KVTC_DECODE_IL;   // blocks processed together
+#ifndef KVTC_DECODE_ZSPLIT
+#define KVTC_DECODE_ZSPLIT 0
+#endif
+// 1: even and odd blocks accumulate the value latents (and l) in separate fragments,
+// halving the MMA dependency chain of each m-tile
+constexpr bool kZSplit = KVTC_DECODE_ZSPLIT != 0;
+#ifndef KVTC_DECODE_HOIST
+#define KVTC_DECODE_HOIST 0
+#endif
+// 1: the packed words of a block group are loaded ahead of the tile jumps
+constexpr bool kHoist = KVTC_DECODE_HOIST != 0;
 #ifndef KVTC_DECODE_MINB
 #define KVTC_DECODE_MINB 2
 #endif
@@ -193,6 +204,8 @@ struct WS {
   float zl[4];
   uint32_t onesA[2][2];
   float z[kNT][4];
+  float z2[kZSplit ? kNT : 1][4];  // odd blocks (kZSplit)
+  float zl2[4];
   float lcvt[2];  // l accumulated from the fp16 P when there is no ones row
 };
 
@@ -298,7 +311,8 @@ __device__ __forceinline__ void p_block(WS<BK, BV, PACK>& w, const float (&x)[4]
     bp[0] = movmatrix_trans(pack_half2(ex2(x[0]), 0.0f));
     bp[1] = movmatrix_trans(pack_half2(ex2(x[1]), 0.0f));
     // l: the ones row times the same rounded P
-    mma_16816(w.zl, w.onesA[BLK & 1][0], 0u, w.onesA[BLK & 1][1], 0u, bp[0], bp[1]);
+    mma_16816((kZSplit && (BLK & 1)) ? w.zl2 : w.zl, w.onesA[BLK & 1][0], 0u, w.onesA[BLK & 1][1], 0u, bp[0],
+              bp[1]);
     return;
   }
   const uint32_t P0 = pack_half2(ex2(x[0]), ex2(x[1]));
@@ -356,19 +370,56 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
   for (int bb = 0; bb < IL; ++bb)
 #pragma unroll
     for (int i = 0; i < 4; ++i) sc[bb][i] = sd[bb][i] = 0.0f;
-  // ---- scores S[tok][head] = sum_j codeK[tok][j] * q^[head][j]; the k-steps run from
-  // a jump into the unrolled sequence (no per-step test)
+  // ---- packed words of the group.  The k-steps and m-tiles below run from a jump into
+  // an unrolled sequence (no per-step test); each case label is a scheduling boundary,
+  // so for the narrow widths (at most two words per row and tile) every word the group
+  // needs is loaded here, ahead of the jumps, predicated on the rank.  Rows past r_K
+  // meet zero q^ coefficients (q~ is zero there) and rows past r_V are never read back,
+  // so both are read unmasked inside the last tile; the shared-memory allocation has
+  // slack for that over-read.
+  constexpr int KB = BK == 0 ? 1 : BK;
+  constexpr int KW0 = (B0 * KB) / 8, KWN = ((B0 + IL - 1) * KB) / 8 - KW0 + 1;
+  constexpr bool kHoistK = kHoist && BK != 0 && KWN <= 2;
+  constexpr int VB = BV == 0 ? 1 : BV;
+  constexpr int VW0 = (B0 * VB) / 8, VWN = ((B0 + IL - 1) * VB) / 8 - VW0 + 1;
+  constexpr bool kHoistV = kHoist && BV != 0 && VWN <= 2;
+  uint32_t KWa[kHoistK ? kNT : 1][KWN], KWb[kHoistK ? kNT : 1][KWN];
+  uint32_t VWa[kHoistV ? kNT : 1][VWN], VWb[kHoistV ? kNT : 1][VWN];
+  if constexpr (kHoistK) {
+#pragma unroll
+    for (int ks = 0; ks < kNT; ++ks) {
+      const bool on = ks < w.nks;
+      const int r0 = 8 * ks + w.tq;
+#pragma unroll
+      for (int q = 0; q < KWN; ++q) {
+        KWa[ks][q] = on ? w.pk[r0 * 8 * BK + w.g * BK + KW0 + q] : 0u;
+        KWb[ks][q] = on ? w.pk[(r0 + 4) * 8 * BK + w.g * BK + KW0 + q] : 0u;
+      }
+    }
+  }
+  if constexpr (kHoistV) {
+#pragma unroll
+    for (int mt = 0; mt < kNT; ++mt) {
+      const bool on = mt < w.nmt;
+      const int j0 = 16 * mt + w.g;
+#pragma unroll
+      for (int q = 0; q < VWN; ++q) {
+        VWa[mt][q] = on ? w.pv[j0 * 4 * BV + w.tq * BV + VW0 + q] : 0u;
+        VWb[mt][q] = on ? w.pv[(j0 + 8) * 4 * BV + w.tq * BV + VW0 + q] : 0u;
+      }
+    }
+  }
+  // ---- scores S[tok][head] = sum_j codeK[tok][j] * q^[head][j]
   auto kstep = [&](auto KSC) {
     constexpr int ks = decltype(KSC)::value;
-    // rows past r_K meet zero q^ coefficients (q~ is zero there), so they are read
-    // unmasked; the shared-memory allocation has slack for the over-read
     const int r0 = 8 * ks + w.tq, r1 = r0 + 4;
-    constexpr int KB = BK == 0 ? 1 : BK;
-    constexpr int KW0 = (B0 * KB) / 8, KWN = ((B0 + IL - 1) * KB) / 8 - KW0 + 1;
     uint32_t W0[KWN], W1[KWN], W0h[KWN], W1h[KWN];
 #pragma unroll
     for (int q = 0; q < KWN; ++q) {
-      if constexpr (BK != 0) {
+      if constexpr (kHoistK) {
+        W0[q] = KWa[ks][q];
+        W1[q] = KWb[ks][q];
+      } else if constexpr (BK != 0) {
         W0[q] = w.pk[r0 * 8 * BK + w.g * BK + KW0 + q];
         W1[q] = w.pk[r1 * 8 * BK + w.g * BK + KW0 + q];
       } else {
@@ -422,9 +473,16 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
         for (int mt = 0; mt < kNT; ++mt) {
           w.z[mt][c] *= resc;
           w.z[mt][2 + c] *= resc;
+          if constexpr (kZSplit) {
+            w.z2[mt][c] *= resc;
+            w.z2[mt][2 + c] *= resc;
+          }
         }
         if constexpr (PACK)
+        {
           w.zl[0] *= resc;
+          if constexpr (kZSplit) w.zl2[0] *= resc;
+        }
         else
           w.lcvt[c] *= resc;
       }
@@ -450,12 +508,13 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
     constexpr int mt = decltype(MTC)::value;
     const int j0 = 16 * mt + w.g, j1 = j0 + 8;
     const bool ones = !PACK && mt == w.ones_mt;
-    constexpr int VB = BV == 0 ? 1 : BV;
-    constexpr int VW0 = (B0 * VB) / 8, VWN = ((B0 + IL - 1) * VB) / 8 - VW0 + 1;
     uint32_t W0[VWN], W1[VWN], W0h[VWN], W1h[VWN];
 #pragma unroll
     for (int q = 0; q < VWN; ++q) {
-      if constexpr (BV != 0) {
+      if constexpr (kHoistV) {
+        W0[q] = VWa[mt][q];
+        W1[q] = VWb[mt][q];
+      } else if constexpr (BV != 0) {
         W0[q] = w.pv[j0 * 4 * BV + w.tq * BV + VW0 + q];
         W1[q] = w.pv[j1 * 4 * BV + w.tq * BV + VW0 + q];
       } else {
@@ -466,7 +525,7 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
     }
     (v_block<BK, BV, PACK, B0 + BB>(w, W0[((B0 + BB) * VB) / 8 - VW0], W0h[((B0 + BB) * VB) / 8 - VW0],
                                     W1[((B0 + BB) * VB) / 8 - VW0], W1h[((B0 + BB) * VB) / 8 - VW0], j0, j1, ones,
-                                    bp[BB], w.z[mt]),
+                                    bp[BB], (kZSplit && ((B0 + BB) & 1)) ? w.z2[mt] : w.z[mt]),
      ...);
   };
   switch (w.nmt) {
@@ -493,13 +552,12 @@ __device__ __forceinline__ void do_page(WS<BK, BV, PACK>& w) {
 
 template <int BK, int BV, bool PACK>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
-  // Programmatic dependent launch.  The first split launch of a call waits here for the
-  // preceding grid (the q~ prep kernel, which completes only after its own predecessor,
-  // e.g. the append that wrote the newest token).  A later split launch of the same call
-  // starts only once every CTA of the one before it is past this point, so it reads at
-  // once and waits at exit instead, which keeps completion ordered for the combine.
-  if (a.wait_first) griddep_wait();
-  griddep_launch_dependents();
+  // Programmatic dependent launch.  The first split launch of a call waits, once it has
+  // read the plan, for the preceding grid (the q~ prep kernel, which completes only after
+  // its own predecessor, e.g. the append that wrote the newest token), and triggers its
+  // dependents only after that wait.  A later split launch of the same call therefore
+  // starts only when the prep grid is complete: it reads at once and waits at exit
+  // instead, which keeps completion ordered for the combine.
   extern __shared__ __align__(128) unsigned char smem[];
   SmemHead& sh = *reinterpret_cast<SmemHead*>(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sizeof(SmemHead));
@@ -516,10 +574,16 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const int s = blockIdx.z;
   const int h = a.heads[hi];
   const int uK = (a.layer * a.H + h) * 2, uV = uK + 1;
+  // the plan is constant: its unit descriptors are read, and the stage barriers set up,
+  // before the wait for the preceding grid
   const UnitDesc dK = a.units[uK], dV = a.units[uV];
   const int rK = dK.r, rV = dV.r;
   const int Hq = a.H * a.G;
   const int g0 = hg * 8, ng = min(8, a.G - g0);
+  if (lane == 0)
+    for (int i = 0; i < a.n_stage; ++i) mbar_init(&bars[warp * 8 + i], 1);
+  if (a.wait_first) griddep_wait();
+  griddep_launch_dependents();
 
   int seq_len = a.seq_lens[s];
   if (seq_len < 0 || seq_len > a.max_pages * kPage) {
@@ -535,9 +599,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const int n_my = static_cast<int>(static_cast<long long>(worker + 1) * n_pages / n_workers) - p_begin;
   const int32_t* bt = a.block_table + static_cast<size_t>(s) * a.max_pages;
 
-  // ---- prologue: barriers, q~, page ids, first copies ----
-  if (lane == 0)
-    for (int i = 0; i < a.n_stage; ++i) mbar_init(&bars[warp * 8 + i], 1);
+  // ---- prologue: q~, page ids, first copies ----
   for (int i = tid; i < 8 * 32; i += kThreads) {
     const int gg = i >> 5, k4 = i & 31;
     float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -672,9 +734,13 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       }
     }
     w.zl[0] = w.zl[1] = w.zl[2] = w.zl[3] = 0.0f;
+    w.zl2[0] = w.zl2[1] = w.zl2[2] = w.zl2[3] = 0.0f;
   }
 #pragma unroll
-  for (int mt = 0; mt < kNT; ++mt) w.z[mt][0] = w.z[mt][1] = w.z[mt][2] = w.z[mt][3] = 0.0f;
+  for (int mt = 0; mt < kNT; ++mt) {
+    w.z[mt][0] = w.z[mt][1] = w.z[mt][2] = w.z[mt][3] = 0.0f;
+    if constexpr (kZSplit) w.z2[mt][0] = w.z2[mt][1] = w.z2[mt][2] = w.z2[mt][3] = 0.0f;
+  }
 
   // ---- main loop over this warp's pages ----
   bool dead = false;
@@ -723,6 +789,13 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     }
   }
 
+  if constexpr (kZSplit) {
+#pragma unroll
+    for (int mt = 0; mt < kNT; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w.z[mt][i] += w.z2[mt][i];
+    w.zl[0] += w.zl2[0];
+  }
   // ---- l: from the ones row, or the per-lane sums ----
   float l_out[2];
 #pragma unroll

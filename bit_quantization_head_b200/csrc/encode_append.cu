@@ -61,14 +61,21 @@ __device__ __forceinline__ void store_code(uint32_t* page, int kind, int r, int 
 // staged in shared memory once; each thread holds its row of M in registers; the fma
 // chains then run in the canonical order from registers and broadcast reads.
 __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constant__ AppendArgs a) {
-  // Programmatic dependent launch: wait for the producer of k/v, then let the next kernel
-  // (typically the decode of this layer) start its prologue.
-  griddep_wait();
-  griddep_launch_dependents();
   __shared__ float xs[kD];
   const int tok = blockIdx.x, ul = blockIdx.y, j = threadIdx.x;
   const int u = a.unit0 + ul;
+  // The plan (unit descriptor, bf16 row of M) is constant: read it before waiting for
+  // the producer of k/v (programmatic dependent launch), so the loads overlap its tail.
   const UnitDesc ud = a.units[u];
+  uint4 mr[16];
+  if (a.bf16 && j < ud.r) {
+    const uint4* m4 = reinterpret_cast<const uint4*>(ud.Mbf + static_cast<size_t>(j) * kD);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) mr[c] = m4[c];
+  }
+  griddep_wait();
+  // let the next kernel (typically the decode of this layer) start its prologue
+  griddep_launch_dependents();
   const int kind = ul & 1;
   const int head = ul >> 1;
   const size_t xoff = (static_cast<size_t>(tok) * a.H + head) * kD;
@@ -83,10 +90,6 @@ __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constan
   // ascending, then ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7))
   float ch[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
   if (a.bf16) {
-    const uint4* m4 = reinterpret_cast<const uint4*>(ud.Mbf + static_cast<size_t>(j) * kD);
-    uint4 mr[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) mr[c] = m4[c];
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       const uint32_t w[4] = {mr[c].x, mr[c].y, mr[c].z, mr[c].w};
