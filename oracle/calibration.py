@@ -29,6 +29,8 @@ import math
 
 import numpy as np
 
+from .codec import RAW_BITS
+
 B_MIN = 2
 B_MAX = 8
 KIND_K = 0
@@ -401,7 +403,8 @@ def gaussian_step(b, lo=1e-3, hi=4.0, iters=200):
 
 # ---------------------------------------------------------------- whole calibration
 def calibrate(k_cal, v_cal, q_cal, n_layers, n_kv_heads, bpd, seed, *,
-              weight_mode="kl", fixed_r=0, fixed_b=0, c2_iters=200, c2_mode="lagrange"):
+              weight_mode="kl", fixed_r=0, fixed_b=0, c2_iters=200, c2_mode="lagrange",
+              k_only=False):
     """Calibrate every unit (layer, KV head, K|V) and allocate (r, b).
 
     k_cal, v_cal: [L, H_kv, N, d]; q_cal: [L, H_kv, G, N, d] (float arrays).
@@ -409,6 +412,12 @@ def calibrate(k_cal, v_cal, q_cal, n_layers, n_kv_heads, bpd, seed, *,
     Returns a list of unit dicts in flat unit order (see ``unit_index``) with keys
     layer, head, kind, r, b, w, lam, V (sorted basis), M (fp64, r x d), sigma,
     delta, inv_delta (fp32 of 1/delta), D.
+
+    k_only (the project page's "k-only" setting: keys compressed, values kept): the
+    allocation runs over the key units alone with bpd * d bits per key unit and token;
+    every value unit is stored uncompressed, r = d, b = RAW_BITS (fp16 values),
+    M = identity, delta = 2^-24 (an fp16 value v read as the integer code v * 2^24,
+    with no centring), D = 0.
     """
     d = k_cal.shape[-1]
     units = []
@@ -424,17 +433,26 @@ def calibrate(k_cal, v_cal, q_cal, n_layers, n_kv_heads, bpd, seed, *,
                     w, lam, V, order = value_unit_weights(v_cal[layer, head])
                 units.append(dict(layer=layer, head=head, kind=kind, w=w, lam=lam, V=V,
                                   order=order))
+    pool = [i for i, u in enumerate(units) if not (k_only and u["kind"] == KIND_V)]
     if fixed_r and fixed_b:
-        rb = [(fixed_r, fixed_b)] * len(units)
+        rb_pool = [(fixed_r, fixed_b)] * len(pool)
         mu = None
     else:
-        total = int(round(bpd * d * len(units)))
+        total = int(round(bpd * d * len(pool)))
+        weights = [units[i]["w"] for i in pool]
         if c2_mode == "damped":
-            rb, mu = c2_damped([u["w"] for u in units], total), 0.0
+            rb_pool, mu = c2_damped(weights, total), 0.0
         else:
-            rb, mu = c2([u["w"] for u in units], total, iters=c2_iters)
+            rb_pool, mu = c2(weights, total, iters=c2_iters)
+    rb = [(d, RAW_BITS)] * len(units)
+    for i, x in zip(pool, rb_pool):
+        rb[i] = x
     steps = {b: gaussian_step(b) for b in range(B_MIN, B_MAX + 1)}
     for idx, (u, (r, b)) in enumerate(zip(units, rb)):
+        if b == RAW_BITS:
+            u.update(r=d, b=b, signs=np.ones(d), M=np.eye(d), sigma=0.0, delta=2.0 ** -24,
+                     inv_delta=np.float32(2.0 ** 24), D=0.0, mu=mu)
+            continue
         signs = hadamard_signs(seed, idx, r)
         M = folded_projection(u["V"], r, signs)
         sigma = math.sqrt(float(np.mean(u["lam"][:r])))

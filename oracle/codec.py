@@ -19,6 +19,10 @@ Readings taken where the page is silent:
     y_hat = delta * (c - (2^b - 1) / 2).
   * Page layout (this build's specification; the page names none): see
     ``field_bit_positions``.
+  * Keys-only mode (the project page's "k-only" results compress keys and keep values
+    as they are): a value unit is then stored uncompressed, r = d and b = 16, each value
+    rounded to fp16 (round to nearest even); ``RAW_BITS`` marks such a unit.  Its page
+    layout is this build's specification too: see ``raw_word_index``.
 """
 
 from __future__ import annotations
@@ -28,6 +32,7 @@ import numpy as np
 PAGE_TOKENS = 128
 KIND_K = 0
 KIND_V = 1
+RAW_BITS = 16  # b of an uncompressed (fp16) value unit in keys-only mode
 
 
 # ---------------------------------------------------------------- fp32 arithmetic
@@ -116,7 +121,10 @@ def quantize(y, inv_delta, b):
 
 
 def dequantize(c, delta, b):
-    """y_hat = delta * (c - (2^b - 1)/2), fp64."""
+    """y_hat = delta * (c - (2^b - 1)/2), fp64.  For an uncompressed unit (b = RAW_BITS)
+    c holds fp16 bit patterns and y_hat is their value."""
+    if b == RAW_BITS:
+        return np.asarray(c, dtype=np.int64).astype(np.uint16).view(np.float16).astype(np.float64)
     return float(delta) * (np.asarray(c, dtype=np.float64) - ((1 << b) - 1) / 2.0)
 
 
@@ -188,8 +196,51 @@ def field_bit_positions(kind, r, b):
     return pos
 
 
+def raw_word_index(j, k):
+    """Index of the 32-bit word that holds coordinate j of tokens 2k (low half) and
+    2k + 1 (high half) in an uncompressed page: row j has 64 words, and pair k sits at
+    position k XOR 4 (j mod 8) of its row.  (Rows are whole coordinates, like the value
+    layout of the coded pages; the XOR spreads the eight rows an MMA fragment reads
+    over distinct shared-memory banks.)"""
+    return j * (PAGE_TOKENS // 2) + (k ^ ((j % 8) << 2))
+
+
+def pack_page_raw(vals):
+    """Pack fp16 bit patterns [128, d] (tokens x coordinates) of one page into
+    128 * d * 2 bytes (little-endian words, see ``raw_word_index``)."""
+    vals = np.asarray(vals, dtype=np.int64)
+    d = vals.shape[1]
+    words = np.zeros(d * (PAGE_TOKENS // 2), dtype=np.uint32)
+    for j in range(d):
+        for k in range(PAGE_TOKENS // 2):
+            lo = int(vals[2 * k, j]) & 0xFFFF
+            hi = int(vals[2 * k + 1, j]) & 0xFFFF
+            words[raw_word_index(j, k)] = lo | (hi << 16)
+    return words.astype("<u4").view(np.uint8)
+
+
+def unpack_page_raw(page, d):
+    """Inverse of ``pack_page_raw``: bytes -> fp16 bit patterns [128, d]."""
+    words = np.asarray(page, dtype=np.uint8).view("<u4")
+    vals = np.zeros((PAGE_TOKENS, d), dtype=np.int64)
+    for j in range(d):
+        for k in range(PAGE_TOKENS // 2):
+            w = int(words[raw_word_index(j, k)])
+            vals[2 * k, j] = w & 0xFFFF
+            vals[2 * k + 1, j] = w >> 16
+    return vals
+
+
+def encode_raw(x):
+    """Uncompressed unit: fp16 (round to nearest even) of every value, as bit
+    patterns [n, d]."""
+    return np.asarray(x, dtype=np.float32).astype(np.float16).view(np.uint16).astype(np.int64)
+
+
 def pack_page(codes, kind, b):
     """Pack codes [128, r] (ints in [0, 2^b)) of one page into 16*r*b bytes."""
+    if b == RAW_BITS:
+        return pack_page_raw(codes)
     codes = np.asarray(codes, dtype=np.int64)
     r = codes.shape[1]
     pos = field_bit_positions(kind, r, b)
@@ -202,6 +253,8 @@ def pack_page(codes, kind, b):
 
 def unpack_page(page, kind, r, b):
     """Inverse of ``pack_page``: bytes -> codes [128, r]."""
+    if b == RAW_BITS:
+        return unpack_page_raw(page, r)
     page = np.asarray(page, dtype=np.uint8)
     bits = np.unpackbits(page, bitorder="little")
     pos = field_bit_positions(kind, r, b)
@@ -210,7 +263,10 @@ def unpack_page(page, kind, r, b):
 
 
 def encode_tokens(x, M_operand, inv_delta, b):
-    """Codes of n tokens of one unit: quantize(project_canonical(x, M))."""
+    """Codes of n tokens of one unit: quantize(project_canonical(x, M)); for an
+    uncompressed unit (b = RAW_BITS) the fp16 bit patterns of x."""
+    if b == RAW_BITS:
+        return encode_raw(x)
     return quantize(project_canonical(x, M_operand), inv_delta, b)
 
 

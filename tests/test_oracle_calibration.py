@@ -333,3 +333,34 @@ def test_c2_damped_moves_budget_toward_the_larger_marginal():
     w = np.sort(np.random.default_rng(4).exponential(1.0, 128))[::-1]
     picks = cal.c2_damped([w, 10.0 * w], 2 * 128)
     assert picks[1][0] * picks[1][1] > picks[0][0] * picks[0][1]
+
+
+# ---------------------------------------------------------------- keys-only mode
+def test_calibrate_keys_only_stores_values_raw_and_spends_the_budget_on_keys():
+    rng = np.random.default_rng(19)
+    L, H, G, N, d = 1, 2, 2, 96, 8
+    k = rng.standard_normal((L, H, N, d)) * np.linspace(2, 0.1, d)
+    v = rng.standard_normal((L, H, N, d)) * np.linspace(1, 0.2, d)
+    q = rng.standard_normal((L, H, G, N, d))
+    bpd = 2.0
+    units = cal.calibrate(k, v, q, L, H, bpd=bpd, seed=3, k_only=True)
+    keys = [u for u in units if u["kind"] == cal.KIND_K]
+    vals = [u for u in units if u["kind"] == cal.KIND_V]
+    for u in vals:
+        assert (u["r"], u["b"], u["D"]) == (d, 16, 0.0)
+        assert np.array_equal(u["M"], np.eye(d)) and u["delta"] == 2.0 ** -24
+    total = int(round(bpd * d * len(keys)))
+    bits = sum(u["r"] * u["b"] for u in keys)
+    D = sum(u["D"] for u in keys)
+    assert bits <= total
+    # the key picks are within the brute-force optimum over the two key units' (r, b)
+    # pairs at that budget and no worse than the Lagrangian point they started from
+    ws = [u["w"] for u in keys]
+    assert D >= _brute_c2(ws, total) - 1e-12
+    tabs = [cal.candidate_table(w) for w in ws]
+    mu = keys[0]["mu"]
+    lag = sum(float(t[2][np.argmin(t[2] + mu * (t[0] * t[1]))]) for t in tabs)
+    assert D <= lag + 1e-12
+    # with fixed (r, b) the keys take it and the values stay raw
+    fixed = cal.calibrate(k, v, q, L, H, bpd=bpd, seed=3, fixed_r=4, fixed_b=3, k_only=True)
+    assert [(u["r"], u["b"]) for u in fixed] == [(4, 3), (d, 16), (4, 3), (d, 16)]

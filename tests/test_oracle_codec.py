@@ -284,3 +284,70 @@ def test_decode_head_reconstructs_from_codes():
     q = rng.standard_normal((2, d))
     o = att.decode_head(q, codes, codes, unit, unit, 0.25)
     assert np.allclose(o, att.softmax_attention(q, K, K, 0.25))
+
+
+# ---------------------------------------------------------------- keys-only: raw pages
+def test_raw_page_hand_example():
+    # token 5, coordinate 9 = fp16 1.0 (0x3C00): pair k = 2, odd token -> high half of
+    # word 9 * 64 + (2 XOR 4) = 582, i.e. bytes 2330..2331 = 00 3C.  Token 6,
+    # coordinate 0 = fp16 -2.0 (0xC000): pair 3, low half of word 0 * 64 + 3 -> bytes
+    # 12..13 = 00 C0.  Nothing else is set.
+    vals = np.zeros((128, 128), dtype=np.int64)
+    vals[5, 9] = 0x3C00
+    vals[6, 0] = 0xC000
+    page = codec.pack_page(vals, codec.KIND_V, codec.RAW_BITS)
+    assert page.size == codec.page_bytes(128, codec.RAW_BITS) == 32768
+    expect = np.zeros(32768, dtype=np.uint8)
+    expect[2331] = 0x3C
+    expect[13] = 0xC0
+    assert np.array_equal(page, expect)
+
+
+def test_raw_page_round_trip():
+    vals = np.random.default_rng(21).integers(0, 1 << 16, size=(128, 128))
+    page = codec.pack_page(vals, codec.KIND_V, codec.RAW_BITS)
+    assert np.array_equal(codec.unpack_page(page, codec.KIND_V, 128, codec.RAW_BITS), vals)
+
+
+def test_raw_swizzle_spreads_each_fragment_read_over_32_banks():
+    # The eight coordinate rows and four token pairs one 16x16 value tile takes per
+    # 32-bit load land in 32 distinct 4-byte banks, for every tile and block.
+    for mt in range(8):
+        for blk in range(8):
+            for half in range(2):
+                banks = {codec.raw_word_index(16 * mt + g + 8 * e, 8 * blk + tq + 4 * half) % 32
+                         for g in range(8) for tq in range(4) for e in (0,)}
+                assert len(banks) == 32
+
+
+def test_encode_raw_rounds_to_nearest_even_fp16():
+    # 1 + 2^-11 is halfway between 1 and 1 + 2^-10 -> 1 (even); 1 + 3 * 2^-11 is halfway
+    # between 1 + 2^-10 and 1 + 2^-9 -> 1 + 2^-9 (even); 2^-25 is halfway between 0 and
+    # the smallest subnormal 2^-24 -> 0; 65520 overflows to +inf.
+    x = np.array([[1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, 2.0 ** -25, -2.0, 65520.0]], dtype=np.float32)
+    got = codec.encode_raw(x)[0]
+    assert list(got) == [0x3C00, 0x3C02, 0x0000, 0xC000, 0x7C00]
+
+
+def test_dequantize_raw_reads_fp16_values():
+    c = np.array([0x3C00, 0xC000, 0x0001, 0x7BFF])
+    y = codec.dequantize(c, 2.0 ** -24, codec.RAW_BITS)
+    assert list(y) == [1.0, -2.0, 2.0 ** -24, 65504.0]
+
+
+def test_decode_head_with_raw_values_equals_sdpa_on_fp16_values():
+    # keys-only: coded keys reconstructed by M^T, values the fp16-rounded inputs
+    rng = np.random.default_rng(23)
+    d, T, r, b = 128, 400, 16, 4
+    Mk, _ = np.linalg.qr(rng.standard_normal((d, r)))
+    Mk = Mk.T
+    kc = rng.integers(0, 1 << b, size=(T, r))
+    V = rng.standard_normal((T, d)).astype(np.float32) * 3
+    vc = codec.encode_raw(V)
+    q = rng.standard_normal((4, d))
+    uk = dict(M=Mk, delta=0.2, b=b)
+    uv = dict(M=np.eye(d), delta=2.0 ** -24, b=codec.RAW_BITS)
+    o = att.decode_head(q, kc, vc, uk, uv, 1 / math.sqrt(d))
+    Khat = (0.2 * (kc - (2 ** b - 1) / 2)) @ Mk
+    ref = _sdpa(q, Khat, V.astype(np.float16).astype(np.float64), 1 / math.sqrt(d))
+    assert np.abs(o - ref).max() < 1e-12
