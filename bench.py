@@ -140,14 +140,14 @@ def algorithmic_bytes(plan, layers, seq_len, n_seq):
 
 
 # ---------------------------------------------------------------------------- our arm
-def build_decode_setup(torch, w, rank):
+def build_decode_setup(torch, w, rank, k_only=False):
     """Calibrate, allocate the cache, prefill 131071 tokens of every layer (encode path),
     and prepare the step's inputs.  Returns a dict of state."""
     t0 = time.time()
     k_cal, v_cal, q_cal = synth.calibration_set(w)
     plan = kvtc.kvtc_calibrate(k_cal, v_cal, q_cal, n_layers=w.n_layers, n_kv_heads=w.n_kv_heads,
                                group=w.group, bpd=w.bpd, seed=w.seed, fixed_r=w.fixed_r,
-                               fixed_b=w.fixed_b).upload()
+                               fixed_b=w.fixed_b, k_only=k_only).upload()
     t_cal = time.time() - t0
     H, G, L, T, B = w.n_kv_heads, w.group, w.n_layers, w.seq_len, w.batch
     pages = (T + 127) // 128
@@ -340,7 +340,7 @@ def run_ours(args, torch, dist, rank, world):
     if args.no_decode:
         return {"encode": encode_bench(torch, synth.WORKLOADS[ENCODE_WORKLOAD], max(1, min(args.steps, 5)),
                                        args.warmup, rank, args.encode_layers)}
-    st = build_decode_setup(torch, w, rank)
+    st = build_decode_setup(torch, w, rank, k_only=args.k_only)
     plan = st["plan"]
     stream = torch.cuda.Stream()
     L = w.n_layers
@@ -428,13 +428,13 @@ def run_ours(args, torch, dist, rank, world):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "layers": L, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
                    "head_dim": 128, "batch": w.batch, "seq_len": w.seq_len, "bpd": w.bpd,
-                   "parallelism": f"replicas x{world}",
+                   "parallelism": f"replicas x{world}", "k_only": bool(args.k_only),
                    "step": f"per layer: append 1 token + decode attention; {L} layers in one CUDA graph",
                    "l2": f"inputs larger than L2: {step_bytes / 1e9:.3f} GB of codes+bases per step vs 126 MB",
                    "compute": "fp16 tensor-core operands (codes exact, q split hi+lo), fp32 accumulation"},
         "pct_of_peak": round(100 * value / world / hbm_peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": DECODE_TRAFFIC.get(w.name),
+                     "frac": round(achieved / hbm_peak, 4), "traffic": None if args.k_only else DECODE_TRAFFIC.get(w.name),
                      "kernel": "decode call of one layer (q~ prep + split kernel + combine)", "peak_kind": peak_kind,
                      "bytes_per_launch": step_bytes // L, "launch_ms": round(dec_ms, 5)},
         "e2e": {"value": round(aggregate_value(world, step_bytes, e2e_ms), 2), "unit": "GB/s",
@@ -618,6 +618,8 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="limit the decode workload's layers (profiling)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the decode workload's context (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--k-only", action="store_true",
+                    help="keys-only plan: keys coded at the budget, values stored as fp16")
     ap.add_argument("--no-sdpa", action="store_true", help="skip the fp16 SDPA context timing")
     ap.add_argument("--efficiency", action="store_true",
                     help="only the project page's Efficiency table (fixed r, b vs fp16 SDPA, 32k-128k)")

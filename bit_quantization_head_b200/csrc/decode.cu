@@ -150,8 +150,11 @@ __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(const __gr
   const int Hq = ca.H * ca.G, h = qh / ca.G;
   const UnitDesc dV = ca.units[(ca.layer * ca.H + h) * 2 + 1];
   const int rV = dV.r;
+  // an uncompressed value unit (keys-only plans) is already in d-space: its latent is
+  // the output (identity back-projection), its codes are v * 2^24, with no centring
+  const bool raw = dV.b == kRawBits;
   // the plan's M_V is not written by the preceding kernels: load it before the wait
-  for (int i = tid; i < rV * (kCombCols / 4); i += kCombThreads) {
+  for (int i = tid; !raw && i < rV * (kCombCols / 4); i += kCombThreads) {
     const int j = i / (kCombCols / 4), c4 = i % (kCombCols / 4);
     reinterpret_cast<float4*>(Ms[j])[c4] =
         reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD + cb * kCombCols)[c4];
@@ -190,22 +193,23 @@ __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(const __gr
   float L = 0.0f;
 #pragma unroll
   for (int w = 0; w < kCombWarps; ++w) L += lsh[w];
-  const float mV = 0.5f * static_cast<float>((1 << dV.b) - 1);
+  const float mV = raw ? 0.0f : 0.5f * static_cast<float>((1 << dV.b) - 1);
+  const float dlt = raw ? 0x1p-24f : dV.delta;
   for (int j = tid; j < rV; j += kCombThreads) {
     float zs = 0.0f;
 #pragma unroll
     for (int w = 0; w < kCombWarps; ++w) zs += zsh[w][j];
     // z holds sum p*c*2^-17 (uncentered codes); center and dequantize
-    y[j] = L > 0.0f ? dV.delta * (ldexpf(zs, 17) - mV * L) / L : 0.0f;
+    y[j] = L > 0.0f ? dlt * (ldexpf(zs, 17) - mV * L) / L : 0.0f;
   }
   __syncthreads();
   // o[k] = sum_j M_V[j][k] y[j] for this CTA's 32 columns: warp w takes j = w, w + 4, ...
   float o = 0.0f;
-  for (int j = warp; j < rV; j += kCombWarps) o = fmaf(Ms[j][lane], y[j], o);
+  for (int j = warp; !raw && j < rV; j += kCombWarps) o = fmaf(Ms[j][lane], y[j], o);
   osh[warp][lane] = o;
   __syncthreads();
   if (warp == 0) {
-    const float v = (osh[0][lane] + osh[1][lane]) + (osh[2][lane] + osh[3][lane]);
+    const float v = raw ? y[cb * kCombCols + lane] : (osh[0][lane] + osh[1][lane]) + (osh[2][lane] + osh[3][lane]);
     const size_t off = (static_cast<size_t>(s) * Hq + qh) * kD + cb * kCombCols + lane;
     if (ca.out_bf16)
       static_cast<__nv_bfloat16*>(ca.out)[off] = __float2bfloat16_rn(v);
@@ -215,8 +219,8 @@ __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(const __gr
 }
 
 // Width class of a code: 2, 4 and 8 have specialised extraction; others share the
-// run-time path (class 0).
-int width_class(int b) { return (b == 2 || b == 4 || b == 8) ? b : 0; }
+// run-time path (class 0); kRawBits marks an uncompressed value unit.
+int width_class(int b) { return (b == 2 || b == 4 || b == 8 || b == kRawBits) ? b : 0; }
 
 // Cost model of one page for the split allocation (warp instructions per page and warp:
 // softmax, bookkeeping and the per-16-coordinate MMA rows).
@@ -355,7 +359,7 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
   double layer_cost = 0.0;
   for (int h = 0; h < plan->H; ++h) {
     const int uK = (layer * plan->H + h) * 2;
-    groups[width_class(plan->b[uK]) * 16 + width_class(plan->b[uK + 1])].push_back(h);
+    groups[width_class(plan->b[uK]) * 32 + width_class(plan->b[uK + 1])].push_back(h);
     head_bytes_pp[h] = 16.0 * (plan->r[uK] * plan->b[uK] + plan->r[uK + 1] * plan->b[uK + 1]);
     head_cost[h] = kPageCost + kTileCost * ((plan->r[uK] + 15) / 16 + (plan->r[uK + 1] + 15) / 16);
     layer_cost += head_cost[h];
@@ -375,7 +379,7 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
   const size_t head_bytes = ((sizeof(SmemHead) + 8 * kWarps * 8 + 127) / 128) * 128;
   bool first = true;
   for (auto& kv : groups) {
-    const int wk = kv.first >> 4, wv = kv.first & 15;
+    const int wk = kv.first >> 5, wv = kv.first & 31;
     const std::vector<int>& hs = kv.second;
     uint32_t stage_bytes = 0;
     double group_cost = 0.0;

@@ -203,6 +203,7 @@ struct WS {
   // fragments of its ones row by block parity (a0, a2; nonzero in lanes g == 0 only)
   float zl[4];
   uint32_t onesA[2][2];
+  int rsw;  // uncompressed value pages: swizzle of this lane's word positions (tq ^ 4 g)
   float z[kNT][4];
   float z2[kZSplit ? kNT : 1][4];  // odd blocks (kZSplit)
   float zl2[4];
@@ -361,6 +362,20 @@ __device__ __forceinline__ void v_block(const WS<BK, BV, PACK>& w, uint32_t W0, 
   mma_16816(z, A0, A1, A2, A3, bp[0], bp[1]);
 }
 
+// Value MMA of one block for an uncompressed value unit (keys-only plans).  Word of
+// coordinate j and token pair k: j * 64 + (k XOR 4 (j mod 8)); the block's pairs are
+// k0 = 8 BLK + tq (a0, a1) and k0 + 4 (a2, a3), and since j mod 8 = g for both rows the
+// positions are (8 BLK) XOR rsw and (8 BLK + 4) XOR rsw with rsw = tq XOR 4 g.  A is
+// the fp16 value v itself, P carries 2^7 (e_V = 0), so z accumulates 2^-17 * (v 2^24) p.
+template <int BK, int BV, bool PACK, int BLK>
+__device__ __forceinline__ void raw_v_block(const WS<BK, BV, PACK>& w, const uint32_t* row0, const uint32_t (&bp)[2],
+                                            float (&z)[4]) {
+  const int c0 = (8 * BLK) ^ w.rsw, c1 = (8 * BLK + 4) ^ w.rsw;
+  const uint32_t A0 = row0[c0], A1 = row0[8 * (kPage / 2) + c0];
+  const uint32_t A2 = row0[c1], A3 = row0[8 * (kPage / 2) + c1];
+  mma_16816(z, A0, A1, A2, A3, bp[0], bp[1]);
+}
+
 // Blocks B0 .. B0 + IL - 1 of the page: scores, lazy online softmax, value accumulation.
 template <int BK, int BV, bool PACK, int B0, int... BB>
 __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_sequence<int, BB...>) {
@@ -506,6 +521,14 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
   // entered by a jump)
   auto vtile = [&](auto MTC) {
     constexpr int mt = decltype(MTC)::value;
+    if constexpr (BV == kRawBits) {
+      // uncompressed values: each A register is one stored word (a token pair of one
+      // coordinate, fp16 as stored); rows 16 mt + g and + 8 of the raw page
+      const uint32_t* row0 = w.pv + (16 * mt + w.g) * (kPage / 2);
+      (raw_v_block<BK, BV, PACK, B0 + BB>(w, row0, bp[BB], (kZSplit && ((B0 + BB) & 1)) ? w.z2[mt] : w.z[mt]),
+       ...);
+      return;
+    }
     const int j0 = 16 * mt + w.g, j1 = j0 + 8;
     const bool ones = !PACK && mt == w.ones_mt;
     uint32_t W0[VWN], W1[VWN], W0h[VWN], W1h[VWN];
@@ -679,6 +702,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   w.nmt = (rV + 15) >> 4;
   w.g = g;
   w.tq = tq;
+  w.rsw = tq ^ (g << 2);
   w.seq_len = seq_len;
   w.partial = false;
   w.partsK = parts_of(dK.b);

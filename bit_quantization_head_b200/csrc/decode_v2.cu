@@ -1,4 +1,5 @@
-// Instantiations of the decode split kernel for key code width class 2 (0 = any width).
+// Instantiations of the decode split kernel for key code width class 2 (0 = any width);
+// value width 16 = uncompressed values.
 #include "decode_kernel.cuh"
 
 namespace kvtc {
@@ -13,6 +14,8 @@ SplitFn split_fn_bk<2>(int bV, bool pack) {
   if (bV == 8 && pack == false) return decode_split_kernel<2, 8, false>;
   if (bV == 0 && pack == true) return decode_split_kernel<2, 0, true>;
   if (bV == 0 && pack == false) return decode_split_kernel<2, 0, false>;
+  if (bV == 16 && pack == true) return decode_split_kernel<2, 16, true>;
+  if (bV == 16 && pack == false) return decode_split_kernel<2, 16, false>;
   return nullptr;
 }
 }  // namespace dec

@@ -7,6 +7,7 @@
 // the oracle reproduces bit for bit), quantizes it and merges its bits into the page
 // word.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "kvtc_internal.h"
@@ -68,7 +69,8 @@ __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constan
   // the producer of k/v (programmatic dependent launch), so the loads overlap its tail.
   const UnitDesc ud = a.units[u];
   uint4 mr[16];
-  if (a.bf16 && j < ud.r) {
+  const bool raw = ud.b == kRawBits;  // uncompressed value unit (keys-only plans)
+  if (a.bf16 && j < ud.r && !raw) {
     const uint4* m4 = reinterpret_cast<const uint4*>(ud.Mbf + static_cast<size_t>(j) * kD);
 #pragma unroll
     for (int c = 0; c < 16; ++c) mr[c] = m4[c];
@@ -86,37 +88,42 @@ __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constan
   __syncthreads();
   if (j >= ud.r) return;
 
-  // canonical projection: eight chains a_e = fma(x_k, M_jk, a_e) over k = e (mod 8)
-  // ascending, then ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7))
-  float ch[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
-  if (a.bf16) {
+  uint32_t code = 0;
+  if (raw) {
+    code = __half_as_ushort(__float2half_rn(xs[j]));
+  } else {
+    // canonical projection: eight chains a_e = fma(x_k, M_jk, a_e) over k = e (mod 8)
+    // ascending, then ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7))
+    float ch[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    if (a.bf16) {
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const uint32_t w[4] = {mr[c].x, mr[c].y, mr[c].z, mr[c].w};
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t w[4] = {mr[c].x, mr[c].y, mr[c].z, mr[c].w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        ch[2 * q] = __fmaf_rn(xs[8 * c + 2 * q], __uint_as_float(w[q] << 16), ch[2 * q]);
-        ch[2 * q + 1] = __fmaf_rn(xs[8 * c + 2 * q + 1], __uint_as_float(w[q] & 0xFFFF0000u), ch[2 * q + 1]);
+        for (int q = 0; q < 4; ++q) {
+          ch[2 * q] = __fmaf_rn(xs[8 * c + 2 * q], __uint_as_float(w[q] << 16), ch[2 * q]);
+          ch[2 * q + 1] = __fmaf_rn(xs[8 * c + 2 * q + 1], __uint_as_float(w[q] & 0xFFFF0000u), ch[2 * q + 1]);
+        }
+      }
+    } else {
+      const float4* m4 = reinterpret_cast<const float4*>(ud.M + static_cast<size_t>(j) * kD);
+#pragma unroll 4
+      for (int c = 0; c < 16; ++c) {
+        const float4 m0 = m4[2 * c], m1 = m4[2 * c + 1];
+        ch[0] = __fmaf_rn(xs[8 * c], m0.x, ch[0]);
+        ch[1] = __fmaf_rn(xs[8 * c + 1], m0.y, ch[1]);
+        ch[2] = __fmaf_rn(xs[8 * c + 2], m0.z, ch[2]);
+        ch[3] = __fmaf_rn(xs[8 * c + 3], m0.w, ch[3]);
+        ch[4] = __fmaf_rn(xs[8 * c + 4], m1.x, ch[4]);
+        ch[5] = __fmaf_rn(xs[8 * c + 5], m1.y, ch[5]);
+        ch[6] = __fmaf_rn(xs[8 * c + 6], m1.z, ch[6]);
+        ch[7] = __fmaf_rn(xs[8 * c + 7], m1.w, ch[7]);
       }
     }
-  } else {
-    const float4* m4 = reinterpret_cast<const float4*>(ud.M + static_cast<size_t>(j) * kD);
-#pragma unroll 4
-    for (int c = 0; c < 16; ++c) {
-      const float4 m0 = m4[2 * c], m1 = m4[2 * c + 1];
-      ch[0] = __fmaf_rn(xs[8 * c], m0.x, ch[0]);
-      ch[1] = __fmaf_rn(xs[8 * c + 1], m0.y, ch[1]);
-      ch[2] = __fmaf_rn(xs[8 * c + 2], m0.z, ch[2]);
-      ch[3] = __fmaf_rn(xs[8 * c + 3], m0.w, ch[3]);
-      ch[4] = __fmaf_rn(xs[8 * c + 4], m1.x, ch[4]);
-      ch[5] = __fmaf_rn(xs[8 * c + 5], m1.y, ch[5]);
-      ch[6] = __fmaf_rn(xs[8 * c + 6], m1.z, ch[6]);
-      ch[7] = __fmaf_rn(xs[8 * c + 7], m1.w, ch[7]);
-    }
+    const float acc = __fadd_rn(__fadd_rn(__fadd_rn(ch[0], ch[1]), __fadd_rn(ch[2], ch[3])),
+                                __fadd_rn(__fadd_rn(ch[4], ch[5]), __fadd_rn(ch[6], ch[7])));
+    code = quantize_code(acc, ud.inv_delta, ud.b);
   }
-  const float acc = __fadd_rn(__fadd_rn(__fadd_rn(ch[0], ch[1]), __fadd_rn(ch[2], ch[3])),
-                              __fadd_rn(__fadd_rn(ch[4], ch[5]), __fadd_rn(ch[6], ch[7])));
-  const uint32_t code = quantize_code(acc, ud.inv_delta, ud.b);
 
   // token -> (sequence, position) -> page
   int lo = 0, hi = a.n_seq - 1;
@@ -142,6 +149,13 @@ __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constan
   }
   uint32_t* page = reinterpret_cast<uint32_t*>(a.pool + a.pages_per_unit * ud.prefix +
                                                static_cast<uint64_t>(pid) * ud.page_bytes);
+  if (raw) {
+    // raw page: row j of 64 words, token pair slot / 2 at position (slot / 2) XOR 4 (j % 8),
+    // the even token in the low half
+    const int word = j * (kPage / 2) + ((slot >> 1) ^ ((j & 7) << 2));
+    reinterpret_cast<uint16_t*>(page)[2 * word + (slot & 1)] = static_cast<uint16_t>(code);
+    return;
+  }
   store_code(page, kind, ud.r, ud.b, slot, j, code);
 }
 

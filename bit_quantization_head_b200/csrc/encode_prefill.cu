@@ -749,6 +749,9 @@ extern "C" kvtc_status kvtc_encode_prefill(const kvtc_plan* plan, const kvtc_cac
   if (st != KVTC_OK) return st;
   if (!cache || !cache->pool || !cache->block_table) return fail(KVTC_EINVAL, "cache is incomplete");
   if (layer < 0 || layer >= plan->L) return fail(KVTC_EINVAL, "layer out of range");
+  for (int u = layer * plan->H * 2; u < (layer + 1) * plan->H * 2; ++u)
+    if (plan->b[u] == kRawBits)
+      return fail(KVTC_EINVAL, "prefill encodes compressed units only; use kvtc_encode_append for keys-only plans");
   if (seq < 0 || seq >= cache->n_seq) return fail(KVTC_EINVAL, "seq out of range");
   if (pos_start < 0 || (pos_start % kPage) != 0) return fail(KVTC_EINVAL, "pos_start must be a multiple of 128");
   if (n_tok <= 0) return fail(KVTC_EINVAL, "n_tok must be > 0");

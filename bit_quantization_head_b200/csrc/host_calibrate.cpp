@@ -417,19 +417,33 @@ extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* 
   double mu = 0.0;
   if (desc->c2_mode != KVTC_C2_LAGRANGE && desc->c2_mode != KVTC_C2_DAMPED)
     return fail(KVTC_EINVAL, "c2_mode must be KVTC_C2_LAGRANGE or KVTC_C2_DAMPED");
+  // The allocation pool: every unit, or the key units alone in keys-only mode (value
+  // units are then stored uncompressed: r = d, b = kRawBits).
+  if (desc->k_only != 0 && desc->k_only != 1) return fail(KVTC_EINVAL, "k_only must be 0 or 1");
+  std::vector<int> pool;
+  for (int u = 0; u < U; ++u)
+    if (!(desc->k_only && (u & 1))) pool.push_back(u);
+  const int P = static_cast<int>(pool.size());
+  std::vector<int> Rp(P), Bp(P);
   if (fixed) {
-    std::fill(R.begin(), R.end(), desc->fixed_r);
-    std::fill(B.begin(), B.end(), desc->fixed_b);
+    std::fill(Rp.begin(), Rp.end(), desc->fixed_r);
+    std::fill(Bp.begin(), Bp.end(), desc->fixed_b);
   } else {
-    const long long total = std::llround(desc->bpd * d * U);
-    if (4ll * U > total) return fail(KVTC_EINFEASIBLE, "budget below 4 bits per unit");
-    std::vector<std::vector<double>> ws(U);
-    for (int u = 0; u < U; ++u) ws[u] = work[u].w;
+    const long long total = std::llround(desc->bpd * d * P);
+    if (4ll * P > total) return fail(KVTC_EINFEASIBLE, "budget below 4 bits per unit");
+    std::vector<std::vector<double>> ws(P);
+    for (int i = 0; i < P; ++i) ws[i] = work[pool[i]].w;
     if (desc->c2_mode == KVTC_C2_DAMPED) {
-      c2_damped(ws, total, R, B);
-    } else if (!c2(ws, total, R, B, mu)) {
+      c2_damped(ws, total, Rp, Bp);
+    } else if (!c2(ws, total, Rp, Bp, mu)) {
       return fail(KVTC_EINFEASIBLE, "no allocation meets the budget");
     }
+  }
+  std::fill(R.begin(), R.end(), d);
+  std::fill(B.begin(), B.end(), kRawBits);
+  for (int i = 0; i < P; ++i) {
+    R[pool[i]] = Rp[i];
+    B[pool[i]] = Bp[i];
   }
 
   std::unique_ptr<kvtc_plan> p(new (std::nothrow) kvtc_plan());
@@ -445,6 +459,20 @@ extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* 
   for (int u = 0; u < U; ++u) {
     const int r = R[u], b = B[u];
     const UnitWork& wk = work[u];
+    if (b == kRawBits) {  // uncompressed value unit: identity basis, c = v * 2^24
+      std::vector<float> M(static_cast<size_t>(d) * d, 0.0f);
+      for (int i = 0; i < d; ++i) M[static_cast<size_t>(i) * d + i] = 1.0f;
+      p->r.push_back(d);
+      p->b.push_back(b);
+      p->delta.push_back(std::ldexp(1.0, -24));
+      p->inv_delta.push_back(std::ldexp(1.0f, 24));
+      p->sigma.push_back(0.0);
+      p->D.push_back(0.0);
+      p->M.push_back(std::move(M));
+      p->w.push_back(wk.w);
+      p->lam.push_back(wk.lam);
+      continue;
+    }
     double mean = 0.0;
     for (int i = 0; i < r; ++i) mean += wk.lam[i];
     mean /= r;

@@ -81,8 +81,8 @@ kvtc_status kvtc_plan_create(int n_layers, int n_kv_heads, int group, int head_d
   p->U = 2 * n_layers * n_kv_heads;
   size_t off = 0;
   for (int u = 0; u < p->U; ++u) {
-    if (r[u] < 2 || r[u] > kD || (r[u] & 1)) return fail(KVTC_EINVAL, "r must be even in [2,128]");
-    if (b[u] < 2 || b[u] > 8) return fail(KVTC_EINVAL, "b must be in [2,8]");
+    if (!valid_rb(r[u], b[u], u & 1))
+      return fail(KVTC_EINVAL, "r must be even in [2,128] and b in [2,8] (or a raw value unit: r = 128, b = 16)");
     if (!(delta[u] > 0.0) || !std::isfinite(delta[u])) return fail(KVTC_EINVAL, "delta must be > 0");
     p->r.push_back(r[u]);
     p->b.push_back(b[u]);
@@ -231,7 +231,7 @@ kvtc_status kvtc_plan_load(const char* path, kvtc_plan** out) {
     get(&inv, 4);
     get(&sigma, 8);
     get(&D, 8);
-    if (!ok || r < 2 || r > kD || (r & 1) || b < 2 || b > 8) return fail(KVTC_EIO, "corrupt unit");
+    if (!ok || !valid_rb(r, b, static_cast<int>(p->r.size()) & 1)) return fail(KVTC_EIO, "corrupt unit");
     p->r.push_back(r);
     p->b.push_back(b);
     p->delta.push_back(delta);

@@ -11,11 +11,19 @@ namespace kvtc {
 
 constexpr int kPage = KVTC_PAGE_TOKENS;
 constexpr int kD = KVTC_HEAD_DIM;
+constexpr int kRawBits = KVTC_RAW_BITS;
+
+// A unit's (r, b) is valid when r is even in [2, d] and b in [2, 8], or when it is an
+// uncompressed value unit (kind 1): r = d, b = kRawBits.
+inline bool valid_rb(int r, int b, int kind) {
+  if (kind == 1 && r == kD && b == kRawBits) return true;
+  return r >= 2 && r <= kD && (r & 1) == 0 && b >= 2 && b <= 8;
+}
 
 // Per-unit parameters as the kernels read them (device array, one per unit).
 struct UnitDesc {
   int r;               // retained coordinates (even, 2..128)
-  int b;               // bits per code (2..8)
+  int b;               // bits per code (2..8), or kRawBits (uncompressed value unit)
   float delta;         // quantizer step
   float inv_delta;     // fp32(1/delta)
   uint64_t page_bytes; // 16 * r * b

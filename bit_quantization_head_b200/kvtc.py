@@ -22,6 +22,7 @@ KVTC_F32, KVTC_BF16 = 0, 1
 KIND_K, KIND_V = 0, 1
 WEIGHTS_KL, WEIGHTS_MSE = 0, 1
 C2_LAGRANGE, C2_DAMPED = 0, 1
+RAW_BITS = 16  # b of an uncompressed value unit (keys-only plans)
 STATUS_BAD_PAGE, STATUS_BAD_POS, STATUS_TIMEOUT = 1, 2, 4
 PAGE_TOKENS = 128
 HEAD_DIM = 128
@@ -38,7 +39,8 @@ class KvtcError(RuntimeError):
 class CalibDesc(C.Structure):
     _fields_ = [("n_layers", C.c_int), ("n_kv_heads", C.c_int), ("group", C.c_int), ("head_dim", C.c_int),
                 ("n_cal", C.c_int), ("bpd", C.c_double), ("weight_mode", C.c_int), ("fixed_r", C.c_int),
-                ("fixed_b", C.c_int), ("seed", C.c_uint64), ("c2_mode", C.c_int)]
+                ("fixed_b", C.c_int), ("seed", C.c_uint64), ("c2_mode", C.c_int),
+                ("k_only", C.c_int)]
 
 
 class UnitInfo(C.Structure):
@@ -194,8 +196,9 @@ class Plan:
 
 
 def kvtc_calibrate(k_cal, v_cal, q_cal, *, n_layers, n_kv_heads, group, bpd=1.0, seed=0,
-                   weight_mode=WEIGHTS_KL, fixed_r=0, fixed_b=0, c2_mode=C2_LAGRANGE):
-    """Host arrays: k_cal, v_cal fp32 [L][H][N][d]; q_cal fp32 [L][H][G][N][d] (or None)."""
+                   weight_mode=WEIGHTS_KL, fixed_r=0, fixed_b=0, c2_mode=C2_LAGRANGE, k_only=False):
+    """Host arrays: k_cal, v_cal fp32 [L][H][N][d]; q_cal fp32 [L][H][G][N][d] (or None).
+    k_only: keys-only plan (value units uncompressed, b = RAW_BITS)."""
     k_cal = np.ascontiguousarray(k_cal, np.float32)
     v_cal = np.ascontiguousarray(v_cal, np.float32)
     qp = None
@@ -203,7 +206,7 @@ def kvtc_calibrate(k_cal, v_cal, q_cal, *, n_layers, n_kv_heads, group, bpd=1.0,
         q_cal = np.ascontiguousarray(q_cal, np.float32)
         qp = _host_ptr(q_cal, np.float32)
     d = CalibDesc(n_layers, n_kv_heads, group, k_cal.shape[-1], k_cal.shape[-2], float(bpd), weight_mode,
-                  fixed_r, fixed_b, seed, c2_mode)
+                  fixed_r, fixed_b, seed, c2_mode, 1 if k_only else 0)
     out = _P()
     _check(lib().kvtc_calibrate(C.byref(d), _host_ptr(k_cal, np.float32), _host_ptr(v_cal, np.float32), qp,
                                 C.byref(out)))

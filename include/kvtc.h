@@ -60,6 +60,14 @@ typedef enum { KVTC_WEIGHTS_KL = 0, KVTC_WEIGHTS_MSE = 1 } kvtc_weight_mode;
  * rounds; "C2, across heads"). */
 typedef enum { KVTC_C2_LAGRANGE = 0, KVTC_C2_DAMPED = 1 } kvtc_c2_mode;
 
+/* b of an uncompressed value unit (keys-only mode, kvtc_calib_desc.k_only): r = d = 128
+ * and every value is stored as fp16 (round to nearest even).  Its page (128 tokens,
+ * 32768 bytes = 16 * r * b like every page) has one row of 64 little-endian 32-bit words
+ * per coordinate j; the word of token pair k (tokens 2k in the low half, 2k + 1 in the
+ * high half) sits at position k XOR 4 (j mod 8) of row j.  The decode reads such a unit
+ * as the integer code c = v * 2^24 with delta = 2^-24 and no centring. */
+#define KVTC_RAW_BITS 16
+
 /* Bits of the device status word. */
 #define KVTC_STATUS_BAD_PAGE 1u      /* block table entry outside [0, pages_per_unit)  */
 #define KVTC_STATUS_BAD_POS 2u       /* position or length beyond max_pages * 128      */
@@ -87,6 +95,9 @@ typedef struct {
   int fixed_b;         /*   fixed_b) and no allocation runs                           */
   uint64_t seed;       /* seed of the random Hadamard signs (splitmix64)              */
   int c2_mode;         /* KVTC_C2_LAGRANGE (default) or KVTC_C2_DAMPED                */
+  int k_only;          /* 1: keys-only ("k-only" results): the allocation covers the  */
+                       /*   key units alone (bpd * d bits per key unit and token) and */
+                       /*   every value unit is stored uncompressed (KVTC_RAW_BITS)   */
 } kvtc_calib_desc;
 
 /*
@@ -105,8 +116,10 @@ typedef struct {
  * k_cal, v_cal: host fp32 [L][H_kv][n_cal][d].  q_cal: host fp32 [L][H_kv][G][n_cal][d]
  * (may be NULL in MSE mode).  Borrowed for the call.  *out receives a new plan
  * (free with kvtc_plan_destroy).  Deterministic for the same inputs and seed; uses
- * host threads.  Errors: EINVAL (shapes, d != 128, fixed_r odd or out of [2,d],
- * fixed_b outside [2,8]), EINFEASIBLE (budget < 4 bits per unit), ENOMEM.
+ * host threads.  With k_only, fixed_r/fixed_b and the budget apply to the key units
+ * only and each value unit gets r = d, b = KVTC_RAW_BITS, M = identity, delta = 2^-24.
+ * Errors: EINVAL (shapes, d != 128, fixed_r odd or out of [2,d], fixed_b outside
+ * [2,8]), EINFEASIBLE (budget < 4 bits per unit), ENOMEM.
  */
 kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* k_cal, const float* v_cal,
                            const float* q_cal, kvtc_plan** out);
@@ -115,6 +128,8 @@ kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* k_cal, cons
  * kvtc_plan_create -- a plan from explicit per-unit parameters (a plan computed
  * elsewhere).  r, b: host [U]; delta: host [U] (step; inv_delta = fp32(1/delta));
  * M: host fp32, the U matrices [r_u][d] concatenated in unit order.  U = 2*L*H_kv.
+ * A value unit may be uncompressed (r = 128, b = KVTC_RAW_BITS; its M and delta are
+ * then not used by the kernels).
  */
 kvtc_status kvtc_plan_create(int n_layers, int n_kv_heads, int group, int head_dim,
                              const int* r, const int* b, const double* delta, const float* M,
@@ -214,7 +229,8 @@ uint64_t kvtc_unit_pool_offset(const kvtc_plan* plan, int unit, uint64_t pages_p
  * sequence's first new token.  The slots written are overwritten (their old bits are
  * cleared, other tokens sharing a 32-bit word are kept).  Positions beyond
  * max_pages * 128 or page ids outside the pool set status bits and are skipped.
- * Calls that write the same slot and overlap on the GPU race.
+ * Calls that write the same slot and overlap on the GPU race.  An uncompressed value unit
+ * (KVTC_RAW_BITS) receives fp16(v) (round to nearest even) in its raw page layout.
  */
 kvtc_status kvtc_encode_append(const kvtc_plan* plan, const kvtc_cache* cache, int layer,
                                const void* k, const void* v, kvtc_dtype dtype,
@@ -227,7 +243,8 @@ kvtc_status kvtc_encode_append(const kvtc_plan* plan, const kvtc_cache* cache, i
  * (tcgen05, TMEM accumulators) whose epilogue quantizes and packs whole pages.  Any
  * coordinate whose tensor-core sum lies within the fp32 accumulation-error bound of a
  * quantizer threshold is recomputed in the canonical order, so the codes equal the
- * canonical ones bit for bit.  bf16 input only.
+ * canonical ones bit for bit.  bf16 input only.  Plans with uncompressed value units
+ * (keys-only) are not handled here (EINVAL): use kvtc_encode_append.
  * seq: sequence index; pos_start: host, multiple of 128; n_tok: host, > 0 (a trailing
  * partial page is written with the same merge rule as append).  k, v: device
  * [n_tok][H_kv][d] bf16.
@@ -259,7 +276,9 @@ uint64_t kvtc_decode_workspace_bytes(const kvtc_plan* plan, int n_seq, int max_s
  *   o = M_V^T (delta_V * z).
  * Equivalent to softmax(scale * q . k_hat_t) v_hat_t with k_hat = M_K^T delta_K (c - m)
  * (the oracle's d-space form).  Split-K over the context with a log-sum-exp merge;
- * the G query heads of a KV head share every code tile.
+ * the G query heads of a KV head share every code tile.  An uncompressed value unit
+ * (keys-only plans) enters the value MMAs with its fp16 values as they are stored
+ * (c_V = v * 2^24, delta_V = 2^-24, m_V = 0, M_V = identity), so o = sum_t p_t v_t.
  * q: device [n_seq][H_q][d] of q_dtype.  seq_lens: device int32 [n_seq] (0 gives an
  * all-zero output).  max_seq_len: host upper bound of seq_lens (sizes the split grid;
  * longer sequences set KVTC_STATUS_BAD_POS).  softmax_scale: 0 means 1/sqrt(d).

@@ -21,12 +21,16 @@ from __future__ import annotations
 
 import numpy as np
 
-from .codec import dequantize
+from .codec import RAW_BITS, dequantize
 
 
 def reconstruct(codes, M, delta, b):
-    """x_hat [T, d] = dequantize(codes) @ M in fp64 (M: [r, d] as stored in the plan)."""
+    """x_hat [T, d] = dequantize(codes) @ M in fp64 (M: [r, d] as stored in the plan).
+    An uncompressed unit (b = RAW_BITS, keys-only plans) is stored in d-space: x_hat is
+    its fp16 values, whatever M and delta the plan carries."""
     y = dequantize(codes, delta, b)
+    if b == RAW_BITS:
+        return y
     return y @ np.asarray(M, dtype=np.float64)
 
 

@@ -149,6 +149,10 @@ def random_plan(n_layers, H, G, rb_pairs, rng):
             Q, _ = np.linalg.qr(rng.standard_normal((128, 128)))
             r.append(rr)
             b.append(bb)
+            if bb == kvtc.RAW_BITS:  # uncompressed value unit: identity, c = v * 2^24
+                delta.append(2.0 ** -24)
+                M.append(np.eye(128, dtype=np.float32))
+                continue
             delta.append(float(rng.uniform(0.05, 0.3)) * 2.0 ** (2 - bb))
             M.append(Q[:rr].astype(np.float32))
     return kvtc.kvtc_plan_create(n_layers, H, G, r, b, delta, M).upload()

@@ -92,6 +92,45 @@ def test_every_code_width_ragged_sequences_and_chunked_appends(dtype):
     _check_decode(plan, cache, 0, q, lens, H, G, dtype)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_keys_only_raw_values_codes_and_attention(dtype):
+    # keys-only plans: coded keys of several widths, values stored as fp16 (raw pages);
+    # packed (G = 4) and unpacked (G = 6) query groups
+    rng = np.random.default_rng(12)
+    for G in (4, 6):
+        pairs = [((16, 2), (128, 16)), ((34, 3), (128, 16)), ((64, 4), (128, 16)), ((8, 8), (128, 16))]
+        H = len(pairs)
+        plan = gh.random_plan(1, H, G, pairs, rng)
+        lens = [777, 130, 0]
+        cache = gh.make_cache(plan, lens, rng)
+        kv = []
+        for T in lens:
+            K = (rng.standard_normal((T, H, 128)) * rng.uniform(0.3, 3.0, (1, H, 1))).astype(np.float32)
+            V = (rng.standard_normal((T, H, 128)) * rng.uniform(0.3, 3.0, (1, H, 1))).astype(np.float32)
+            kv.append((synth.round_dtype(K, dtype), synth.round_dtype(V, dtype)))
+        gh.encode_all(plan, cache, 0, kv, dtype, chunk=200)
+        assert gh.check_encode(plan, cache, 0, kv, dtype, H) == 0
+        q = synth.round_dtype((rng.standard_normal((len(lens), H * G, 128)) * 0.7).astype(np.float32), dtype)
+        _check_decode(plan, cache, 0, q, lens, H, G, dtype)
+
+
+def test_keys_only_calibrated_llama_layer():
+    w = synth.WORKLOADS["llama8b-layer-32k-2bpd"]
+    k, v, q = synth.calibration_set(w)
+    plan = kvtc.kvtc_calibrate(k, v, q, n_layers=1, n_kv_heads=w.n_kv_heads, group=w.group, bpd=w.bpd,
+                               seed=w.seed, k_only=True).upload()
+    rng = np.random.default_rng(13)
+    T = 5000
+    cache = gh.make_cache(plan, [T], rng)
+    K, V = _kv(w, 0, T)
+    gh.encode_all(plan, cache, 0, [(K, V)], "bf16")
+    assert gh.check_encode(plan, cache, 0, [(K, V)], "bf16", w.n_kv_heads) == 0
+    with pytest.raises(kvtc.KvtcError):   # prefill encodes compressed units only
+        kvtc.kvtc_encode_prefill(plan, cache, 0, gh.to_dev(K, "bf16"), gh.to_dev(V, "bf16"), 0, 0)
+    q = synth.decode_queries(w, 0)[None]
+    _check_decode(plan, cache, 0, q, [T], w.n_kv_heads, w.group, "bf16")
+
+
 def test_query_groups_larger_than_eight_and_peaked_attention():
     rng = np.random.default_rng(3)
     H, G = 2, 12

@@ -86,6 +86,30 @@ def test_calibrate_damped_c2_matches_oracle_and_sits_between_bounds():
     assert D_lagrange <= D_damped <= D_equal
 
 
+def test_calibrate_keys_only_matches_oracle():
+    # keys-only ("k-only" results): the allocation covers the key units, values raw
+    w = synth.scaled(synth.WORKLOADS["llama8b-32L-128k-1bpd"], n_layers=2, n_cal=256)
+    k, v, q = synth.calibration_set(w)
+    plan = kvtc.kvtc_calibrate(k, v, q, n_layers=2, n_kv_heads=8, group=4, bpd=1.0, seed=w.seed, k_only=True)
+    units = ocal.calibrate(k, v, q, 2, 8, bpd=1.0, seed=w.seed, k_only=True)
+    _compare_plans(plan, units)
+    for u in range(1, 32, 2):
+        info = plan.unit(u)
+        assert (info["r"], info["b"]) == (128, kvtc.RAW_BITS)
+        assert info["page_bytes"] == 32768
+    assert sum(plan.unit(u)["r"] * plan.unit(u)["b"] for u in range(0, 32, 2)) <= 1.0 * 128 * 16
+
+
+def test_plan_create_accepts_raw_value_units_only_as_values():
+    rng = np.random.default_rng(8)
+    M = [np.linalg.qr(rng.standard_normal((128, 128)))[0][:16].astype(np.float32), np.eye(128, dtype=np.float32)]
+    kvtc.kvtc_plan_create(1, 1, 1, [16, 128], [2, 16], [0.1, 2.0 ** -24], M)
+    with pytest.raises(kvtc.KvtcError):
+        kvtc.kvtc_plan_create(1, 1, 1, [128, 16], [16, 2], [2.0 ** -24, 0.1], M[::-1])
+    with pytest.raises(kvtc.KvtcError):
+        kvtc.kvtc_plan_create(1, 1, 1, [16, 64], [2, 16], [0.1, 2.0 ** -24], [M[0], M[1][:64]])
+
+
 def test_plan_save_load_round_trip(tmp_path):
     w = synth.WORKLOADS["head1-fp32-1k"]
     k, v, q = synth.calibration_set(w)
