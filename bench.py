@@ -46,7 +46,7 @@ ENCODE_WORKLOAD = "qwen7b-28L-128k-2bpd"
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the current decode kernels
 # on layers 0-3 of the workload; reported as roofline.traffic beside the algorithmic
 # bytes.  Set to None whenever a decode kernel changes, until it is captured again.
-DECODE_TRAFFIC = {"llama8b-32L-128k-1bpd": 34413312}
+DECODE_TRAFFIC = {"llama8b-32L-128k-1bpd": 34413056}
 METRIC = "decode-attn effective HBM GB/s (% of peak) at 128k ctx; encode Mtok/s"
 
 

@@ -16,10 +16,10 @@
 // fp32.  q~ is split into fp16 hi + lo (about 22 bits).  Online softmax per block; P goes
 // to fp16 (scaled by 2^(7-e) so P * A = p * c * 2^-17 whatever e is), is transposed into
 // the B fragment with movmatrix, and multiplies the value codes (A = V codes, rows =
-// latent coordinates) into fp32 accumulators.  Each CTA writes one (m, l, z) partial per
-// query head.
-// Kernel 2 (decode_combine_kernel): log-sum-exp merge of the partials, centering
-// (z - m_V * l), dequantization (delta_V) and the back-projection o = M_V^T y.
+// latent coordinates) into fp32 accumulators, centring them (z - m_V * l) as it goes.
+// Each CTA writes one (m, l, z) partial per query head.
+// Kernel 2 (decode_combine_kernel): log-sum-exp merge of the partials, dequantization
+// (delta_V) and the back-projection o = M_V^T y.
 // All launches use programmatic dependent launch, so each kernel's set-up overlaps the
 // tail of the one before it.
 #include <cuda_runtime.h>
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(const __grid_constant_
   }
 }
 
-// ---- kernel 2: merge the partials, centre, dequantise, back-project --------------------
+// ---- kernel 2: merge the partials, dequantise, back-project -----------------------------
 // CTA = (query head, sequence, block of 32 output columns), 128 threads.  The CTA's slice
 // M_V[:, 32c .. 32c + 31] is loaded into shared memory before the wait for the split
 // kernels; then the four warps fold the partials (lane l holds latent coordinates
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(const __gr
   const UnitDesc dV = ca.units[(ca.layer * ca.H + h) * 2 + 1];
   const int rV = dV.r;
   // an uncompressed value unit (keys-only plans) is already in d-space: its latent is
-  // the output (identity back-projection), its codes are v * 2^24, with no centring
+  // the output (identity back-projection), its codes are v * 2^24
   const bool raw = dV.b == kRawBits;
   // the plan's M_V is not written by the preceding kernels: load it before the wait
   for (int i = tid; !raw && i < rV * (kCombCols / 4); i += kCombThreads) {
@@ -163,44 +163,57 @@ __global__ void __launch_bounds__(kCombThreads) decode_combine_kernel(const __gr
   griddep_launch_dependents();
   const int n_part = ca.nparts[h];
   const float* base = ca.ws + (static_cast<size_t>(s) * Hq + qh) * ca.part_stride * kPartStride;
-  // global max of the partial maxima (log2 domain)
-  float mx = -INFINITY;
-  for (int i = tid; i < n_part; i += kCombThreads) mx = fmaxf(mx, base[static_cast<size_t>(i) * kPartStride]);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) mxsh[warp] = mx;
-  __syncthreads();
-  mx = mxsh[0];
-#pragma unroll
-  for (int w = 1; w < kCombWarps; ++w) mx = fmaxf(mx, mxsh[w]);
+  // One pass over the partials per warp (partials warp, warp + 4, ...) with a running
+  // maximum (log2 domain); the four warps then meet at the largest of their maxima.
+  float mw = -INFINITY;
   float4 zacc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   float lacc = 0.0f;
 #pragma unroll 4
   for (int i = warp; i < n_part; i += kCombWarps) {
     const float* pp = base + static_cast<size_t>(i) * kPartStride;
     const float mi = pp[0];
-    const float wi = mi == -INFINITY ? 0.0f : exp2f(mi - mx);
+    const float li = pp[1];
     const float4 z4 = 4 * lane < rV ? reinterpret_cast<const float4*>(pp + 4)[lane] : make_float4(0, 0, 0, 0);
-    lacc = fmaf(wi, pp[1], lacc);
+    if (mi == -INFINITY) continue;  // a split without live tokens
+    if (mi > mw) {
+      const float sc = mw == -INFINITY ? 0.0f : exp2f(mw - mi);
+      zacc.x *= sc;
+      zacc.y *= sc;
+      zacc.z *= sc;
+      zacc.w *= sc;
+      lacc *= sc;
+      mw = mi;
+    }
+    const float wi = exp2f(mi - mw);
+    lacc = fmaf(wi, li, lacc);
     zacc.x = fmaf(wi, z4.x, zacc.x);
     zacc.y = fmaf(wi, z4.y, zacc.y);
     zacc.z = fmaf(wi, z4.z, zacc.z);
     zacc.w = fmaf(wi, z4.w, zacc.w);
   }
+  if (lane == 0) mxsh[warp] = mw;
+  __syncthreads();
+  float mx = mxsh[0];
+#pragma unroll
+  for (int w = 1; w < kCombWarps; ++w) mx = fmaxf(mx, mxsh[w]);
+  const float sw = mw == -INFINITY ? 0.0f : exp2f(mw - mx);
+  zacc.x *= sw;
+  zacc.y *= sw;
+  zacc.z *= sw;
+  zacc.w *= sw;
   reinterpret_cast<float4*>(zsh[warp])[lane] = zacc;
-  if (lane == 0) lsh[warp] = lacc;
+  if (lane == 0) lsh[warp] = lacc * sw;
   __syncthreads();
   float L = 0.0f;
 #pragma unroll
   for (int w = 0; w < kCombWarps; ++w) L += lsh[w];
-  const float mV = raw ? 0.0f : 0.5f * static_cast<float>((1 << dV.b) - 1);
   const float dlt = raw ? 0x1p-24f : dV.delta;
   for (int j = tid; j < rV; j += kCombThreads) {
     float zs = 0.0f;
 #pragma unroll
     for (int w = 0; w < kCombWarps; ++w) zs += zsh[w][j];
-    // z holds sum p*c*2^-17 (uncentered codes); center and dequantize
-    y[j] = L > 0.0f ? dlt * (ldexpf(zs, 17) - mV * L) / L : 0.0f;
+    // z holds sum p*(c - m_V)*2^-17 (the split kernel centres it); dequantize
+    y[j] = L > 0.0f ? dlt * ldexpf(zs, 17) / L : 0.0f;
   }
   __syncthreads();
   // o[k] = sum_j M_V[j][k] y[j] for this CTA's 32 columns: warp w takes j = w, w + 4, ...

@@ -19,6 +19,9 @@
 //     accumulated from the same rounded P, so z - m_V * l cancels consistently: in packed
 //     mode by one more MMA whose A operand is a constant row of ones, otherwise by one
 //     extra A row of ones (when r_V is not a multiple of 16) or per-lane sums.
+// The value codes enter their MMAs shifted by floor(m_V) (an exact fp16x2 subtraction),
+// so the tensor core accumulates signed terms near the size of the result; the 0.5 l left
+// over is folded into z after every page in packed mode (once at the end otherwise).
 // IL blocks are processed together (their MMA chains interleave).  The four warps'
 // (m, l, z) partials meet in shared memory and each CTA writes one partial per query
 // head; decode.cu's combine kernel merges those and back-projects.  q~ = M_K q comes from
@@ -125,6 +128,21 @@ __device__ __forceinline__ uint32_t fast_pair(uint32_t W, uint32_t Wh) {
   }
 }
 
+// fp16x2 a - b (round to nearest, subnormals kept).  On the code operands it is exact:
+// both are multiples of the same 2^(e-24) and the difference stays below 2^(b+e-24).
+__device__ __forceinline__ uint32_t hsub2_bits(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// floor(m_V) = 2^(b-1) - 1 at the bit offset e of the value codes of block BLK, row
+// eta, in both halves: the offset the value operand is shifted by before its MMA.
+template <int B, int BLK, int ETA>
+__host__ __device__ constexpr uint32_t centre_bits() {
+  return ((((1u << (B - 1)) - 1u) << e_of<B>(BLK, ETA)) * 0x10001u);
+}
+
 // Run-time part description of a b-bit code, indexed by log2 of the width (8/4/2/1):
 // has[lw] says whether the width-2^lw part exists, lo[lw] its lowest code bit.
 struct Parts {
@@ -204,6 +222,13 @@ struct WS {
   float zl[4];
   uint32_t onesA[2][2];
   int rsw;  // uncompressed value pages: swizzle of this lane's word positions (tq ^ 4 g)
+  // Centring of the value sums: the operands are c - floor(m_V), so z accumulates
+  // p * (c - m_V + 0.5); the 0.5 l left over is folded into z after every page (packed
+  // mode) or once at the end.  mV = 0.5 (0 for raw values); lfold = the part of l
+  // (times 2^-17) already folded.
+  float mV;
+  float lfold;
+  uint32_t cmV;  // generic widths: floor(m_V) * 2^-24 as fp16x2 bits
   float z[kNT][4];
   float z2[kZSplit ? kNT : 1][4];  // odd blocks (kZSplit)
   float zl2[4];
@@ -351,6 +376,18 @@ __device__ __forceinline__ void v_block(const WS<BK, BV, PACK>& w, uint32_t W0, 
     A2 = gen_pair<BLK, 1>(G0, w.partsV);
     A3 = gen_pair<BLK, 1>(G1, w.partsV);
   }
+  // Signed operands: the codes enter the MMA as c - floor(m_V), so the tensor core sums
+  // terms of both signs near the size of the result (an unsigned sum of p c, about
+  // m_V l, loses the centred result in the accumulation).  The remaining 0.5 l is
+  // folded into z separately.
+  {
+    const uint32_t c0 = BV == 0 ? w.cmV : centre_bits<BV == 0 ? 2 : BV, BLK, 0>();
+    const uint32_t c1 = BV == 0 ? w.cmV : centre_bits<BV == 0 ? 2 : BV, BLK, 1>();
+    A0 = hsub2_bits(A0, c0);
+    A1 = hsub2_bits(A1, c0);
+    A2 = hsub2_bits(A2, c1);
+    A3 = hsub2_bits(A3, c1);
+  }
   if (ones) {  // the ones row (row r_V) accumulates l: its A value is all ones
     constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
     constexpr uint32_t one0 = (1u << ev0) | (1u << (ev0 + 16)), one1 = (1u << ev1) | (1u << (ev1 + 16));
@@ -374,6 +411,23 @@ __device__ __forceinline__ void raw_v_block(const WS<BK, BV, PACK>& w, const uin
   const uint32_t A0 = row0[c0], A1 = row0[8 * (kPage / 2) + c0];
   const uint32_t A2 = row0[c1], A3 = row0[8 * (kPage / 2) + c1];
   mma_16816(z, A0, A1, A2, A3, bp[0], bp[1]);
+}
+
+// Packed mode: subtract m_V times the l gathered since the last fold from this lane's
+// value sums (head tq: z columns 2 tq, rows g and g + 8 of every tile).  zl[0] holds
+// head tq's l * 2^-17 in lane tq (g = 0).
+template <int BK, int BV, bool PACK>
+__device__ __forceinline__ void fold_centre(WS<BK, BV, PACK>& w) {
+  float lt = w.zl[0];
+  if constexpr (kZSplit) lt += w.zl2[0];
+  const float lnow = __shfl_sync(0xffffffffu, lt, w.tq);
+  const float dl = w.mV * (lnow - w.lfold);
+  w.lfold = lnow;
+#pragma unroll
+  for (int mt = 0; mt < kNT; ++mt) {
+    w.z[mt][0] -= dl;
+    w.z[mt][2] -= dl;
+  }
 }
 
 // Blocks B0 .. B0 + IL - 1 of the page: scores, lazy online softmax, value accumulation.
@@ -497,6 +551,7 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
         {
           w.zl[0] *= resc;
           if constexpr (kZSplit) w.zl2[0] *= resc;
+          w.lfold *= resc;
         }
         else
           w.lcvt[c] *= resc;
@@ -622,18 +677,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const int n_my = static_cast<int>(static_cast<long long>(worker + 1) * n_pages / n_workers) - p_begin;
   const int32_t* bt = a.block_table + static_cast<size_t>(s) * a.max_pages;
 
-  // ---- prologue: q~, page ids, first copies ----
-  for (int i = tid; i < 8 * 32; i += kThreads) {
-    const int gg = i >> 5, k4 = i & 31;
-    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    if (gg < ng && 4 * k4 < rK) {
-      v = reinterpret_cast<const float4*>(a.qt + (static_cast<size_t>(s) * Hq + h * a.G + g0 + gg) * kD)[k4];
-      if (4 * k4 + 2 >= rK) v.z = v.w = 0.0f;  // r_K is even: only the upper pair can be past it
-    }
-    reinterpret_cast<float4*>(sh.qt[gg])[k4] = v;
-  }
+  // ---- prologue: first copies (the barriers were set up by lane 0 of each warp, which
+  // also issues the copies), then q~ while they are in flight ----
   fence_mbar_init();
-  __syncthreads();
+  __syncwarp();
 
   const uint32_t bytesK = static_cast<uint32_t>(dK.page_bytes), bytesV = static_cast<uint32_t>(dV.page_bytes);
   const char* poolK = a.pool + a.pages_per_unit * dK.prefix;
@@ -675,6 +722,17 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     const int pid = pid_of(i);
     if (lane == 0) issue(i, pid);  // page i < n_stage uses slot i
   }
+
+  for (int i = tid; i < 8 * 32; i += kThreads) {
+    const int gg = i >> 5, k4 = i & 31;
+    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (gg < ng && 4 * k4 < rK) {
+      v = reinterpret_cast<const float4*>(a.qt + (static_cast<size_t>(s) * Hq + h * a.G + g0 + gg) * kD)[k4];
+      if (4 * k4 + 2 >= rK) v.z = v.w = 0.0f;  // r_K is even: only the upper pair can be past it
+    }
+    reinterpret_cast<float4*>(sh.qt[gg])[k4] = v;
+  }
+  __syncthreads();
 
   // per head: S = sum_j q~_j and the fp16 normalisation exponent (warp w: heads 2w, 2w+1)
 #pragma unroll
@@ -759,6 +817,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     }
     w.zl[0] = w.zl[1] = w.zl[2] = w.zl[3] = 0.0f;
     w.zl2[0] = w.zl2[1] = w.zl2[2] = w.zl2[3] = 0.0f;
+    w.mV = dV.b == kRawBits ? 0.0f : 0.5f;
+    w.lfold = 0.0f;
+    w.cmV = dV.b == kRawBits ? 0u : ((1u << (dV.b - 1)) - 1u) * 0x10001u;
   }
 #pragma unroll
   for (int mt = 0; mt < kNT; ++mt) {
@@ -796,6 +857,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       w.tok0 = p * kPage;
       w.partial = w.tok0 + kPage > w.seq_len;
       do_page<BK, BV, PACK>(w);
+      if constexpr (PACK) fold_centre(w);
     } else if (lane == 0 && a.status) {
       atomicOr(a.status, KVTC_STATUS_BAD_PAGE);
     }
@@ -846,6 +908,21 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       l += __shfl_xor_sync(0xffffffffu, l, 8);
       l += __shfl_xor_sync(0xffffffffu, l, 16);
       l_out[c] = l;
+    }
+  }
+
+  // ---- finish centring: the partial carries sum p (c - m_V) (times 2^-17) ----
+  if constexpr (PACK) {
+    fold_centre(w);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const float dl = w.mV * ldexpf(l_out[c], -17);
+#pragma unroll
+      for (int mt = 0; mt < kNT; ++mt) {
+        w.z[mt][c] -= dl;
+        w.z[mt][2 + c] -= dl;
+      }
     }
   }
 
