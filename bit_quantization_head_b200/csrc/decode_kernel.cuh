@@ -59,6 +59,11 @@ constexpr bool kZSplit = KVTC_DECODE_ZSPLIT != 0;
 #endif
 // 1: the packed words of a block group are loaded ahead of the tile jumps
 constexpr bool kHoist = KVTC_DECODE_HOIST != 0;
+#ifndef KVTC_DECODE_VORDER
+#define KVTC_DECODE_VORDER 0
+#endif
+// 1: the value phase of the fast code widths runs blocks outer, tiles inner
+constexpr bool kBlockOuterV = KVTC_DECODE_VORDER != 0;
 #ifndef KVTC_DECODE_MINB
 #define KVTC_DECODE_MINB 2
 #endif
@@ -606,15 +611,56 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
                                     bp[BB], (kZSplit && ((B0 + BB) & 1)) ? w.z2[mt] : w.z[mt]),
      ...);
   };
-  switch (w.nmt) {
-    default: vtile(std::integral_constant<int, 7>{}); [[fallthrough]];
-    case 7: vtile(std::integral_constant<int, 6>{}); [[fallthrough]];
-    case 6: vtile(std::integral_constant<int, 5>{}); [[fallthrough]];
-    case 5: vtile(std::integral_constant<int, 4>{}); [[fallthrough]];
-    case 4: vtile(std::integral_constant<int, 3>{}); [[fallthrough]];
-    case 3: vtile(std::integral_constant<int, 2>{}); [[fallthrough]];
-    case 2: vtile(std::integral_constant<int, 1>{}); [[fallthrough]];
-    case 1: vtile(std::integral_constant<int, 0>{});
+  if constexpr (kBlockOuterV && (BV == 2 || BV == 4 || BV == 8)) {
+    // One fully unrolled value phase per m-tile count: the packed words of every tile
+    // first, then blocks outer and tiles inner, so consecutive MMAs feed different
+    // accumulators (no MMA waits on the one before it).
+    auto vphase = [&](auto NMTC) {
+      constexpr int NMT = decltype(NMTC)::value;
+      uint32_t W0[NMT][VWN], W1[NMT][VWN], W0h[NMT][VWN], W1h[NMT][VWN];
+#pragma unroll
+      for (int mt = 0; mt < NMT; ++mt) {
+        const int j0 = 16 * mt + w.g;
+#pragma unroll
+        for (int q = 0; q < VWN; ++q) {
+          W0[mt][q] = w.pv[j0 * 4 * BV + w.tq * BV + VW0 + q];
+          W1[mt][q] = w.pv[(j0 + 8) * 4 * BV + w.tq * BV + VW0 + q];
+          W0h[mt][q] = shr8(W0[mt][q]);
+          W1h[mt][q] = shr8(W1[mt][q]);
+        }
+      }
+      auto blk = [&](auto BBC) {
+        constexpr int BB = decltype(BBC)::value;
+        constexpr int qi = ((B0 + BB) * VB) / 8 - VW0;
+#pragma unroll
+        for (int mt = 0; mt < NMT; ++mt)
+          v_block<BK, BV, PACK, B0 + BB>(w, W0[mt][qi], W0h[mt][qi], W1[mt][qi], W1h[mt][qi], 16 * mt + w.g,
+                                         16 * mt + w.g + 8, !PACK && mt == w.ones_mt, bp[BB],
+                                         (kZSplit && ((B0 + BB) & 1)) ? w.z2[mt] : w.z[mt]);
+      };
+      (blk(std::integral_constant<int, BB>{}), ...);
+    };
+    switch (w.nmt) {
+      case 1: vphase(std::integral_constant<int, 1>{}); break;
+      case 2: vphase(std::integral_constant<int, 2>{}); break;
+      case 3: vphase(std::integral_constant<int, 3>{}); break;
+      case 4: vphase(std::integral_constant<int, 4>{}); break;
+      case 5: vphase(std::integral_constant<int, 5>{}); break;
+      case 6: vphase(std::integral_constant<int, 6>{}); break;
+      case 7: vphase(std::integral_constant<int, 7>{}); break;
+      default: vphase(std::integral_constant<int, 8>{}); break;
+    }
+  } else {
+    switch (w.nmt) {
+      default: vtile(std::integral_constant<int, 7>{}); [[fallthrough]];
+      case 7: vtile(std::integral_constant<int, 6>{}); [[fallthrough]];
+      case 6: vtile(std::integral_constant<int, 5>{}); [[fallthrough]];
+      case 5: vtile(std::integral_constant<int, 4>{}); [[fallthrough]];
+      case 4: vtile(std::integral_constant<int, 3>{}); [[fallthrough]];
+      case 3: vtile(std::integral_constant<int, 2>{}); [[fallthrough]];
+      case 2: vtile(std::integral_constant<int, 1>{}); [[fallthrough]];
+      case 1: vtile(std::integral_constant<int, 0>{});
+    }
   }
 }
 
