@@ -1,0 +1,108 @@
+"""The oracle's pins must catch plausible mistakes.  Each test plants one mistake in an
+oracle function (a dropped term, a wrong constant, a swapped index, a transposed
+operand, a wrong rounding), runs the pin that guards that function, and expects it to
+fail.  The mistakes live only inside these tests (monkeypatch, CPU)."""
+
+import math
+
+import numpy as np
+import pytest
+
+from oracle import attention as att
+from oracle import calibration as cal
+from oracle import codec
+from tests import test_oracle_calibration as pins_cal
+from tests import test_oracle_codec as pins_codec
+
+
+def _fails(pin, *args):
+    with pytest.raises(AssertionError):
+        pin(*args)
+
+
+def test_dropped_quantization_term_is_caught(monkeypatch):
+    monkeypatch.setattr(cal, "q_of_b", lambda b: 0.0)
+    _fails(pins_cal.test_distortion_is_truncation_plus_quantization_terms)
+
+
+def test_wrong_quantization_constant_is_caught(monkeypatch):
+    monkeypatch.setattr(cal, "q_of_b", lambda b: 2.0 ** (-2.0 * b) / 6.0)
+    _fails(pins_cal.test_q_of_b_is_uniform_quantizer_mse_on_unit_range_exact, 3)
+
+
+def test_c1_rounding_the_bit_width_up_is_caught(monkeypatch):
+    def c1_ceil(w, B, d=None):
+        d = len(w) if d is None else d
+        best = None
+        for r in range(2, d + 1, 2):
+            b = min(cal.B_MAX, -(-B // r))   # ceil instead of floor
+            if b < cal.B_MIN:
+                continue
+            key = (cal.distortion(w, r, b), r * b, r)
+            if best is None or key < best[0]:
+                best = (key, (r, b))
+        return None if best is None else best[1]
+    monkeypatch.setattr(cal, "c1", c1_ceil)
+    _fails(pins_cal.test_c1_equals_brute_force_on_d8)
+
+
+def test_hadamard_sign_error_is_caught(monkeypatch):
+    good = cal.sylvester
+
+    def bad(n):
+        H = good(n).copy()
+        if n >= 2:
+            H[-1, -1] = -H[-1, -1]
+        return H
+    monkeypatch.setattr(cal, "sylvester", bad)
+    _fails(pins_cal.test_sylvester_hadamard_orthogonality, 4)
+
+
+def test_quantizer_rounding_instead_of_floor_is_caught(monkeypatch):
+    def quantize_round(y, inv_delta, b):
+        y = np.asarray(y, dtype=np.float32)
+        t = (y * np.float32(inv_delta)).astype(np.float32)
+        u = (t + np.float32(1 << (b - 1))).astype(np.float32)
+        f = np.fmin(np.fmax(np.rint(u), 0), (1 << b) - 1)
+        return f.astype(np.int64)
+    monkeypatch.setattr(codec, "quantize", quantize_round)
+    _fails(pins_codec.test_quantizer_matches_exact_rational_definition, 4)
+
+
+def test_dequantize_without_centring_is_caught(monkeypatch):
+    monkeypatch.setattr(codec, "dequantize", lambda c, delta, b: delta * np.asarray(c, np.float64))
+    _fails(pins_codec.test_dequantize_returns_cell_midpoint, 5)
+
+
+def test_transposed_operand_in_projection_is_caught(monkeypatch):
+    good = codec.project_canonical
+
+    def bad(x, M):
+        M = np.array(M, copy=True)
+        M[:, [0, 1]] = M[:, [1, 0]]          # two columns of M exchanged
+        return good(x, M)
+    monkeypatch.setattr(codec, "project_canonical", bad)
+    _fails(pins_codec.test_canonical_projection_equals_exact_rational_evaluation_of_its_order)
+
+
+def test_swapped_tokens_in_layout_are_caught_by_the_hand_example(monkeypatch):
+    # a bijection still round-trips, so only the hand-computed example can catch it
+    good = codec.field_bit_positions
+
+    def bad(kind, r, b):
+        pos = good(kind, r, b)
+        return pos[np.arange(codec.PAGE_TOKENS) ^ 1]
+    monkeypatch.setattr(codec, "field_bit_positions", bad)
+    _fails(pins_codec.test_layout_hand_computed_example)
+
+
+def test_raw_layout_without_swizzle_is_caught(monkeypatch):
+    monkeypatch.setattr(codec, "raw_word_index", lambda j, k: j * (codec.PAGE_TOKENS // 2) + k)
+    _fails(pins_codec.test_raw_page_hand_example)
+    _fails(pins_codec.test_raw_swizzle_spreads_each_fragment_read_over_32_banks)
+
+
+def test_attention_scale_error_is_caught(monkeypatch):
+    good = att.softmax_attention
+    monkeypatch.setattr(att, "softmax_attention", lambda q, K, V, scale: good(q, K, V, scale * math.sqrt(2)))
+    _fails(pins_codec.test_attention_full_rank_unquantized_equals_textbook_sdpa)
