@@ -63,6 +63,44 @@ def decode_head(q, k_codes, v_codes, unit_k, unit_v, scale):
     return softmax_attention(q, K, V, scale)
 
 
+# ---------------------------------------------------------------- pre-RoPE keys
+# The project page's Results caption states that keys are compressed pre-RoPE: the codes
+# hold keys before the rotary position embedding, which is applied when they are read.
+# The pages name no RoPE variant.  Readings: the common rotate-half form over pairs
+# (i, i + d/2) with angle t * base^(-2i/d), base 500000 (the Llama-3.1 value), no
+# frequency scaling; cached token t sits at position t; the query arrives already
+# rotated to its own position (as a model applies RoPE to q before attention).
+ROPE_BASE = 500000.0
+
+
+def rope_angles(positions, d, base=ROPE_BASE):
+    """Angles [n, d/2]: position * base^(-2i/d) for i < d/2, fp64."""
+    pos = np.asarray(positions, dtype=np.float64)
+    inv = base ** (-np.arange(0, d, 2, dtype=np.float64) / d)
+    return pos[:, None] * inv[None, :]
+
+
+def apply_rope(x, positions, base=ROPE_BASE):
+    """Rotary embedding of rows x [n, d] at the given positions (rotate-half form):
+    (x_i, x_{i+d/2}) -> (x_i cos a_i - x_{i+d/2} sin a_i, x_{i+d/2} cos a_i + x_i sin a_i)."""
+    x = np.asarray(x, dtype=np.float64)
+    h = x.shape[1] // 2
+    a = rope_angles(positions, x.shape[1], base)
+    c, s = np.cos(a), np.sin(a)
+    x1, x2 = x[:, :h], x[:, h:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=1)
+
+
+def decode_head_prerope(q_rot, k_codes, v_codes, unit_k, unit_v, scale, base=ROPE_BASE):
+    """One KV head with keys coded before RoPE: each reconstructed key k_hat_t is
+    rotated to its position t, then scored against the already-rotated queries
+    q_rot [G, d]; values as in ``decode_head``."""
+    K = reconstruct(k_codes, unit_k["M"], unit_k["delta"], unit_k["b"])
+    K = apply_rope(K, np.arange(K.shape[0]), base)
+    V = reconstruct(v_codes, unit_v["M"], unit_v["delta"], unit_v["b"])
+    return softmax_attention(q_rot, K, V, scale)
+
+
 def split_merge_attention(q, K, V, scale, n_split):
     """The same attention computed over ``n_split`` contiguous token ranges with an
     online (max, sum, weighted-sum) state per range, merged by log-sum-exp.  Used

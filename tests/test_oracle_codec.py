@@ -351,3 +351,48 @@ def test_decode_head_with_raw_values_equals_sdpa_on_fp16_values():
     Khat = (0.2 * (kc - (2 ** b - 1) / 2)) @ Mk
     ref = _sdpa(q, Khat, V.astype(np.float16).astype(np.float64), 1 / math.sqrt(d))
     assert np.abs(o - ref).max() < 1e-12
+
+
+# ---------------------------------------------------------------- pre-RoPE keys
+def test_rope_hand_example():
+    # d = 4, base 100: angles t * 100^0 = t and t * 100^(-1/2) = t / 10.  x = e_0 at
+    # position 2 -> (cos 2, 0, sin 2, 0); x = e_1 -> (0, cos 0.2, 0, sin 0.2).
+    x = np.array([[1.0, 0, 0, 0], [0, 1.0, 0, 0]])
+    got = att.apply_rope(x, [2, 2], base=100.0)
+    want = np.array([[math.cos(2), 0, math.sin(2), 0], [0, math.cos(0.2), 0, math.sin(0.2)]])
+    assert np.abs(got - want).max() < 1e-15
+
+
+def test_rope_is_a_rotation_by_relative_position():
+    rng = np.random.default_rng(31)
+    d = 128
+    q, k = rng.standard_normal((1, d)), rng.standard_normal((1, d))
+    assert np.allclose(att.apply_rope(q, [0]), q, atol=0)                       # identity at 0
+    for m, n in ((5, 9), (1000, 70000), (131071, 3)):
+        qm, kn = att.apply_rope(q, [m]), att.apply_rope(k, [n])
+        assert abs(np.linalg.norm(kn) - np.linalg.norm(k)) < 1e-12                # orthogonal
+        # R(m)^T R(n) = R(n - m): the score depends on the distance only
+        assert abs((qm @ kn.T).item() - (q @ att.apply_rope(k, [n - m]).T).item()) < 1e-9
+
+
+def test_decode_head_prerope_equals_sdpa_on_keys_rotated_as_complex_numbers():
+    # independent form of the rotation: pair (x_i, x_{i+d/2}) as x_i + j x_{i+d/2} times
+    # exp(j t theta_i); full rank, quantisation bypassed through an identity basis
+    rng = np.random.default_rng(32)
+    d, T, G = 128, 500, 4
+    K = rng.standard_normal((T, d))
+    V = rng.standard_normal((T, d))
+    theta = att.ROPE_BASE ** (-np.arange(0, d, 2) / d)
+    z = (K[:, :d // 2] + 1j * K[:, d // 2:]) * np.exp(1j * np.arange(T)[:, None] * theta[None, :])
+    K_rot = np.concatenate([z.real, z.imag], axis=1)
+    q_rot = rng.standard_normal((G, d)) * 0.3
+    unit = dict(M=np.eye(d), delta=1.0, b=codec.RAW_BITS)
+    kc = codec.encode_raw(K)           # fp16 patterns: reconstruct gives fp16(K)
+    vc = codec.encode_raw(V)
+    o = att.decode_head_prerope(q_rot, kc, vc, unit, unit, 1 / math.sqrt(d))
+    K16 = K.astype(np.float32).astype(np.float16).astype(np.float64)
+    z16 = (K16[:, :d // 2] + 1j * K16[:, d // 2:]) * np.exp(1j * np.arange(T)[:, None] * theta[None, :])
+    ref = _sdpa(q_rot, np.concatenate([z16.real, z16.imag], axis=1),
+                V.astype(np.float32).astype(np.float16).astype(np.float64), 1 / math.sqrt(d))
+    assert np.abs(o - ref).max() < 1e-12
+    assert np.abs(K_rot - att.apply_rope(K, np.arange(T))).max() < 1e-12

@@ -106,3 +106,14 @@ def test_attention_scale_error_is_caught(monkeypatch):
     good = att.softmax_attention
     monkeypatch.setattr(att, "softmax_attention", lambda q, K, V, scale: good(q, K, V, scale * math.sqrt(2)))
     _fails(pins_codec.test_attention_full_rank_unquantized_equals_textbook_sdpa)
+
+
+def test_rope_without_the_cross_term_is_caught(monkeypatch):
+    def bad(x, positions, base=att.ROPE_BASE):
+        x = np.asarray(x, dtype=np.float64)
+        h = x.shape[1] // 2
+        a = att.rope_angles(positions, x.shape[1], base)
+        return np.concatenate([x[:, :h] * np.cos(a), x[:, h:] * np.cos(a)], axis=1)
+    monkeypatch.setattr(att, "apply_rope", bad)
+    _fails(pins_codec.test_rope_hand_example)
+    _fails(pins_codec.test_decode_head_prerope_equals_sdpa_on_keys_rotated_as_complex_numbers)
