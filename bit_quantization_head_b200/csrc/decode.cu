@@ -7,7 +7,7 @@
 // are accumulated in their latent basis, back-projected once per query head.
 //
 // Kernel 0 (decode_prep_kernel): q~ = M_K q for every query head, once per call.
-// Kernel 1 (decode_split_kernel<BK, BV, PACK, NT>): CTA = (context split, KV head [, head
+// Kernel 1 (decode_split_kernel<BK, BV, PACK>): CTA = (context split, KV head [, head
 // group of 8], sequence), four warps, each streaming its own pages through a ring of
 // cp.async.bulk + mbarrier stages.  Per 16-token block a warp computes the G (<= 8) query
 // heads' scores with m16n8k16 tensor-core MMAs whose A operand is taken directly from the
@@ -15,9 +15,10 @@
 // the subnormal c * 2^(e-24) (exact), with e the field's bit offset; e is undone per row in
 // fp32.  q~ is split into fp16 hi + lo (about 22 bits).  Online softmax per block; P goes
 // to fp16 (scaled by 2^(7-e) so P * A = p * c * 2^-17 whatever e is), is transposed into
-// the B fragment with movmatrix, and multiplies the value codes (A = V codes, rows =
-// latent coordinates) into fp32 accumulators, centring them (z - m_V * l) as it goes.
-// Each CTA writes one (m, l, z) partial per query head.
+// the B fragment with movmatrix, and multiplies the value codes (A = V codes shifted by
+// floor(m_V), rows = latent coordinates) into fp32 accumulators; the remaining 0.5 l is
+// folded in, so each CTA writes one centred (m, l, z) partial per query head.  Keys-only
+// plans feed the stored fp16 values to the same MMAs.
 // Kernel 2 (decode_combine_kernel): log-sum-exp merge of the partials, dequantization
 // (delta_V) and the back-projection o = M_V^T y.
 // All launches use programmatic dependent launch, so each kernel's set-up overlaps the
