@@ -441,7 +441,9 @@ def run_ours(args, torch, dist, rank, world):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": kernels_per_step(plan, w) * args.steps,
         "clocks": clk.summary(),
-        "setup_s": {"calibrate": round(st["t_cal"], 1), "total": round(st["t_setup"], 1)},
+        "setup_s": {"calibrate": round(st["t_cal"], 1), "total": round(st["t_setup"], 1),
+                    "calib_stats": round(plan.calib_seconds()[0], 3),
+                    "calib_c1_c2": round(plan.calib_seconds()[1], 4)},
     }
     if not args.no_sdpa:
         res["sdpa_context"] = sdpa_context(torch, w, dec_ms)

@@ -8,6 +8,7 @@
 // over units.
 #include <algorithm>
 #include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstring>
 #include <memory>
@@ -306,21 +307,27 @@ uint64_t splitmix64_at(uint64_t seed, uint64_t n) {
   return z ^ (z >> 31);
 }
 
-// Entry (i, j) of the orthonormal block Walsh-Hadamard of order r (blocks: powers of two
-// of r's binary expansion, largest first; Sylvester entry sign = (-1)^popcount(i & j)).
-double block_hadamard_entry(int r, int i, int j) {
+// y = H_r x in place for the orthonormal block Walsh-Hadamard of order r: diagonal
+// blocks of the powers of two of r's binary expansion, largest first; a block of order n
+// is the Sylvester matrix (entry sign (-1)^popcount(i & j), H_2n = [[H_n, H_n],
+// [H_n, -H_n]], applied as butterflies) times 1/sqrt(n).
+void block_hadamard_apply(int r, double* x) {
   int off = 0;
   for (int bit = 30; bit >= 0; --bit) {
-    int n = 1 << bit;
+    const int n = 1 << bit;
     if (!(r & n)) continue;
-    if (i >= off && i < off + n) {
-      if (j < off || j >= off + n) return 0.0;
-      int a = i - off, c = j - off;
-      return (__builtin_popcount(a & c) & 1 ? -1.0 : 1.0) / std::sqrt(static_cast<double>(n));
-    }
+    double* y = x + off;
+    for (int len = 1; len < n; len <<= 1)
+      for (int i = 0; i < n; i += 2 * len)
+        for (int j = i; j < i + len; ++j) {
+          const double a = y[j], c = y[j + len];
+          y[j] = a + c;
+          y[j + len] = a - c;
+        }
+    const double s = 1.0 / std::sqrt(static_cast<double>(n));
+    for (int j = 0; j < n; ++j) y[j] *= s;
     off += n;
   }
-  return 0.0;
 }
 
 struct UnitWork {
@@ -347,6 +354,8 @@ extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* 
                 desc->fixed_b > 8))
     return fail(KVTC_EINVAL, "fixed_r must be even in [2,128] and fixed_b in [2,8]");
   const int U = 2 * L * H;
+  using clock = std::chrono::steady_clock;
+  const auto t0 = clock::now();
   if (!fixed && !(desc->bpd > 0.0)) return fail(KVTC_EINVAL, "bpd must be > 0");
 
   std::vector<UnitWork> work(U);
@@ -412,6 +421,7 @@ extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* 
     worker();
     for (auto& t : pool) t.join();
   }
+  const auto t1 = clock::now();
 
   std::vector<int> R(U), B(U);
   double mu = 0.0;
@@ -445,6 +455,7 @@ extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* 
     R[pool[i]] = Rp[i];
     B[pool[i]] = Bp[i];
   }
+  const auto t2 = clock::now();
 
   std::unique_ptr<kvtc_plan> p(new (std::nothrow) kvtc_plan());
   if (!p) return fail(KVTC_ENOMEM, "out of host memory");
@@ -454,6 +465,8 @@ extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* 
   p->d = d;
   p->U = U;
   p->mu = mu;
+  p->t_stats = std::chrono::duration<double>(t1 - t0).count();
+  p->t_alloc = std::chrono::duration<double>(t2 - t1).count();
   double gstep[9] = {0};
   for (int b = 2; b <= 8; ++b) gstep[b] = gaussian_step(b);
   for (int u = 0; u < U; ++u) {
@@ -480,16 +493,14 @@ extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* 
     const double delta = gstep[b] * sigma;
     std::vector<double> eps(r);
     for (int i = 0; i < r; ++i) eps[i] = (splitmix64_at(desc->seed, static_cast<uint64_t>(u) * 256 + i) >> 63) ? -1.0 : 1.0;
+    // M = H_r diag(eps) V_r^T, one column k at a time: the transform of eps .* V_r[k, :]
     std::vector<float> M(static_cast<size_t>(r) * d);
-    for (int i = 0; i < r; ++i)
-      for (int k = 0; k < d; ++k) {
-        double acc = 0.0;
-        for (int j = 0; j < r; ++j) {
-          const double h = block_hadamard_entry(r, i, j);
-          if (h != 0.0) acc += h * eps[j] * wk.Vs[static_cast<size_t>(k) * d + j];
-        }
-        M[static_cast<size_t>(i) * d + k] = static_cast<float>(acc);
-      }
+    std::vector<double> col(r);
+    for (int k = 0; k < d; ++k) {
+      for (int j = 0; j < r; ++j) col[j] = eps[j] * wk.Vs[static_cast<size_t>(k) * d + j];
+      block_hadamard_apply(r, col.data());
+      for (int i = 0; i < r; ++i) M[static_cast<size_t>(i) * d + k] = static_cast<float>(col[i]);
+    }
     p->r.push_back(r);
     p->b.push_back(b);
     p->delta.push_back(delta);

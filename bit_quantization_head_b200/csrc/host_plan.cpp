@@ -157,6 +157,13 @@ kvtc_status kvtc_plan_budget(const kvtc_plan* plan, double* mu, uint64_t* total_
   return KVTC_OK;
 }
 
+extern "C" kvtc_status kvtc_plan_calib_seconds(const kvtc_plan* plan, double* stats_s, double* alloc_s) {
+  if (!plan) return fail(KVTC_EINVAL, "plan is NULL");
+  if (stats_s) *stats_s = plan->t_stats;
+  if (alloc_s) *alloc_s = plan->t_alloc;
+  return KVTC_OK;
+}
+
 // File format (little-endian): "KVTCPLAN", u32 version, i32 L, H, G, d, U, f64 mu,
 // u32 has_weights; per unit: i32 r, i32 b, f64 delta, f32 inv_delta, f64 sigma, f64 D,
 // f32 M[r*d], then (if has_weights) f64 w[d], f64 lam[d].

@@ -47,6 +47,7 @@ struct kvtc_plan {
   std::vector<std::vector<float>> M;       // [U][r*d]
   std::vector<std::vector<double>> w, lam; // [U][d] (empty for imported plans)
   double mu = 0.0;
+  double t_stats = 0.0, t_alloc = 0.0;     // kvtc_calibrate: seconds in the eigen step and in C1 + C2
   // device copy (kvtc_plan_upload)
   int device = -1;
   kvtc::UnitDesc* d_units = nullptr;

@@ -78,6 +78,7 @@ def lib():
         "kvtc_plan_matrix": (st, [_P, C.c_int, _P]),
         "kvtc_plan_weights": (st, [_P, C.c_int, _P, _P]),
         "kvtc_plan_budget": (st, [_P, C.POINTER(C.c_double), C.POINTER(C.c_uint64)]),
+        "kvtc_plan_calib_seconds": (st, [_P, C.POINTER(C.c_double), C.POINTER(C.c_double)]),
         "kvtc_plan_save": (st, [_P, C.c_char_p]),
         "kvtc_plan_load": (st, [C.c_char_p, C.POINTER(_P)]),
         "kvtc_plan_upload": (st, [_P, _P]),
@@ -186,6 +187,12 @@ class Plan:
         mu, bits = C.c_double(), C.c_uint64()
         _check(lib().kvtc_plan_budget(self._h, C.byref(mu), C.byref(bits)))
         return mu.value, bits.value
+
+    def calib_seconds(self):
+        """(statistics and eigen step, C1 + C2 allocation) seconds of kvtc_calibrate."""
+        a, b = C.c_double(), C.c_double()
+        _check(lib().kvtc_plan_calib_seconds(self._h, C.byref(a), C.byref(b)))
+        return a.value, b.value
 
     def save(self, path):
         _check(lib().kvtc_plan_save(self._h, str(path).encode()))

@@ -160,6 +160,11 @@ kvtc_status kvtc_plan_matrix(const kvtc_plan* plan, int unit, float* M_out);
 kvtc_status kvtc_plan_weights(const kvtc_plan* plan, int unit, double* w_out, double* lam_out);
 /* The C2 multiplier mu* (0 for fixed or imported plans) and the total bits per token. */
 kvtc_status kvtc_plan_budget(const kvtc_plan* plan, double* mu, uint64_t* total_bits);
+/* Wall-clock seconds kvtc_calibrate spent on the per-unit statistics (second moments,
+ * eigen-decompositions, weights; host threads) and on the allocation (C1 + C2, the step
+ * the project page's "per-token overhead" figure times); 0 for imported plans.  Either
+ * pointer may be NULL. */
+kvtc_status kvtc_plan_calib_seconds(const kvtc_plan* plan, double* stats_s, double* alloc_s);
 
 /* Versioned binary plan file: header, then per unit r, b, delta, inv_delta and M. */
 kvtc_status kvtc_plan_save(const kvtc_plan* plan, const char* path);

@@ -86,6 +86,15 @@ def test_calibrate_damped_c2_matches_oracle_and_sits_between_bounds():
     assert D_lagrange <= D_damped <= D_equal
 
 
+def test_calibration_times_are_reported_per_phase():
+    w = synth.scaled(synth.WORKLOADS["llama8b-32L-128k-1bpd"], n_layers=2, n_cal=256)
+    k, v, q = synth.calibration_set(w)
+    plan = kvtc.kvtc_calibrate(k, v, q, n_layers=2, n_kv_heads=8, group=4, bpd=1.0, seed=w.seed)
+    stats_s, alloc_s = plan.calib_seconds()
+    assert stats_s > 0.0 and alloc_s > 0.0
+    assert stats_s + alloc_s < 120.0
+
+
 def test_calibrate_keys_only_matches_oracle():
     # keys-only ("k-only" results): the allocation covers the key units, values raw
     w = synth.scaled(synth.WORKLOADS["llama8b-32L-128k-1bpd"], n_layers=2, n_cal=256)
