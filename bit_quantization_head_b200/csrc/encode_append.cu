@@ -159,9 +159,67 @@ __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constan
   store_code(page, kind, ud.r, ud.b, slot, j, code);
 }
 
+// Test-only: the fp32 latent y = M x of rows of one unit in the same canonical order as
+// encode_append_kernel (CTA = token, thread j = coordinate), written instead of codes.
+// Raw value units (keys-only plans) have no projection: y = x.
+__global__ void __launch_bounds__(128) debug_latent_kernel(const UnitDesc* units, int u, const void* x, int bf16,
+                                                            float* y) {
+  __shared__ float xs[kD];
+  const int tok = blockIdx.x, j = threadIdx.x;
+  const UnitDesc ud = units[u];
+  const size_t xoff = static_cast<size_t>(tok) * kD;
+  xs[j] = bf16 ? __bfloat162float((static_cast<const __nv_bfloat16*>(x) + xoff)[j])
+               : (static_cast<const float*>(x) + xoff)[j];
+  __syncthreads();
+  if (j >= ud.r) return;
+  float out;
+  if (ud.b == kRawBits) {
+    out = xs[j];
+  } else {
+    float ch[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    if (bf16) {
+      const uint4* m4 = reinterpret_cast<const uint4*>(ud.Mbf + static_cast<size_t>(j) * kD);
+      for (int c = 0; c < 16; ++c) {
+        const uint4 mr = m4[c];
+        const uint32_t w[4] = {mr.x, mr.y, mr.z, mr.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          ch[2 * q] = __fmaf_rn(xs[8 * c + 2 * q], __uint_as_float(w[q] << 16), ch[2 * q]);
+          ch[2 * q + 1] = __fmaf_rn(xs[8 * c + 2 * q + 1], __uint_as_float(w[q] & 0xFFFF0000u), ch[2 * q + 1]);
+        }
+      }
+    } else {
+      const float* m = ud.M + static_cast<size_t>(j) * kD;
+      for (int k = 0; k < kD; ++k) ch[k & 7] = __fmaf_rn(xs[k], m[k], ch[k & 7]);
+    }
+    out = __fadd_rn(__fadd_rn(__fadd_rn(ch[0], ch[1]), __fadd_rn(ch[2], ch[3])),
+                    __fadd_rn(__fadd_rn(ch[4], ch[5]), __fadd_rn(ch[6], ch[7])));
+  }
+  y[static_cast<size_t>(tok) * ud.r + j] = out;
+}
+
 }  // namespace kvtc
 
 using namespace kvtc;
+
+extern "C" kvtc_status kvtc_debug_encode_latent(const kvtc_plan* plan, int layer, int head, int kind, const void* x,
+                                                kvtc_dtype dtype, int n_tok, float* y_out, void* stream) {
+  kvtc_status st = check_uploaded(plan);
+  if (st != KVTC_OK) return st;
+  if (layer < 0 || layer >= plan->L || head < 0 || head >= plan->H || (kind != 0 && kind != 1))
+    return fail(KVTC_EINVAL, "layer, head or kind out of range");
+  if (dtype != KVTC_F32 && dtype != KVTC_BF16) return fail(KVTC_EINVAL, "dtype must be F32 or BF16");
+  if (n_tok < 0) return fail(KVTC_EINVAL, "n_tok must be >= 0");
+  if (n_tok == 0) return KVTC_OK;
+  if (!x || !y_out) return fail(KVTC_EINVAL, "null device pointer");
+  if (reinterpret_cast<uintptr_t>(x) & 15) return fail(KVTC_EINVAL, "x must be 16-byte aligned");
+  const int u = (layer * plan->H + head) * 2 + kind;
+  debug_latent_kernel<<<n_tok, 128, 0, static_cast<cudaStream_t>(stream)>>>(plan->d_units, u, x,
+                                                                            dtype == KVTC_BF16 ? 1 : 0, y_out);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "debug latent launch");
+  return KVTC_OK;
+}
 
 extern "C" kvtc_status kvtc_encode_append(const kvtc_plan* plan, const kvtc_cache* cache, int layer,
                                           const void* k, const void* v, kvtc_dtype dtype,

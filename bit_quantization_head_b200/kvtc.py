@@ -87,6 +87,7 @@ def lib():
         "kvtc_encode_append": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, _P, C.c_int, _P, _P, C.c_int, _P]),
         "kvtc_encode_prefill": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, _P, C.c_int, C.c_int, C.c_int, _P]),
         "kvtc_plan_prefill_stats": (st, [_P, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64), C.c_int]),
+        "kvtc_debug_encode_latent": (st, [_P, C.c_int, C.c_int, C.c_int, _P, C.c_int, C.c_int, _P, _P]),
         "kvtc_decode_workspace_bytes": (C.c_uint64, [_P, C.c_int, C.c_int]),
         "kvtc_decode_attention": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, C.c_int, _P, C.c_int, C.c_float,
                                        _P, C.c_int, _P, C.c_uint64, _P]),
@@ -277,6 +278,12 @@ def kvtc_encode_append(plan, cache, layer, k, v, cu_seqlens, pos_start, stream=N
 def kvtc_encode_prefill(plan, cache, layer, k, v, seq, pos_start, stream=None):
     _check(lib().kvtc_encode_prefill(plan.handle, C.byref(cache.desc), layer, _dev_ptr(k), _dev_ptr(v), seq,
                                      pos_start, k.shape[0], _stream(stream)))
+
+
+def kvtc_debug_encode_latent(plan, layer, head, kind, x, y_out, stream=None):
+    """Test-only: fp32 latents [n, r] of rows x [n, d] of one unit (the append's order)."""
+    _check(lib().kvtc_debug_encode_latent(plan.handle, layer, head, kind, _dev_ptr(x), _dtype_code(x), x.shape[0],
+                                          _dev_ptr(y_out), _stream(stream)))
 
 
 def kvtc_plan_prefill_stats(plan, reset=False):

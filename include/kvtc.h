@@ -259,6 +259,16 @@ kvtc_status kvtc_encode_prefill(const kvtc_plan* plan, const kvtc_cache* cache, 
                                 void* stream);
 
 /*
+ * kvtc_debug_encode_latent -- test-only: the fp32 latent y = M_u x of n_tok rows of one
+ * unit (layer, head, kind) in the canonical order of kvtc_encode_append (what it
+ * quantizes), so a checker can quantize and pack it independently.  An uncompressed
+ * value unit returns x itself.  x: device [n_tok][d] of dtype (16-byte aligned);
+ * y_out: device fp32 [n_tok][r_u].  Asynchronous on the stream.
+ */
+kvtc_status kvtc_debug_encode_latent(const kvtc_plan* plan, int layer, int head, int kind, const void* x,
+                                     kvtc_dtype dtype, int n_tok, float* y_out, void* stream);
+
+/*
  * kvtc_plan_prefill_stats -- diagnostics of kvtc_encode_prefill since the plan was
  * uploaded (or last reset): codes produced and codes whose tensor-core sum fell within
  * the error bound of a quantizer threshold and were recomputed in canonical order.

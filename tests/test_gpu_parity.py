@@ -131,6 +131,36 @@ def test_keys_only_calibrated_llama_layer():
     _check_decode(plan, cache, 0, q, [T], w.n_kv_heads, w.group, "bf16")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_debug_latent_is_the_canonical_projection(dtype):
+    # the fp32 latents the append quantizes, bit for bit against the oracle's canonical
+    # projection; the oracle's quantizer applied to them gives the canonical codes
+    from oracle import codec as ocodec
+    rng = np.random.default_rng(14)
+    plan = gh.random_plan(1, 2, 1, [((34, 3), (128, 16)), ((128, 8), (16, 2))], rng)
+    n = 300
+    x = synth.round_dtype((rng.standard_normal((n, 128)) * 2).astype(np.float32), dtype)
+    for h in range(2):
+        for kind in (0, 1):
+            u = h * 2 + kind
+            info = plan.unit(u)
+            M = plan.matrix(u)
+            y = torch.empty((n, info["r"]), dtype=torch.float32, device="cuda")
+            kvtc.kvtc_debug_encode_latent(plan, 0, h, kind, gh.to_dev(x, dtype), y)
+            torch.cuda.synchronize()
+            got = y.cpu().numpy()
+            if info["b"] == kvtc.RAW_BITS:
+                want = x.astype(np.float32)
+            else:
+                Mop = ocodec.to_bf16(M) if dtype == "bf16" else M.astype(np.float32)
+                want = ocodec.project_canonical(x, Mop).astype(np.float32)
+            assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), (h, kind)
+            if info["b"] != kvtc.RAW_BITS:
+                unit = dict(info, M=M)
+                assert np.array_equal(ocodec.quantize(got, np.float32(info["inv_delta"]), info["b"]),
+                                      gh.oracle_codes(x, unit, dtype))
+
+
 def test_query_groups_larger_than_eight_and_peaked_attention():
     rng = np.random.default_rng(3)
     H, G = 2, 12
