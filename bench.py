@@ -336,6 +336,8 @@ def run_ours(args, torch, dist, rank, world):
         w = synth.scaled(w, n_layers=args.layers)
     if args.seq_len:
         w = synth.scaled(w, seq_len=args.seq_len)
+    if args.bpd:
+        w = synth.with_bpd(w, args.bpd)
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
     if args.no_decode:
         return {"encode": encode_bench(torch, synth.WORKLOADS[ENCODE_WORKLOAD], max(1, min(args.steps, 5)),
@@ -619,6 +621,8 @@ def main():
     ap.add_argument("--encode-layers", type=int, default=0, help="limit the encode workload's layers")
     ap.add_argument("--layers", type=int, default=0, help="limit the decode workload's layers (profiling)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the decode workload's context (profiling)")
+    ap.add_argument("--bpd", type=float, default=0.0,
+                    help="override the decode workload's budget (e.g. the 16 x 32k sweep at 0.5/1/2/4)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--k-only", action="store_true",
                     help="keys-only plan: keys coded at the budget, values stored as fp16")
