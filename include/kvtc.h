@@ -12,8 +12,10 @@
  * Vocabulary.  A *unit* is one (layer, KV head, kind) with kind K (keys) or V (values);
  * unit index u = ((layer * n_kv_heads) + head) * 2 + kind.  d = head dimension (128).
  * G = query heads per KV head.  Unit u keeps r_u coordinates (r even, 2..d) at b_u bits
- * (2..8): R_u = r_u * b_u bits per token.  A *page* holds 128 tokens of one unit and is
- * exactly 16 * R_u bytes (no per-token overhead, the "0 per-token overhead" figure).
+ * (2..8): R_u = r_u * b_u bits per token; in keys-only plans a value unit is stored
+ * uncompressed (r = d, b = KVTC_RAW_BITS, fp16).  A *page* holds 128 tokens of one unit
+ * and is exactly 16 * R_u bytes (no per-token overhead, the "0 per-token overhead"
+ * figure).
  *
  * Conventions for every call:
  *   - Every call returns a kvtc_status; nothing throws or exits across the ABI.  On an
