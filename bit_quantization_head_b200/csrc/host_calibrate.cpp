@@ -3,9 +3,10 @@
 //
 // Source: KV-COBRA project page, "How KV-COBRA Works" (distortion D(r,b), calibration),
 // "C1, per head", "C2, across heads", "Hadamard rotation", "Attention-KL reordering";
-// joint K+V pool per the KV-COBRA abstract.  The eigen-solver here is cyclic Jacobi
-// (a different algorithm from the LAPACK routine the oracle uses), run on host threads
-// over units.
+// joint K+V pool per the KV-COBRA abstract.  The eigen-solver here is Householder
+// tridiagonalisation plus implicit QR with a Wilkinson shift, with cyclic Jacobi as a
+// fallback (both written here, independent of the LAPACK routine the oracle uses), run on
+// host threads over units.
 #include <algorithm>
 #include <atomic>
 #include <chrono>
@@ -79,6 +80,117 @@ void jacobi_eig(std::vector<double>& A, int n, std::vector<double>& lam, std::ve
     for (int k = 0; k < n; ++k) W[k * n + j] = sgn * V[k * n + src];
   }
   V.swap(W);
+}
+
+// Householder tridiagonalisation followed by implicit symmetric QR steps with a Wilkinson
+// shift (the textbook method for dense symmetric matrices).  A (row-major, symmetric,
+// destroyed) -> eigenvalues (diagonal of the converged T) and eigenvectors (columns of
+// the accumulated orthogonal Q), in the same order and sign convention as jacobi_eig.
+// Returns false if the QR iteration does not converge within its step limit.
+bool tridiag_qr_eig(std::vector<double>& A, int n, std::vector<double>& lam, std::vector<double>& V) {
+  auto at = [&](int i, int j) -> double& { return A[static_cast<size_t>(i) * n + j]; };
+  std::vector<double> Q(static_cast<size_t>(n) * n, 0.0);
+  for (int i = 0; i < n; ++i) Q[static_cast<size_t>(i) * n + i] = 1.0;
+  auto q = [&](int i, int j) -> double& { return Q[static_cast<size_t>(i) * n + j]; };
+  // ---- A = Q T Q^T with T tridiagonal: reflection H_k = I - beta v v^T zeroes column k
+  // below its subdiagonal; the trailing block becomes H A22 H = A22 - v w^T - w v^T with
+  // p = beta A22 v, w = p - (beta / 2)(v^T p) v.
+  std::vector<double> v(n), p(n), w(n);
+  for (int k = 0; k + 2 < n; ++k) {
+    double sigma = 0.0;
+    for (int i = k + 1; i < n; ++i) sigma += at(i, k) * at(i, k);
+    if (sigma == 0.0) continue;
+    const double x0 = at(k + 1, k);
+    const double alpha = x0 > 0.0 ? -std::sqrt(sigma) : std::sqrt(sigma);
+    for (int i = k + 1; i < n; ++i) v[i] = at(i, k);
+    v[k + 1] -= alpha;
+    const double vtv = sigma - 2.0 * alpha * x0 + alpha * alpha;
+    if (!(vtv > 0.0)) continue;
+    const double beta = 2.0 / vtv;
+    double vp = 0.0;
+    for (int i = k + 1; i < n; ++i) {
+      double acc = 0.0;
+      for (int j = k + 1; j < n; ++j) acc += at(i, j) * v[j];
+      p[i] = beta * acc;
+      vp += v[i] * p[i];
+    }
+    const double K = 0.5 * beta * vp;
+    for (int i = k + 1; i < n; ++i) w[i] = p[i] - K * v[i];
+    for (int i = k + 1; i < n; ++i)
+      for (int j = k + 1; j < n; ++j) at(i, j) -= v[i] * w[j] + w[i] * v[j];
+    at(k + 1, k) = at(k, k + 1) = alpha;
+    for (int i = k + 2; i < n; ++i) at(i, k) = at(k, i) = 0.0;
+    for (int r = 0; r < n; ++r) {  // Q <- Q H_k
+      double t = 0.0;
+      for (int i = k + 1; i < n; ++i) t += q(r, i) * v[i];
+      t *= beta;
+      for (int i = k + 1; i < n; ++i) q(r, i) -= t * v[i];
+    }
+  }
+  // ---- implicit QR on the unreduced blocks of T, deflating from the bottom.  A plane
+  // rotation J on (k, k+1) (c, s with J^T [x; z] = [r; 0]) is applied as T <- J^T T J on
+  // the band window rows/columns k-1 .. k+2 and accumulated as Q <- Q J.
+  const double eps = std::ldexp(1.0, -52);
+  auto rotate = [&](int k, double c, double s) {
+    const int lo = std::max(0, k - 1), hi = std::min(n - 1, k + 2);
+    for (int i = lo; i <= hi; ++i) {  // columns k, k+1
+      const double a = at(i, k), b = at(i, k + 1);
+      at(i, k) = c * a - s * b;
+      at(i, k + 1) = s * a + c * b;
+    }
+    for (int j = lo; j <= hi; ++j) {  // rows k, k+1
+      const double a = at(k, j), b = at(k + 1, j);
+      at(k, j) = c * a - s * b;
+      at(k + 1, j) = s * a + c * b;
+    }
+    for (int r = 0; r < n; ++r) {
+      const double a = q(r, k), b = q(r, k + 1);
+      q(r, k) = c * a - s * b;
+      q(r, k + 1) = s * a + c * b;
+    }
+  };
+  int steps = 0;
+  for (;;) {
+    for (int i = 0; i + 1 < n; ++i)
+      if (std::fabs(at(i + 1, i)) <= eps * (std::fabs(at(i, i)) + std::fabs(at(i + 1, i + 1))))
+        at(i + 1, i) = at(i, i + 1) = 0.0;
+    int hi = n - 1;
+    while (hi > 0 && at(hi, hi - 1) == 0.0) --hi;
+    if (hi == 0) break;
+    int lo = hi - 1;
+    while (lo > 0 && at(lo, lo - 1) != 0.0) --lo;
+    if (++steps > 60 * n) return false;
+    // Wilkinson shift: the eigenvalue of the trailing 2x2 block nearer to its last entry
+    const double a = at(hi - 1, hi - 1), b = at(hi, hi - 1), cc = at(hi, hi);
+    const double t = 0.5 * (a - cc);
+    const double mu = cc - b * b / (t + std::copysign(std::hypot(t, b), t == 0.0 ? 1.0 : t));
+    double x = at(lo, lo) - mu, z = at(lo + 1, lo);
+    for (int k = lo; k < hi; ++k) {
+      const double r = std::hypot(x, z);
+      const double c = r == 0.0 ? 1.0 : x / r, s = r == 0.0 ? 0.0 : -z / r;
+      rotate(k, c, s);
+      if (k + 1 < hi) {
+        x = at(k + 1, k);
+        z = at(k + 2, k);
+      }
+    }
+  }
+  // ---- order and signs as jacobi_eig
+  std::vector<int> idx(n);
+  for (int i = 0; i < n; ++i) idx[i] = i;
+  std::stable_sort(idx.begin(), idx.end(), [&](int x1, int x2) { return at(x1, x1) > at(x2, x2); });
+  lam.resize(n);
+  V.assign(static_cast<size_t>(n) * n, 0.0);
+  for (int j = 0; j < n; ++j) {
+    const int src = idx[j];
+    lam[j] = at(src, src);
+    int kmax = 0;
+    for (int k = 1; k < n; ++k)
+      if (std::fabs(q(k, src)) > std::fabs(q(kmax, src))) kmax = k;
+    const double sgn = q(kmax, src) < 0 ? -1.0 : 1.0;
+    for (int k = 0; k < n; ++k) V[static_cast<size_t>(k) * n + j] = sgn * q(k, src);
+  }
+  return true;
 }
 
 // ------------------------------------------------------------------ model pieces
@@ -381,7 +493,8 @@ extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* 
           C[i * d + j] /= N;
           C[j * d + i] = C[i * d + j];
         }
-      jacobi_eig(C, d, lam, V);
+      std::vector<double> C0 = C;
+      if (!tridiag_qr_eig(C, d, lam, V)) jacobi_eig(C0, d, lam, V);
       std::vector<double> wraw(lam);
       if (kind == 0 && kl) {
         const float* Q = q_cal + (static_cast<size_t>(layer) * H + head) * G * N * d;
