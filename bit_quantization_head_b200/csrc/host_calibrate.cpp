@@ -14,6 +14,7 @@
 #include <cstring>
 #include <memory>
 #include <thread>
+#include <utility>
 #include <vector>
 
 #include "kvtc_internal.h"
@@ -243,56 +244,158 @@ std::vector<Cand> candidates(int d) {
   return c;
 }
 
+// Lower convex hull of one unit's candidate points (bits, D), given in (bits, r) order:
+// the corners of C1's distortion-versus-budget curve.  x increasing, y strictly falling.
+std::vector<std::pair<int, double>> hull_points(const std::vector<Cand>& cand, const double* D) {
+  std::vector<std::pair<int, double>> stair, hull;
+  for (size_t c = 0; c < cand.size(); ++c) {
+    const int x = cand[c].bits;
+    const double y = D[c];
+    if (!stair.empty() && y >= stair.back().second) continue;
+    if (!stair.empty() && stair.back().first == x) stair.pop_back();
+    stair.emplace_back(x, y);
+  }
+  for (const auto& p : stair) {
+    while (hull.size() >= 2) {
+      const auto& a = hull[hull.size() - 2];
+      const auto& b = hull.back();
+      // b on or above the segment a -> p
+      if ((b.second - a.second) * static_cast<double>(p.first - a.first) >=
+          (p.second - a.second) * static_cast<double>(b.first - a.first))
+        hull.pop_back();
+      else
+        break;
+    }
+    hull.push_back(p);
+  }
+  return hull;
+}
+
+// Distortion saved per extra bit at budget B on a unit's hull: the slope of the segment
+// holding B, the mean of the two adjacent slopes at a corner, 0 past the last corner.
+double hull_marginal(const std::vector<std::pair<int, double>>& h, double B) {
+  const size_t n = h.size();
+  size_t k = 0;
+  while (k + 1 < n && static_cast<double>(h[k + 1].first) <= B) ++k;
+  if (k + 1 >= n) return 0.0;
+  const double right = (h[k].second - h[k + 1].second) / static_cast<double>(h[k + 1].first - h[k].first);
+  if (B == static_cast<double>(h[k].first) && k > 0) {
+    const double left = (h[k - 1].second - h[k].second) / static_cast<double>(h[k].first - h[k - 1].first);
+    return 0.5 * (left + right);
+  }
+  return right;
+}
+
 // C2 in the pages' iterative form ("C2, across heads": with C1 as the oracle, budget moves
-// between heads until their marginal distortions equalize; a damped update converges in
-// five rounds).  Step rule (the pages give none): start at equal real-valued budgets;
-// each round m_u = (D*_u(B_u - 8) - D*_u(B_u + 8)) / 16 with D*_u(B) the distortion of
-// C1's pick at floor(B) (sum w when no rank fits); B_u <- B_u (1 + (m_u - m) / (2 m)) with
-// m the mean marginal; clip to [4, 8d] and rescale the unclipped units to the total.
-// After five rounds each unit gets C1 at floor(B_u).  Only + - * / and sequential sums,
-// in the oracle's order.
-void c2_damped(const std::vector<std::vector<double>>& ws, long long total_bits, std::vector<int>& r_out,
-               std::vector<int>& b_out) {
+// between heads until their marginal distortions equalize, the water-filling condition; a
+// damped update converges in five rounds).  The water-filling condition is a common level
+// mu of marginal distortion per bit: at a level every unit holds the corner of C1's
+// distortion-versus-budget curve where its marginal falls to mu (argmin D + mu * bits,
+// ties to fewer bits, then smaller r), so only the level is iterated.  Level 0: the mean
+// hull marginal at the equal split.  Each round, with S the bits and R the summed ranks of
+// the picks: ln mu <- ln mu - 0.7 * 2 ln 2 * (total - S) / R (a damped Newton step; R / 2 ln 2
+// is the high-rate model's -dS/d ln mu).  After five rounds the picks at the final level
+// are fitted: while over budget, the downgrade with the smallest distortion increase per
+// bit saved; then the leftover bits go to the upgrade with the largest drop per bit.  Each
+// unit gets C1 at its pick's bits.  Same operations and order as the oracle.
+bool c2_damped(const std::vector<std::vector<double>>& ws, long long total_bits, std::vector<int>& r_out,
+               std::vector<int>& b_out, double& mu_out) {
   const int U = static_cast<int>(ws.size());
   const int d = static_cast<int>(ws[0].size());
-  const double lo_b = 4.0, hi_b = 8.0 * d, step = 8.0, damping = 0.5;
-  auto dstar = [&](int u, double Bv) {
-    const int Bi = static_cast<int>(std::floor(std::min(std::max(Bv, 0.0), hi_b)));
-    int r = 0, b = 0;
-    if (!c1(ws[u], Bi, r, b)) {
-      double tot = 0.0;
-      for (double x : ws[u]) tot += x;
-      return tot;
-    }
-    return distortion(ws[u], r, b);
-  };
-  std::vector<double> bud(U, static_cast<double>(total_bits) / U), m(U);
-  for (int round = 0; round < 5; ++round) {
-    for (int u = 0; u < U; ++u) m[u] = (dstar(u, bud[u] - step) - dstar(u, bud[u] + step)) / (2.0 * step);
-    double msum = 0.0;
-    for (int u = 0; u < U; ++u) msum += m[u];
-    const double mbar = msum / U;
-    if (!(mbar > 0.0)) break;
-    for (int u = 0; u < U; ++u) bud[u] = bud[u] * (1.0 + damping * (m[u] - mbar) / mbar);
-    for (int it = 0; it < 8; ++it) {
-      for (int u = 0; u < U; ++u) bud[u] = std::min(std::max(bud[u], lo_b), hi_b);
-      double fixed = 0.0, free = 0.0;
-      for (int u = 0; u < U; ++u) {
-        if (bud[u] <= lo_b || bud[u] >= hi_b)
-          fixed += bud[u];
-        else
-          free += bud[u];
+  const std::vector<Cand> cand = candidates(d);
+  const int n = static_cast<int>(cand.size());
+  const int rounds = 5;
+  const double damping = 0.7;
+  std::vector<double> D(static_cast<size_t>(U) * n);
+  for (int u = 0; u < U; ++u)
+    for (int c = 0; c < n; ++c) D[static_cast<size_t>(u) * n + c] = distortion(ws[u], cand[c].r, cand[c].b);
+  auto pick = [&](int u, double mu) {
+    int best = 0;
+    double bv = D[static_cast<size_t>(u) * n] + mu * static_cast<double>(cand[0].bits);
+    for (int c = 1; c < n; ++c) {
+      const double v = D[static_cast<size_t>(u) * n + c] + mu * static_cast<double>(cand[c].bits);
+      if (v < bv) {
+        bv = v;
+        best = c;
       }
-      if (free <= 0.0) break;
-      const double scale = (static_cast<double>(total_bits) - fixed) / free;
-      for (int u = 0; u < U; ++u)
-        if (!(bud[u] <= lo_b || bud[u] >= hi_b)) bud[u] = bud[u] * scale;
     }
+    return best;
+  };
+  const double B0 = static_cast<double>(total_bits) / U;
+  double msum = 0.0;
+  for (int u = 0; u < U; ++u) msum += hull_marginal(hull_points(cand, &D[static_cast<size_t>(u) * n]), B0);
+  const double mbar = msum / U;
+  double mu = 0.0;
+  if (mbar > 0.0) {
+    double lmu = std::log(mbar);
+    for (int round = 0; round < rounds; ++round) {
+      const double m = std::exp(lmu);
+      long long S = 0, rsum = 0;
+      for (int u = 0; u < U; ++u) {
+        const int c = pick(u, m);
+        S += cand[c].bits;
+        rsum += cand[c].r;
+      }
+      lmu = lmu - damping * (2.0 * std::log(2.0)) * static_cast<double>(total_bits - S) / static_cast<double>(rsum);
+    }
+    mu = std::exp(lmu);
+  }
+  std::vector<int> sel(U);
+  long long used = 0;
+  for (int u = 0; u < U; ++u) {
+    sel[u] = pick(u, mu);
+    used += cand[sel[u]].bits;
+  }
+  while (used > total_bits) {  // over budget: the cheapest downgrade per bit saved
+    int bu = -1, bc = -1;
+    double bcost = 0.0;
+    for (int u = 0; u < U; ++u) {
+      const int b0 = cand[sel[u]].bits;
+      const double D0 = D[static_cast<size_t>(u) * n + sel[u]];
+      for (int c = 0; c < n; ++c) {
+        const int saved = b0 - cand[c].bits;
+        if (saved <= 0) continue;
+        const double cost = (D[static_cast<size_t>(u) * n + c] - D0) / saved;
+        if (bu < 0 || cost < bcost) {
+          bu = u;
+          bc = c;
+          bcost = cost;
+        }
+      }
+    }
+    if (bu < 0) return false;
+    used -= cand[sel[bu]].bits - cand[bc].bits;
+    sel[bu] = bc;
+  }
+  long long left = total_bits - used;
+  for (;;) {  // leftover: the best drop per bit that fits
+    int bu = -1, bc = -1;
+    double bg = 0.0;
+    for (int u = 0; u < U; ++u) {
+      const int b0 = cand[sel[u]].bits;
+      const double D0 = D[static_cast<size_t>(u) * n + sel[u]];
+      for (int c = 0; c < n; ++c) {
+        const int extra = cand[c].bits - b0;
+        const double Dc = D[static_cast<size_t>(u) * n + c];
+        if (extra <= 0 || extra > left || !(Dc < D0)) continue;
+        const double g = (D0 - Dc) / extra;
+        if (bu < 0 || g > bg) {
+          bu = u;
+          bc = c;
+          bg = g;
+        }
+      }
+    }
+    if (bu < 0) break;
+    left -= cand[bc].bits - cand[sel[bu]].bits;
+    sel[bu] = bc;
   }
   r_out.assign(U, 0);
   b_out.assign(U, 0);
   for (int u = 0; u < U; ++u)
-    c1(ws[u], static_cast<int>(std::floor(std::min(std::max(bud[u], lo_b), hi_b))), r_out[u], b_out[u]);
+    if (!c1(ws[u], cand[sel[u]].bits, r_out[u], b_out[u])) return false;
+  mu_out = mu;
+  return true;
 }
 
 // C2 in Lagrangian form: bisect mu so that sum_u bits(argmin D_u + mu*bits) fits the
@@ -557,7 +660,7 @@ extern "C" kvtc_status kvtc_calibrate(const kvtc_calib_desc* desc, const float* 
     std::vector<std::vector<double>> ws(P);
     for (int i = 0; i < P; ++i) ws[i] = work[pool[i]].w;
     if (desc->c2_mode == KVTC_C2_DAMPED) {
-      c2_damped(ws, total, Rp, Bp);
+      if (!c2_damped(ws, total, Rp, Bp, mu)) return fail(KVTC_EINFEASIBLE, "no allocation meets the budget");
     } else if (!c2(ws, total, Rp, Bp, mu)) {
       return fail(KVTC_EINFEASIBLE, "no allocation meets the budget");
     }

@@ -57,9 +57,11 @@ typedef enum {
 typedef enum { KVTC_F32 = 0, KVTC_BF16 = 1 } kvtc_dtype;
 typedef enum { KVTC_KIND_K = 0, KVTC_KIND_V = 1 } kvtc_kind;
 typedef enum { KVTC_WEIGHTS_KL = 0, KVTC_WEIGHTS_MSE = 1 } kvtc_weight_mode;
-/* C2 solver: the Lagrangian water-filling (exact on the convex hull), or the pages'
- * iterative form (budget moved toward the larger marginal distortion, damped, five
- * rounds; "C2, across heads"). */
+/* C2 solver: the Lagrangian water-filling (mu bisected, exact on the convex hull), or the
+ * pages' iterative form ("C2, across heads": marginal distortions equalized by a damped
+ * update in five rounds): every unit sits where its marginal distortion on C1's
+ * distortion-versus-budget hull falls to a common level mu, and five damped Newton steps
+ * in log mu bring the level to the budget. */
 typedef enum { KVTC_C2_LAGRANGE = 0, KVTC_C2_DAMPED = 1 } kvtc_c2_mode;
 
 /* b of an uncompressed value unit (keys-only mode, kvtc_calib_desc.k_only): r = d = 128

@@ -16,7 +16,8 @@ Readings taken where the page is silent:
     floor(B/r) >= 2, so r*b <= B always;
   * C2 is solved in Lagrangian form (each unit minimises D + mu*r*b; mu is bisected
     so the pool meets its budget) plus a greedy spend of the leftover bits; each
-    unit's final (r, b) is C1 at the budget C2 gave it;
+    unit's final (r, b) is C1 at the budget C2 gave it; the pages' damped five-round
+    form iterates the same common level mu with damped Newton steps (``c2_damped``);
   * the Walsh-Hadamard of a non-power-of-two order r is block diagonal (normalised
     Sylvester blocks from the binary expansion of r, largest first);
   * one uniform quantizer per unit, step = g(b) * sqrt(mean retained eigenvalue),
@@ -218,66 +219,140 @@ def c2(weights, total_bits, iters=200):
     return out, hi
 
 
-def c2_damped(weights, total_bits, rounds=5, step=8, damping=0.5):
-    """C2, across heads, in the pages' iterative form ("C2, across heads": with C1 as the
-    oracle, budget moves between heads until their marginal distortions equalize; a
-    damped update converges in five rounds).  The pages give no step rule; the one
-    taken here:
-      * every unit starts at B_u = total_bits / U (real-valued budgets);
-      * a round measures each unit's marginal distortion with C1 as the oracle,
-        m_u = (D*_u(B_u - step) - D*_u(B_u + step)) / (2 step), where D*_u(B) is the
-        distortion of C1's pick at floor(B) (all-truncated sum(w) when no rank fits);
-      * and moves budget toward the units above the mean marginal m = mean_u m_u:
-        B_u <- B_u * (1 + damping * (m_u - m) / m), then clips to [4, 8 d] and rescales
-        the unclipped units so that the budgets add up to total_bits again;
-      * after ``rounds`` rounds each unit gets C1 at floor(B_u).
-    Only +, -, *, / and sequential sums are used, so a C++ restatement reproduces the
-    budgets bit for bit.  Returns the list of (r, b).  Raises ValueError if even 4 bits
-    per unit exceed the budget.
-    Pinned: identical units stay at equal budgets; the result fits the budget; its total
-    D lies between the Lagrangian optimum and the equal-budget start.
+def hull_points(bits, D):
+    """Lower convex hull of one unit's candidate points (bits, D) given in (bits, r)
+    order: the corners of C1's distortion-versus-budget curve B -> min{D(r, b) : r*b <= B}
+    that a marginal exchange of budget can reach.  Returns a list of (x, y) with x
+    increasing and y strictly decreasing."""
+    stair = []
+    for x, y in zip(bits, D):
+        x, y = int(x), float(y)
+        if stair and y >= stair[-1][1]:
+            continue
+        if stair and stair[-1][0] == x:
+            stair.pop()
+        stair.append((x, y))
+    hull = []
+    for x, y in stair:
+        while len(hull) >= 2:
+            (xa, ya), (xb, yb) = hull[-2], hull[-1]
+            if (yb - ya) * (x - xa) >= (y - ya) * (xb - xa):  # b on or above segment a -> (x, y)
+                hull.pop()
+            else:
+                break
+        hull.append((x, y))
+    return hull
+
+
+def hull_marginal(hull, B):
+    """Marginal distortion of a unit at budget B (bits per token) on its hull: the
+    distortion saved per extra bit, i.e. the slope of the hull segment that holds B; at
+    a corner the mean of the two adjacent slopes; 0 past the last corner."""
+    n = len(hull)
+    k = 0
+    while k + 1 < n and hull[k + 1][0] <= B:
+        k += 1
+    if k + 1 >= n:
+        return 0.0
+    right = (hull[k][1] - hull[k + 1][1]) / (hull[k + 1][0] - hull[k][0])
+    if B == hull[k][0] and k > 0:
+        left = (hull[k - 1][1] - hull[k][1]) / (hull[k][0] - hull[k - 1][0])
+        return 0.5 * (left + right)
+    return right
+
+
+def c2_damped(weights, total_bits, rounds=5, damping=0.7, trace=None):
+    """C2, across heads, in the pages' iterative form ("C2, across heads": with C1 as
+    the oracle, budget moves between heads until their marginal distortions equalize,
+    the water-filling condition; a damped update converges in five rounds).
+
+    Reading (the pages give no step rule): the water-filling condition is a common
+    level mu of marginal distortion per bit.  At a level mu every unit holds the budget
+    at which its marginal distortion falls to mu, i.e. the pick argmin D + mu * r*b on
+    the corners of C1's distortion-versus-budget curve (ties: fewer bits, then smaller
+    r), so the marginals are equal by construction and only the level has to be found.
+      * Level 0: the mean, over units, of the hull marginal distortion at the equal
+        split total_bits / U (``hull_marginal``).
+      * Each round: S = the bits the picks at mu spend and R = the sum of their ranks;
+        a damped Newton step in log mu,
+            ln mu <- ln mu - damping * 2 ln 2 * (total_bits - S) / R,
+        where R / (2 ln 2) is the high-rate model's -dS/d ln mu (D ~ 2^(-2B/r) for a
+        unit of rank r).
+      * After ``rounds`` rounds the picks at the final level are made to fit: while
+        over budget, the downgrade to a cheaper candidate with the smallest distortion
+        increase per bit saved; then the leftover bits go greedily to the upgrade with
+        the largest drop per bit (as in ``c2``).  Each unit's (r, b) is C1 at the bits
+        of its pick.
+    log and exp are the C library's (math.log / math.exp); every other step is +, -,
+    *, / or a comparison, so a C++ restatement reproduces the picks.
+    Returns (list of (r, b), final mu).  ``trace``, if a list, receives (mu, S) per round
+    and once more for the final level.  Raises ValueError if even 4 bits per unit exceed
+    the budget.
+    Pinned: after five rounds the picks spend the budget to within 1 % and every unit's
+    marginal interval on its hull brackets the common level; the final total D is
+    within 2 % of the Lagrangian solver's; identical units stay equal.
     """
-    U = len(weights)
+    tabs = [candidate_table(w) for w in weights]
+    U = len(tabs)
     if 4 * U > total_bits:
         raise ValueError("budget below 4 bits per unit")
-    d = len(weights[0])
-    lo_b, hi_b = 4.0, float(8 * d)
+    R = np.stack([t[0] for t in tabs])
+    Bq = np.stack([t[1] for t in tabs])
+    D = np.stack([t[2] for t in tabs])
+    bits = R * Bq
+    rows = np.arange(U)
 
-    def dstar(u, B):
-        w = weights[u]
-        Bi = int(np.floor(min(max(B, 0.0), hi_b)))
-        rb = c1(w, Bi, d)
-        if rb is None:
-            tot = 0.0
-            for x in w:
-                tot += float(x)
-            return tot
-        return distortion(w, rb[0], rb[1])
+    def pick(mu):
+        return np.argmin(D + mu * bits, axis=1)
 
-    budgets = [float(total_bits) / U] * U
-    for _ in range(rounds):
-        m = [(dstar(u, budgets[u] - step) - dstar(u, budgets[u] + step)) / (2.0 * step) for u in range(U)]
-        msum = 0.0
-        for x in m:
-            msum += x
-        mbar = msum / U
-        if not mbar > 0.0:
+    B0 = float(total_bits) / U
+    msum = 0.0
+    for u in range(U):
+        msum += hull_marginal(hull_points(bits[u], D[u]), B0)
+    mbar = msum / U
+    if mbar > 0.0:
+        lmu = math.log(mbar)
+        for _ in range(rounds):
+            sel = pick(math.exp(lmu))
+            S = 0
+            rsum = 0
+            for u in range(U):
+                S += int(bits[u, sel[u]])
+                rsum += int(R[u, sel[u]])
+            if trace is not None:
+                trace.append((math.exp(lmu), S))
+            lmu = lmu - damping * (2.0 * math.log(2.0)) * float(total_bits - S) / float(rsum)
+        mu = math.exp(lmu)
+    else:
+        mu = 0.0
+    sel = pick(mu)
+    used = int(bits[rows, sel].sum())
+    if trace is not None:
+        trace.append((mu, used))
+    while used > total_bits:  # over budget: cheapest downgrade per bit saved
+        b0 = bits[rows, sel][:, None]
+        D0 = D[rows, sel][:, None]
+        saved = b0 - bits
+        ok = saved > 0
+        cost = np.where(ok, (D - D0) / np.where(ok, saved, 1), np.inf)
+        flat = int(np.argmin(cost))
+        u, c = divmod(flat, bits.shape[1])
+        used -= int(saved[u, c])
+        sel[u] = c
+    left = total_bits - used
+    while True:  # leftover: best drop per bit that fits
+        b0 = bits[rows, sel][:, None]
+        D0 = D[rows, sel][:, None]
+        extra = bits - b0
+        ok = (extra > 0) & (extra <= left) & (D < D0)
+        if not ok.any():
             break
-        budgets = [budgets[u] * (1.0 + damping * (m[u] - mbar) / mbar) for u in range(U)]
-        for _ in range(8):  # clip, then rescale the free units to the total
-            budgets = [min(max(x, lo_b), hi_b) for x in budgets]
-            fixed = 0.0
-            free = 0.0
-            for x in budgets:
-                if x <= lo_b or x >= hi_b:
-                    fixed += x
-                else:
-                    free += x
-            if free <= 0.0:
-                break
-            scale = (float(total_bits) - fixed) / free
-            budgets = [x if (x <= lo_b or x >= hi_b) else x * scale for x in budgets]
-    return [c1(weights[u], int(np.floor(min(max(budgets[u], lo_b), hi_b))), d) for u in range(U)]
+        gain = np.where(ok, (D0 - D) / np.where(ok, extra, 1), -np.inf)
+        flat = int(np.argmax(gain))
+        u, c = divmod(flat, bits.shape[1])
+        left -= int(extra[u, c])
+        sel[u] = c
+    return [c1(w, int(bits[u, sel[u]])) for u, w in enumerate(weights)], mu
 
 
 # ---------------------------------------------------------------- Hadamard + signs
@@ -441,7 +516,7 @@ def calibrate(k_cal, v_cal, q_cal, n_layers, n_kv_heads, bpd, seed, *,
         total = int(round(bpd * d * len(pool)))
         weights = [units[i]["w"] for i in pool]
         if c2_mode == "damped":
-            rb_pool, mu = c2_damped(weights, total), 0.0
+            rb_pool, mu = c2_damped(weights, total)
         else:
             rb_pool, mu = c2(weights, total, iters=c2_iters)
     rb = [(d, RAW_BITS)] * len(units)

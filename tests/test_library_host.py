@@ -23,7 +23,10 @@ def test_library_exports_every_header_entry_point(L):
     assert L.kvtc_version() == 1
 
 
-def _compare_plans(plan, units, atol_M=2e-5):
+def _compare_plans(plan, units, rtol_M=1e-6):
+    # Calibration parity: (r, b) identical; delta and inv_delta equal to rounding; M
+    # (fp32, after sign canonicalisation) within 1e-6 of the oracle's fp64 M normwise
+    # (max |dM| <= 1e-6 max |M|); measured differences are a few fp32 ulp (~3e-8).
     assert plan.shape["n_units"] == len(units)
     for u, ou in enumerate(units):
         info = plan.unit(u)
@@ -34,7 +37,7 @@ def _compare_plans(plan, units, atol_M=2e-5):
         assert np.allclose(w, ou["w"], rtol=1e-8, atol=1e-12 * ou["w"].max())
         assert np.allclose(lam, ou["lam"], rtol=1e-8, atol=1e-12 * ou["lam"].max())
         M = plan.matrix(u)
-        assert np.abs(M - ou["M"]).max() <= atol_M, (u, np.abs(M - ou["M"]).max())
+        assert np.abs(M - ou["M"]).max() <= rtol_M * np.abs(ou["M"]).max(), (u, np.abs(M - ou["M"]).max())
         assert info["distortion"] == pytest.approx(ou["D"], rel=1e-8)
 
 
@@ -83,7 +86,11 @@ def test_calibrate_damped_c2_matches_oracle_and_sits_between_bounds():
     D_lagrange = sum(u["D"] for u in lag)
     per_unit = int(total) // 32
     D_equal = sum(ocal.distortion(u["w"], *ocal.c1(u["w"], per_unit)) for u in lag)
-    assert D_lagrange <= D_damped <= D_equal
+    # the damped level iteration reaches the water-filling point: within 2 % of the
+    # Lagrangian solver's total distortion, and far below the equal split
+    assert D_damped <= 1.02 * D_lagrange and D_damped < D_equal
+    mu, _ = plan.budget()
+    assert mu == pytest.approx(units[0]["mu"], rel=1e-12)
 
 
 def test_calibration_times_are_reported_per_phase():

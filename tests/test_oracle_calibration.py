@@ -307,19 +307,77 @@ def test_calibrate_small_model_meets_budget_and_is_deterministic():
 
 
 # ---------------------------------------------------------------- C2, damped form
+def _random_pool(seed, n=12):
+    rng = np.random.default_rng(seed)
+    return [np.sort(rng.exponential(1.0, 128) * np.arange(1, 129) ** -rng.uniform(0.5, 2.0))[::-1]
+            for _ in range(n)]
+
+
+_QWEN_WEIGHTS = []
+
+
+def _qwen_pool():
+    # the 224 units (28 layers x 4 KV heads x K, V) of the Qwen2.5-7B-shaped workload
+    if not _QWEN_WEIGHTS:
+        from bit_quantization_head_b200 import synth
+        w = synth.WORKLOADS["qwen7b-28L-128k-2bpd"]
+        k, v, q = synth.calibration_set(w)
+        for layer in range(w.n_layers):
+            for h in range(w.n_kv_heads):
+                _QWEN_WEIGHTS.append(cal.key_unit_weights(k[layer, h], q[layer, h])[0])
+                _QWEN_WEIGHTS.append(cal.value_unit_weights(v[layer, h])[0])
+    return _QWEN_WEIGHTS
+
+
+def _marginal_interval(w, bits):
+    """(left, right) slopes of the unit's hull at a corner budget: the distortion saved
+    per bit by the last bits spent and by the next ones; None off the hull."""
+    r, b, D = cal.candidate_table(w)
+    h = cal.hull_points(r * b, D)
+    xs = [p[0] for p in h]
+    if bits not in xs:
+        return None
+    k = xs.index(bits)
+    left = (h[k - 1][1] - h[k][1]) / (h[k][0] - h[k - 1][0]) if k > 0 else math.inf
+    right = (h[k][1] - h[k + 1][1]) / (h[k + 1][0] - h[k][0]) if k + 1 < len(h) else 0.0
+    return left, right
+
+
+def test_hull_points_are_the_convex_corners_of_c1s_distortion_curve():
+    # every hull corner is a candidate, D strictly falls, slopes strictly fall, and C1's
+    # distortion at any budget lies on or above the hull (brute force over budgets)
+    w = _random_pool(7, 1)[0][:16].copy()
+    r, b, D = cal.candidate_table(w)
+    h = cal.hull_points(r * b, D)
+    assert h[0][0] == 4
+    sl = [(h[i][1] - h[i + 1][1]) / (h[i + 1][0] - h[i][0]) for i in range(len(h) - 1)]
+    assert all(h[i + 1][1] < h[i][1] for i in range(len(h) - 1))
+    assert all(sl[i + 1] < sl[i] for i in range(len(sl) - 1))
+    for B in range(4, 8 * 16 + 1):
+        r1, b1 = cal.c1(w, B)
+        Dstar = cal.distortion(w, r1, b1)
+        k = max(i for i in range(len(h)) if h[i][0] <= B)
+        if k + 1 < len(h):
+            t = (B - h[k][0]) / (h[k + 1][0] - h[k][0])
+            Dh = h[k][1] + t * (h[k + 1][1] - h[k][1])
+        else:
+            Dh = h[k][1]
+        assert Dstar >= Dh - 1e-12
+        if B == h[k][0]:
+            assert Dstar == pytest.approx(h[k][1], rel=1e-12)
+
+
 def test_c2_damped_keeps_identical_units_at_equal_budgets():
     w = np.sort(np.random.default_rng(3).exponential(1.0, 128))[::-1]
-    picks = cal.c2_damped([w] * 6, 6 * 96)
+    picks, _ = cal.c2_damped([w] * 6, 6 * 96)
     assert len(set(picks)) == 1 and picks[0][0] * picks[0][1] <= 96
 
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_c2_damped_fits_the_budget_and_lies_between_optimum_and_equal_split(seed):
-    rng = np.random.default_rng(seed)
-    ws = [np.sort(rng.exponential(1.0, 128) * np.arange(1, 129) ** -rng.uniform(0.5, 2.0))[::-1]
-          for _ in range(12)]
+    ws = _random_pool(seed)
     total = 12 * 128
-    picks = cal.c2_damped(ws, total)
+    picks, _ = cal.c2_damped(ws, total)
     assert sum(r * b for r, b in picks) <= total
     D = sum(cal.distortion(w, r, b) for w, (r, b) in zip(ws, picks))
     lag, _ = cal.c2(ws, total)
@@ -328,10 +386,40 @@ def test_c2_damped_fits_the_budget_and_lies_between_optimum_and_equal_split(seed
     assert D_opt <= D <= D_eq
 
 
+def _check_damped_equalises(ws, total):
+    """"C2, across heads": after the five damped rounds the marginal distortions are
+    equal (water-filling) -- the level's picks spend the budget to within 2 %, every
+    final pick is a corner of its unit's hull, one common level brackets every unit's
+    marginal interval to within 5 % (max right slope <= 1.05 x min left slope), and the
+    total distortion is within 2 % of the Lagrangian solver's exact water-filling."""
+    trace = []
+    picks, mu = cal.c2_damped(ws, total, trace=trace)
+    assert len(trace) == 6
+    assert abs(trace[-1][1] - total) <= 0.02 * total
+    assert sum(r * b for r, b in picks) <= total
+    iv = [_marginal_interval(w, r * b) for w, (r, b) in zip(ws, picks)]
+    assert all(x is not None for x in iv)
+    assert max(x[1] for x in iv) <= 1.05 * min(x[0] for x in iv)
+    lag, _ = cal.c2(ws, total)
+    D = sum(cal.distortion(w, r, b) for w, (r, b) in zip(ws, picks))
+    D_lag = sum(cal.distortion(w, r, b) for w, (r, b) in zip(ws, lag))
+    assert D <= 1.02 * D_lag
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_c2_damped_equalises_marginal_distortion_in_five_rounds(seed):
+    _check_damped_equalises(_random_pool(seed), 12 * 128)
+
+
+def test_c2_damped_equalises_marginal_distortion_on_the_qwen_plan():
+    ws = _qwen_pool()
+    _check_damped_equalises(ws, 2 * 128 * len(ws))
+
+
 def test_c2_damped_moves_budget_toward_the_larger_marginal():
     # two units, one with ten times the weight: it must end with more bits
     w = np.sort(np.random.default_rng(4).exponential(1.0, 128))[::-1]
-    picks = cal.c2_damped([w, 10.0 * w], 2 * 128)
+    picks, _ = cal.c2_damped([w, 10.0 * w], 2 * 128)
     assert picks[1][0] * picks[1][1] > picks[0][0] * picks[0][1]
 
 

@@ -117,3 +117,38 @@ def test_rope_without_the_cross_term_is_caught(monkeypatch):
     monkeypatch.setattr(att, "apply_rope", bad)
     _fails(pins_codec.test_rope_hand_example)
     _fails(pins_codec.test_decode_head_prerope_equals_sdpa_on_keys_rotated_as_complex_numbers)
+
+
+def test_undamped_budget_exchange_is_caught(monkeypatch):
+    # the earlier step rule: budgets moved in proportion to their marginal's excess over
+    # the mean (no common level); it never reaches equal marginals in five rounds
+    def linear_exchange(weights, total_bits, rounds=5, damping=0.5, trace=None):
+        U = len(weights)
+        B = [float(total_bits) / U] * U
+
+        def dstar(u, x):
+            rb = cal.c1(weights[u], int(max(4.0, min(x, 1024.0))))
+            return cal.distortion(weights[u], *rb) if rb else float(np.sum(weights[u]))
+        for _ in range(rounds):
+            m = [(dstar(u, B[u] - 8) - dstar(u, B[u] + 8)) / 16.0 for u in range(U)]
+            mb = sum(m) / U
+            B = [b * (1 + damping * (x - mb) / mb) for b, x in zip(B, m)]
+            s = total_bits / sum(B)
+            B = [b * s for b in B]
+            if trace is not None:
+                trace.append((mb, int(sum(B))))
+        if trace is not None:
+            trace.append((mb, int(sum(B))))
+        return [cal.c1(w, int(max(4.0, min(b, 1024.0)))) for w, b in zip(weights, B)], 0.0
+    monkeypatch.setattr(cal, "c2_damped", linear_exchange)
+    _fails(pins_cal.test_c2_damped_equalises_marginal_distortion_in_five_rounds, 1)
+
+
+def test_damped_level_step_with_the_wrong_sign_is_caught(monkeypatch):
+    # the level moves away from the budget (ln mu + step instead of ln mu - step)
+    good = cal.c2_damped
+
+    def flipped(weights, total_bits, rounds=5, damping=0.7, trace=None):
+        return good(weights, total_bits, rounds=rounds, damping=-damping, trace=trace)
+    monkeypatch.setattr(cal, "c2_damped", flipped)
+    _fails(pins_cal.test_c2_damped_equalises_marginal_distortion_in_five_rounds, 0)
