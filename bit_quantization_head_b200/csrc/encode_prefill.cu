@@ -582,6 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const UnitDesc& ud = nk ? dV : dK;
         const unsigned char* row = sm.x[s][nk] + t * 128;
         float ss = 0.0f;
+        uint32_t any = 0u;  // OR of the magnitude bits: 0 only for a row of +-0
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -594,14 +595,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q = 0; q < 4; ++q) {
               const float x0 = __uint_as_float(xw[q] << 16), x1 = __uint_as_float(xw[q] & 0xFFFF0000u);
               ss = fmaf(x1, x1, fmaf(x0, x0, ss));
+              any |= xw[q] & 0x7FFF7FFFu;
             }
           }
         }
-        const float nrm = sqrtf(ss) * 1.001f;
+        float nrm = sqrtf(ss) * 1.001f;
+        // a row of tiny values can underflow ss (or lose it to subnormal rounding) while its
+        // sums still matter at a small step: bound ||x||_2 by sqrt(128) * max |x| instead
+        if (ss < 0x1p-100f && any != 0u) {
+          float am = 0.0f;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(row + (c >> 3) * kHalfBytes + ((c & 7) << 4));
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              am = fmaxf(am, fmaxf(fabsf(__uint_as_float(xw[q] << 16)), fabsf(__uint_as_float(xw[q] & 0xFFFF0000u))));
+          }
+          nrm = am * 11.32f;
+        }
         float e = ldexpf(nrm, -14) * ud.mnorm * ud.inv_delta * (1.0f + 0x1p-20f) +
                   0x1p-21f * static_cast<float>((1 << ud.b) + 1);
         if (!(nrm < INFINITY)) e = INFINITY;  // non-finite input: recompute every code
-        if (ss == 0.0f) e = -1.0f;            // zero token: every sum is exactly 0
+        if (any == 0u) e = -1.0f;             // zero token: every sum is exactly 0
         sm.eps[nk][t] = e;
       }
       epi_sync();
