@@ -12,7 +12,16 @@ new token's K/V (encode: project, quantize, pack) and run decode attention over 
 accumulation in the latent basis, split merge, back-projection).  The 32 layers are
 captured in one CUDA graph and replayed; inputs are resident in HBM.  GB/s counts the
 algorithmic bytes of a step: packed codes of every cached token plus the projection
-bases (fp32 M_K and M_V) of every KV head.
+bases (fp32 M_K and M_V) of every KV head.  roofline: the decode call of one layer, timed
+as the mean call of a graph of the 32 decode calls alone.
+
+Beside the headline the same line carries the other workloads of the method's scope:
+layer32k (one 32k-token layer at 2 bpd, L2 evicted before every call), sweep (16
+sequences x 32k tokens, 32 layers, at 0.5 / 1 / 2 / 4 bpd), k_only (keys coded, values
+fp16), encode (the 28-layer Qwen-shaped prefill of 131072 tokens, tensor cores) and
+qwen_decode (one decode step over that cache, 7 query heads per KV head), sdpa_context
+(torch fp16 SDPA at the headline shape) and cpu_baseline (the oracle on host cores:
+decode sample, whole-plan calibration, canonical encode sample).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -42,11 +51,11 @@ from bit_quantization_head_b200 import kvtc, synth  # noqa: E402
 DECODE_WORKLOAD = "llama8b-32L-128k-1bpd"
 ENCODE_WORKLOAD = "qwen7b-28L-128k-2bpd"
 
-# DRAM bytes (read + write) of one decode call (prep + split + combine) per layer, from an
-# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the current decode kernels
-# on layers 0-3 of the workload; reported as roofline.traffic beside the algorithmic
-# bytes.  Set to None whenever a decode kernel changes, until it is captured again.
-DECODE_TRAFFIC = {"llama8b-32L-128k-1bpd": 34413056}
+# DRAM bytes (read + write) of one decode call per layer, from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum) of the current decode kernels on layers
+# 0-3 of the workload (the file named beside it); reported as roofline.traffic next to the
+# algorithmic bytes.  None whenever a decode kernel has changed since the capture.
+DECODE_TRAFFIC = {"llama8b-32L-128k-1bpd": (None, None)}
 METRIC = "decode-attn effective HBM GB/s (% of peak) at 128k ctx; encode Mtok/s"
 
 
@@ -195,17 +204,14 @@ def build_decode_setup(torch, w, rank, k_only=False):
                 seq_lens=seq_lens, ws=ws, t_cal=t_cal, t_setup=time.time() - t0)
 
 
-def decode_step(st, w, events=None, stream=None):
+def decode_step(st, w, stream=None):
+    """One decode step of the whole model: per layer, append the new token, then decode."""
     plan, cache = st["plan"], st["cache"]
     for layer in range(w.n_layers):
         kvtc.kvtc_encode_append(plan, cache, layer, st["k_new"][layer], st["v_new"][layer], st["cu"], st["pos"],
                                 stream=stream)
-        if events is not None:
-            record_external(events[layer][0], stream)
         kvtc.kvtc_decode_attention(plan, cache, layer, st["q"][layer], st["seq_lens"], w.seq_len,
                                    st["out"][layer], st["ws"], stream=stream)
-        if events is not None:
-            record_external(events[layer][1], stream)
 
 
 def kernels_per_step(plan, w):
@@ -254,17 +260,17 @@ def cpu_baseline_decode(torch, st, w, budget_s=12.0):
     return done_bytes, t_used, heads
 
 
-def blas_threads():
+def host_cores():
+    """Host cores this process may run on (the oracle's numpy/BLAS threads use them)."""
     try:
-        from threadpoolctl import threadpool_info
-        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
+        return len(os.sched_getaffinity(0))
     except Exception:
-        return 1
+        return os.cpu_count() or 1
 
 
-def encode_bench(torch, w, steps, warmup, rank, n_layers=None):
-    """Encode Mtok/s: every layer's K and V of 131072 tokens, resident in HBM."""
+def encode_bench(torch, w, steps, warmup, rank, n_layers=None, keep=False):
+    """Encode Mtok/s: every layer's K and V of 131072 tokens, resident in HBM.  With keep,
+    also returns the encoded cache (plan, cache) for the decode leg over it."""
     dev = torch.device("cuda")
     if n_layers:
         w = synth.scaled(w, n_layers=n_layers)
@@ -304,13 +310,182 @@ def encode_bench(torch, w, steps, warmup, rank, n_layers=None):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
+    fix = kvtc.kvtc_plan_prefill_stats(plan) if use_prefill else (0, 0)
     in_bytes = w.n_layers * T * w.n_kv_heads * 128 * 2 * 2
     code_bytes = sum(T * plan.unit(u)["r"] * plan.unit(u)["b"] // 8 for u in range(plan.shape["n_units"]))
     flops = sum(2 * 128 * plan.unit(u)["r"] for u in range(plan.shape["n_units"])) * T
-    return {"workload": w.name, "path": "prefill (tensor cores)" if use_prefill else "append (CUDA cores)",
-            "recomputed_fraction": (fix[1] / fix[0]) if fix[0] else None,
-            "ms_per_pass": ms, "mtok_s": T / ms / 1e3, "gb_s": (in_bytes + code_bytes) / ms / 1e6,
-            "bytes_per_pass": in_bytes + code_bytes, "tflop_s": flops / ms / 1e9, "layers": w.n_layers}
+    hbm_peak, tf_peak, peak_kind = measured_peaks()
+    gbs = (in_bytes + code_bytes) / ms / 1e6
+    res = {"workload": w.name, "path": "prefill (tensor cores)" if use_prefill else "append (CUDA cores)",
+           "recomputed_fraction": (fix[1] / fix[0]) if fix[0] else None,
+           "ms_per_pass": round(ms, 4), "mtok_s": round(T / ms / 1e3, 3), "gb_s": round(gbs, 1),
+           "bytes_per_pass": in_bytes + code_bytes, "tflop_s": round(flops / ms / 1e9, 2), "layers": w.n_layers,
+           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                        "frac": round(gbs / hbm_peak, 4), "peak_kind": peak_kind,
+                        "hbm_roof_mtok_s": round(hbm_peak * 1e9 / ((in_bytes + code_bytes) / T) / 1e6, 2)}}
+    del kv
+    torch.cuda.empty_cache()
+    if keep:
+        return res, (w, plan, cache)
+    return res
+
+
+def graph_of(torch, stream, fn):
+    """fn() captured in a CUDA graph on stream (after one eager run that warms it)."""
+    with torch.cuda.stream(stream):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(torch, g, stream, steps, warmup):
+    """Mean ms per replay of g: warm-up replays, then steps replays bracketed by events."""
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, warmup)):
+            g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def decode_calls(st, w, stream):
+    """The decode calls of every layer alone (no appends): the per-call timing graph."""
+    for layer in range(w.n_layers):
+        kvtc.kvtc_decode_attention(st["plan"], st["cache"], layer, st["q"][layer], st["seq_lens"], w.seq_len,
+                                   st["out"][layer], st["ws"], stream=stream)
+
+
+def decode_leg(torch, w, steps, warmup, rank, k_only=False, setup=None):
+    """Throughput of one decode step over a workload: the step graph (append + decode per
+    layer) and the decode calls alone (the roofline figure: algorithmic bytes of one
+    call / mean call time from a graph of the calls with no events inside)."""
+    st = setup or build_decode_setup(torch, w, rank, k_only=k_only)
+    plan = st["plan"]
+    stream = torch.cuda.Stream()
+    per_layer = algorithmic_bytes(plan, range(w.n_layers), w.seq_len, w.batch)
+    step_bytes = sum(per_layer)
+    g_step = graph_of(torch, stream, lambda: decode_step(st, w, stream=stream))
+    g_dec = graph_of(torch, stream, lambda: decode_calls(st, w, stream))
+    ms_step = time_graph(torch, g_step, stream, steps, warmup)
+    ms_dec = time_graph(torch, g_dec, stream, steps, warmup) / w.n_layers
+    hbm_peak, _, peak_kind = measured_peaks()
+    achieved = (step_bytes / w.n_layers) / (ms_dec * 1e-3) / 1e9
+    out = {"workload": w.name, "layers": w.n_layers, "batch": w.batch, "seq_len": w.seq_len, "bpd": w.bpd,
+           "group": w.group, "k_only": bool(k_only), "bytes_per_step": step_bytes,
+           "ms_per_step": round(ms_step, 4), "gb_s": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
+           "decode_call_ms": round(ms_dec, 5), "decode_call_gb_s": round(achieved, 1),
+           "frac": round(achieved / hbm_peak, 4), "peak": hbm_peak, "peak_kind": peak_kind}
+    del g_step, g_dec
+    return out, st
+
+
+def layer32k_leg(torch, reps=30):
+    """One 32k-token layer at 2 bpd (16.8 MB of codes, L2-resident unless evicted): each
+    timed decode call follows a 512 MB write that evicts L2; median of reps."""
+    w = synth.WORKLOADS["llama8b-layer-32k-2bpd"]
+    st = build_decode_setup(torch, w, 0)
+    stream = torch.cuda.Stream()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        decode_step(st, w, stream=stream)  # the newest token
+        for ea, eb in evs:                 # torch creates its events lazily, on first record
+            ea.record(stream)
+            eb.record(stream)
+    torch.cuda.synchronize()
+
+    def call():
+        kvtc.kvtc_decode_attention(st["plan"], st["cache"], 0, st["q"][0], st["seq_lens"], w.seq_len, st["out"][0],
+                                   st["ws"], stream=stream)
+    with torch.cuda.stream(stream):
+        call()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for ea, eb in evs:
+            flush.fill_(1)
+            record_external(ea, stream)
+            call()
+            record_external(eb, stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+        g.replay()
+    torch.cuda.synchronize()
+    ms = statistics.median(ea.elapsed_time(eb) for ea, eb in evs)
+    b = algorithmic_bytes(st["plan"], [0], w.seq_len, 1)[0]
+    hbm_peak, _, peak_kind = measured_peaks()
+    del g, flush, st
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "bytes_per_call": b, "decode_call_us": round(ms * 1e3, 2),
+            "gb_s": round(b / (ms * 1e-3) / 1e9, 1), "frac": round(b / (ms * 1e-3) / 1e9 / hbm_peak, 4),
+            "peak": hbm_peak, "peak_kind": peak_kind, "l2": "512 MB write before every timed call"}
+
+
+def qwen_decode_leg(torch, enc_state, steps, warmup):
+    """One decode step over the 28-layer Qwen cache the encode leg wrote (G = 7)."""
+    w, plan, cache = enc_state
+    dev = torch.device("cuda")
+    T = w.seq_len
+    q = torch.stack([torch.from_numpy(synth.decode_queries(w, l)) for l in range(w.n_layers)]).to(dev, torch.bfloat16)
+    st = dict(plan=plan, cache=cache, q=q.reshape(w.n_layers, 1, w.n_q_heads, 128),
+              out=torch.empty((w.n_layers, 1, w.n_q_heads, 128), dtype=torch.bfloat16, device=dev),
+              seq_lens=torch.full((1,), T, dtype=torch.int32, device=dev),
+              ws=torch.empty(kvtc.kvtc_decode_workspace_bytes(plan, 1, T), dtype=torch.uint8, device=dev))
+    stream = torch.cuda.Stream()
+    g = graph_of(torch, stream, lambda: decode_calls(st, w, stream))
+    ms = time_graph(torch, g, stream, steps, warmup)
+    b = sum(algorithmic_bytes(plan, range(w.n_layers), T, 1))
+    hbm_peak, _, peak_kind = measured_peaks()
+    del g
+    return {"workload": w.name, "group": w.group, "layers": w.n_layers, "bytes_per_step": b,
+            "ms_per_step": round(ms, 4), "decode_call_ms": round(ms / w.n_layers, 5),
+            "gb_s": round(b / (ms * 1e-3) / 1e9, 1), "frac": round(b / (ms * 1e-3) / 1e9 / hbm_peak, 4),
+            "peak": hbm_peak, "peak_kind": peak_kind, "step": "decode calls of every layer (no append)"}
+
+
+def oracle_calibrate_and_encode(budget_s=6.0):
+    """The oracle timed on the host: the whole-model calibration of the 32-layer llama
+    plan (eigen-decompositions, KL weights, C1 + C2, Hadamard folds), and its canonical
+    fp32 encode (project, quantize) of a sample of the Qwen prefill workload (layer 0,
+    every KV head, K and V), reported per whole-model token."""
+    from oracle import calibration as ocal
+    from oracle import codec as ocodec
+    w = synth.WORKLOADS[DECODE_WORKLOAD]
+    k_cal, v_cal, q_cal = synth.calibration_set(w)
+    t0 = time.perf_counter()
+    ocal.calibrate(k_cal, v_cal, q_cal, w.n_layers, w.n_kv_heads, bpd=w.bpd, seed=w.seed)
+    t_cal = time.perf_counter() - t0
+    we = synth.WORKLOADS[ENCODE_WORKLOAD]
+    kc, vc, qc = synth.calibration_set(we, layers=[0])
+    units = ocal.calibrate(kc, vc, qc, 1, we.n_kv_heads, bpd=we.bpd, seed=we.seed)
+    n_tok, t_enc = 0, 0.0
+    chunk = 512
+    while t_enc < budget_s:
+        for h in range(we.n_kv_heads):
+            for kind in (0, 1):
+                u = units[h * 2 + kind]
+                x = synth.cache_tokens(we, 0, h, kind, chunk, seq=1 + n_tok // chunk)
+                t0 = time.perf_counter()
+                ocodec.encode_tokens(x, ocodec.to_bf16(u["M"].astype(np.float32)), u["inv_delta"], u["b"])
+                t_enc += time.perf_counter() - t0
+        n_tok += chunk
+    units_model = we.n_layers * we.n_kv_heads * 2
+    tok_s = n_tok * (2 * we.n_kv_heads) / units_model / t_enc
+    return {"calibrate_s": round(t_cal, 2),
+            "calibrate_sample": f"whole {w.name} plan ({w.n_layers * w.n_kv_heads * 2} units, C2 over all)",
+            "encode_mtok_s": round(tok_s / 1e6, 6),
+            "encode_sample": f"layer 0 of {we.name}: {n_tok} tokens x {we.n_kv_heads} KV heads x K, V "
+                             f"(canonical fp32 projection + quantize), scaled to whole-model tokens"}
 
 
 def max_over_ranks(torch, dist, x):
@@ -349,23 +524,9 @@ def run_ours(args, torch, dist, rank, world):
     per_layer_bytes = algorithmic_bytes(plan, range(L), w.seq_len, w.batch)
     step_bytes = sum(per_layer_bytes)
 
-    # warm the kernels (sets function attributes) before capture
-    with torch.cuda.stream(stream):
-        decode_step(st, w, stream=stream)
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        decode_step(st, w, stream=stream)
-    # a second graph with timing events around every layer's decode call
-    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
-    for ea, eb in events:            # torch creates the CUDA events lazily, on first record
-        ea.record(stream)
-        eb.record(stream)
-    torch.cuda.synchronize()
-    g_ev = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_ev, stream=stream):
-        decode_step(st, w, events=events, stream=stream)
-    torch.cuda.synchronize()
+    g = graph_of(torch, stream, lambda: decode_step(st, w, stream=stream))
+    # the decode calls alone (no appends, no events inside): the per-call roofline figure
+    g_dec = graph_of(torch, stream, lambda: decode_calls(st, w, stream))
 
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
@@ -386,14 +547,7 @@ def run_ours(args, torch, dist, rank, world):
     if dist:
         dist.barrier()
 
-    # per-launch duration of the dominant kernel (decode call of one layer)
-    durs = []
-    for _ in range(max(1, min(args.steps, 10))):
-        with torch.cuda.stream(stream):
-            g_ev.replay()
-        torch.cuda.synchronize()
-        durs.extend(events[l][0].elapsed_time(events[l][1]) for l in range(L))
-    dec_ms = statistics.mean(durs)
+    dec_ms = time_graph(torch, g_dec, stream, max(10, min(args.steps, 50)), args.warmup) / L
     hbm_peak, tf_peak, peak_kind = measured_peaks()
     achieved = (step_bytes / L) / (dec_ms * 1e-3) / 1e9
 
@@ -422,23 +576,27 @@ def run_ours(args, torch, dist, rank, world):
         f1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(torch, dist, f0.elapsed_time(f1) / args.steps)
+    del g, g_dec
 
+    traffic, traffic_from = (None, None) if args.k_only else DECODE_TRAFFIC.get(w.name, (None, None))
     value = aggregate_value(world, step_bytes, ms)
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "layers": L, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
                    "head_dim": 128, "batch": w.batch, "seq_len": w.seq_len, "bpd": w.bpd,
                    "parallelism": f"replicas x{world}", "k_only": bool(args.k_only),
                    "step": f"per layer: append 1 token + decode attention; {L} layers in one CUDA graph",
                    "l2": f"inputs larger than L2: {step_bytes / 1e9:.3f} GB of codes+bases per step vs 126 MB",
-                   "compute": "fp16 tensor-core operands (codes exact, q split hi+lo), fp32 accumulation"},
+                   "compute": "bf16 in/out; fp16 tensor-core operands (codes exact, q split hi+lo), "
+                              "fp32 accumulation"},
         "pct_of_peak": round(100 * value / world / hbm_peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": None if args.k_only else DECODE_TRAFFIC.get(w.name),
-                     "kernel": "decode call of one layer (q~ prep + split kernel + combine)", "peak_kind": peak_kind,
-                     "bytes_per_launch": step_bytes // L, "launch_ms": round(dec_ms, 5)},
+                     "frac": round(achieved / hbm_peak, 4), "traffic": traffic, "traffic_from": traffic_from,
+                     "kernel": "decode call of one layer (all its launches)", "peak_kind": peak_kind,
+                     "bytes_per_launch": step_bytes // L, "launch_ms": round(dec_ms, 5),
+                     "launch_ms_from": "graph of the 32 decode calls alone (no events inside), mean per call"},
         "e2e": {"value": round(aggregate_value(world, step_bytes, e2e_ms), 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": kernels_per_step(plan, w) * args.steps,
@@ -449,15 +607,43 @@ def run_ours(args, torch, dist, rank, world):
     }
     if not args.no_sdpa:
         res["sdpa_context"] = sdpa_context(torch, w, dec_ms)
-    if not args.no_encode:
-        res["encode"] = encode_bench(torch, synth.WORKLOADS[ENCODE_WORKLOAD], max(1, min(args.steps, 5)),
-                                     args.warmup, rank, args.encode_layers)
+    cpu_decode = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        b, t, heads = cpu_baseline_decode(torch, st, w)
-        res["cpu_baseline"] = {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": blas_threads(),
+        cpu_decode = cpu_baseline_decode(torch, st, w, budget_s=8.0)
+    del st
+    torch.cuda.empty_cache()
+    side_steps = max(3, min(args.steps, 20))
+    if not args.no_extra:
+        # the scope table's other decode workloads (each set up, timed and freed in turn)
+        res["layer32k"] = layer32k_leg(torch)
+        sweep = []
+        for bpd in (0.5, 1.0, 2.0, 4.0):
+            ws = synth.with_bpd(synth.WORKLOADS["llama8b-32L-b16x32k"], bpd)
+            out, st2 = decode_leg(torch, ws, side_steps, 3, rank)
+            sweep.append(out)
+            del st2
+            torch.cuda.empty_cache()
+        res["sweep"] = sweep
+        if not args.k_only:
+            out, st2 = decode_leg(torch, w, side_steps, 3, rank, k_only=True)
+            res["k_only"] = out
+            del st2
+            torch.cuda.empty_cache()
+    if not args.no_encode:
+        enc, enc_state = encode_bench(torch, synth.WORKLOADS[ENCODE_WORKLOAD], max(1, min(args.steps, 5)),
+                                      args.warmup, rank, args.encode_layers, keep=True)
+        res["encode"] = enc
+        if not args.no_extra:
+            res["qwen_decode"] = qwen_decode_leg(torch, enc_state, side_steps, 3)
+        del enc_state
+        torch.cuda.empty_cache()
+    if cpu_decode is not None:
+        b, t, heads = cpu_decode
+        res["cpu_baseline"] = {"value": round(b / t / 1e9, 5), "unit": "GB/s", "cores": host_cores(),
                                "kind": "oracle",
                                "sample": f"{heads} KV head(s) of layer 0 (G={w.group} queries each) over the "
                                          f"{w.seq_len}-token cache: unpack + fp64 d-space attention"}
+        res["cpu_baseline"].update(oracle_calibrate_and_encode())
     return res
 
 
@@ -597,7 +783,7 @@ def run_reference(args):
     dt = (time.perf_counter() - t0) / args.steps
     b = sum(Ts * u["r"] * u["b"] // 8 + u["r"] * 128 * 4 for u in (uK, uV))
     value = b / dt / 1e9
-    cores = blas_threads()
+    cores = host_cores()
     sample = (f"1 KV head (G={w.group} queries) of layer 0 over the first {Ts} tokens of a {T}-token cache "
               "encoded by the oracle; unpack + fp64 d-space attention per step")
     return {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s", "n_gpus": 1,
@@ -627,6 +813,8 @@ def main():
     ap.add_argument("--k-only", action="store_true",
                     help="keys-only plan: keys coded at the budget, values stored as fp16")
     ap.add_argument("--no-sdpa", action="store_true", help="skip the fp16 SDPA context timing")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other decode workloads (32k layer, 16 x 32k budget sweep, keys-only, Qwen decode)")
     ap.add_argument("--efficiency", action="store_true",
                     help="only the project page's Efficiency table (fixed r, b vs fp16 SDPA, 32k-128k)")
     args = ap.parse_args()
