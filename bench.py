@@ -18,7 +18,7 @@ as the mean call of a graph of the 32 decode calls alone.
 Beside the headline the same line carries the other workloads of the method's scope:
 layer32k (one 32k-token layer at 2 bpd, L2 evicted before every call), sweep (16
 sequences x 32k tokens, 32 layers, at 0.5 / 1 / 2 / 4 bpd), k_only (keys coded, values
-fp16), encode (the 28-layer Qwen-shaped prefill of 131072 tokens, tensor cores) and
+fp16), prerope (the same cache read as keys coded before the rotary embedding), encode (the 28-layer Qwen-shaped prefill of 131072 tokens, tensor cores) and
 qwen_decode (one decode step over that cache, 7 query heads per KV head), sdpa_context
 (torch fp16 SDPA at the headline shape) and cpu_baseline (the oracle on host cores:
 decode sample, whole-plan calibration, canonical encode sample).
@@ -198,7 +198,7 @@ def build_decode_setup(torch, w, rank, k_only=False):
     cu = torch.arange(B + 1, dtype=torch.int32, device=dev)
     pos = torch.full((B,), prefix, dtype=torch.int32, device=dev)
     seq_lens = torch.full((B,), T, dtype=torch.int32, device=dev)
-    ws = torch.empty(kvtc.kvtc_decode_workspace_bytes(plan, B, T), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(kvtc.kvtc_decode_workspace_bytes(plan, B, T), dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
     return dict(plan=plan, cache=cache, k_new=k_new, v_new=v_new, q=q, out=out, cu=cu, pos=pos,
                 seq_lens=seq_lens, ws=ws, t_cal=t_cal, t_setup=time.time() - t0)
@@ -365,6 +365,32 @@ def decode_calls(st, w, stream):
                                    st["out"][layer], st["ws"], stream=stream)
 
 
+def rope_leg(torch, st, w, steps, warmup):
+    """The pre-RoPE decode (keys coded before the rotary embedding; kvtc_decode_attention_rope)
+    over the same cache: every layer's call in one graph, mean call time.  Its work is
+    dominated by the per-block key reconstruction on the tensor cores (16 tokens x r_K x
+    128, fp16 hi + lo parts of M_K), so the line also reports those MMA flops."""
+    stream = torch.cuda.Stream()
+
+    def calls():
+        for layer in range(w.n_layers):
+            kvtc.kvtc_decode_attention_rope(st["plan"], st["cache"], layer, st["q"][layer], st["seq_lens"], w.seq_len,
+                                            st["out"][layer], st["ws"], stream=stream)
+    g = graph_of(torch, stream, calls)
+    ms = time_graph(torch, g, stream, steps, warmup) / w.n_layers
+    del g
+    plan = st["plan"]
+    b = sum(algorithmic_bytes(plan, range(w.n_layers), w.seq_len, w.batch)) / w.n_layers
+    H = plan.shape["n_kv_heads"]
+    rec_flops = sum(2 * 2 * 16 * ((plan.unit((l * H + h) * 2)["r"] + 15) // 16) * 128
+                    for l in range(w.n_layers) for h in range(H)) * w.seq_len * w.batch / w.n_layers
+    hbm_peak, tf_peak, peak_kind = measured_peaks()
+    return {"workload": w.name, "decode_call_ms": round(ms, 5), "gb_s": round(b / (ms * 1e-3) / 1e9, 1),
+            "frac": round(b / (ms * 1e-3) / 1e9 / hbm_peak, 4), "peak": hbm_peak, "peak_kind": peak_kind,
+            "reconstruction_tflop_s": round(rec_flops / (ms * 1e-3) / 1e12, 1),
+            "rope_base": 500000.0, "bytes_per_call": int(b)}
+
+
 def decode_leg(torch, w, steps, warmup, rank, k_only=False, setup=None):
     """Throughput of one decode step over a workload: the step graph (append + decode per
     layer) and the decode calls alone (the roofline figure: algorithmic bytes of one
@@ -440,7 +466,7 @@ def qwen_decode_leg(torch, enc_state, steps, warmup):
     st = dict(plan=plan, cache=cache, q=q.reshape(w.n_layers, 1, w.n_q_heads, 128),
               out=torch.empty((w.n_layers, 1, w.n_q_heads, 128), dtype=torch.bfloat16, device=dev),
               seq_lens=torch.full((1,), T, dtype=torch.int32, device=dev),
-              ws=torch.empty(kvtc.kvtc_decode_workspace_bytes(plan, 1, T), dtype=torch.uint8, device=dev))
+              ws=torch.zeros(kvtc.kvtc_decode_workspace_bytes(plan, 1, T), dtype=torch.uint8, device=dev))
     stream = torch.cuda.Stream()
     g = graph_of(torch, stream, lambda: decode_calls(st, w, stream))
     ms = time_graph(torch, g, stream, steps, warmup)
@@ -607,6 +633,8 @@ def run_ours(args, torch, dist, rank, world):
     }
     if not args.no_sdpa:
         res["sdpa_context"] = sdpa_context(torch, w, dec_ms)
+    if not args.no_extra and not args.k_only:
+        res["prerope"] = rope_leg(torch, st, w, max(3, min(args.steps, 10)), 3)
     cpu_decode = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu_decode = cpu_baseline_decode(torch, st, w, budget_s=8.0)

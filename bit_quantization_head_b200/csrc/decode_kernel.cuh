@@ -1,15 +1,18 @@
 // Decode split kernel (templates).  Included by decode.cu and the per-variant
 // instantiation units decode_v*.cu.
 //
-// CTA = (context split, KV head [, head group of 8], sequence); four warps, each streaming
-// its own pages through a ring of cp.async.bulk + mbarrier stages.  Per 16-token block a
-// warp
-//   * scores its G (<= 8) query heads with m16n8k16 MMAs whose A operand comes straight
-//     from the packed words: one AND leaves each code in the low mantissa bits of an fp16
-//     half, the exact subnormal c * 2^(e-24), e the field's bit offset (undone in fp32);
-//     q~ is split into fp16 hi + lo; for G <= 4 (packed mode) head n's hi and lo parts sit
-//     in columns 2n and 2n + 1 of one MMA, so each lane adds its own two columns and
-//     holds one head's scores for two token rows;
+// One launch per layer and width-class group.  CTA = (context split, KV head [, head group
+// of 8], sequence); four warps, each streaming its own pages through a ring of
+// cp.async.bulk + mbarrier stages.  The CTA
+//   * forms q~ = M_K q for its query heads on the tensor cores (M_K as fp16 hi + lo
+//     fragments from the plan, q scaled to fp16 by a power of two per head), and keeps the
+//     B fragments of q^ = q~ 2^-E (fp16 hi + lo) in shared memory for all four warps;
+//   * per 16-token block scores its G (<= 8) query heads with m16n8k16 MMAs whose A operand
+//     comes straight from the packed words: one AND leaves each code in the low mantissa
+//     bits of an fp16 half, the exact subnormal c * 2^(e-24), e the field's bit offset
+//     (undone in fp32); for G <= 4 (packed mode) head n's hi and lo parts sit in columns
+//     2n and 2n + 1 of one MMA, so each lane adds its own two columns and holds one head's
+//     scores for two token rows;
 //   * runs an online softmax whose rescale is lazy: it happens only when a score exceeds
 //     the running max by more than 2^8 (a warp vote), so the common block costs one FFMA
 //     and one ex2 per score;
@@ -22,10 +25,11 @@
 // The value codes enter their MMAs shifted by floor(m_V) (an exact fp16x2 subtraction),
 // so the tensor core accumulates signed terms near the size of the result; the 0.5 l left
 // over is folded into z after every page in packed mode (once at the end otherwise).
-// IL blocks are processed together (their MMA chains interleave).  The four warps'
-// (m, l, z) partials meet in shared memory and each CTA writes one partial per query
-// head; decode.cu's combine kernel merges those and back-projects.  q~ = M_K q comes from
-// decode.cu's prep kernel through the workspace.
+// A page's eight 16-token blocks are processed together (their MMA chains interleave).
+// The four warps' (m, l, z) meet in shared memory and each CTA writes one partial per
+// query head; the CTA that completes a (sequence, KV head, head group) last (an atomic
+// ticket in the workspace) merges every split's partial with a log-sum-exp, dequantizes
+// (delta_V) and back-projects o = M_V^T y itself, then re-arms the ticket.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -37,39 +41,19 @@
 #include "kvtc_internal.h"
 #include "ptx.cuh"
 
-#ifndef KVTC_DECODE_IL
-#define KVTC_DECODE_IL 8
-#endif
-
 namespace kvtc {
 namespace dec {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kNT = 8;                // 16-row tiles of a rank (r <= 128)
-constexpr int kIL = KVTC_DECODE_IL;   // blocks processed together
-#ifndef KVTC_DECODE_ZSPLIT
-#define KVTC_DECODE_ZSPLIT 0
-#endif
-// 1: even and odd blocks accumulate the value latents (and l) in separate fragments,
-// halving the MMA dependency chain of each m-tile
-constexpr bool kZSplit = KVTC_DECODE_ZSPLIT != 0;
-#ifndef KVTC_DECODE_HOIST
-#define KVTC_DECODE_HOIST 0
-#endif
-// 1: the packed words of a block group are loaded ahead of the tile jumps
-constexpr bool kHoist = KVTC_DECODE_HOIST != 0;
-#ifndef KVTC_DECODE_VORDER
-#define KVTC_DECODE_VORDER 0
-#endif
-// 1: the value phase of the fast code widths runs blocks outer, tiles inner
-constexpr bool kBlockOuterV = KVTC_DECODE_VORDER != 0;
-#ifndef KVTC_DECODE_MINB
-#define KVTC_DECODE_MINB 2
-#endif
-constexpr int kMinBlocks = KVTC_DECODE_MINB;  // resident CTAs per SM aimed for (registers, stages)
+constexpr int kIL = 8;                // blocks processed together (one page)
+constexpr int kMinBlocks = 3;         // resident CTAs per SM the registers are sized for
 constexpr int kPartStride = 132;      // floats per partial: m, l, 2 pad, z[128]
 constexpr int kMaxHeadsPerLaunch = 64;
+constexpr int kMaxSplits = 128;       // context splits per KV head (bounds the merge scratch)
+// floats of merge scratch the last CTA needs (weights, y, the warps' back-projections)
+constexpr int kMergeFloats = 8 * kMaxSplits + 8 * 128 + 4 * 8 * 128;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;         // log2 of the growth allowed before a rescale
 
@@ -80,7 +64,10 @@ struct DecodeArgs {
   int split_prefix[kMaxHeadsPerLaunch + 1];  // CTAs of head i: [prefix[i], prefix[i+1])
   int n_heads;
   int part_stride;                       // partial slots per query head in the workspace
-  const float* qt;    // q~ = M_K q per query head [n_seq][Hq][128] (the prep kernel's output)
+  const void* q;      // [n_seq][Hq][128] of q dtype
+  int q_bf16;
+  void* out;          // [n_seq][Hq][128] of out dtype
+  int out_bf16;
   int wait_first;     // 1: wait for the preceding grid before reading; 0: at exit (see decode.cu)
   const int32_t* seq_lens;
   int n_seq;
@@ -92,7 +79,8 @@ struct DecodeArgs {
   float scale;
   int n_stage;
   uint32_t stage_bytes;
-  float* ws;  // partials [n_seq][Hq][part_stride][kPartStride]
+  int* tickets;       // [n_seq][H][n_hg] arrival counters (zero between calls)
+  float* ws;          // partials [n_seq][Hq][part_stride][kPartStride]
 };
 
 // ------------------------------------------------------------------ code extraction
@@ -200,9 +188,18 @@ __device__ __forceinline__ void gen_words(const uint32_t* page, int r, int row, 
 
 // ------------------------------------------------------------------ shared memory
 struct SmemHead {
-  float qt[8][128];  // q~ = M_K q (zero beyond the head group and beyond r_K)
-  float S[8];        // sum_j q~_j
-  int E[8];          // power-of-two normalisation of q~ for fp16
+  float qt[8][128];        // q~ = M_K q (zero beyond the head group and beyond r_K)
+  union {
+    struct {
+      uint16_t hi[8][136];  // q of the group as fp16, scaled by 2^-Eq (rows padded: no conflicts)
+      uint16_t lo[8][136];  // the fp16 residual of an fp32 q
+    } q16;
+    uint32_t frag[2][8][2][32];  // B fragments of q^: [hi, lo][k-step][half][lane]
+  } u;
+  float S[8];              // sum_j q~_j
+  int E[8];                // power-of-two normalisation of q~ for fp16
+  int Eq[8];               // power-of-two normalisation of q for fp16
+  int last;                // this CTA merges the (sequence, KV head, head group)
 };
 
 // ------------------------------------------------------------------ per-warp state
@@ -210,16 +207,13 @@ template <int BK, int BV, bool PACK>
 struct WS {
   const uint32_t* pk;  // K page in shared memory
   const uint32_t* pv;  // V page in shared memory
+  const uint32_t* fr;  // this lane's B fragments of q^ in shared memory (hi; lo at + 512)
   int tok0, seq_len;
   bool partial;        // the page holds positions at or beyond seq_len
   int rK, rV, nks, nmt, g, tq;
   Parts partsK, partsV;
   int ones_mt, ones_lr;  // m-tile / local row of the ones row (ones_mt < 0: none)
   uint32_t ones_m0, ones_m1;  // lane masks: this lane's A rows g / g+8 are the ones row
-  // B fragments of q^: PACK -> bh[ks] (column g: head g / 2, hi for even g, lo for odd);
-  // else bh (hi), bl (lo), column g: head g
-  uint32_t bh[kNT][2];
-  uint32_t bl[PACK ? 1 : kNT][2];
   float alpha[2], beta[2], m_run[2];
   float al[2][n_e<BK == 0 ? 8 : BK>()], nb[2][n_e<BV == 0 ? 8 : BV>()];
   // PACK: l accumulator (row 0, column 2n: l of head n, times 2^-17) and the constant A
@@ -235,8 +229,6 @@ struct WS {
   float lfold;
   uint32_t cmV;  // generic widths: floor(m_V) * 2^-24 as fp16x2 bits
   float z[kNT][4];
-  float z2[kZSplit ? kNT : 1][4];  // odd blocks (kZSplit)
-  float zl2[4];
   float lcvt[2];  // l accumulated from the fp16 P when there is no ones row
 };
 
@@ -266,8 +258,9 @@ __device__ __forceinline__ void refresh_constants(WS<BK, BV, PACK>& w) {
 // r0, r1 of this lane that hold the block's fields (Wh = W >> 8).  Generic widths: the
 // words are read here (rows r0, r1).
 template <int BK, int BV, bool PACK, int BLK>
-__device__ __forceinline__ void k_block(const WS<BK, BV, PACK>& w, int ks, uint32_t W0, uint32_t W0h, uint32_t W1,
-                                        uint32_t W1h, int r0, int r1, float (&sc)[4], float (&sd)[4]) {
+__device__ __forceinline__ void k_block(const WS<BK, BV, PACK>& w, const uint32_t (&bh)[2], const uint32_t (&bl)[2],
+                                        uint32_t W0, uint32_t W0h, uint32_t W1, uint32_t W1h, int r0, int r1,
+                                        float (&sc)[4], float (&sd)[4]) {
   uint32_t A0, A1, A2, A3;
   if constexpr (BK != 0) {
     A0 = fast_pair<BK, BLK, 0>(W0, W0h);
@@ -283,8 +276,8 @@ __device__ __forceinline__ void k_block(const WS<BK, BV, PACK>& w, int ks, uint3
     A2 = gen_pair<BLK, 0>(G1, w.partsK);
     A3 = gen_pair<BLK, 1>(G1, w.partsK);
   }
-  mma_16816(sc, A0, A1, A2, A3, w.bh[ks][0], w.bh[ks][1]);
-  if constexpr (!PACK) mma_16816(sd, A0, A1, A2, A3, w.bl[ks][0], w.bl[ks][1]);
+  mma_16816(sc, A0, A1, A2, A3, bh[0], bh[1]);
+  if constexpr (!PACK) mma_16816(sd, A0, A1, A2, A3, bl[0], bl[1]);
 }
 
 // Score arguments of one block: x = s - m_run + 7 - e_V (log2 domain), -inf if masked.
@@ -342,8 +335,7 @@ __device__ __forceinline__ void p_block(WS<BK, BV, PACK>& w, const float (&x)[4]
     bp[0] = movmatrix_trans(pack_half2(ex2(x[0]), 0.0f));
     bp[1] = movmatrix_trans(pack_half2(ex2(x[1]), 0.0f));
     // l: the ones row times the same rounded P
-    mma_16816((kZSplit && (BLK & 1)) ? w.zl2 : w.zl, w.onesA[BLK & 1][0], 0u, w.onesA[BLK & 1][1], 0u, bp[0],
-              bp[1]);
+    mma_16816(w.zl, w.onesA[BLK & 1][0], 0u, w.onesA[BLK & 1][1], 0u, bp[0], bp[1]);
     return;
   }
   const uint32_t P0 = pack_half2(ex2(x[0]), ex2(x[1]));
@@ -423,9 +415,7 @@ __device__ __forceinline__ void raw_v_block(const WS<BK, BV, PACK>& w, const uin
 // head tq's l * 2^-17 in lane tq (g = 0).
 template <int BK, int BV, bool PACK>
 __device__ __forceinline__ void fold_centre(WS<BK, BV, PACK>& w) {
-  float lt = w.zl[0];
-  if constexpr (kZSplit) lt += w.zl2[0];
-  const float lnow = __shfl_sync(0xffffffffu, lt, w.tq);
+  const float lnow = __shfl_sync(0xffffffffu, w.zl[0], w.tq);
   const float dl = w.mV * (lnow - w.lfold);
   w.lfold = lnow;
 #pragma unroll
@@ -444,56 +434,31 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
   for (int bb = 0; bb < IL; ++bb)
 #pragma unroll
     for (int i = 0; i < 4; ++i) sc[bb][i] = sd[bb][i] = 0.0f;
-  // ---- packed words of the group.  The k-steps and m-tiles below run from a jump into
-  // an unrolled sequence (no per-step test); each case label is a scheduling boundary,
-  // so for the narrow widths (at most two words per row and tile) every word the group
-  // needs is loaded here, ahead of the jumps, predicated on the rank.  Rows past r_K
-  // meet zero q^ coefficients (q~ is zero there) and rows past r_V are never read back,
-  // so both are read unmasked inside the last tile; the shared-memory allocation has
-  // slack for that over-read.
+  // The k-steps and m-tiles below run from a jump into an unrolled sequence (no per-step
+  // test).  Rows past r_K meet zero q^ coefficients (q~ is zero there) and rows past r_V
+  // are never read back, so both are read unmasked inside the last tile; the
+  // shared-memory allocation has slack for that over-read.
   constexpr int KB = BK == 0 ? 1 : BK;
   constexpr int KW0 = (B0 * KB) / 8, KWN = ((B0 + IL - 1) * KB) / 8 - KW0 + 1;
-  constexpr bool kHoistK = kHoist && BK != 0 && KWN <= 2;
   constexpr int VB = BV == 0 ? 1 : BV;
   constexpr int VW0 = (B0 * VB) / 8, VWN = ((B0 + IL - 1) * VB) / 8 - VW0 + 1;
-  constexpr bool kHoistV = kHoist && BV != 0 && VWN <= 2;
-  uint32_t KWa[kHoistK ? kNT : 1][KWN], KWb[kHoistK ? kNT : 1][KWN];
-  uint32_t VWa[kHoistV ? kNT : 1][VWN], VWb[kHoistV ? kNT : 1][VWN];
-  if constexpr (kHoistK) {
-#pragma unroll
-    for (int ks = 0; ks < kNT; ++ks) {
-      const bool on = ks < w.nks;
-      const int r0 = 8 * ks + w.tq;
-#pragma unroll
-      for (int q = 0; q < KWN; ++q) {
-        KWa[ks][q] = on ? w.pk[r0 * 8 * BK + w.g * BK + KW0 + q] : 0u;
-        KWb[ks][q] = on ? w.pk[(r0 + 4) * 8 * BK + w.g * BK + KW0 + q] : 0u;
-      }
-    }
-  }
-  if constexpr (kHoistV) {
-#pragma unroll
-    for (int mt = 0; mt < kNT; ++mt) {
-      const bool on = mt < w.nmt;
-      const int j0 = 16 * mt + w.g;
-#pragma unroll
-      for (int q = 0; q < VWN; ++q) {
-        VWa[mt][q] = on ? w.pv[j0 * 4 * BV + w.tq * BV + VW0 + q] : 0u;
-        VWb[mt][q] = on ? w.pv[(j0 + 8) * 4 * BV + w.tq * BV + VW0 + q] : 0u;
-      }
-    }
-  }
   // ---- scores S[tok][head] = sum_j codeK[tok][j] * q^[head][j]
   auto kstep = [&](auto KSC) {
     constexpr int ks = decltype(KSC)::value;
     const int r0 = 8 * ks + w.tq, r1 = r0 + 4;
+    uint32_t bh[2], bl[2];
+    bh[0] = w.fr[ks * 64];
+    bh[1] = w.fr[ks * 64 + 32];
+    if constexpr (!PACK) {
+      bl[0] = w.fr[512 + ks * 64];
+      bl[1] = w.fr[512 + ks * 64 + 32];
+    } else {
+      bl[0] = bl[1] = 0u;
+    }
     uint32_t W0[KWN], W1[KWN], W0h[KWN], W1h[KWN];
 #pragma unroll
     for (int q = 0; q < KWN; ++q) {
-      if constexpr (kHoistK) {
-        W0[q] = KWa[ks][q];
-        W1[q] = KWb[ks][q];
-      } else if constexpr (BK != 0) {
+      if constexpr (BK != 0) {
         W0[q] = w.pk[r0 * 8 * BK + w.g * BK + KW0 + q];
         W1[q] = w.pk[r1 * 8 * BK + w.g * BK + KW0 + q];
       } else {
@@ -502,7 +467,7 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
       W0h[q] = shr8(W0[q]);
       W1h[q] = shr8(W1[q]);
     }
-    (k_block<BK, BV, PACK, B0 + BB>(w, ks, W0[((B0 + BB) * KB) / 8 - KW0], W0h[((B0 + BB) * KB) / 8 - KW0],
+    (k_block<BK, BV, PACK, B0 + BB>(w, bh, bl, W0[((B0 + BB) * KB) / 8 - KW0], W0h[((B0 + BB) * KB) / 8 - KW0],
                                     W1[((B0 + BB) * KB) / 8 - KW0], W1h[((B0 + BB) * KB) / 8 - KW0], r0, r1,
                                     sc[BB], sd[BB]),
      ...);
@@ -547,19 +512,13 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
         for (int mt = 0; mt < kNT; ++mt) {
           w.z[mt][c] *= resc;
           w.z[mt][2 + c] *= resc;
-          if constexpr (kZSplit) {
-            w.z2[mt][c] *= resc;
-            w.z2[mt][2 + c] *= resc;
-          }
         }
-        if constexpr (PACK)
-        {
+        if constexpr (PACK) {
           w.zl[0] *= resc;
-          if constexpr (kZSplit) w.zl2[0] *= resc;
           w.lfold *= resc;
-        }
-        else
+        } else {
           w.lcvt[c] *= resc;
+        }
       }
 #pragma unroll
       for (int bb = 0; bb < IL; ++bb) {
@@ -585,8 +544,7 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
       // uncompressed values: each A register is one stored word (a token pair of one
       // coordinate, fp16 as stored); rows 16 mt + g and + 8 of the raw page
       const uint32_t* row0 = w.pv + (16 * mt + w.g) * (kPage / 2);
-      (raw_v_block<BK, BV, PACK, B0 + BB>(w, row0, bp[BB], (kZSplit && ((B0 + BB) & 1)) ? w.z2[mt] : w.z[mt]),
-       ...);
+      (raw_v_block<BK, BV, PACK, B0 + BB>(w, row0, bp[BB], w.z[mt]), ...);
       return;
     }
     const int j0 = 16 * mt + w.g, j1 = j0 + 8;
@@ -594,10 +552,7 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
     uint32_t W0[VWN], W1[VWN], W0h[VWN], W1h[VWN];
 #pragma unroll
     for (int q = 0; q < VWN; ++q) {
-      if constexpr (kHoistV) {
-        W0[q] = VWa[mt][q];
-        W1[q] = VWb[mt][q];
-      } else if constexpr (BV != 0) {
+      if constexpr (BV != 0) {
         W0[q] = w.pv[j0 * 4 * BV + w.tq * BV + VW0 + q];
         W1[q] = w.pv[j1 * 4 * BV + w.tq * BV + VW0 + q];
       } else {
@@ -608,59 +563,18 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
     }
     (v_block<BK, BV, PACK, B0 + BB>(w, W0[((B0 + BB) * VB) / 8 - VW0], W0h[((B0 + BB) * VB) / 8 - VW0],
                                     W1[((B0 + BB) * VB) / 8 - VW0], W1h[((B0 + BB) * VB) / 8 - VW0], j0, j1, ones,
-                                    bp[BB], (kZSplit && ((B0 + BB) & 1)) ? w.z2[mt] : w.z[mt]),
+                                    bp[BB], w.z[mt]),
      ...);
   };
-  if constexpr (kBlockOuterV && (BV == 2 || BV == 4 || BV == 8)) {
-    // One fully unrolled value phase per m-tile count: the packed words of every tile
-    // first, then blocks outer and tiles inner, so consecutive MMAs feed different
-    // accumulators (no MMA waits on the one before it).
-    auto vphase = [&](auto NMTC) {
-      constexpr int NMT = decltype(NMTC)::value;
-      uint32_t W0[NMT][VWN], W1[NMT][VWN], W0h[NMT][VWN], W1h[NMT][VWN];
-#pragma unroll
-      for (int mt = 0; mt < NMT; ++mt) {
-        const int j0 = 16 * mt + w.g;
-#pragma unroll
-        for (int q = 0; q < VWN; ++q) {
-          W0[mt][q] = w.pv[j0 * 4 * BV + w.tq * BV + VW0 + q];
-          W1[mt][q] = w.pv[(j0 + 8) * 4 * BV + w.tq * BV + VW0 + q];
-          W0h[mt][q] = shr8(W0[mt][q]);
-          W1h[mt][q] = shr8(W1[mt][q]);
-        }
-      }
-      auto blk = [&](auto BBC) {
-        constexpr int BB = decltype(BBC)::value;
-        constexpr int qi = ((B0 + BB) * VB) / 8 - VW0;
-#pragma unroll
-        for (int mt = 0; mt < NMT; ++mt)
-          v_block<BK, BV, PACK, B0 + BB>(w, W0[mt][qi], W0h[mt][qi], W1[mt][qi], W1h[mt][qi], 16 * mt + w.g,
-                                         16 * mt + w.g + 8, !PACK && mt == w.ones_mt, bp[BB],
-                                         (kZSplit && ((B0 + BB) & 1)) ? w.z2[mt] : w.z[mt]);
-      };
-      (blk(std::integral_constant<int, BB>{}), ...);
-    };
-    switch (w.nmt) {
-      case 1: vphase(std::integral_constant<int, 1>{}); break;
-      case 2: vphase(std::integral_constant<int, 2>{}); break;
-      case 3: vphase(std::integral_constant<int, 3>{}); break;
-      case 4: vphase(std::integral_constant<int, 4>{}); break;
-      case 5: vphase(std::integral_constant<int, 5>{}); break;
-      case 6: vphase(std::integral_constant<int, 6>{}); break;
-      case 7: vphase(std::integral_constant<int, 7>{}); break;
-      default: vphase(std::integral_constant<int, 8>{}); break;
-    }
-  } else {
-    switch (w.nmt) {
-      default: vtile(std::integral_constant<int, 7>{}); [[fallthrough]];
-      case 7: vtile(std::integral_constant<int, 6>{}); [[fallthrough]];
-      case 6: vtile(std::integral_constant<int, 5>{}); [[fallthrough]];
-      case 5: vtile(std::integral_constant<int, 4>{}); [[fallthrough]];
-      case 4: vtile(std::integral_constant<int, 3>{}); [[fallthrough]];
-      case 3: vtile(std::integral_constant<int, 2>{}); [[fallthrough]];
-      case 2: vtile(std::integral_constant<int, 1>{}); [[fallthrough]];
-      case 1: vtile(std::integral_constant<int, 0>{});
-    }
+  switch (w.nmt) {
+    default: vtile(std::integral_constant<int, 7>{}); [[fallthrough]];
+    case 7: vtile(std::integral_constant<int, 6>{}); [[fallthrough]];
+    case 6: vtile(std::integral_constant<int, 5>{}); [[fallthrough]];
+    case 5: vtile(std::integral_constant<int, 4>{}); [[fallthrough]];
+    case 4: vtile(std::integral_constant<int, 3>{}); [[fallthrough]];
+    case 3: vtile(std::integral_constant<int, 2>{}); [[fallthrough]];
+    case 2: vtile(std::integral_constant<int, 1>{}); [[fallthrough]];
+    case 1: vtile(std::integral_constant<int, 0>{});
   }
 }
 
@@ -674,22 +588,154 @@ __device__ __forceinline__ void do_page(WS<BK, BV, PACK>& w) {
   do_page_groups<BK, BV, PACK>(w, std::make_integer_sequence<int, 8 / kIL>{});
 }
 
+// Bytes before the stage ring: the head, then the stage barriers (8 per warp, 16-byte
+// aligned), rounded to 128.
+constexpr size_t kBarOffset = (sizeof(SmemHead) + 15) / 16 * 16;
+constexpr size_t kHeadBytes = ((kBarOffset + 8 * kWarps * 8 + 127) / 128) * 128;
+
+// ---- q~ = M_K q for the CTA's query heads, on the tensor cores -------------------------
+// q of head n (n < ng) is scaled by 2^-Eq[n] and stored as fp16 hi (+ lo for fp32 input);
+// A = M_K's fp16 hi and lo fragments (plan), so q~ = (M_hi + M_lo)(q_hi + q_lo) with the
+// lo x lo product dropped (below 2^-22 relative).  Warp w forms m-tiles w, w + 4; the
+// result (column n = head n) lands in sh.qt, rows past r_K exactly zero (zero A rows).
+__device__ __forceinline__ void form_qtilde(SmemHead& sh, const uint32_t* mfrag, int nmtK, int warp, int lane,
+                                            bool q_lo) {
+  const int g = lane >> 2, tq = lane & 3;
+  for (int mt = warp; mt < nmtK; mt += kWarps) {
+    float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const uint4* fr = reinterpret_cast<const uint4*>(mfrag) + static_cast<size_t>(mt) * 8 * 2 * 32 + lane;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint4 ah = __ldg(fr + (ks * 2 + 0) * 32);
+      const uint4 alo = __ldg(fr + (ks * 2 + 1) * 32);
+      const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.hi[g][16 * ks + 2 * tq]);
+      const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.hi[g][16 * ks + 8 + 2 * tq]);
+      mma_16816(c, ah.x, ah.y, ah.z, ah.w, b0, b1);
+      mma_16816(c, alo.x, alo.y, alo.z, alo.w, b0, b1);
+      if (q_lo) {
+        const uint32_t l0 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.lo[g][16 * ks + 2 * tq]);
+        const uint32_t l1 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.lo[g][16 * ks + 8 + 2 * tq]);
+        mma_16816(c, ah.x, ah.y, ah.z, ah.w, l0, l1);
+      }
+    }
+    const int j = 16 * mt + g;
+    const float s0 = ldexpf(1.0f, sh.Eq[2 * tq]), s1 = ldexpf(1.0f, sh.Eq[2 * tq + 1]);
+    sh.qt[2 * tq][j] = c[0] * s0;
+    sh.qt[2 * tq + 1][j] = c[1] * s1;
+    sh.qt[2 * tq][j + 8] = c[2] * s0;
+    sh.qt[2 * tq + 1][j + 8] = c[3] * s1;
+  }
+}
+
+// ---- the last CTA of a (sequence, KV head, head group): merge and back-project ------------
+// Partials (m in the log2 domain, l, centred z times 2^-17) of every split; warp w merges
+// heads w and w + 4.  y = delta_V 2^17 z / l, then o = M_V^T y: warp w takes the rows
+// j = w, w + 4, ... of M_V (lane l: columns 4l..4l+3), the four warps' sums meet in shared
+// memory.  scratch: ng * n_split + 8 * 128 + 4 * 8 * 128 floats.
+__device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDesc& dV, float* scratch, int s,
+                                              int qh0, int ng, int n_split, int warp, int lane, int tid) {
+  const int Hq = a.H * a.G;
+  const int rV = dV.r;
+  const bool raw = dV.b == kRawBits;
+  float* wbuf = scratch;                                       // [ng][n_split]
+  float* ybuf = scratch + ((ng * n_split + 31) & ~31);         // [8][128]
+  float* obuf = ybuf + 8 * 128;                                // [4][8][128]
+  const float dlt = raw ? 0x1p-24f : dV.delta;
+  for (int n = warp; n < ng; n += kWarps) {
+    const float* base = a.ws + (static_cast<size_t>(s) * Hq + qh0 + n) * a.part_stride * kPartStride;
+    float M = -INFINITY;
+    for (int i = lane; i < n_split; i += 32) M = fmaxf(M, __ldcg(base + static_cast<size_t>(i) * kPartStride));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.0f;
+    for (int i = lane; i < n_split; i += 32) {
+      const float* pp = base + static_cast<size_t>(i) * kPartStride;
+      const float mi = __ldcg(pp);
+      const float wi = (mi == -INFINITY || M == -INFINITY) ? 0.0f : ex2(mi - M);
+      wbuf[n * n_split + i] = wi;
+      L = fmaf(wi, __ldcg(pp + 1), L);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    __syncwarp();
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (4 * lane < rV) {
+#pragma unroll 8
+      for (int i = 0; i < n_split; ++i) {
+        const float wi = wbuf[n * n_split + i];
+        const float4 z4 = __ldcg(reinterpret_cast<const float4*>(base + static_cast<size_t>(i) * kPartStride + 4) + lane);
+        acc.x = fmaf(wi, z4.x, acc.x);
+        acc.y = fmaf(wi, z4.y, acc.y);
+        acc.z = fmaf(wi, z4.z, acc.z);
+        acc.w = fmaf(wi, z4.w, acc.w);
+      }
+    }
+    // z holds sum p (c - m_V) 2^-17: dequantize
+    const float f = L > 0.0f ? dlt * 131072.0f / L : 0.0f;
+    reinterpret_cast<float4*>(ybuf + n * 128)[lane] =
+        4 * lane < rV ? make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  }
+  __syncthreads();
+  if (raw) {
+    // an uncompressed value unit is already in d-space (identity back-projection)
+    for (int i = tid; i < ng * 128; i += kThreads) {
+      const int n = i >> 7, k = i & 127;
+      const size_t off = (static_cast<size_t>(s) * Hq + qh0 + n) * kD + k;
+      if (a.out_bf16)
+        static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(ybuf[n * 128 + k]);
+      else
+        static_cast<float*>(a.out)[off] = ybuf[n * 128 + k];
+    }
+    return;
+  }
+  float4 o[8];
+#pragma unroll
+  for (int n = 0; n < 8; ++n) o[n] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll 4
+  for (int j = warp; j < rV; j += kWarps) {
+    const float4 m4 = __ldg(reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD) + lane);
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      if (n < ng) {
+        const float yj = ybuf[n * 128 + j];
+        o[n].x = fmaf(m4.x, yj, o[n].x);
+        o[n].y = fmaf(m4.y, yj, o[n].y);
+        o[n].z = fmaf(m4.z, yj, o[n].z);
+        o[n].w = fmaf(m4.w, yj, o[n].w);
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < 8; ++n)
+    if (n < ng) reinterpret_cast<float4*>(obuf + (warp * 8 + n) * 128)[lane] = o[n];
+  __syncthreads();
+  for (int i = tid; i < ng * 128; i += kThreads) {
+    const int n = i >> 7, k = i & 127;
+    const float v = (obuf[(0 * 8 + n) * 128 + k] + obuf[(1 * 8 + n) * 128 + k]) +
+                    (obuf[(2 * 8 + n) * 128 + k] + obuf[(3 * 8 + n) * 128 + k]);
+    const size_t off = (static_cast<size_t>(s) * Hq + qh0 + n) * kD + k;
+    if (a.out_bf16)
+      static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(v);
+    else
+      static_cast<float*>(a.out)[off] = v;
+  }
+}
+
 template <int BK, int BV, bool PACK>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
   // Programmatic dependent launch.  The first split launch of a call waits, once it has
-  // read the plan, for the preceding grid (the q~ prep kernel, which completes only after
-  // its own predecessor, e.g. the append that wrote the newest token), and triggers its
-  // dependents only after that wait.  A later split launch of the same call therefore
-  // starts only when the prep grid is complete: it reads at once and waits at exit
-  // instead, which keeps completion ordered for the combine.
+  // read the plan, for the preceding grid (whatever wrote q and the newest cache slots),
+  // and triggers its dependents only after that wait.  A later split launch of the same
+  // call starts only after that point, so it reads at once and waits at exit instead,
+  // which keeps the call's completion ordered behind every launch of it.
   extern __shared__ __align__(128) unsigned char smem[];
   SmemHead& sh = *reinterpret_cast<SmemHead*>(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sizeof(SmemHead));
-  unsigned char* stages = smem + ((sizeof(SmemHead) + 8 * kWarps * 8 + 127) / 128) * 128;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
+  unsigned char* stages = smem + kHeadBytes;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
-  // CTA -> (KV head, context split): heads get splits in proportion to their bytes
+  // CTA -> (KV head, context split): heads get splits in proportion to their work
   int hi = 0;
   while (hi + 1 < a.n_heads && static_cast<int>(blockIdx.x) >= a.split_prefix[hi + 1]) ++hi;
   const int split = blockIdx.x - a.split_prefix[hi];
@@ -698,14 +744,16 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const int s = blockIdx.z;
   const int h = a.heads[hi];
   const int uK = (a.layer * a.H + h) * 2, uV = uK + 1;
-  // the plan is constant: its unit descriptors are read, and the stage barriers set up,
-  // before the wait for the preceding grid
+  // the plan is constant: its unit descriptors are read, the stage barriers set up and
+  // M_V prefetched into L2 (for the merge) before the wait for the preceding grid
   const UnitDesc dK = a.units[uK], dV = a.units[uV];
   const int rK = dK.r, rV = dV.r;
   const int Hq = a.H * a.G;
   const int g0 = hg * 8, ng = min(8, a.G - g0);
+  const int nmtK = (rK + 15) >> 4;
   if (lane == 0)
     for (int i = 0; i < a.n_stage; ++i) mbar_init(&bars[warp * 8 + i], 1);
+  if (tid == 0 && dV.b != kRawBits) prefetch_l2(dV.M, static_cast<uint32_t>(rV) * kD * 4);
   if (a.wait_first) griddep_wait();
   griddep_launch_dependents();
 
@@ -769,15 +817,41 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     if (lane == 0) issue(i, pid);  // page i < n_stage uses slot i
   }
 
-  for (int i = tid; i < 8 * 32; i += kThreads) {
-    const int gg = i >> 5, k4 = i & 31;
+  // ---- q of the group into shared memory as fp16, scaled per head (warp w: heads 2w,
+  // 2w + 1; lane l: elements 4l .. 4l + 3); q~ cleared
+  const bool q_lo = !a.q_bf16;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int gg = 2 * warp + hh;
     float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    if (gg < ng && 4 * k4 < rK) {
-      v = reinterpret_cast<const float4*>(a.qt + (static_cast<size_t>(s) * Hq + h * a.G + g0 + gg) * kD)[k4];
-      if (4 * k4 + 2 >= rK) v.z = v.w = 0.0f;  // r_K is even: only the upper pair can be past it
+    if (gg < ng) {
+      const size_t off = (static_cast<size_t>(s) * Hq + h * a.G + g0 + gg) * kD + 4 * lane;
+      if (a.q_bf16) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.q) + off);
+        v = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                        __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u));
+      } else {
+        v = *reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + off);
+      }
     }
-    reinterpret_cast<float4*>(sh.qt[gg])[k4] = v;
+    float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    // max |q| 2^-Eq in [2^14, 2^15): fp16 holds it with headroom
+    const int Eq = (amax > 0.0f && amax < INFINITY) ? ilogbf(amax) - 14 : 0;
+    const float sc = ldexpf(1.0f, -Eq);
+    const float xs[4] = {v.x * sc, v.y * sc, v.z * sc, v.w * sc};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __half hq = __float2half_rn(xs[e]);
+      sh.u.q16.hi[gg][4 * lane + e] = __half_as_ushort(hq);
+      sh.u.q16.lo[gg][4 * lane + e] = __half_as_ushort(__float2half_rn(xs[e] - __half2float(hq)));
+    }
+    if (lane == 0) sh.Eq[gg] = Eq;
   }
+  for (int i = tid; i < 8 * 128; i += kThreads) sh.qt[i >> 7][i & 127] = 0.0f;
+  __syncthreads();
+  form_qtilde(sh, dK.Mfrag, nmtK, warp, lane, q_lo);
   __syncthreads();
 
   // per head: S = sum_j q~_j and the fp16 normalisation exponent (warp w: heads 2w, 2w+1)
@@ -799,10 +873,34 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   }
   __syncthreads();
 
+  // B fragments of q^ = q~ * 2^-E, shared by the four warps: [hi, lo][k-step][half][lane]
+  // (lane (g, t): rows 16 ks + 8 half + 2t, + 1, column g).  Packed (G <= 4): column n
+  // holds head n / 2, its hi part for even n and its lo part for odd n.
+  for (int idx = tid; idx < 8 * 2 * 32; idx += kThreads) {
+    const int ks = idx >> 6, half = (idx >> 5) & 1, ln = idx & 31;
+    const int gl = ln >> 2, tql = ln & 3;
+    const int hsrc = PACK ? (gl >> 1) : gl;
+    const float scl = ldexpf(1.0f, -sh.E[hsrc]);
+    const int k0 = 16 * ks + 8 * half + 2 * tql;
+    const float x0 = sh.qt[hsrc][k0] * scl, x1 = sh.qt[hsrc][k0 + 1] * scl;
+    const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+    const __half l0 = __float2half_rn(x0 - __half2float(h0)), l1 = __float2half_rn(x1 - __half2float(h1));
+    const uint32_t hw = static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
+    const uint32_t lw = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
+    if constexpr (PACK) {
+      sh.u.frag[0][ks][half][ln] = (gl & 1) ? lw : hw;
+    } else {
+      sh.u.frag[0][ks][half][ln] = hw;
+      sh.u.frag[1][ks][half][ln] = lw;
+    }
+  }
+  __syncthreads();
+
   WS<BK, BV, PACK> w;
+  w.fr = &sh.u.frag[0][0][0][lane];
   w.rK = rK;
   w.rV = rV;
-  w.nks = (rK + 15) >> 4;
+  w.nks = nmtK;
   w.nmt = (rV + 15) >> 4;
   w.g = g;
   w.tq = tq;
@@ -815,30 +913,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   w.ones_lr = rV & 15;
   w.ones_m0 = (w.ones_mt >= 0 && w.ones_lr == g) ? 0xFFFFFFFFu : 0u;
   w.ones_m1 = (w.ones_mt >= 0 && w.ones_lr == g + 8) ? 0xFFFFFFFFu : 0u;
-  // B fragments of q^ = q~ * 2^-E.  Packed (G <= 4): column n holds head n / 2, its hi
-  // part for even n and its lo part for odd n.
-  {
-    const int hsrc = PACK ? (g >> 1) : g;
-    const float scl = ldexpf(1.0f, -sh.E[hsrc]);
-#pragma unroll
-    for (int ks = 0; ks < kNT; ++ks) {
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int k0 = 16 * ks + 8 * half + 2 * tq;
-        const float x0 = sh.qt[hsrc][k0] * scl, x1 = sh.qt[hsrc][k0 + 1] * scl;
-        const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
-        const __half l0 = __float2half_rn(x0 - __half2float(h0)), l1 = __float2half_rn(x1 - __half2float(h1));
-        const uint32_t hw = static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
-        const uint32_t lw = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
-        if constexpr (PACK) {
-          w.bh[ks][half] = (g & 1) ? lw : hw;
-        } else {
-          w.bh[ks][half] = hw;
-          w.bl[ks][half] = lw;
-        }
-      }
-    }
-  }
   // Score constants (log2 domain) for this lane's heads.
   {
     const float mK = 0.5f * static_cast<float>((1 << dK.b) - 1);
@@ -862,16 +936,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       }
     }
     w.zl[0] = w.zl[1] = w.zl[2] = w.zl[3] = 0.0f;
-    w.zl2[0] = w.zl2[1] = w.zl2[2] = w.zl2[3] = 0.0f;
     w.mV = dV.b == kRawBits ? 0.0f : 0.5f;
     w.lfold = 0.0f;
     w.cmV = dV.b == kRawBits ? 0u : ((1u << (dV.b - 1)) - 1u) * 0x10001u;
   }
 #pragma unroll
-  for (int mt = 0; mt < kNT; ++mt) {
-    w.z[mt][0] = w.z[mt][1] = w.z[mt][2] = w.z[mt][3] = 0.0f;
-    if constexpr (kZSplit) w.z2[mt][0] = w.z2[mt][1] = w.z2[mt][2] = w.z2[mt][3] = 0.0f;
-  }
+  for (int mt = 0; mt < kNT; ++mt) w.z[mt][0] = w.z[mt][1] = w.z[mt][2] = w.z[mt][3] = 0.0f;
 
   // ---- main loop over this warp's pages ----
   bool dead = false;
@@ -921,13 +991,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     }
   }
 
-  if constexpr (kZSplit) {
-#pragma unroll
-    for (int mt = 0; mt < kNT; ++mt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) w.z[mt][i] += w.z2[mt][i];
-    w.zl[0] += w.zl2[0];
-  }
   // ---- l: from the ones row, or the per-lane sums ----
   float l_out[2];
 #pragma unroll
@@ -1023,6 +1086,19 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     } else if (e <= rV) {
       dst[4 + (e - 1)] = acc;
     }
+  }
+
+  // ---- arrival ticket: the CTA that completes the (sequence, KV head, head group) last
+  // merges every split's partial and writes the output, then re-arms the ticket ----
+  __threadfence();
+  __syncthreads();
+  int* ticket = a.tickets + (static_cast<size_t>(s) * a.H + h) * a.n_hg + hg;
+  if (tid == 0) sh.last = atomicAdd(ticket, 1) == n_split - 1;
+  __syncthreads();
+  if (sh.last) {
+    __threadfence();
+    merge_project(a, dV, mb, s, h * a.G + g0, ng, n_split, warp, lane, tid);
+    if (tid == 0) atomicExch(ticket, 0);
   }
   if (!a.wait_first) griddep_wait();
 }

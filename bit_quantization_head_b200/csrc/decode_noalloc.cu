@@ -18,13 +18,15 @@
 namespace kvtc {
 namespace {
 
-// 16 MiB: enough for the split-K partials of one 131072-token sequence of a 32-query-head
-// model (kvtc_decode_workspace_bytes gives the exact need of a call).
+// 16 MiB: the arrival tickets and split-K partials of seven 131072-token sequences of a
+// 32-query-head model (kvtc_decode_workspace_bytes gives the exact need of a call).  The
+// array is zero when the module loads and every call returns its tickets to zero.
 constexpr size_t kScratchBytes = 16u << 20;
 constexpr int kMaxDevices = 64;
 
 // In host code this name is only a handle for cudaGetSymbolAddress; it is not a device
-// address and must never be passed to a kernel directly.
+// address and must never be passed to a kernel directly.  The address found for a device
+// is kept for the life of the process (it does not survive cudaDeviceReset).
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 std::mutex g_mu;

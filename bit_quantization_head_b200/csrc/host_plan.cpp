@@ -43,17 +43,58 @@ static uint16_t bf16_bits(float x) {
   return static_cast<uint16_t>((u + rounding) >> 16);
 }
 
+// fp16 bits of x, round to nearest even (subnormals kept, overflow to infinity).
+static uint16_t fp16_bits(float x) {
+  uint32_t u;
+  std::memcpy(&u, &x, 4);
+  const uint32_t sign = (u >> 16) & 0x8000u;
+  const uint32_t ax = u & 0x7FFFFFFFu;
+  if (ax >= 0x7F800000u) return static_cast<uint16_t>(sign | 0x7C00u | (ax > 0x7F800000u ? 0x200u : 0u));
+  if (ax >= 0x477FF000u) return static_cast<uint16_t>(sign | 0x7C00u);  // rounds past 65504
+  if (ax < 0x33000001u) return static_cast<uint16_t>(sign);              // below half the least subnormal
+  int e = static_cast<int>(ax >> 23) - 127;
+  uint32_t m = (ax & 0x7FFFFFu) | 0x800000u;                             // 24-bit significand
+  // value = m * 2^(e - 23); fp16 keeps 11 bits for normals (e >= -14), fewer below
+  const int shift = e >= -14 ? 13 : 13 + (-14 - e);
+  const uint32_t q = m >> shift, rem = m & ((1u << shift) - 1u), half = 1u << (shift - 1);
+  uint32_t r = q + ((rem > half || (rem == half && (q & 1u))) ? 1u : 0u);
+  if (e >= -14) {
+    // r holds 11 significant bits (or 2^11 after rounding up)
+    uint32_t exp = static_cast<uint32_t>(e + 15);
+    if (r == 0x800u) {
+      r = 0x400u;
+      ++exp;
+    }
+    if (exp >= 31) return static_cast<uint16_t>(sign | 0x7C00u);
+    return static_cast<uint16_t>(sign | (exp << 10) | (r & 0x3FFu));
+  }
+  return static_cast<uint16_t>(sign | r);  // subnormal (r == 0x400 is the least normal)
+}
+
+static float fp16_value(uint16_t h) {
+  const uint32_t sign = (h & 0x8000u) ? 1u : 0u;
+  const int exp = (h >> 10) & 31;
+  const int man = h & 0x3FF;
+  float v = exp == 0 ? std::ldexp(static_cast<float>(man), -24) : std::ldexp(static_cast<float>(man | 0x400), exp - 25);
+  return sign ? -v : v;
+}
+
 static void free_device(kvtc_plan* p) {
   if (p->d_units) cudaFree(p->d_units);
   if (p->d_M) cudaFree(p->d_M);
   if (p->d_Mbf) cudaFree(p->d_Mbf);
+  if (p->d_Mfrag) cudaFree(p->d_Mfrag);
+  if (p->d_Mrec) cudaFree(p->d_Mrec);
   if (p->d_stats) cudaFree(p->d_stats);
   p->d_stats = nullptr;
   p->d_units = nullptr;
   p->d_M = nullptr;
   p->d_Mbf = nullptr;
+  p->d_Mfrag = nullptr;
+  p->d_Mrec = nullptr;
   p->device = -1;
   p->h_units.clear();
+  p->dec_groups.clear();
 }
 
 }  // namespace kvtc
@@ -277,8 +318,70 @@ kvtc_status kvtc_plan_upload(kvtc_plan* plan, void* stream) {
       hM.push_back(x);
       hMbf.push_back(bf16_bits(x));
     }
+  // fp16 hi/lo A fragments of every M (m16n8k16 layout: lane (g, t) holds rows g, g + 8
+  // and columns 2t, 2t + 1, 2t + 8, 2t + 9 of a 16 x 16 tile)
+  std::vector<uint32_t> hFrag;
+  std::vector<size_t> frag_off(plan->U);
+  for (int u = 0; u < plan->U; ++u) {
+    frag_off[u] = hFrag.size();
+    const int r = plan->r[u], nmt = (r + 15) / 16;
+    const std::vector<float>& Mu = plan->M[u];
+    auto part = [&](int row, int col, int p) -> uint32_t {
+      if (row >= r) return 0u;
+      const float x = Mu[static_cast<size_t>(row) * kD + col];
+      const uint16_t hi = fp16_bits(x);
+      return p == 0 ? hi : fp16_bits(x - fp16_value(hi));
+    };
+    for (int mt = 0; mt < nmt; ++mt)
+      for (int ks = 0; ks < 8; ++ks)
+        for (int p = 0; p < 2; ++p)
+          for (int lane = 0; lane < 32; ++lane) {
+            const int g = lane >> 2, t = lane & 3;
+            const int r0 = 16 * mt + g, c0 = 16 * ks + 2 * t;
+            const int rows[4] = {r0, r0 + 8, r0, r0 + 8};
+            const int cols[4] = {c0, c0, c0 + 8, c0 + 8};
+            for (int i = 0; i < 4; ++i)
+              hFrag.push_back(part(rows[i], cols[i], p) | (part(rows[i], cols[i] + 1, p) << 16));
+          }
+  }
+  // key units: M^T in B-fragment order for the reconstruction K-hat = C M (lane (g, t) of
+  // n-tile nt, k-step ks: b0 = M[16ks + 2t .. + 1][8nt + g], b1 = M[16ks + 8 + 2t .. + 1][8nt + g]),
+  // hi and lo parts, followed by the fp32 column sums of M
+  std::vector<uint32_t> hRec;
+  std::vector<size_t> rec_off(plan->U, 0);
+  for (int u = 0; u < plan->U; u += 2) {
+    rec_off[u] = hRec.size();
+    const int r = plan->r[u], nks = (r + 15) / 16;
+    const std::vector<float>& Mu = plan->M[u];
+    auto el = [&](int row, int col, int p) -> uint32_t {
+      if (row >= r) return 0u;
+      const float x = Mu[static_cast<size_t>(row) * kD + col];
+      const uint16_t hi = fp16_bits(x);
+      return p == 0 ? hi : fp16_bits(x - fp16_value(hi));
+    };
+    for (int ks = 0; ks < nks; ++ks)
+      for (int nt = 0; nt < 16; ++nt)
+        for (int lane = 0; lane < 32; ++lane) {
+          const int g = lane >> 2, t = lane & 3;
+          const int col = 8 * nt + g, r0 = 16 * ks + 2 * t;
+          for (int p = 0; p < 2; ++p) {
+            hRec.push_back(el(r0, col, p) | (el(r0 + 1, col, p) << 16));
+            hRec.push_back(el(r0 + 8, col, p) | (el(r0 + 9, col, p) << 16));
+          }
+        }
+    for (int col = 0; col < kD; ++col) {
+      double cs = 0.0;
+      for (int row = 0; row < r; ++row) cs += Mu[static_cast<size_t>(row) * kD + col];
+      const float f = static_cast<float>(cs);
+      uint32_t bits;
+      std::memcpy(&bits, &f, 4);
+      hRec.push_back(bits);
+    }
+  }
   if ((e = cudaMalloc(&plan->d_M, total * sizeof(float))) != cudaSuccess ||
+      (e = cudaMalloc(&plan->d_Mrec, std::max<size_t>(1, hRec.size()) * sizeof(uint32_t))) != cudaSuccess ||
       (e = cudaMalloc(&plan->d_Mbf, total * sizeof(uint16_t))) != cudaSuccess ||
+      (e = cudaMalloc(&plan->d_Mfrag, std::max<size_t>(1, hFrag.size()) * sizeof(uint32_t))) != cudaSuccess ||
       (e = cudaMalloc(&plan->d_units, plan->U * sizeof(UnitDesc))) != cudaSuccess ||
       (e = cudaMalloc(&plan->d_stats, 2 * sizeof(uint64_t))) != cudaSuccess ||
       (e = cudaMemsetAsync(plan->d_stats, 0, 2 * sizeof(uint64_t), st)) != cudaSuccess) {
@@ -298,6 +401,14 @@ kvtc_status kvtc_plan_upload(kvtc_plan* plan, void* stream) {
     ud.prefix = prefix;
     ud.M = plan->d_M + off;
     ud.Mbf = plan->d_Mbf + off;
+    ud.Mfrag = plan->d_Mfrag + frag_off[u];
+    if (u % 2 == 0) {
+      ud.Mrec = plan->d_Mrec + rec_off[u];
+      ud.Msum = reinterpret_cast<const float*>(plan->d_Mrec + rec_off[u] + static_cast<size_t>((ud.r + 15) / 16) * 16 * 32 * 4);
+    } else {
+      ud.Mrec = nullptr;
+      ud.Msum = nullptr;
+    }
     double mn = 0.0;
     for (int i = 0; i < ud.r; ++i) {
       double ss = 0.0;
@@ -317,6 +428,10 @@ kvtc_status kvtc_plan_upload(kvtc_plan* plan, void* stream) {
           cudaSuccess ||
       (e = cudaMemcpyAsync(plan->d_Mbf, hMbf.data(), total * sizeof(uint16_t), cudaMemcpyHostToDevice,
                            st)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(plan->d_Mfrag, hFrag.data(), hFrag.size() * sizeof(uint32_t), cudaMemcpyHostToDevice,
+                           st)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(plan->d_Mrec, hRec.data(), hRec.size() * sizeof(uint32_t), cudaMemcpyHostToDevice,
+                           st)) != cudaSuccess ||
       (e = cudaMemcpyAsync(plan->d_units, plan->h_units.data(), plan->U * sizeof(UnitDesc),
                            cudaMemcpyHostToDevice, st)) != cudaSuccess ||
       (e = cudaStreamSynchronize(st)) != cudaSuccess) {
@@ -324,6 +439,11 @@ kvtc_status kvtc_plan_upload(kvtc_plan* plan, void* stream) {
     return cuda_fail(e, "plan upload copy");
   }
   plan->device = dev;
+  const kvtc_status ds = prepare_decode(plan);
+  if (ds != KVTC_OK) {
+    free_device(plan);
+    return ds;
+  }
   return KVTC_OK;
 }
 

@@ -30,7 +30,29 @@ struct UnitDesc {
   uint64_t prefix;     // sum of page_bytes over the units before this one
   const float* M;      // device fp32 [r][d]
   const uint16_t* Mbf; // device bf16 bits [r][d] (round-to-nearest-even of M)
+  // device: M as fp16 hi + lo parts (hi = RN16(M), lo = RN16(M - hi)) in m16n8k16
+  // A-fragment order, [ceil(r/16)][8 k-steps][2 parts][32 lanes][4 registers] (rows past r
+  // are zero); the decode forms q~ = M q from it on the tensor cores
+  const uint32_t* Mfrag;
+  // device, key units only (else null): M^T as fp16 hi + lo parts in m16n8k16 B-fragment
+  // order for K-hat = C M (C: codes, tokens x r), [ceil(r/16)][16 n-tiles][32 lanes][4]
+  // = (hi b0, hi b1, lo b0, lo b1); then the column sums sum_j M[j][i] (fp32 [128])
+  const uint32_t* Mrec;
+  const float* Msum;
   float mnorm;         // largest row 2-norm of the bf16 M (rounded up)
+};
+
+// One decode launch of a layer: the KV heads whose (b_K, b_V) width classes share a split
+// kernel variant, with the variant's shared-memory plan (decided once, at plan upload).
+struct DecodeGroup {
+  int wk = 0, wv = 0;           // width classes (2, 4, 8, 16 raw, 0 any)
+  std::vector<int> heads;       // KV heads of the layer in this launch
+  std::vector<double> cost;     // modelled cost of one page of each head (warp instructions)
+  uint32_t stage_bytes = 0;     // one K + V page of the widest head, 128-byte rounded
+  int n_stage = 0;              // stages per warp
+  size_t smem = 0;              // dynamic shared memory per CTA
+  int per_sm = 1;               // resident CTAs per SM at that size
+  const void* fn = nullptr;     // the kernel variant
 };
 
 // Sets the thread-local error message and returns the status.
@@ -53,11 +75,19 @@ struct kvtc_plan {
   kvtc::UnitDesc* d_units = nullptr;
   float* d_M = nullptr;
   uint16_t* d_Mbf = nullptr;
+  uint32_t* d_Mfrag = nullptr;
+  uint32_t* d_Mrec = nullptr;                // key units: reconstruction fragments + column sums
   uint64_t* d_stats = nullptr;               // prefill counters (codes, recomputed)
   std::vector<kvtc::UnitDesc> h_units;      // descriptors with device pointers
+  // decode launch plan, per layer (set at upload): the launches and the device's SM count
+  std::vector<std::vector<kvtc::DecodeGroup>> dec_groups;
+  int sm_count = 0;
 };
 
 namespace kvtc {
 // Validates that the plan is uploaded to the current device.
 kvtc_status check_uploaded(const kvtc_plan* plan);
+// Fills plan->dec_groups and plan->sm_count for the current device and sets the kernel
+// attributes the decode launches need (decode.cu; called by kvtc_plan_upload).
+kvtc_status prepare_decode(kvtc_plan* plan);
 }  // namespace kvtc

@@ -93,6 +93,8 @@ def lib():
                                        _P, C.c_int, _P, C.c_uint64, _P]),
         "kvtc_decode_attention_noalloc": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, C.c_int, _P, C.c_int,
                                                C.c_float, _P, C.c_int, _P]),
+        "kvtc_decode_attention_rope": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, C.c_int, _P, C.c_int, C.c_float,
+                                            C.c_double, _P, C.c_int, _P, C.c_uint64, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -311,3 +313,12 @@ def kvtc_decode_attention_noalloc(plan, cache, layer, q, seq_lens, max_seq_len, 
     _check(lib().kvtc_decode_attention_noalloc(plan.handle, C.byref(cache.desc), layer, _dev_ptr(q),
                                                _dtype_code(q), _dev_ptr(seq_lens), max_seq_len, scale,
                                                _dev_ptr(out), _dtype_code(out), _stream(stream)))
+
+
+def kvtc_decode_attention_rope(plan, cache, layer, q, seq_lens, max_seq_len, out, workspace, scale=0.0,
+                               rope_base=0.0, stream=None):
+    """Decode attention for keys coded before the rotary embedding (q already rotated)."""
+    _check(lib().kvtc_decode_attention_rope(plan.handle, C.byref(cache.desc), layer, _dev_ptr(q), _dtype_code(q),
+                                            _dev_ptr(seq_lens), max_seq_len, scale, float(rope_base), _dev_ptr(out),
+                                            _dtype_code(out), _dev_ptr(workspace),
+                                            workspace.numel() * workspace.element_size(), _stream(stream)))

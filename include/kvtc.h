@@ -283,7 +283,8 @@ kvtc_status kvtc_plan_prefill_stats(const kvtc_plan* plan, uint64_t* codes, uint
 /* ------------------------------------------------------------------ decode ------- */
 
 /* Workspace bytes kvtc_decode_attention needs for n_seq sequences of at most
- * max_seq_len tokens (split-K partials). */
+ * max_seq_len tokens: arrival tickets (one int32 per sequence, KV head and group of 8
+ * query heads) followed by the split-K partials. */
 uint64_t kvtc_decode_workspace_bytes(const kvtc_plan* plan, int n_seq, int max_seq_len);
 
 /*
@@ -294,21 +295,48 @@ uint64_t kvtc_decode_workspace_bytes(const kvtc_plan* plan, int n_seq, int max_s
  *   with m = (2^b - 1)/2, p = softmax over t < seq_len, z = sum_t p_t (c_V,t - m_V),
  *   o = M_V^T (delta_V * z).
  * Equivalent to softmax(scale * q . k_hat_t) v_hat_t with k_hat = M_K^T delta_K (c - m)
- * (the oracle's d-space form).  Split-K over the context with a log-sum-exp merge;
- * the G query heads of a KV head share every code tile.  An uncompressed value unit
- * (keys-only plans) enters the value MMAs with its fp16 values as they are stored
+ * (the oracle's d-space form).  Split-K over the context; the G query heads of a KV head
+ * share every code tile; the last split of a (sequence, KV head) to finish merges the
+ * partials (log-sum-exp) and back-projects, in the same kernel.  An uncompressed value
+ * unit (keys-only plans) enters the value MMAs with its fp16 values as they are stored
  * (c_V = v * 2^24, delta_V = 2^-24, m_V = 0, M_V = identity), so o = sum_t p_t v_t.
  * q: device [n_seq][H_q][d] of q_dtype.  seq_lens: device int32 [n_seq] (0 gives an
  * all-zero output).  max_seq_len: host upper bound of seq_lens (sizes the split grid;
  * longer sequences set KVTC_STATUS_BAD_POS).  softmax_scale: 0 means 1/sqrt(d).
  * out: device [n_seq][H_q][d] of out_dtype.  workspace: device, at least
- * kvtc_decode_workspace_bytes(plan, n_seq, max_seq_len) bytes (else ECAPACITY).
+ * kvtc_decode_workspace_bytes(plan, n_seq, max_seq_len) bytes (else ECAPACITY), 16-byte
+ * aligned and zero-filled before its first use; every call leaves its tickets at zero
+ * again, so one workspace serves any number of consecutive calls (of any plan and shape
+ * that fits), but two calls that share a workspace and overlap on the GPU race.
+ * Launches one kernel per group of KV heads whose code widths share a kernel variant
+ * (one per layer when every head has the same widths); nothing is allocated.
  */
 kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_cache* cache, int layer,
                                   const void* q, kvtc_dtype q_dtype, const int32_t* seq_lens,
                                   int max_seq_len, float softmax_scale, void* out,
                                   kvtc_dtype out_dtype, void* workspace, uint64_t workspace_bytes,
                                   void* stream);
+
+/*
+ * kvtc_decode_attention_rope -- kvtc_decode_attention for caches whose keys were coded
+ * before the rotary position embedding (KV-COBRA project page, Results: keys compressed
+ * pre-RoPE).  The rotation of a key depends on its position, so q is not moved into the
+ * key basis: per 16-token block the keys are reconstructed in d-space,
+ * k_t = delta_K (c_K,t - m_K) M_K (tensor cores), rotated to position t and scored:
+ *   s_t = scale * q . R(t) k_t,  R(t): (x_i, x_{i+64}) -> (x_i cos a - x_{i+64} sin a,
+ *   x_{i+64} cos a + x_i sin a), a = t * rope_base^(-2i/128), i < 64
+ * (the rotate-half form; cached token t of a sequence sits at position t; q arrives
+ * already rotated to its own position, as a model applies RoPE to q before attention).
+ * Values, softmax, split merge and back-projection as kvtc_decode_attention, through the
+ * same workspace (kvtc_decode_workspace_bytes, zero-filled before its first use).
+ * rope_base: 0 means 500000 (the Llama-3.1 value), else > 1.  The codes are those of
+ * kvtc_encode_append / kvtc_encode_prefill applied to the un-rotated keys.
+ */
+kvtc_status kvtc_decode_attention_rope(const kvtc_plan* plan, const kvtc_cache* cache, int layer,
+                                       const void* q, kvtc_dtype q_dtype, const int32_t* seq_lens,
+                                       int max_seq_len, float softmax_scale, double rope_base, void* out,
+                                       kvtc_dtype out_dtype, void* workspace, uint64_t workspace_bytes,
+                                       void* stream);
 
 /*
  * kvtc_decode_attention_noalloc -- kvtc_decode_attention without a caller workspace.
@@ -319,12 +347,16 @@ kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_cache* cache
  * (a file-scope __device__ array: every GPU that loads the library holds it until the
  * process exits); nothing is allocated per call.
  *   - The first call on a device looks up the array's device address (once per device,
- *     with that device current).  Make that first call before any stream capture.
+ *     with that device current).  Make that first call before any stream capture.  The
+ *     address is kept for the life of the process: after cudaDeviceReset (or anything
+ *     else that destroys the device's primary context) it is stale, and this call must
+ *     not be used on that device again.
  *   - Calls whose kvtc_decode_workspace_bytes(plan, n_seq, max_seq_len) exceeds 16 MiB
  *     return KVTC_ECAPACITY; use kvtc_decode_attention with a workspace for those.
- *   - Every call shares the one array and leaves its contents behind.  No part of it has
- *     to start at zero (each call writes every slot it later reads), but two calls that
- *     run at the same time on the GPU (different streams, or overlapping graphs) race.
+ *   - Every call shares the one array and leaves its contents behind.  The array starts
+ *     at zero when the library is loaded and every call returns its arrival tickets to
+ *     zero, so nothing has to be cleared between calls; but two calls that run at the
+ *     same time on the GPU (different streams, or overlapping graphs) race.
  * Arguments, results and error codes otherwise as kvtc_decode_attention.
  */
 kvtc_status kvtc_decode_attention_noalloc(const kvtc_plan* plan, const kvtc_cache* cache, int layer,

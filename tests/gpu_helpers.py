@@ -125,7 +125,7 @@ def run_decode(plan, cache, layer, q, seq_lens, out_dtype="f32", q_dtype="f32", 
     qd = to_dev(q, q_dtype)
     sl = torch.tensor(seq_lens, dtype=torch.int32).cuda()
     mx = max(seq_lens + [0])
-    ws = torch.empty(max(1, kvtc.kvtc_decode_workspace_bytes(plan, n_seq, mx)), dtype=torch.uint8).cuda()
+    ws = torch.zeros(max(1, kvtc.kvtc_decode_workspace_bytes(plan, n_seq, mx)), dtype=torch.uint8, device="cuda")
     out = torch.empty((n_seq, Hq, 128), dtype=torch.float32 if out_dtype == "f32" else torch.bfloat16).cuda()
     kvtc.kvtc_decode_attention(plan, cache, layer, qd, sl, mx, out, ws, scale)
     torch.cuda.synchronize()
