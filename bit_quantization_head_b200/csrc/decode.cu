@@ -80,8 +80,7 @@ size_t tickets_bytes(const kvtc_plan* plan, int n_seq) {
 
 // The decode launches of every layer: heads grouped by the kernel variant of their
 // (b_K, b_V) width classes, the stage size of each group, and the stage count and
-// occupancy that fit (three CTAs per SM with two or more stages per warp where the pages
-// allow it, else as many CTAs as fit one stage per warp).
+// occupancy that fit (the most CTAs per SM, up to three, that leave a stage per warp).
 // Sets each variant's shared-memory attribute once, here, so decode calls do no host
 // allocation and no attribute calls.
 kvtc_status prepare_decode(kvtc_plan* plan) {
@@ -119,18 +118,14 @@ kvtc_status prepare_decode(kvtc_plan* plan) {
       SplitFn fn = split_fn(gr.wk == 0 ? 3 : gr.wk, gr.wv == 0 ? 3 : gr.wv, pack);
       if (!fn) return fail(KVTC_EINVAL, "no decode kernel for this code width");
       gr.fn = reinterpret_cast<const void*>(fn);
-      // the most CTAs per SM that leave two stages per warp, else the most that leave one
-      int n_stage = 0, fallback = 0;
-      for (int target = kMinBlocks; target >= 1; --target) {
+      // the most CTAs per SM that leave at least one stage per warp (more resident warps
+      // beat deeper rings: with one stage a warp waits for its next page, but the other
+      // warps of the SM keep the pipes and the memory system busy)
+      int n_stage = 0;
+      for (int target = kMinBlocks; target >= 1 && n_stage < 1; --target) {
         const size_t budget = kSmemPerSM / target - kSmemReserved - kReadSlack - kHeadBytes;
-        const int n = static_cast<int>(budget / (static_cast<size_t>(kWarps) * gr.stage_bytes));
-        if (n >= 2) {
-          n_stage = n;
-          break;
-        }
-        if (n >= 1 && fallback == 0) fallback = n;
+        n_stage = static_cast<int>(budget / (static_cast<size_t>(kWarps) * gr.stage_bytes));
       }
-      if (n_stage == 0) n_stage = fallback;
       if (n_stage < 1) return fail(KVTC_EINVAL, "a page of this plan does not fit in shared memory");
       gr.n_stage = std::min(n_stage, 6);
       // + slack: the kernel reads whole 16-row tiles, up to 2 KB past a page's last row

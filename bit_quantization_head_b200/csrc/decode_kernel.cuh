@@ -52,8 +52,9 @@ constexpr int kMinBlocks = 3;         // resident CTAs per SM the registers are 
 constexpr int kPartStride = 132;      // floats per partial: m, l, 2 pad, z[128]
 constexpr int kMaxHeadsPerLaunch = 64;
 constexpr int kMaxSplits = 128;       // context splits per KV head (bounds the merge scratch)
-// floats of merge scratch the last CTA needs (weights, y, the warps' back-projections)
-constexpr int kMergeFloats = 8 * kMaxSplits + 8 * 128 + 4 * 8 * 128;
+// floats of merge scratch the last CTA needs ((m, l) of every split, y, the warps'
+// back-projections)
+constexpr int kMergeFloats = 16 * kMaxSplits + 8 * 128 + 4 * 8 * 128;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;         // log2 of the growth allowed before a rescale
 
@@ -628,52 +629,99 @@ __device__ __forceinline__ void form_qtilde(SmemHead& sh, const uint32_t* mfrag,
 }
 
 // ---- the last CTA of a (sequence, KV head, head group): merge and back-project ------------
-// Partials (m in the log2 domain, l, centred z times 2^-17) of every split; warp w merges
-// heads w and w + 4.  y = delta_V 2^17 z / l, then o = M_V^T y: warp w takes the rows
-// j = w, w + 4, ... of M_V (lane l: columns 4l..4l+3), the four warps' sums meet in shared
-// memory.  scratch: ng * n_split + 8 * 128 + 4 * 8 * 128 floats.
+// Partials (m in the log2 domain, l, centred z times 2^-17) of every split.  The merge is
+// the serial tail of the call, so it is written for memory-level parallelism: every
+// (m, l) is fetched at once, then each thread owns one (head, 4-coordinate) slice of z
+// over a share of the splits (all of its loads independent), the shares meet in shared
+// memory, y = delta_V 2^17 z / l, and o = M_V^T y (warp w: rows w, w + 4, ... of M_V,
+// lane: four output columns; the four warps' sums meet in shared memory).
+// scratch: 2 * 8 * kMaxSplits (m, l) + 8 * 128 (y) + 4 * 8 * 128 floats (the reduction
+// of the split shares and of the back-projection reuse the last region).
 __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDesc& dV, float* scratch, int s,
                                               int qh0, int ng, int n_split, int warp, int lane, int tid) {
   const int Hq = a.H * a.G;
   const int rV = dV.r;
   const bool raw = dV.b == kRawBits;
-  float* wbuf = scratch;                                       // [ng][n_split]
-  float* ybuf = scratch + ((ng * n_split + 31) & ~31);         // [8][128]
-  float* obuf = ybuf + 8 * 128;                                // [4][8][128]
+  float* mbuf = scratch;                     // [ng][n_split]: m, then the weights 2^(m - M)
+  float* lbuf = scratch + 8 * kMaxSplits;    // [ng][n_split]: l
+  float* ybuf = scratch + 16 * kMaxSplits;   // [8][128]
+  float* obuf = ybuf + 8 * 128;              // [4][8][128] (also the split-share reduction)
+  float* Lsum = obuf + 4 * 8 * 128 - 8;      // [8] (the last floats of obuf; free until the back-projection)
   const float dlt = raw ? 0x1p-24f : dV.delta;
+  const size_t head_stride = static_cast<size_t>(a.part_stride) * kPartStride;
+  const float* base0 = a.ws + (static_cast<size_t>(s) * Hq + qh0) * head_stride;
+  // (1) every (m, l) at once
+  for (int idx = tid; idx < ng * n_split; idx += kThreads) {
+    const int n = idx / n_split, i = idx - n * n_split;
+    const float* pp = base0 + n * head_stride + static_cast<size_t>(i) * kPartStride;
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(pp));
+    mbuf[idx] = ml.x;
+    lbuf[idx] = ml.y;
+  }
+  __syncthreads();
+  // (2) per head: the largest m, the weights and l (warp per head)
   for (int n = warp; n < ng; n += kWarps) {
-    const float* base = a.ws + (static_cast<size_t>(s) * Hq + qh0 + n) * a.part_stride * kPartStride;
     float M = -INFINITY;
-    for (int i = lane; i < n_split; i += 32) M = fmaxf(M, __ldcg(base + static_cast<size_t>(i) * kPartStride));
+    for (int i = lane; i < n_split; i += 32) M = fmaxf(M, mbuf[n * n_split + i]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.0f;
     for (int i = lane; i < n_split; i += 32) {
-      const float* pp = base + static_cast<size_t>(i) * kPartStride;
-      const float mi = __ldcg(pp);
+      const float mi = mbuf[n * n_split + i];
       const float wi = (mi == -INFINITY || M == -INFINITY) ? 0.0f : ex2(mi - M);
-      wbuf[n * n_split + i] = wi;
-      L = fmaf(wi, __ldcg(pp + 1), L);
+      mbuf[n * n_split + i] = wi;
+      L = fmaf(wi, lbuf[n * n_split + i], L);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    __syncwarp();
+    if (lane == 0) Lsum[n] = L;
+  }
+  __syncthreads();
+  const float Ls[8] = {Lsum[0], Lsum[1], Lsum[2], Lsum[3], Lsum[4], Lsum[5], Lsum[6], Lsum[7]};
+  __syncthreads();  // obuf (which holds Lsum) is reused below
+  // (3) z: slice p = (head, 4-coordinate group) and split share u; U shares per slice
+  const int quads = (rV + 3) >> 2;
+  const int P = ng * quads;
+  const int U = P >= kThreads ? 1 : kThreads / P;
+  float4* red = reinterpret_cast<float4*>(obuf);  // [U][P] when U > 1 (U * P <= 128)
+  for (int t = tid; t < P * U; t += kThreads) {
+    const int p = t % P, u = t / P;
+    const int n = p / quads, q = p - n * quads;
+    const float* zp = base0 + n * head_stride + 4 + 4 * q;
+    const float* wn = mbuf + n * n_split;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    if (4 * lane < rV) {
 #pragma unroll 8
-      for (int i = 0; i < n_split; ++i) {
-        const float wi = wbuf[n * n_split + i];
-        const float4 z4 = __ldcg(reinterpret_cast<const float4*>(base + static_cast<size_t>(i) * kPartStride + 4) + lane);
-        acc.x = fmaf(wi, z4.x, acc.x);
-        acc.y = fmaf(wi, z4.y, acc.y);
-        acc.z = fmaf(wi, z4.z, acc.z);
-        acc.w = fmaf(wi, z4.w, acc.w);
-      }
+    for (int i = u; i < n_split; i += U) {
+      const float wi = wn[i];
+      const float4 z4 = __ldcg(reinterpret_cast<const float4*>(zp + static_cast<size_t>(i) * kPartStride));
+      acc.x = fmaf(wi, z4.x, acc.x);
+      acc.y = fmaf(wi, z4.y, acc.y);
+      acc.z = fmaf(wi, z4.z, acc.z);
+      acc.w = fmaf(wi, z4.w, acc.w);
     }
-    // z holds sum p (c - m_V) 2^-17: dequantize
-    const float f = L > 0.0f ? dlt * 131072.0f / L : 0.0f;
-    reinterpret_cast<float4*>(ybuf + n * 128)[lane] =
-        4 * lane < rV ? make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (U > 1) {
+      red[u * P + p] = acc;
+    } else {
+      // z holds sum p (c - m_V) 2^-17: dequantize
+      const float f = Ls[n] > 0.0f ? dlt * 131072.0f / Ls[n] : 0.0f;
+      reinterpret_cast<float4*>(ybuf + n * 128)[q] = make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f);
+    }
+  }
+  if (U > 1) {
+    __syncthreads();
+    for (int p = tid; p < P; p += kThreads) {
+      const int n = p / quads, q = p - n * quads;
+      float4 acc = red[p];
+      for (int u = 1; u < U; ++u) {
+        const float4 v = red[u * P + p];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      const float f = Ls[n] > 0.0f ? dlt * 131072.0f / Ls[n] : 0.0f;
+      reinterpret_cast<float4*>(ybuf + n * 128)[q] = make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f);
+    }
   }
   __syncthreads();
   if (raw) {
@@ -688,10 +736,11 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     }
     return;
   }
+  // (4) o = M_V^T y
   float4 o[8];
 #pragma unroll
   for (int n = 0; n < 8; ++n) o[n] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 4
+#pragma unroll 8
   for (int j = warp; j < rV; j += kWarps) {
     const float4 m4 = __ldg(reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD) + lane);
 #pragma unroll
