@@ -54,7 +54,7 @@ constexpr int kMaxHeadsPerLaunch = 64;
 constexpr int kMaxSplits = 128;       // context splits per KV head (bounds the merge scratch)
 // floats of merge scratch the last CTA needs ((m, l) of every split, y, the warps'
 // back-projections)
-constexpr int kMergeFloats = 16 * kMaxSplits + 8 * 128 + 4 * 8 * 128;
+constexpr int kMergeFloats = 16 * kMaxSplits + 8 * 128 + 4 * 8 * 128 + 8;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;         // log2 of the growth allowed before a rescale
 
@@ -635,8 +635,8 @@ __device__ __forceinline__ void form_qtilde(SmemHead& sh, const uint32_t* mfrag,
 // over a share of the splits (all of its loads independent), the shares meet in shared
 // memory, y = delta_V 2^17 z / l, and o = M_V^T y (warp w: rows w, w + 4, ... of M_V,
 // lane: four output columns; the four warps' sums meet in shared memory).
-// scratch: 2 * 8 * kMaxSplits (m, l) + 8 * 128 (y) + 4 * 8 * 128 floats (the reduction
-// of the split shares and of the back-projection reuse the last region).
+// scratch: 2 * 8 * kMaxSplits (m, l) + 8 * 128 (y) + 4 * 8 * 128 (the reductions of the
+// split shares and of the back-projection) + 8 (l per head) floats.
 __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDesc& dV, float* scratch, int s,
                                               int qh0, int ng, int n_split, int warp, int lane, int tid) {
   const int Hq = a.H * a.G;
@@ -646,7 +646,7 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
   float* lbuf = scratch + 8 * kMaxSplits;    // [ng][n_split]: l
   float* ybuf = scratch + 16 * kMaxSplits;   // [8][128]
   float* obuf = ybuf + 8 * 128;              // [4][8][128] (also the split-share reduction)
-  float* Lsum = obuf + 4 * 8 * 128 - 8;      // [8] (the last floats of obuf; free until the back-projection)
+  float* Lsum = ybuf + 8 * 128 + 4 * 8 * 128;  // [8]
   const float dlt = raw ? 0x1p-24f : dV.delta;
   const size_t head_stride = static_cast<size_t>(a.part_stride) * kPartStride;
   const float* base0 = a.ws + (static_cast<size_t>(s) * Hq + qh0) * head_stride;
@@ -677,9 +677,9 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     if (lane == 0) Lsum[n] = L;
   }
   __syncthreads();
-  const float Ls[8] = {Lsum[0], Lsum[1], Lsum[2], Lsum[3], Lsum[4], Lsum[5], Lsum[6], Lsum[7]};
-  __syncthreads();  // obuf (which holds Lsum) is reused below
-  // (3) z: slice p = (head, 4-coordinate group) and split share u; U shares per slice
+  // (3) z: slice p = (head, 4-coordinate group) and split share u; U shares per slice.
+  // The loads go out in explicit batches of eight (a register array filled before it is
+  // used), so every batch costs one L2 round trip whatever the compiler does with the loop.
   const int quads = (rV + 3) >> 2;
   const int P = ng * quads;
   const int U = P >= kThreads ? 1 : kThreads / P;
@@ -690,20 +690,31 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     const float* zp = base0 + n * head_stride + 4 + 4 * q;
     const float* wn = mbuf + n * n_split;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 8
-    for (int i = u; i < n_split; i += U) {
-      const float wi = wn[i];
-      const float4 z4 = __ldcg(reinterpret_cast<const float4*>(zp + static_cast<size_t>(i) * kPartStride));
-      acc.x = fmaf(wi, z4.x, acc.x);
-      acc.y = fmaf(wi, z4.y, acc.y);
-      acc.z = fmaf(wi, z4.z, acc.z);
-      acc.w = fmaf(wi, z4.w, acc.w);
+    for (int i0 = u; i0 < n_split; i0 += 8 * U) {
+      float4 zz[8];
+      float ww[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = i0 + k * U;
+        const bool in = i < n_split;
+        zz[k] = in ? __ldcg(reinterpret_cast<const float4*>(zp + static_cast<size_t>(i) * kPartStride))
+                   : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        ww[k] = in ? wn[i] : 0.0f;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        acc.x = fmaf(ww[k], zz[k].x, acc.x);
+        acc.y = fmaf(ww[k], zz[k].y, acc.y);
+        acc.z = fmaf(ww[k], zz[k].z, acc.z);
+        acc.w = fmaf(ww[k], zz[k].w, acc.w);
+      }
     }
     if (U > 1) {
       red[u * P + p] = acc;
     } else {
       // z holds sum p (c - m_V) 2^-17: dequantize
-      const float f = Ls[n] > 0.0f ? dlt * 131072.0f / Ls[n] : 0.0f;
+      const float L = Lsum[n];
+      const float f = L > 0.0f ? dlt * 131072.0f / L : 0.0f;
       reinterpret_cast<float4*>(ybuf + n * 128)[q] = make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f);
     }
   }
@@ -719,7 +730,8 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
         acc.z += v.z;
         acc.w += v.w;
       }
-      const float f = Ls[n] > 0.0f ? dlt * 131072.0f / Ls[n] : 0.0f;
+      const float L = Lsum[n];
+      const float f = L > 0.0f ? dlt * 131072.0f / L : 0.0f;
       reinterpret_cast<float4*>(ybuf + n * 128)[q] = make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f);
     }
   }
@@ -736,21 +748,32 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     }
     return;
   }
-  // (4) o = M_V^T y
+  // (4) o = M_V^T y: warp w takes rows w, w + 4, ... in batches of eight rows (one L2
+  // round trip per batch; M_V was prefetched into L2 by every CTA of the head)
   float4 o[8];
 #pragma unroll
   for (int n = 0; n < 8; ++n) o[n] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 8
-  for (int j = warp; j < rV; j += kWarps) {
-    const float4 m4 = __ldg(reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD) + lane);
+  for (int j0 = warp; j0 < rV; j0 += 8 * kWarps) {
+    float4 m4[8];
 #pragma unroll
-    for (int n = 0; n < 8; ++n) {
-      if (n < ng) {
-        const float yj = ybuf[n * 128 + j];
-        o[n].x = fmaf(m4.x, yj, o[n].x);
-        o[n].y = fmaf(m4.y, yj, o[n].y);
-        o[n].z = fmaf(m4.z, yj, o[n].z);
-        o[n].w = fmaf(m4.w, yj, o[n].w);
+    for (int k = 0; k < 8; ++k) {
+      const int j = j0 + k * kWarps;
+      m4[k] = j < rV ? __ldg(reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD) + lane)
+                     : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int j = j0 + k * kWarps;
+      const bool in = j < rV;
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        if (n < ng) {
+          const float yj = in ? ybuf[n * 128 + j] : 0.0f;
+          o[n].x = fmaf(m4[k].x, yj, o[n].x);
+          o[n].y = fmaf(m4[k].y, yj, o[n].y);
+          o[n].z = fmaf(m4[k].z, yj, o[n].z);
+          o[n].w = fmaf(m4[k].w, yj, o[n].w);
+        }
       }
     }
   }
@@ -794,7 +817,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const int h = a.heads[hi];
   const int uK = (a.layer * a.H + h) * 2, uV = uK + 1;
   // the plan is constant: its unit descriptors are read, the stage barriers set up and
-  // M_V prefetched into L2 (for the merge) before the wait for the preceding grid
+  // M_K's fragments (for q~) and M_V (for the merge) prefetched into L2 before the wait for
+  // the preceding grid
   const UnitDesc dK = a.units[uK], dV = a.units[uV];
   const int rK = dK.r, rV = dV.r;
   const int Hq = a.H * a.G;
@@ -802,7 +826,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const int nmtK = (rK + 15) >> 4;
   if (lane == 0)
     for (int i = 0; i < a.n_stage; ++i) mbar_init(&bars[warp * 8 + i], 1);
-  if (tid == 0 && dV.b != kRawBits) prefetch_l2(dV.M, static_cast<uint32_t>(rV) * kD * 4);
+  if (tid == 0) {
+    prefetch_l2(dK.Mfrag, static_cast<uint32_t>(nmtK) * 8 * 2 * 32 * 16);
+    if (dV.b != kRawBits) prefetch_l2(dV.M, static_cast<uint32_t>(rV) * kD * 4);
+  }
   if (a.wait_first) griddep_wait();
   griddep_launch_dependents();
 

@@ -5,8 +5,8 @@
 // hold keys before the rotation, so q~ = M_K q (the shortcut of kvtc_decode_attention)
 // no longer applies: the rotation of token t depends on t.  Per 16-token block a warp
 //   * reconstructs K-hat = delta_K (C - m_K) M_K in d-space on the tensor cores (A = the
-//     codes as exact fp16 subnormals, B = M_K^T as fp16 hi + lo fragments; the centring is
-//     the column sums of M_K times m_K, subtracted in fp32);
+//     codes as exact fp16 subnormals, B = M_K^T as fp16 hi + lo fragments read through L1;
+//     the centring is the column sums of M_K times m_K, subtracted in fp32);
 //   * rotates each row by its offset rho < 16 inside the block (rotate-half pairs
 //     (i, i + 64), angles rho w_i from a table), and scores it against the query rotated
 //     back by the block's start: s_t = q . R(t) k_t = (R(-(t0 + 16 a)) q) . (R(rho) k_t)
@@ -137,7 +137,7 @@ __device__ __forceinline__ void rope_block(RopeWS& w, const RopeSmem& sm, const 
     const uint4* fr = reinterpret_cast<const uint4*>(mrec) + static_cast<size_t>(ks) * 16 * 32 + (g * 4 + tq);
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) {
-      const uint4 b = fr[nt * 32];
+      const uint4 b = __ldg(fr + nt * 32);
       mma_16816(acc[nt], A0, A1, A2, A3, b.x, b.y);
       mma_16816(acc[nt], A0, A1, A2, A3, b.z, b.w);
     }
@@ -267,15 +267,13 @@ __device__ __forceinline__ void rotate_back(float (&x)[8][4], const float2* cs, 
 }
 
 template <int BK, int BV>
-__global__ void __launch_bounds__(kThreads, 1) decode_rope_kernel(const __grid_constant__ RopeArgs ra) {
+__global__ void __launch_bounds__(kThreads, 2) decode_rope_kernel(const __grid_constant__ RopeArgs ra) {
   const DecodeArgs& a = ra.d;
   extern __shared__ __align__(128) unsigned char smem[];
   RopeSmem& sm = *reinterpret_cast<RopeSmem*>(smem);
   constexpr size_t kBar = (sizeof(RopeSmem) + 15) / 16 * 16;
-  constexpr size_t kRec = ((kBar + 8 * kWarps * 8 + 8 + 127) / 128) * 128;
+  constexpr size_t kRing = ((kBar + 8 * kWarps * 8 + 127) / 128) * 128;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBar);
-  uint64_t* rec_bar = bars + 8 * kWarps;
-  uint32_t* mrec = reinterpret_cast<uint32_t*>(smem + kRec);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tq = lane & 3;
@@ -292,17 +290,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_rope_kernel(const __grid_c
   const int nks = (rK + 15) >> 4, nmt = (rV + 15) >> 4;
   const int Hq = a.H * a.G;
   const int g0 = hg * 8, ng = min(8, a.G - g0);
-  const uint32_t rec_bytes = static_cast<uint32_t>(nks) * 16 * 32 * 16;
-  unsigned char* stages = smem + kRec + rec_bytes;
-  // constant plan data and tables before the wait: the reconstruction fragments of M_K
-  // (one bulk copy), the rotation tables, the centring sums
+  const uint32_t* mrec = dK.Mrec;  // read through L1: every CTA of the head on an SM shares it
+  unsigned char* stages = smem + kRing;
+  // constant plan data and tables before the wait: the rotation tables, the centring sums,
+  // L2 prefetches of the reconstruction fragments of M_K and of M_V
   if (lane == 0)
     for (int i = 0; i < a.n_stage; ++i) mbar_init(&bars[warp * 8 + i], 1);
   if (tid == 0) {
-    mbar_init(rec_bar, 1);
-    fence_mbar_init();
-    mbar_arrive_expect_tx(rec_bar, rec_bytes);
-    bulk_copy_g2s(mrec, dK.Mrec, rec_bytes, rec_bar);
+    prefetch_l2(dK.Mrec, static_cast<uint32_t>(nks) * 16 * 32 * 16);
     if (dV.b != kRawBits) prefetch_l2(dV.M, static_cast<uint32_t>(rV) * kD * 4);
   }
   for (int i = tid; i < 16 * 64; i += kThreads) sm.rot1[i >> 6][i & 63] = ra.rot1[i >> 6][i & 63];
@@ -412,10 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_rope_kernel(const __grid_c
   const Parts PK = parts_of(dK.b), PV = parts_of(dV.b);
   const float mV = dV.b == kRawBits ? 0.0f : 0.5f;
   const uint32_t cmV = dV.b == kRawBits ? 0u : ((1u << (dV.b - 1)) - 1u) * 0x10001u;
-  const bool rec_ok = mbar_wait_bounded_warp(rec_bar, 0);
-
-  bool dead = !rec_ok;
-  if (dead && lane == 0 && a.status) atomicOr(a.status, KVTC_STATUS_TIMEOUT);
+  bool dead = false;
   int next_issue = n_first;
   int slot = 0;
   uint32_t phase = 0;
@@ -568,9 +560,9 @@ RopeFn rope_fn(int bK, int bV) {
 constexpr size_t kSmemPerSM = 233472;
 constexpr size_t kReadSlack = 2048;
 
-size_t head_bytes(int nks) {
+size_t head_bytes() {
   const size_t bar = (sizeof(RopeSmem) + 15) / 16 * 16;
-  return ((bar + 8 * kWarps * 8 + 8 + 127) / 128) * 128 + static_cast<size_t>(nks) * 16 * 32 * 16;
+  return ((bar + 8 * kWarps * 8 + 127) / 128) * 128;
 }
 
 template <typename... KArgs, typename... Args>
@@ -661,7 +653,6 @@ extern "C" kvtc_status kvtc_decode_attention_rope(const kvtc_plan* plan, const k
     RopeFn fn;
     std::vector<int> heads;
     uint32_t stage_bytes = 0;
-    int nks = 1;
   };
   std::vector<Group> groups;
   for (int h = 0; h < plan->H; ++h) {
@@ -669,13 +660,12 @@ extern "C" kvtc_status kvtc_decode_attention_rope(const kvtc_plan* plan, const k
     RopeFn fn = rope_fn(plan->b[uK], plan->b[uK + 1]);
     auto it = std::find_if(groups.begin(), groups.end(), [&](const Group& x) { return x.fn == fn; });
     if (it == groups.end()) {
-      groups.push_back(Group{fn, {}, 0, 1});
+      groups.push_back(Group{fn, {}, 0});
       it = groups.end() - 1;
     }
     it->heads.push_back(h);
     const uint32_t pb = static_cast<uint32_t>(16 * (plan->r[uK] * plan->b[uK] + plan->r[uK + 1] * plan->b[uK + 1]));
     it->stage_bytes = std::max(it->stage_bytes, (pb + 127u) / 128u * 128u);
-    it->nks = std::max(it->nks, (plan->r[uK] + 15) / 16);
   }
   const size_t merge_bytes = std::max<size_t>(static_cast<size_t>(kWarps) * 8 * kPartStride, kMergeFloats) * sizeof(float);
   bool first = true;
@@ -683,9 +673,10 @@ extern "C" kvtc_status kvtc_decode_attention_rope(const kvtc_plan* plan, const k
     int n_stage = kRopeStages;
     size_t smem = 0;
     for (; n_stage >= 1; --n_stage) {
-      smem = head_bytes(gr.nks) + std::max<size_t>(static_cast<size_t>(kWarps) * n_stage * gr.stage_bytes, merge_bytes) +
+      smem = head_bytes() + std::max<size_t>(static_cast<size_t>(kWarps) * n_stage * gr.stage_bytes, merge_bytes) +
              kReadSlack;
-      if (smem <= kSmemPerSM - 1024) break;
+      // two CTAs per SM (the register limit) when the ring allows it
+      if (smem <= kSmemPerSM / 2 - 1024 || (n_stage == 1 && smem <= kSmemPerSM - 1024)) break;
     }
     if (n_stage < 1) return fail(KVTC_EINVAL, "a page of this plan does not fit in shared memory");
     // the attribute is per kernel (shared with other plans and calls): the largest size
