@@ -600,15 +600,19 @@ constexpr size_t kHeadBytes = ((kBarOffset + 8 * kWarps * 8 + 127) / 128) * 128;
 // lo x lo product dropped (below 2^-22 relative).  Warp w forms m-tiles w, w + 4; the
 // result (column n = head n) lands in sh.qt, rows past r_K exactly zero (zero A rows).
 __device__ __forceinline__ void form_qtilde(SmemHead& sh, const uint32_t* mfrag, int nmtK, int warp, int lane,
-                                            bool q_lo) {
+                                            bool q_lo, const uint4 (&pre)[16]) {
   const int g = lane >> 2, tq = lane & 3;
   for (int mt = warp; mt < nmtK; mt += kWarps) {
+    // this tile's 16 fragments (hi, lo for 8 k-steps): the first tile's were loaded before
+    // the wait for the preceding grid; a second tile's are loaded here in one batch
+    uint4 fr[16];
+    const uint4* src = reinterpret_cast<const uint4*>(mfrag) + static_cast<size_t>(mt) * 8 * 2 * 32 + lane;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) fr[k] = mt == warp ? pre[k] : __ldg(src + k * 32);
     float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const uint4* fr = reinterpret_cast<const uint4*>(mfrag) + static_cast<size_t>(mt) * 8 * 2 * 32 + lane;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      const uint4 ah = __ldg(fr + (ks * 2 + 0) * 32);
-      const uint4 alo = __ldg(fr + (ks * 2 + 1) * 32);
+      const uint4 ah = fr[2 * ks], alo = fr[2 * ks + 1];
       const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.hi[g][16 * ks + 2 * tq]);
       const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.hi[g][16 * ks + 8 + 2 * tq]);
       mma_16816(c, ah.x, ah.y, ah.z, ah.w, b0, b1);
@@ -642,35 +646,38 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
   const int Hq = a.H * a.G;
   const int rV = dV.r;
   const bool raw = dV.b == kRawBits;
-  float* mbuf = scratch;                     // [ng][n_split]: m, then the weights 2^(m - M)
-  float* lbuf = scratch + 8 * kMaxSplits;    // [ng][n_split]: l
+  float* mbuf = scratch;                     // [ng][n_split]: the weights 2^(m - M)
   float* ybuf = scratch + 16 * kMaxSplits;   // [8][128]
   float* obuf = ybuf + 8 * 128;              // [4][8][128] (also the split-share reduction)
   float* Lsum = ybuf + 8 * 128 + 4 * 8 * 128;  // [8]
   const float dlt = raw ? 0x1p-24f : dV.delta;
   const size_t head_stride = static_cast<size_t>(a.part_stride) * kPartStride;
   const float* base0 = a.ws + (static_cast<size_t>(s) * Hq + qh0) * head_stride;
-  // (1) every (m, l) at once
-  for (int idx = tid; idx < ng * n_split; idx += kThreads) {
-    const int n = idx / n_split, i = idx - n * n_split;
-    const float* pp = base0 + n * head_stride + static_cast<size_t>(i) * kPartStride;
-    const float2 ml = __ldcg(reinterpret_cast<const float2*>(pp));
-    mbuf[idx] = ml.x;
-    lbuf[idx] = ml.y;
-  }
-  __syncthreads();
-  // (2) per head: the largest m, the weights and l (warp per head)
+  // (1) per head (warp per head): every split's (m, l) in one batch of loads (lane i,
+  // i + 32, ...), the largest m, the weights 2^(m - M) and l
   for (int n = warp; n < ng; n += kWarps) {
+    const float* hb = base0 + n * head_stride;
+    float mi[kMaxSplits / 32], li[kMaxSplits / 32];
+#pragma unroll
+    for (int k = 0; k < kMaxSplits / 32; ++k) {
+      const int i = lane + 32 * k;
+      float2 ml = make_float2(-INFINITY, 0.0f);
+      if (i < n_split) ml = __ldcg(reinterpret_cast<const float2*>(hb + static_cast<size_t>(i) * kPartStride));
+      mi[k] = ml.x;
+      li[k] = ml.y;
+    }
     float M = -INFINITY;
-    for (int i = lane; i < n_split; i += 32) M = fmaxf(M, mbuf[n * n_split + i]);
+#pragma unroll
+    for (int k = 0; k < kMaxSplits / 32; ++k) M = fmaxf(M, mi[k]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.0f;
-    for (int i = lane; i < n_split; i += 32) {
-      const float mi = mbuf[n * n_split + i];
-      const float wi = (mi == -INFINITY || M == -INFINITY) ? 0.0f : ex2(mi - M);
-      mbuf[n * n_split + i] = wi;
-      L = fmaf(wi, lbuf[n * n_split + i], L);
+#pragma unroll
+    for (int k = 0; k < kMaxSplits / 32; ++k) {
+      const int i = lane + 32 * k;
+      const float wi = (mi[k] == -INFINITY || M == -INFINITY) ? 0.0f : ex2(mi[k] - M);
+      if (i < n_split) mbuf[n * n_split + i] = wi;
+      L = fmaf(wi, li[k], L);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
@@ -678,7 +685,7 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
   }
   __syncthreads();
   // (3) z: slice p = (head, 4-coordinate group) and split share u; U shares per slice.
-  // The loads go out in explicit batches of eight (a register array filled before it is
+  // The loads go out in explicit batches of sixteen (a register array filled before it is
   // used), so every batch costs one L2 round trip whatever the compiler does with the loop.
   const int quads = (rV + 3) >> 2;
   const int P = ng * quads;
@@ -690,11 +697,11 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     const float* zp = base0 + n * head_stride + 4 + 4 * q;
     const float* wn = mbuf + n * n_split;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int i0 = u; i0 < n_split; i0 += 8 * U) {
-      float4 zz[8];
-      float ww[8];
+    for (int i0 = u; i0 < n_split; i0 += 16 * U) {
+      float4 zz[16];
+      float ww[16];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < 16; ++k) {
         const int i = i0 + k * U;
         const bool in = i < n_split;
         zz[k] = in ? __ldcg(reinterpret_cast<const float4*>(zp + static_cast<size_t>(i) * kPartStride))
@@ -702,7 +709,7 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
         ww[k] = in ? wn[i] : 0.0f;
       }
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < 16; ++k) {
         acc.x = fmaf(ww[k], zz[k].x, acc.x);
         acc.y = fmaf(ww[k], zz[k].y, acc.y);
         acc.z = fmaf(ww[k], zz[k].z, acc.z);
@@ -748,21 +755,21 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     }
     return;
   }
-  // (4) o = M_V^T y: warp w takes rows w, w + 4, ... in batches of eight rows (one L2
+  // (4) o = M_V^T y: warp w takes rows w, w + 4, ... in batches of sixteen rows (one L2
   // round trip per batch; M_V was prefetched into L2 by every CTA of the head)
   float4 o[8];
 #pragma unroll
   for (int n = 0; n < 8; ++n) o[n] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  for (int j0 = warp; j0 < rV; j0 += 8 * kWarps) {
-    float4 m4[8];
+  for (int j0 = warp; j0 < rV; j0 += 16 * kWarps) {
+    float4 m4[16];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < 16; ++k) {
       const int j = j0 + k * kWarps;
       m4[k] = j < rV ? __ldg(reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD) + lane)
                      : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < 16; ++k) {
       const int j = j0 + k * kWarps;
       const bool in = j < rV;
 #pragma unroll
@@ -830,10 +837,37 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     prefetch_l2(dK.Mfrag, static_cast<uint32_t>(nmtK) * 8 * 2 * 32 * 16);
     if (dV.b != kRawBits) prefetch_l2(dV.M, static_cast<uint32_t>(rV) * kD * 4);
   }
+  // this warp's first m-tile of M_K fragments for q~ (16 x 16 bytes per lane)
+  uint4 mfrag[16];
+  {
+    // (a warp without a tile reads the unit's first tile, in bounds, and never uses it)
+    const uint4* src = reinterpret_cast<const uint4*>(dK.Mfrag) + static_cast<size_t>(warp < nmtK ? warp : 0) * 8 * 2 * 32 + lane;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) mfrag[k] = __ldg(src + k * 32);
+  }
   if (a.wait_first) griddep_wait();
   griddep_launch_dependents();
 
+  // the inputs the preceding kernels may have written: the sequence length and the
+  // group's queries (warp w: heads 2w, 2w + 1; lane l: elements 4l .. 4l + 3), all loads
+  // issued together
   int seq_len = a.seq_lens[s];
+  float4 qv[2];
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int gg = 2 * warp + hh;
+    qv[hh] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (gg < ng) {
+      const size_t off = (static_cast<size_t>(s) * Hq + h * a.G + g0 + gg) * kD + 4 * lane;
+      if (a.q_bf16) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.q) + off);
+        qv[hh] = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                             __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u));
+      } else {
+        qv[hh] = *reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + off);
+      }
+    }
+  }
   if (seq_len < 0 || seq_len > a.max_pages * kPage) {
     if (tid == 0 && a.status) atomicOr(a.status, KVTC_STATUS_BAD_POS);
     seq_len = seq_len < 0 ? 0 : a.max_pages * kPage;
@@ -893,23 +927,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     if (lane == 0) issue(i, pid);  // page i < n_stage uses slot i
   }
 
-  // ---- q of the group into shared memory as fp16, scaled per head (warp w: heads 2w,
-  // 2w + 1; lane l: elements 4l .. 4l + 3); q~ cleared
+  // ---- q of the group into shared memory as fp16, scaled per head; q~ cleared
   const bool q_lo = !a.q_bf16;
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     const int gg = 2 * warp + hh;
-    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    if (gg < ng) {
-      const size_t off = (static_cast<size_t>(s) * Hq + h * a.G + g0 + gg) * kD + 4 * lane;
-      if (a.q_bf16) {
-        const uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.q) + off);
-        v = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
-                        __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u));
-      } else {
-        v = *reinterpret_cast<const float4*>(static_cast<const float*>(a.q) + off);
-      }
-    }
+    const float4 v = qv[hh];
     float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 #pragma unroll
     for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -927,7 +950,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   }
   for (int i = tid; i < 8 * 128; i += kThreads) sh.qt[i >> 7][i & 127] = 0.0f;
   __syncthreads();
-  form_qtilde(sh, dK.Mfrag, nmtK, warp, lane, q_lo);
+  form_qtilde(sh, dK.Mfrag, nmtK, warp, lane, q_lo, mfrag);
   __syncthreads();
 
   // per head: S = sum_j q~_j and the fp16 normalisation exponent (warp w: heads 2w, 2w+1)

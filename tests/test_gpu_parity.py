@@ -59,6 +59,15 @@ def test_llama_layer_32k_2bpd_codes_and_attention():
     plan = _calibrated(w)
     bs = {plan.unit(u)["b"] for u in range(16)}
     assert len(bs) >= 2            # a real mix of widths from C2
+    # the plan the GPU runs with is the oracle's calibration of the same inputs: identical
+    # (r, b) per unit, and M within 1e-6 of the oracle's normwise
+    from oracle import calibration as ocal
+    k, v, q = synth.calibration_set(w)
+    units = ocal.calibrate(k, v, q, 1, w.n_kv_heads, bpd=w.bpd, seed=w.seed)
+    for u, ou in enumerate(units):
+        info = plan.unit(u)
+        assert (info["r"], info["b"]) == (ou["r"], ou["b"]), u
+        assert np.abs(plan.matrix(u) - ou["M"]).max() <= 1e-6 * np.abs(ou["M"]).max(), u
     rng = np.random.default_rng(1)
     cache = gh.make_cache(plan, [w.seq_len], rng)
     K, V = _kv(w, 0, w.seq_len)
