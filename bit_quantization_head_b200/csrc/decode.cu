@@ -127,6 +127,8 @@ kvtc_status prepare_decode(kvtc_plan* plan) {
         n_stage = static_cast<int>(budget / (static_cast<size_t>(kWarps) * gr.stage_bytes));
       }
       if (n_stage < 1) return fail(KVTC_EINVAL, "a page of this plan does not fit in shared memory");
+      // the ring of each warp takes the whole budget (up to six of the widest stages): the
+      // kernel fits as many stages of its own head's pages as the ring holds
       gr.n_stage = std::min(n_stage, 6);
       // + slack: the kernel reads whole 16-row tiles, up to 2 KB past a page's last row
       gr.smem = kHeadBytes + std::max<size_t>(static_cast<size_t>(kWarps) * gr.n_stage * gr.stage_bytes, merge_bytes) +

@@ -78,8 +78,8 @@ struct DecodeArgs {
   int max_pages;
   int32_t* status;
   float scale;
-  int n_stage;
-  uint32_t stage_bytes;
+  int n_stage;          // stages per warp of the widest head of the launch
+  uint32_t stage_bytes;  // that head's stage (K + V page, 128-byte rounded)
   int* tickets;       // [n_seq][H][n_hg] arrival counters (zero between calls)
   float* ws;          // partials [n_seq][Hq][part_stride][kPartStride]
 };
@@ -685,8 +685,8 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
   }
   __syncthreads();
   // (3) z: slice p = (head, 4-coordinate group) and split share u; U shares per slice.
-  // The loads go out in explicit batches of sixteen (a register array filled before it is
-  // used), so every batch costs one L2 round trip whatever the compiler does with the loop.
+  // The merge runs once per head and call, from cold instruction caches, so its loops are
+  // kept small (a few loads in flight per thread, no long unrolled bodies).
   const int quads = (rV + 3) >> 2;
   const int P = ng * quads;
   const int U = P >= kThreads ? 1 : kThreads / P;
@@ -697,24 +697,14 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     const float* zp = base0 + n * head_stride + 4 + 4 * q;
     const float* wn = mbuf + n * n_split;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int i0 = u; i0 < n_split; i0 += 16 * U) {
-      float4 zz[16];
-      float ww[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int i = i0 + k * U;
-        const bool in = i < n_split;
-        zz[k] = in ? __ldcg(reinterpret_cast<const float4*>(zp + static_cast<size_t>(i) * kPartStride))
-                   : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        ww[k] = in ? wn[i] : 0.0f;
-      }
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        acc.x = fmaf(ww[k], zz[k].x, acc.x);
-        acc.y = fmaf(ww[k], zz[k].y, acc.y);
-        acc.z = fmaf(ww[k], zz[k].z, acc.z);
-        acc.w = fmaf(ww[k], zz[k].w, acc.w);
-      }
+#pragma unroll 4
+    for (int i = u; i < n_split; i += U) {
+      const float wi = wn[i];
+      const float4 z4 = __ldcg(reinterpret_cast<const float4*>(zp + static_cast<size_t>(i) * kPartStride));
+      acc.x = fmaf(wi, z4.x, acc.x);
+      acc.y = fmaf(wi, z4.y, acc.y);
+      acc.z = fmaf(wi, z4.z, acc.z);
+      acc.w = fmaf(wi, z4.w, acc.w);
     }
     if (U > 1) {
       red[u * P + p] = acc;
@@ -755,32 +745,22 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     }
     return;
   }
-  // (4) o = M_V^T y: warp w takes rows w, w + 4, ... in batches of sixteen rows (one L2
-  // round trip per batch; M_V was prefetched into L2 by every CTA of the head)
+  // (4) o = M_V^T y: warp w takes rows w, w + 4, ... (lane: four output columns; M_V was
+  // prefetched into L2 by every CTA of the head)
   float4 o[8];
 #pragma unroll
   for (int n = 0; n < 8; ++n) o[n] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  for (int j0 = warp; j0 < rV; j0 += 16 * kWarps) {
-    float4 m4[16];
+#pragma unroll 2
+  for (int j = warp; j < rV; j += kWarps) {
+    const float4 m4 = __ldg(reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD) + lane);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int j = j0 + k * kWarps;
-      m4[k] = j < rV ? __ldg(reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD) + lane)
-                     : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    }
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int j = j0 + k * kWarps;
-      const bool in = j < rV;
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        if (n < ng) {
-          const float yj = in ? ybuf[n * 128 + j] : 0.0f;
-          o[n].x = fmaf(m4[k].x, yj, o[n].x);
-          o[n].y = fmaf(m4[k].y, yj, o[n].y);
-          o[n].z = fmaf(m4[k].z, yj, o[n].z);
-          o[n].w = fmaf(m4[k].w, yj, o[n].w);
-        }
+    for (int n = 0; n < 8; ++n) {
+      if (n < ng) {
+        const float yj = ybuf[n * 128 + j];
+        o[n].x = fmaf(m4.x, yj, o[n].x);
+        o[n].y = fmaf(m4.y, yj, o[n].y);
+        o[n].z = fmaf(m4.z, yj, o[n].z);
+        o[n].w = fmaf(m4.w, yj, o[n].w);
       }
     }
   }
@@ -831,8 +811,13 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const int Hq = a.H * a.G;
   const int g0 = hg * 8, ng = min(8, a.G - g0);
   const int nmtK = (rK + 15) >> 4;
+  // this head's stage (a K and a V page) and how many fit in the warp's share of the ring
+  // (the launch sizes the ring for its widest head; narrower heads get deeper rings)
+  const uint32_t stage_b = static_cast<uint32_t>((dK.page_bytes + dV.page_bytes + 127) / 128 * 128);
+  const uint32_t ring_b = static_cast<uint32_t>(a.n_stage) * a.stage_bytes;
+  const int n_stage = min(6, static_cast<int>(ring_b / stage_b));
   if (lane == 0)
-    for (int i = 0; i < a.n_stage; ++i) mbar_init(&bars[warp * 8 + i], 1);
+    for (int i = 0; i < n_stage; ++i) mbar_init(&bars[warp * 8 + i], 1);
   if (tid == 0) {
     prefetch_l2(dK.Mfrag, static_cast<uint32_t>(nmtK) * 8 * 2 * 32 * 16);
     if (dV.b != kRawBits) prefetch_l2(dV.M, static_cast<uint32_t>(rV) * kD * 4);
@@ -889,8 +874,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const uint32_t bytesK = static_cast<uint32_t>(dK.page_bytes), bytesV = static_cast<uint32_t>(dV.page_bytes);
   const char* poolK = a.pool + a.pages_per_unit * dK.prefix;
   const char* poolV = a.pool + a.pages_per_unit * dV.prefix;
-  unsigned char* const warp_stages = stages + static_cast<size_t>(warp) * a.n_stage * a.stage_bytes;
-  auto stage_ptr = [&](int slot) { return warp_stages + static_cast<size_t>(slot) * a.stage_bytes; };
+  unsigned char* const warp_stages = stages + static_cast<size_t>(warp) * ring_b;
+  auto stage_ptr = [&](int slot) { return warp_stages + static_cast<size_t>(slot) * stage_b; };
   // Page ids of this warp's pages, 32 at a time: lane l holds the id of page base + l of
   // the current window (-1 past the end), so no dependent global load is left in the loop.
   int pid_win = -1;
@@ -921,7 +906,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     bulk_copy_g2s(st, poolK + static_cast<uint64_t>(pid) * bytesK, bytesK, bar);
     bulk_copy_g2s(st + bytesK, poolV + static_cast<uint64_t>(pid) * bytesV, bytesV, bar);
   };
-  const int n_first = min(a.n_stage, n_my);
+  const int n_first = min(n_stage, n_my);
   for (int i = 0; i < n_first; ++i) {
     const int pid = pid_of(i);
     if (lane == 0) issue(i, pid);  // page i < n_stage uses slot i
@@ -1057,7 +1042,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       int s2 = slot;
       uint32_t ph2 = phase;
       for (int i2 = i + 1; i2 < next_issue; ++i2) {
-        if (++s2 == a.n_stage) {
+        if (++s2 == n_stage) {
           s2 = 0;
           ph2 ^= 1u;
         }
@@ -1078,13 +1063,13 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     }
     // release the stage: every lane is done reading it, then refill it
     __syncwarp();
-    if (next_issue < n_my && next_issue == i + a.n_stage) {
+    if (next_issue < n_my && next_issue == i + n_stage) {
       const int npid = pid_of(next_issue);
       if (lane == 0) issue(slot, npid);  // page i + n_stage reuses page i's stage
       ++next_issue;
     }
     __syncwarp();
-    if (++slot == a.n_stage) {
+    if (++slot == n_stage) {
       slot = 0;
       phase ^= 1u;
     }
