@@ -20,7 +20,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "-I" + os.path.join(ROOT, "include")]
 
-SOURCES = ["host_plan.cpp", "host_calibrate.cpp", "encode_append.cu", "encode_prefill.cu", "decode.cu", "decode_rope.cu", "decode_noalloc.cu"] + [f"decode_v{b}.cu" for b in (2, 4, 8, 0)]
+SOURCES = ["host_plan.cpp", "host_calibrate.cpp", "encode_append.cu", "encode_prefill.cu", "decode.cu", "decode_rope.cu", "decode_noalloc.cu"] + [f"decode_v{b}.cu" for b in range(2, 9)]
 
 
 def _deps_hash(src):

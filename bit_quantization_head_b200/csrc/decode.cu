@@ -25,26 +25,31 @@ namespace kvtc {
 namespace dec {
 namespace {
 
-// Width class of a code: 2, 4 and 8 have specialised extraction; others share the
-// run-time path (class 0); kRawBits marks an uncompressed value unit.
-int width_class(int b) { return (b == 2 || b == 4 || b == 8 || b == kRawBits) ? b : 0; }
-
 // Cost model of one page for the split allocation (warp instructions per page and warp:
-// softmax, bookkeeping and the per-16-coordinate MMA rows).
+// softmax, bookkeeping and the per-16-coordinate MMA rows; a code width with minor parts
+// adds a shift and an AND-OR per part to every A register of its rows).
 constexpr double kPageCost = 320.0;
 constexpr size_t kReadSlack = 2048;
 constexpr double kTileCost = 56.0;
+constexpr double kMinorCost = 24.0;
 constexpr size_t kSmemPerSM = 233472;  // 228 KB of shared memory per SM
 constexpr size_t kSmemReserved = 1024; // reserved by the system per resident CTA
 
+// The kernel variant of a (b_K, b_V) pair: b_K in 2..8; b_V in 2..8 or kRawBits.
 SplitFn split_fn(int bK, int bV, bool pack) {
-  switch (width_class(bK)) {
-    case 2: return split_fn_bk<2>(width_class(bV), pack);
-    case 4: return split_fn_bk<4>(width_class(bV), pack);
-    case 8: return split_fn_bk<8>(width_class(bV), pack);
-    default: return split_fn_bk<0>(width_class(bV), pack);
+  switch (bK) {
+    case 2: return split_fn_bk<2>(bV, pack);
+    case 3: return split_fn_bk<3>(bV, pack);
+    case 4: return split_fn_bk<4>(bV, pack);
+    case 5: return split_fn_bk<5>(bV, pack);
+    case 6: return split_fn_bk<6>(bV, pack);
+    case 7: return split_fn_bk<7>(bV, pack);
+    case 8: return split_fn_bk<8>(bV, pack);
+    default: return nullptr;
   }
 }
+
+double tile_cost(int b) { return kTileCost + kMinorCost * (b == kRawBits ? 0 : n_minor(b)); }
 
 // Partial slots per query head: at most one context split per 8 pages (2 per warp), and
 // at most kMaxSplits.
@@ -55,18 +60,24 @@ int split_cap(int max_seq_len) {
 
 // Launch with programmatic stream serialization: the kernel may start while the previous
 // kernel in the stream finishes; it calls griddepcontrol.wait before reading its inputs.
+// With cluster > 1 the grid is launched in clusters of that many consecutive CTAs along x.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*fn)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+cudaError_t launch_pdl(void (*fn)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster,
+                       Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cluster > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, fn, std::forward<Args>(args)...);
 }
 
@@ -95,12 +106,14 @@ kvtc_status prepare_decode(kvtc_plan* plan) {
     optin = 232448;
   plan->dec_groups.assign(plan->L, {});
   const bool pack = plan->G <= 4;
-  const size_t merge_bytes = std::max<size_t>(static_cast<size_t>(kWarps) * 8 * kPartStride, kMergeFloats) * sizeof(float);
+  // the epilogue's scratch: the warps' partials and a cluster leader's slots, then the merge
+  const size_t merge_bytes =
+      std::max<size_t>(static_cast<size_t>(kWarps + kCluster) * 8 * kPartStride, kMergeFloats) * sizeof(float);
   for (int layer = 0; layer < plan->L; ++layer) {
     std::vector<DecodeGroup>& gs = plan->dec_groups[layer];
     for (int h = 0; h < plan->H; ++h) {
       const int uK = (layer * plan->H + h) * 2;
-      const int wk = width_class(plan->b[uK]), wv = width_class(plan->b[uK + 1]);
+      const int wk = plan->b[uK], wv = plan->b[uK + 1];
       auto it = std::find_if(gs.begin(), gs.end(), [&](const DecodeGroup& x) { return x.wk == wk && x.wv == wv; });
       if (it == gs.end()) {
         gs.emplace_back();
@@ -109,13 +122,14 @@ kvtc_status prepare_decode(kvtc_plan* plan) {
         it->wv = wv;
       }
       it->heads.push_back(h);
-      it->cost.push_back(kPageCost + kTileCost * ((plan->r[uK] + 15) / 16 + (plan->r[uK + 1] + 15) / 16));
+      it->cost.push_back(kPageCost + tile_cost(wk) * ((plan->r[uK] + 15) / 16) +
+                         tile_cost(wv) * ((plan->r[uK + 1] + 15) / 16));
       const uint32_t pb = static_cast<uint32_t>(16 * (plan->r[uK] * plan->b[uK] + plan->r[uK + 1] * plan->b[uK + 1]));
       it->stage_bytes = std::max(it->stage_bytes, (pb + 127u) / 128u * 128u);
     }
     for (DecodeGroup& gr : gs) {
       if (static_cast<int>(gr.heads.size()) > kMaxHeadsPerLaunch) return fail(KVTC_EINVAL, "at most 64 KV heads per layer");
-      SplitFn fn = split_fn(gr.wk == 0 ? 3 : gr.wk, gr.wv == 0 ? 3 : gr.wv, pack);
+      SplitFn fn = split_fn(gr.wk, gr.wv, pack);
       if (!fn) return fail(KVTC_EINVAL, "no decode kernel for this code width");
       gr.fn = reinterpret_cast<const void*>(fn);
       // the most CTAs per SM that leave at least one stage per warp (more resident warps
@@ -141,6 +155,25 @@ kvtc_status prepare_decode(kvtc_plan* plan) {
       int occ = 1;
       if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kThreads, gr.smem) != cudaSuccess || occ < 1) occ = 1;
       gr.per_sm = occ;
+      // clusters are placed whole inside a GPC, so fewer CTAs may be resident in clusters
+      // than alone: the launch sizes its cluster grid by this count
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(kCluster * 64);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = gr.smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = kCluster;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int ncl = 0;
+      if (cudaOccupancyMaxActiveClusters(&ncl, fn, &cfg) != cudaSuccess || ncl < 1) {
+        (void)cudaGetLastError();
+        ncl = 0;
+      }
+      gr.clusters = ncl;
     }
   }
   return KVTC_OK;
@@ -204,8 +237,19 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     const int nh = static_cast<int>(gr.heads.size());
     double group_cost = 0.0;
     for (double c : gr.cost) group_cost += c;
-    const int wave = static_cast<int>(gr.per_sm * plan->sm_count * (group_cost / layer_cost));
-    const int columns = std::max(nh, wave / std::max(1, n_hg * n_seq));
+    const double share = group_cost / layer_cost;
+    const int rows = std::max(1, n_hg * n_seq);
+    const int wave = static_cast<int>(gr.per_sm * plan->sm_count * share);
+    int columns = std::max(nh, wave / rows);
+    // Splits come in clusters of C = kCluster CTAs that merge their partials among
+    // themselves first, where every head can take two clusters within the resident
+    // clusters' share.
+    int C = 1;
+    const int cl_columns = static_cast<int>(gr.clusters * share) / rows * kCluster;
+    if (cl_columns >= 2 * kCluster * nh && cap >= 2 * kCluster) {
+      C = kCluster;
+      columns = cl_columns;
+    }
     DecodeArgs a;
     a.units = plan->d_units;
     a.layer = layer;
@@ -216,17 +260,17 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     a.part_stride = cap;
     // Splits per head: greedy on the modelled finishing time.  A head with s splits
     // gives each of its 4 s warps at most ceil(P / 4 s) pages, so it ends after about
-    // ceil(P / 4 s) * cost; the column goes to the head that ends last, while columns
-    // remain (and the head has at least 8 pages per split).
+    // ceil(P / 4 s) * cost; the next C columns go to the head that ends last, while
+    // columns remain (and the head has at least 8 pages per split).
     int ns[kMaxHeadsPerLaunch];
-    for (int i = 0; i < nh; ++i) ns[i] = 1;
+    for (int i = 0; i < nh; ++i) ns[i] = C;
     auto ends = [&](int i) { return std::ceil(static_cast<double>(max_pages_seq) / (kWarps * ns[i])) * gr.cost[i]; };
-    for (int used = nh; used < columns; ++used) {
+    for (int used = C * nh; used + C <= columns; used += C) {
       int best = -1;
       for (int i = 0; i < nh; ++i)
-        if (ns[i] < cap && (best < 0 || ends(i) > ends(best))) best = i;
+        if (ns[i] + C <= cap && (best < 0 || ends(i) > ends(best))) best = i;
       if (best < 0) break;
-      ++ns[best];
+      ns[best] += C;
     }
     a.split_prefix[0] = 0;
     for (int i = 0; i < nh; ++i) {
@@ -251,7 +295,7 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     a.tickets = tickets;
     a.ws = parts;
     dim3 grid(a.split_prefix[nh], n_hg, n_seq);
-    cudaError_t e = launch_pdl(reinterpret_cast<SplitFn>(const_cast<void*>(gr.fn)), grid, dim3(kThreads), gr.smem, cs, a);
+    cudaError_t e = launch_pdl(reinterpret_cast<SplitFn>(const_cast<void*>(gr.fn)), grid, dim3(kThreads), gr.smem, cs, C, a);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     first = false;
   }

@@ -1,7 +1,7 @@
 // Decode split kernel (templates).  Included by decode.cu and the per-variant
 // instantiation units decode_v*.cu.
 //
-// One launch per layer and width-class group.  CTA = (context split, KV head [, head group
+// One launch per layer and (b_K, b_V) group.  CTA = (context split, KV head [, head group
 // of 8], sequence); four warps, each streaming its own pages through a ring of
 // cp.async.bulk + mbarrier stages.  The CTA
 //   * forms q~ = M_K q for its query heads on the tensor cores (M_K as fp16 hi + lo
@@ -10,7 +10,8 @@
 //   * per 16-token block scores its G (<= 8) query heads with m16n8k16 MMAs whose A operand
 //     comes straight from the packed words: one AND leaves each code in the low mantissa
 //     bits of an fp16 half, the exact subnormal c * 2^(e-24), e the field's bit offset
-//     (undone in fp32); for G <= 4 (packed mode) head n's hi and lo parts sit in columns
+//     (undone in fp32), and widths 3, 5, 6 and 7 add their one or two minor parts with a
+//     shift and an AND-OR each; for G <= 4 (packed mode) head n's hi and lo parts sit in columns
 //     2n and 2n + 1 of one MMA, so each lane adds its own two columns and holds one head's
 //     scores for two token rows;
 //   * runs an online softmax whose rescale is lazy: it happens only when a score exceeds
@@ -26,11 +27,14 @@
 // so the tensor core accumulates signed terms near the size of the result; the 0.5 l left
 // over is folded into z after every page in packed mode (once at the end otherwise).
 // A page's eight 16-token blocks are processed together (their MMA chains interleave).
-// The four warps' (m, l, z) meet in shared memory and each CTA writes one partial per
-// query head; the CTA that completes a (sequence, KV head, head group) last (an atomic
-// ticket in the workspace) merges every split's partial with a log-sum-exp, dequantizes
+// The four warps' (m, l, z) meet in shared memory.  In a launch with clusters, the CTAs
+// of a cluster (consecutive splits of one head) then merge into the leader's shared
+// memory, and each cluster writes one partial per query head (else each CTA does); the
+// CTA that writes the last partial of a (sequence, KV head, head group) (an atomic
+// ticket in the workspace) merges every partial with a log-sum-exp, dequantizes
 // (delta_V) and back-projects o = M_V^T y itself, then re-arms the ticket.
 #pragma once
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -44,7 +48,10 @@
 namespace kvtc {
 namespace dec {
 
+namespace cg = cooperative_groups;
+
 constexpr int kWarps = 4;
+constexpr int kCluster = 4;           // CTAs (consecutive splits of one head) per cluster
 constexpr int kThreads = kWarps * 32;
 constexpr int kNT = 8;                // 16-row tiles of a rank (r <= 128)
 constexpr int kIL = 8;                // blocks processed together (one page)
@@ -85,21 +92,35 @@ struct DecodeArgs {
 };
 
 // ------------------------------------------------------------------ code extraction
-// B in {2, 4, 8}: a single part of width B.  B == 0: any width, parts at run time.
+// A b-bit code is stored as parts of width 8, 4, 2 and 1 (its binary expansion, lowest
+// code bits first, each part in its own plane of the page).  The widest part (the major
+// part, holding the code's low bits) decides where a pair's field lands after one AND:
+// at bit offset e of each fp16 half.  Widths 2, 4 and 8 are a major part alone; 3 = 2 + 1,
+// 5 = 4 + 1, 6 = 4 + 2 and 7 = 4 + 2 + 1 add one or two minor parts, each moved to bit
+// e + (its low code bit).  The code then occupies bits [e, e + b) with e + b <= 11, where
+// an fp16 bit pattern x still has the value x 2^-24 (the subnormals and the first normal
+// binade).
+__host__ __device__ constexpr int major_w(int B) { return B == 3 ? 2 : ((B >= 5 && B <= 7) ? 4 : B); }
+__host__ __device__ constexpr int n_minor(int B) { return (B == 3 || B == 5 || B == 6) ? 1 : (B == 7 ? 2 : 0); }
+// width and low code bit of minor part i
+__host__ __device__ constexpr int minor_w(int B, int i) { return (B == 6 || (B == 7 && i == 0)) ? 2 : 1; }
+__host__ __device__ constexpr int minor_lo(int B, int i) { return B == 3 ? 2 : ((B == 7 && i == 1) ? 6 : 4); }
+
+// bit position of pair (blk, eta)'s field in its word, for a part of width w
 __host__ __device__ constexpr int pair_offset(int w, int blk, int eta) { return ((2 * blk + eta) % (16 / w)) * w; }
 
 // bit offset e of the code inside each fp16 half after extraction
 template <int B>
 __host__ __device__ constexpr int e_of(int blk, int eta) {
-  return B == 2 ? 4 * (blk & 1) + 2 * eta : (B == 4 ? 4 * eta : 0);
+  return major_w(B) == 2 ? 4 * (blk & 1) + 2 * eta : (major_w(B) == 4 ? 4 * eta : 0);
 }
 template <int B>
 __host__ __device__ constexpr int n_e() {
-  return B == 2 ? 4 : (B == 4 ? 2 : 1);
+  return major_w(B) == 2 ? 4 : (major_w(B) == 4 ? 2 : 1);
 }
 template <int B>
 __host__ __device__ constexpr int e_idx(int blk, int eta) {
-  return B == 2 ? 2 * (blk & 1) + eta : (B == 4 ? eta : 0);
+  return major_w(B) == 2 ? 2 * (blk & 1) + eta : (major_w(B) == 4 ? eta : 0);
 }
 
 // W >> 8 as mul.hi (the FMA pipe), leaving the ALU pipe to the field extraction.
@@ -137,54 +158,38 @@ __host__ __device__ constexpr uint32_t centre_bits() {
   return ((((1u << (B - 1)) - 1u) << e_of<B>(BLK, ETA)) * 0x10001u);
 }
 
-// Run-time part description of a b-bit code, indexed by log2 of the width (8/4/2/1):
-// has[lw] says whether the width-2^lw part exists, lo[lw] its lowest code bit.
-struct Parts {
-  bool has[4];
-  int lo[4];
-};
-__device__ __forceinline__ Parts parts_of(int b) {
-  Parts P;
-  int lo = 0;
-#pragma unroll
-  for (int lw = 3; lw >= 0; --lw) {
-    P.has[lw] = (b >> lw) & 1;
-    P.lo[lw] = lo;
-    if (P.has[lw]) lo += 1 << lw;
+// Minor part I of a width-B code for pair (BLK, ETA): its field in word Wm, moved to bit
+// e + (its low code bit) of each half.
+template <int B, int BLK, int ETA, int I>
+__device__ __forceinline__ uint32_t minor_field(uint32_t Wm) {
+  constexpr int wm = minor_w(B, I);
+  constexpr int off = pair_offset(wm, BLK, ETA);
+  constexpr int to = e_of<B>(BLK, ETA) + minor_lo(B, I);
+  constexpr uint32_t m = (1u << wm) - 1u;
+  constexpr uint32_t mask = (m << to) | (m << (to + 16));
+  if constexpr (to >= off) {
+    return (Wm << (to - off)) & mask;
+  } else {
+    return (Wm >> (off - to)) & mask;
   }
-  return P;
 }
 
-// Generic pair extraction: the code assembled at bits [0, b) of each half (e = 0).
-// W[lw] is the word of the width-2^lw part.
-template <int BLK, int ETA>
-__device__ __forceinline__ uint32_t gen_pair(const uint32_t (&W)[4], const Parts& P) {
-  uint32_t v = 0;
-#pragma unroll
-  for (int lw = 3; lw >= 0; --lw) {
-    if (P.has[lw]) {
-      const int off = ((2 * BLK + ETA) & ((16 >> lw) - 1)) << lw;
-      const uint32_t m = (1u << (1 << lw)) - 1u;
-      v |= ((W[lw] >> off) & (m | (m << 16))) << P.lo[lw];
-    }
-  }
+// A-fragment pair (BLK, ETA) of a width-B code: the major part's field from W (or from
+// Wh = W >> 8), the minor parts' fields from Wm[0], Wm[1].
+template <int B, int BLK, int ETA>
+__device__ __forceinline__ uint32_t code_pair(uint32_t W, uint32_t Wh, const uint32_t (&Wm)[2]) {
+  uint32_t v = fast_pair<major_w(B), BLK, ETA>(W, Wh);
+  if constexpr (n_minor(B) >= 1) v |= minor_field<B, BLK, ETA, 0>(Wm[0]);
+  if constexpr (n_minor(B) >= 2) v |= minor_field<B, BLK, ETA, 1>(Wm[1]);
   return v;
 }
 
-// Generic words of a K row (or V row) for block BLK: one word per part.
-template <int BLK>
-__device__ __forceinline__ void gen_words(const uint32_t* page, int r, int row, bool ok, int owner, bool is_k,
-                                          const Parts& P, uint32_t (&W)[4]) {
-#pragma unroll
-  for (int lw = 3; lw >= 0; --lw) {
-    W[lw] = 0u;
-    if (P.has[lw] && ok) {
-      const int wd = 1 << lw;
-      const uint32_t* plane = page + 4 * r * P.lo[lw];
-      const int row_words = (is_k ? 8 : 4) * wd;
-      W[lw] = plane[row * row_words + owner * wd + ((BLK * wd) >> 3)];
-    }
-  }
+// Minor-part words of block BLK out of a group's words M[part][word] (group of blocks
+// starting at B0).
+template <int B, int B0, int BLK>
+__device__ __forceinline__ void pick_minor(const uint32_t (&M)[2][2], uint32_t (&out)[2]) {
+  out[0] = M[0][(BLK * minor_w(B, 0)) / 8 - (B0 * minor_w(B, 0)) / 8];
+  out[1] = M[1][(BLK * minor_w(B, 1)) / 8 - (B0 * minor_w(B, 1)) / 8];
 }
 
 // ------------------------------------------------------------------ shared memory
@@ -212,11 +217,11 @@ struct WS {
   int tok0, seq_len;
   bool partial;        // the page holds positions at or beyond seq_len
   int rK, rV, nks, nmt, g, tq;
-  Parts partsK, partsV;
+  int kmo[2], vmo[2];  // word offsets of the minor parts' planes in a K / V page
   int ones_mt, ones_lr;  // m-tile / local row of the ones row (ones_mt < 0: none)
   uint32_t ones_m0, ones_m1;  // lane masks: this lane's A rows g / g+8 are the ones row
   float alpha[2], beta[2], m_run[2];
-  float al[2][n_e<BK == 0 ? 8 : BK>()], nb[2][n_e<BV == 0 ? 8 : BV>()];
+  float al[2][n_e<BK>()], nb[2][n_e<BV>()];
   // PACK: l accumulator (row 0, column 2n: l of head n, times 2^-17) and the constant A
   // fragments of its ones row by block parity (a0, a2; nonzero in lanes g == 0 only)
   float zl[4];
@@ -228,7 +233,6 @@ struct WS {
   // (times 2^-17) already folded.
   float mV;
   float lfold;
-  uint32_t cmV;  // generic widths: floor(m_V) * 2^-24 as fp16x2 bits
   float z[kNT][4];
   float lcvt[2];  // l accumulated from the fp16 P when there is no ones row
 };
@@ -237,46 +241,34 @@ struct WS {
 // scale 2^(7 - e_V) folded into nb (value side).
 template <int BK, int BV, bool PACK>
 __device__ __forceinline__ void refresh_constants(WS<BK, BV, PACK>& w) {
-  constexpr int NEK = n_e<BK == 0 ? 8 : BK>();
-  constexpr int NEV = n_e<BV == 0 ? 8 : BV>();
+  constexpr int NEK = n_e<BK>();
+  constexpr int NEV = n_e<BV>();
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
 #pragma unroll
     for (int i = 0; i < NEK; ++i) {
-      const int e = BK == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (BK == 4 ? 4 * i : 0);
+      const int e = major_w(BK) == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (major_w(BK) == 4 ? 4 * i : 0);
       w.al[c][i] = w.alpha[c] * (1.0f / static_cast<float>(1 << e));
     }
     const float base = -(w.beta[c] + (w.m_run[c] == -INFINITY ? 0.0f : w.m_run[c])) + 7.0f;
 #pragma unroll
     for (int i = 0; i < NEV; ++i) {
-      const int e = BV == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (BV == 4 ? 4 * i : 0);
+      const int e = major_w(BV) == 2 ? (i >> 1) * 4 + (i & 1) * 2 : (major_w(BV) == 4 ? 4 * i : 0);
       w.nb[c][i] = base - static_cast<float>(e);
     }
   }
 }
 
-// Score MMA(s) of one block for k-step ks.  Fast widths: W0, W1 are the words of rows
-// r0, r1 of this lane that hold the block's fields (Wh = W >> 8).  Generic widths: the
-// words are read here (rows r0, r1).
+// Score MMA(s) of one block for k-step ks: W0, W1 are the major-part words of rows r0, r1
+// of this lane that hold the block's fields (Wh = W >> 8), M0, M1 their minor-part words.
 template <int BK, int BV, bool PACK, int BLK>
-__device__ __forceinline__ void k_block(const WS<BK, BV, PACK>& w, const uint32_t (&bh)[2], const uint32_t (&bl)[2],
-                                        uint32_t W0, uint32_t W0h, uint32_t W1, uint32_t W1h, int r0, int r1,
+__device__ __forceinline__ void k_block(const uint32_t (&bh)[2], const uint32_t (&bl)[2], uint32_t W0, uint32_t W0h,
+                                        uint32_t W1, uint32_t W1h, const uint32_t (&M0)[2], const uint32_t (&M1)[2],
                                         float (&sc)[4], float (&sd)[4]) {
-  uint32_t A0, A1, A2, A3;
-  if constexpr (BK != 0) {
-    A0 = fast_pair<BK, BLK, 0>(W0, W0h);
-    A1 = fast_pair<BK, BLK, 1>(W0, W0h);
-    A2 = fast_pair<BK, BLK, 0>(W1, W1h);
-    A3 = fast_pair<BK, BLK, 1>(W1, W1h);
-  } else {
-    uint32_t G0[4], G1[4];
-    gen_words<BLK>(w.pk, w.rK, r0, true, w.g, true, w.partsK, G0);
-    gen_words<BLK>(w.pk, w.rK, r1, true, w.g, true, w.partsK, G1);
-    A0 = gen_pair<BLK, 0>(G0, w.partsK);
-    A1 = gen_pair<BLK, 1>(G0, w.partsK);
-    A2 = gen_pair<BLK, 0>(G1, w.partsK);
-    A3 = gen_pair<BLK, 1>(G1, w.partsK);
-  }
+  const uint32_t A0 = code_pair<BK, BLK, 0>(W0, W0h, M0);
+  const uint32_t A1 = code_pair<BK, BLK, 1>(W0, W0h, M0);
+  const uint32_t A2 = code_pair<BK, BLK, 0>(W1, W1h, M1);
+  const uint32_t A3 = code_pair<BK, BLK, 1>(W1, W1h, M1);
   mma_16816(sc, A0, A1, A2, A3, bh[0], bh[1]);
   if constexpr (!PACK) mma_16816(sd, A0, A1, A2, A3, bl[0], bl[1]);
 }
@@ -286,9 +278,9 @@ __device__ __forceinline__ void k_block(const WS<BK, BV, PACK>& w, const uint32_
 template <int BK, int BV, bool PACK, int BLK>
 __device__ __forceinline__ bool x_block(const WS<BK, BV, PACK>& w, const float (&sc)[4], const float (&sd)[4],
                                         float (&x)[4]) {
-  constexpr int ik0 = e_idx<BK == 0 ? 8 : BK>(BLK, 0), ik1 = e_idx<BK == 0 ? 8 : BK>(BLK, 1);
-  constexpr int iv0 = e_idx<BV == 0 ? 8 : BV>(BLK, 0), iv1 = e_idx<BV == 0 ? 8 : BV>(BLK, 1);
-  constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
+  constexpr int ik0 = e_idx<BK>(BLK, 0), ik1 = e_idx<BK>(BLK, 1);
+  constexpr int iv0 = e_idx<BV>(BLK, 0), iv1 = e_idx<BV>(BLK, 1);
+  constexpr int ev0 = e_of<BV>(BLK, 0), ev1 = e_of<BV>(BLK, 1);
   constexpr float lim0 = kLazy + 7.0f - ev0, lim1 = kLazy + 7.0f - ev1;
   if constexpr (PACK) {
     // columns 2 tq (hi) and 2 tq + 1 (lo) of head tq: x[0] row g, x[1] row g + 8
@@ -321,7 +313,7 @@ __device__ __forceinline__ bool x_block(const WS<BK, BV, PACK>& w, const float (
 // Block maximum of s - m_run for head column c of one block (x with the e_V offset removed).
 template <int BK, int BV, bool PACK, int BLK>
 __device__ __forceinline__ float xmax_block(const WS<BK, BV, PACK>& w, const float (&x)[4], int c) {
-  constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
+  constexpr int ev0 = e_of<BV>(BLK, 0), ev1 = e_of<BV>(BLK, 1);
   if constexpr (PACK) return fmaxf(x[0] - (7.0f - ev0), x[1] - (7.0f - ev1));
   return fmaxf(x[c] - (7.0f - ev0), x[2 + c] - (7.0f - ev1));
 }
@@ -342,7 +334,7 @@ __device__ __forceinline__ void p_block(WS<BK, BV, PACK>& w, const float (&x)[4]
   const uint32_t P0 = pack_half2(ex2(x[0]), ex2(x[1]));
   const uint32_t P1 = pack_half2(ex2(x[2]), ex2(x[3]));
   if (w.ones_mt < 0) {
-    constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
+    constexpr int ev0 = e_of<BV>(BLK, 0), ev1 = e_of<BV>(BLK, 1);
     const float2 f0 = half2_to_float2(P0), f1 = half2_to_float2(P1);
     constexpr float u0 = 1.0f / static_cast<float>(1 << (7 - ev0)), u1 = 1.0f / static_cast<float>(1 << (7 - ev1));
     w.lcvt[0] += fmaf(f0.x, u0, f1.x * u1);
@@ -352,42 +344,30 @@ __device__ __forceinline__ void p_block(WS<BK, BV, PACK>& w, const float (&x)[4]
   bp[1] = movmatrix_trans(P1);
 }
 
-// Value MMA of one block for m-tile mt (words as in k_block; rows j0, j1).  Rows past
-// r_V hold whatever follows the page in shared memory: their z rows are never read,
-// except the ones row, whose A value is replaced whole.
+// Value MMA of one block for m-tile mt (words as in k_block, of rows j0 and j0 + 8).
+// Rows past r_V hold whatever follows the page in shared memory: their z rows are never
+// read, except the ones row, whose A value is replaced whole.
 template <int BK, int BV, bool PACK, int BLK>
 __device__ __forceinline__ void v_block(const WS<BK, BV, PACK>& w, uint32_t W0, uint32_t W0h, uint32_t W1,
-                                        uint32_t W1h, int j0, int j1, bool ones, const uint32_t (&bp)[2],
-                                        float (&z)[4]) {
-  uint32_t A0, A1, A2, A3;
-  if constexpr (BV != 0) {
-    A0 = fast_pair<BV, BLK, 0>(W0, W0h);
-    A1 = fast_pair<BV, BLK, 0>(W1, W1h);
-    A2 = fast_pair<BV, BLK, 1>(W0, W0h);
-    A3 = fast_pair<BV, BLK, 1>(W1, W1h);
-  } else {
-    uint32_t G0[4], G1[4];
-    gen_words<BLK>(w.pv, w.rV, j0, true, w.tq, false, w.partsV, G0);
-    gen_words<BLK>(w.pv, w.rV, j1, true, w.tq, false, w.partsV, G1);
-    A0 = gen_pair<BLK, 0>(G0, w.partsV);
-    A1 = gen_pair<BLK, 0>(G1, w.partsV);
-    A2 = gen_pair<BLK, 1>(G0, w.partsV);
-    A3 = gen_pair<BLK, 1>(G1, w.partsV);
-  }
+                                        uint32_t W1h, const uint32_t (&M0)[2], const uint32_t (&M1)[2], bool ones,
+                                        const uint32_t (&bp)[2], float (&z)[4]) {
+  uint32_t A0 = code_pair<BV, BLK, 0>(W0, W0h, M0);
+  uint32_t A1 = code_pair<BV, BLK, 0>(W1, W1h, M1);
+  uint32_t A2 = code_pair<BV, BLK, 1>(W0, W0h, M0);
+  uint32_t A3 = code_pair<BV, BLK, 1>(W1, W1h, M1);
   // Signed operands: the codes enter the MMA as c - floor(m_V), so the tensor core sums
   // terms of both signs near the size of the result (an unsigned sum of p c, about
   // m_V l, loses the centred result in the accumulation).  The remaining 0.5 l is
   // folded into z separately.
   {
-    const uint32_t c0 = BV == 0 ? w.cmV : centre_bits<BV == 0 ? 2 : BV, BLK, 0>();
-    const uint32_t c1 = BV == 0 ? w.cmV : centre_bits<BV == 0 ? 2 : BV, BLK, 1>();
+    constexpr uint32_t c0 = centre_bits<BV, BLK, 0>(), c1 = centre_bits<BV, BLK, 1>();
     A0 = hsub2_bits(A0, c0);
     A1 = hsub2_bits(A1, c0);
     A2 = hsub2_bits(A2, c1);
     A3 = hsub2_bits(A3, c1);
   }
   if (ones) {  // the ones row (row r_V) accumulates l: its A value is all ones
-    constexpr int ev0 = BV == 0 ? 0 : e_of<BV>(BLK, 0), ev1 = BV == 0 ? 0 : e_of<BV>(BLK, 1);
+    constexpr int ev0 = e_of<BV>(BLK, 0), ev1 = e_of<BV>(BLK, 1);
     constexpr uint32_t one0 = (1u << ev0) | (1u << (ev0 + 16)), one1 = (1u << ev1) | (1u << (ev1 + 16));
     A0 = (A0 & ~w.ones_m0) | (one0 & w.ones_m0);
     A2 = (A2 & ~w.ones_m0) | (one1 & w.ones_m0);
@@ -439,9 +419,10 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
   // test).  Rows past r_K meet zero q^ coefficients (q~ is zero there) and rows past r_V
   // are never read back, so both are read unmasked inside the last tile; the
   // shared-memory allocation has slack for that over-read.
-  constexpr int KB = BK == 0 ? 1 : BK;
+  // major-part words: the first one the group needs and how many
+  constexpr int KB = major_w(BK);
   constexpr int KW0 = (B0 * KB) / 8, KWN = ((B0 + IL - 1) * KB) / 8 - KW0 + 1;
-  constexpr int VB = BV == 0 ? 1 : BV;
+  constexpr int VB = major_w(BV);
   constexpr int VW0 = (B0 * VB) / 8, VWN = ((B0 + IL - 1) * VB) / 8 - VW0 + 1;
   // ---- scores S[tok][head] = sum_j codeK[tok][j] * q^[head][j]
   auto kstep = [&](auto KSC) {
@@ -459,19 +440,32 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
     uint32_t W0[KWN], W1[KWN], W0h[KWN], W1h[KWN];
 #pragma unroll
     for (int q = 0; q < KWN; ++q) {
-      if constexpr (BK != 0) {
-        W0[q] = w.pk[r0 * 8 * BK + w.g * BK + KW0 + q];
-        W1[q] = w.pk[r1 * 8 * BK + w.g * BK + KW0 + q];
-      } else {
-        W0[q] = W1[q] = 0u;
-      }
+      W0[q] = w.pk[r0 * 8 * KB + w.g * KB + KW0 + q];
+      W1[q] = w.pk[r1 * 8 * KB + w.g * KB + KW0 + q];
       W0h[q] = shr8(W0[q]);
       W1h[q] = shr8(W1[q]);
     }
-    (k_block<BK, BV, PACK, B0 + BB>(w, bh, bl, W0[((B0 + BB) * KB) / 8 - KW0], W0h[((B0 + BB) * KB) / 8 - KW0],
-                                    W1[((B0 + BB) * KB) / 8 - KW0], W1h[((B0 + BB) * KB) / 8 - KW0], r0, r1,
-                                    sc[BB], sd[BB]),
-     ...);
+    // minor-part words (K row of width-w part: 8 w words, owner g's at g w)
+    uint32_t M0[2][2] = {{0u, 0u}, {0u, 0u}}, M1[2][2] = {{0u, 0u}, {0u, 0u}};
+#pragma unroll
+    for (int i = 0; i < n_minor(BK); ++i) {
+      const int wm = minor_w(BK, i), m0 = (B0 * wm) / 8, mn = ((B0 + IL - 1) * wm) / 8 - m0 + 1;
+      const uint32_t* plane = w.pk + w.kmo[i];
+#pragma unroll
+      for (int q = 0; q < mn; ++q) {
+        M0[i][q] = plane[r0 * 8 * wm + w.g * wm + m0 + q];
+        M1[i][q] = plane[r1 * 8 * wm + w.g * wm + m0 + q];
+      }
+    }
+    auto kb = [&](auto BLKC) {
+      constexpr int BLK = decltype(BLKC)::value;
+      constexpr int q = (BLK * KB) / 8 - KW0;
+      uint32_t m0[2], m1[2];
+      pick_minor<BK, B0, BLK>(M0, m0);
+      pick_minor<BK, B0, BLK>(M1, m1);
+      k_block<BK, BV, PACK, BLK>(bh, bl, W0[q], W0h[q], W1[q], W1h[q], m0, m1, sc[BLK - B0], sd[BLK - B0]);
+    };
+    (kb(std::integral_constant<int, B0 + BB>{}), ...);
   };
   switch (w.nks) {
     default: kstep(std::integral_constant<int, 7>{}); [[fallthrough]];
@@ -553,19 +547,32 @@ __device__ __forceinline__ void do_group(WS<BK, BV, PACK>& w, std::integer_seque
     uint32_t W0[VWN], W1[VWN], W0h[VWN], W1h[VWN];
 #pragma unroll
     for (int q = 0; q < VWN; ++q) {
-      if constexpr (BV != 0) {
-        W0[q] = w.pv[j0 * 4 * BV + w.tq * BV + VW0 + q];
-        W1[q] = w.pv[j1 * 4 * BV + w.tq * BV + VW0 + q];
-      } else {
-        W0[q] = W1[q] = 0u;
-      }
+      W0[q] = w.pv[j0 * 4 * VB + w.tq * VB + VW0 + q];
+      W1[q] = w.pv[j1 * 4 * VB + w.tq * VB + VW0 + q];
       W0h[q] = shr8(W0[q]);
       W1h[q] = shr8(W1[q]);
     }
-    (v_block<BK, BV, PACK, B0 + BB>(w, W0[((B0 + BB) * VB) / 8 - VW0], W0h[((B0 + BB) * VB) / 8 - VW0],
-                                    W1[((B0 + BB) * VB) / 8 - VW0], W1h[((B0 + BB) * VB) / 8 - VW0], j0, j1, ones,
-                                    bp[BB], w.z[mt]),
-     ...);
+    // minor-part words (V row of width-w part: 4 w words, owner tq's at tq w)
+    uint32_t M0[2][2] = {{0u, 0u}, {0u, 0u}}, M1[2][2] = {{0u, 0u}, {0u, 0u}};
+#pragma unroll
+    for (int i = 0; i < n_minor(BV); ++i) {
+      const int wm = minor_w(BV, i), m0 = (B0 * wm) / 8, mn = ((B0 + IL - 1) * wm) / 8 - m0 + 1;
+      const uint32_t* plane = w.pv + w.vmo[i];
+#pragma unroll
+      for (int q = 0; q < mn; ++q) {
+        M0[i][q] = plane[j0 * 4 * wm + w.tq * wm + m0 + q];
+        M1[i][q] = plane[j1 * 4 * wm + w.tq * wm + m0 + q];
+      }
+    }
+    auto vb = [&](auto BLKC) {
+      constexpr int BLK = decltype(BLKC)::value;
+      constexpr int q = (BLK * VB) / 8 - VW0;
+      uint32_t m0[2], m1[2];
+      pick_minor<BV, B0, BLK>(M0, m0);
+      pick_minor<BV, B0, BLK>(M1, m1);
+      v_block<BK, BV, PACK, BLK>(w, W0[q], W0h[q], W1[q], W1h[q], m0, m1, ones, bp[BLK - B0], w.z[mt]);
+    };
+    (vb(std::integral_constant<int, B0 + BB>{}), ...);
   };
   switch (w.nmt) {
     default: vtile(std::integral_constant<int, 7>{}); [[fallthrough]];
@@ -685,8 +692,8 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
   }
   __syncthreads();
   // (3) z: slice p = (head, 4-coordinate group) and split share u; U shares per slice.
-  // The merge runs once per head and call, from cold instruction caches, so its loops are
-  // kept small (a few loads in flight per thread, no long unrolled bodies).
+  // The loads go out in explicit batches of sixteen (a register array filled before it is
+  // used): measured here, a plain loop over the splits issued one L2 round trip per split.
   const int quads = (rV + 3) >> 2;
   const int P = ng * quads;
   const int U = P >= kThreads ? 1 : kThreads / P;
@@ -697,14 +704,24 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     const float* zp = base0 + n * head_stride + 4 + 4 * q;
     const float* wn = mbuf + n * n_split;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 4
-    for (int i = u; i < n_split; i += U) {
-      const float wi = wn[i];
-      const float4 z4 = __ldcg(reinterpret_cast<const float4*>(zp + static_cast<size_t>(i) * kPartStride));
-      acc.x = fmaf(wi, z4.x, acc.x);
-      acc.y = fmaf(wi, z4.y, acc.y);
-      acc.z = fmaf(wi, z4.z, acc.z);
-      acc.w = fmaf(wi, z4.w, acc.w);
+    for (int i0 = u; i0 < n_split; i0 += 16 * U) {
+      float4 zz[16];
+      float ww[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int i = i0 + k * U;
+        const bool in = i < n_split;
+        zz[k] = in ? __ldcg(reinterpret_cast<const float4*>(zp + static_cast<size_t>(i) * kPartStride))
+                   : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        ww[k] = in ? wn[i] : 0.0f;
+      }
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        acc.x = fmaf(ww[k], zz[k].x, acc.x);
+        acc.y = fmaf(ww[k], zz[k].y, acc.y);
+        acc.z = fmaf(ww[k], zz[k].z, acc.z);
+        acc.w = fmaf(ww[k], zz[k].w, acc.w);
+      }
     }
     if (U > 1) {
       red[u * P + p] = acc;
@@ -991,8 +1008,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   w.rsw = tq ^ (g << 2);
   w.seq_len = seq_len;
   w.partial = false;
-  w.partsK = parts_of(dK.b);
-  w.partsV = parts_of(dV.b);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    w.kmo[i] = 4 * rK * minor_lo(BK, i);
+    w.vmo[i] = 4 * rV * minor_lo(BV, i);
+  }
   w.ones_mt = (!PACK && (rV & 15)) ? (rV >> 4) : -1;
   w.ones_lr = rV & 15;
   w.ones_m0 = (w.ones_mt >= 0 && w.ones_lr == g) ? 0xFFFFFFFFu : 0u;
@@ -1015,14 +1035,13 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     for (int p = 0; p < 2; ++p) {
 #pragma unroll
       for (int eta = 0; eta < 2; ++eta) {
-        const int e = BV == 2 ? 4 * p + 2 * eta : (BV == 4 ? 4 * eta : 0);
+        const int e = e_of<BV>(p, eta);
         w.onesA[p][eta] = g == 0 ? ((1u << e) | (1u << (e + 16))) : 0u;
       }
     }
     w.zl[0] = w.zl[1] = w.zl[2] = w.zl[3] = 0.0f;
     w.mV = dV.b == kRawBits ? 0.0f : 0.5f;
     w.lfold = 0.0f;
-    w.cmV = dV.b == kRawBits ? 0u : ((1u << (dV.b - 1)) - 1u) * 0x10001u;
   }
 #pragma unroll
   for (int mt = 0; mt < kNT; ++mt) w.z[mt][0] = w.z[mt][1] = w.z[mt][2] = w.z[mt][3] = 0.0f;
@@ -1146,6 +1165,24 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     }
   }
   __syncthreads();
+  // ---- a launch with clusters of C CTAs (C consecutive splits of one head) first merges
+  // inside the cluster: after every CTA of the cluster has left its main loop (the
+  // leader's stage buffers are free), each CTA stores its partial into the leader's
+  // shared memory, and the leader merges the C partials into the one it writes.  The
+  // final merge then reads C times fewer partials. ----
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int rank = C > 1 ? static_cast<int>(cluster.block_rank()) : 0;
+  float* slots = mb + kWarps * 8 * kPartStride;  // leader: [kCluster][8][kPartStride]
+  float* to = nullptr;
+  if (C > 1) {
+    cluster.sync();
+    to = cluster.map_shared_rank(slots, 0) + rank * 8 * kPartStride;
+  } else {
+    to = a.ws + (static_cast<size_t>(s) * Hq + h * a.G + g0) * a.part_stride * kPartStride +
+         static_cast<size_t>(split) * kPartStride;
+  }
+  const size_t to_head = C > 1 ? kPartStride : static_cast<size_t>(a.part_stride) * kPartStride;
   for (int idx = tid; idx < ng * (rV + 2); idx += kThreads) {
     const int n = idx / (rV + 2), e = idx - n * (rV + 2);
     float mw[kWarps], M = -INFINITY;
@@ -1163,7 +1200,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
           if (mw[q] != -INFINITY) acc = fmaf(ex2(mw[q] - M), mb[(q * 8 + n) * kPartStride + src], acc);
       }
     }
-    float* dst = a.ws + ((static_cast<size_t>(s) * Hq + h * a.G + g0 + n) * a.part_stride + split) * kPartStride;
+    float* dst = to + n * to_head;
     if (e == 0) {
       dst[0] = M;
       dst[1] = acc;
@@ -1171,17 +1208,47 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       dst[4 + (e - 1)] = acc;
     }
   }
+  if (C > 1) {
+    cluster.sync();  // the partials have landed in the leader's shared memory
+    if (rank != 0) return;  // (the leader's wait below keeps the launch ordered)
+    float* dstb = a.ws + (static_cast<size_t>(s) * Hq + h * a.G + g0) * a.part_stride * kPartStride +
+                  static_cast<size_t>(split / C) * kPartStride;
+    for (int idx = tid; idx < ng * (rV + 2); idx += kThreads) {
+      const int n = idx / (rV + 2), e = idx - n * (rV + 2);
+      float mw[kCluster], M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < kCluster; ++r) {
+        mw[r] = r < C ? slots[(r * 8 + n) * kPartStride] : -INFINITY;
+        M = fmaxf(M, mw[r]);
+      }
+      const int src = e == 0 ? 1 : 4 + (e - 1);
+      float acc = 0.0f;
+      if (M != -INFINITY && e <= rV) {
+#pragma unroll
+        for (int r = 0; r < kCluster; ++r)
+          if (mw[r] != -INFINITY) acc = fmaf(ex2(mw[r] - M), slots[(r * 8 + n) * kPartStride + src], acc);
+      }
+      float* dst = dstb + static_cast<size_t>(n) * a.part_stride * kPartStride;
+      if (e == 0) {
+        dst[0] = M;
+        dst[1] = acc;
+      } else if (e <= rV) {
+        dst[src] = acc;
+      }
+    }
+  }
 
-  // ---- arrival ticket: the CTA that completes the (sequence, KV head, head group) last
-  // merges every split's partial and writes the output, then re-arms the ticket ----
+  // ---- arrival ticket: the CTA that writes the last partial of a (sequence, KV head,
+  // head group) merges every partial and writes the output, then re-arms the ticket ----
+  const int n_part = n_split / C;
   __threadfence();
   __syncthreads();
   int* ticket = a.tickets + (static_cast<size_t>(s) * a.H + h) * a.n_hg + hg;
-  if (tid == 0) sh.last = atomicAdd(ticket, 1) == n_split - 1;
+  if (tid == 0) sh.last = atomicAdd(ticket, 1) == n_part - 1;
   __syncthreads();
   if (sh.last) {
     __threadfence();
-    merge_project(a, dV, mb, s, h * a.G + g0, ng, n_split, warp, lane, tid);
+    merge_project(a, dV, mb, s, h * a.G + g0, ng, n_part, warp, lane, tid);
     if (tid == 0) atomicExch(ticket, 0);
   }
   if (!a.wait_first) griddep_wait();

@@ -63,6 +63,24 @@ __device__ __forceinline__ uint32_t pair_rt(const uint32_t* row_words, int blk, 
   return (W >> off) & (m | (m << 16));
 }
 
+// Run-time part description of a b-bit code, indexed by log2 of the width (8/4/2/1):
+// has[lw] says whether the width-2^lw part exists, lo[lw] its lowest code bit.
+struct Parts {
+  bool has[4];
+  int lo[4];
+};
+__device__ __forceinline__ Parts parts_of(int b) {
+  Parts P;
+  int lo = 0;
+#pragma unroll
+  for (int lw = 3; lw >= 0; --lw) {
+    P.has[lw] = (b >> lw) & 1;
+    P.lo[lw] = lo;
+    if (P.has[lw]) lo += 1 << lw;
+  }
+  return P;
+}
+
 // Generic widths at run-time block index (parts of width 8/4/2/1, assembled at e = 0).
 __device__ __forceinline__ uint32_t pair_gen_rt(const uint32_t* page, int r, int row, int owner, bool is_k,
                                                 const Parts& P, int blk, int eta) {

@@ -1,22 +1,22 @@
-// Instantiations of the decode split kernel for key code width class 4 (0 = any width);
-// value width 16 = uncompressed values.
+// Instantiations of the decode split kernel for 4-bit key codes; value widths 2..8,
+// or 16 = uncompressed values.
 #include "decode_kernel.cuh"
 
 namespace kvtc {
 namespace dec {
 template <>
 SplitFn split_fn_bk<4>(int bV, bool pack) {
-  if (bV == 2 && pack == true) return decode_split_kernel<4, 2, true>;
-  if (bV == 2 && pack == false) return decode_split_kernel<4, 2, false>;
-  if (bV == 4 && pack == true) return decode_split_kernel<4, 4, true>;
-  if (bV == 4 && pack == false) return decode_split_kernel<4, 4, false>;
-  if (bV == 8 && pack == true) return decode_split_kernel<4, 8, true>;
-  if (bV == 8 && pack == false) return decode_split_kernel<4, 8, false>;
-  if (bV == 0 && pack == true) return decode_split_kernel<4, 0, true>;
-  if (bV == 0 && pack == false) return decode_split_kernel<4, 0, false>;
-  if (bV == 16 && pack == true) return decode_split_kernel<4, 16, true>;
-  if (bV == 16 && pack == false) return decode_split_kernel<4, 16, false>;
-  return nullptr;
+  switch (bV) {
+    case 2: return pack ? decode_split_kernel<4, 2, true> : decode_split_kernel<4, 2, false>;
+    case 3: return pack ? decode_split_kernel<4, 3, true> : decode_split_kernel<4, 3, false>;
+    case 4: return pack ? decode_split_kernel<4, 4, true> : decode_split_kernel<4, 4, false>;
+    case 5: return pack ? decode_split_kernel<4, 5, true> : decode_split_kernel<4, 5, false>;
+    case 6: return pack ? decode_split_kernel<4, 6, true> : decode_split_kernel<4, 6, false>;
+    case 7: return pack ? decode_split_kernel<4, 7, true> : decode_split_kernel<4, 7, false>;
+    case 8: return pack ? decode_split_kernel<4, 8, true> : decode_split_kernel<4, 8, false>;
+    case 16: return pack ? decode_split_kernel<4, 16, true> : decode_split_kernel<4, 16, false>;
+    default: return nullptr;
+  }
 }
 }  // namespace dec
 }  // namespace kvtc

@@ -1,0 +1,22 @@
+// Instantiations of the decode split kernel for 5-bit key codes; value widths 2..8,
+// or 16 = uncompressed values.
+#include "decode_kernel.cuh"
+
+namespace kvtc {
+namespace dec {
+template <>
+SplitFn split_fn_bk<5>(int bV, bool pack) {
+  switch (bV) {
+    case 2: return pack ? decode_split_kernel<5, 2, true> : decode_split_kernel<5, 2, false>;
+    case 3: return pack ? decode_split_kernel<5, 3, true> : decode_split_kernel<5, 3, false>;
+    case 4: return pack ? decode_split_kernel<5, 4, true> : decode_split_kernel<5, 4, false>;
+    case 5: return pack ? decode_split_kernel<5, 5, true> : decode_split_kernel<5, 5, false>;
+    case 6: return pack ? decode_split_kernel<5, 6, true> : decode_split_kernel<5, 6, false>;
+    case 7: return pack ? decode_split_kernel<5, 7, true> : decode_split_kernel<5, 7, false>;
+    case 8: return pack ? decode_split_kernel<5, 8, true> : decode_split_kernel<5, 8, false>;
+    case 16: return pack ? decode_split_kernel<5, 16, true> : decode_split_kernel<5, 16, false>;
+    default: return nullptr;
+  }
+}
+}  // namespace dec
+}  // namespace kvtc

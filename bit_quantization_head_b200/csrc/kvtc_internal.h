@@ -45,13 +45,14 @@ struct UnitDesc {
 // One decode launch of a layer: the KV heads whose (b_K, b_V) width classes share a split
 // kernel variant, with the variant's shared-memory plan (decided once, at plan upload).
 struct DecodeGroup {
-  int wk = 0, wv = 0;           // width classes (2, 4, 8, 16 raw, 0 any)
+  int wk = 0, wv = 0;           // code widths b_K (2..8) and b_V (2..8, or 16: raw values)
   std::vector<int> heads;       // KV heads of the layer in this launch
   std::vector<double> cost;     // modelled cost of one page of each head (warp instructions)
   uint32_t stage_bytes = 0;     // one K + V page of the widest head, 128-byte rounded
   int n_stage = 0;              // stages per warp
   size_t smem = 0;              // dynamic shared memory per CTA
   int per_sm = 1;               // resident CTAs per SM at that size
+  int clusters = 0;             // resident clusters of 4 CTAs on the device (0: none)
   const void* fn = nullptr;     // the kernel variant
 };
 

@@ -101,6 +101,27 @@ def test_every_code_width_ragged_sequences_and_chunked_appends(dtype):
     _check_decode(plan, cache, 0, q, lens, H, G, dtype)
 
 
+@pytest.mark.parametrize("G", [2, 6])
+def test_every_pair_of_key_and_value_widths(G):
+    # one KV head per (b_K, b_V) pair of 2..8 (each pair is its own kernel variant; G = 2
+    # runs the packed score mode, G = 6 the unpacked one), random even ranks from 2 to 128
+    rng = np.random.default_rng(20 + G)
+    pairs = []
+    for bk in range(2, 9):
+        for bv in range(2, 9):
+            rk, rv = (int(x) for x in 2 * rng.integers(1, 65, 2))
+            pairs.append(((rk, bk), (rv, bv)))
+    H = len(pairs)
+    plan = gh.random_plan(1, H, G, pairs, rng)
+    lens = [700, 129]
+    cache = gh.make_cache(plan, lens, rng)
+    kv = [((rng.standard_normal((T, H, 128)) * 1.5).astype(np.float32),
+           (rng.standard_normal((T, H, 128)) * 1.5).astype(np.float32)) for T in lens]
+    gh.encode_all(plan, cache, 0, kv, "f32")
+    q = (rng.standard_normal((len(lens), H * G, 128)) * 0.5).astype(np.float32)
+    _check_decode(plan, cache, 0, q, lens, H, G, "f32")
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_keys_only_raw_values_codes_and_attention(dtype):
     # keys-only plans: coded keys of several widths, values stored as fp16 (raw pages);
