@@ -60,24 +60,18 @@ int split_cap(int max_seq_len) {
 
 // Launch with programmatic stream serialization: the kernel may start while the previous
 // kernel in the stream finishes; it calls griddepcontrol.wait before reading its inputs.
-// With cluster > 1 the grid is launched in clusters of that many consecutive CTAs along x.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*fn)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster,
-                       Args&&... args) {
+cudaError_t launch_pdl(void (*fn)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = cluster > 1 ? 2 : 1;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, fn, std::forward<Args>(args)...);
 }
 
@@ -106,9 +100,8 @@ kvtc_status prepare_decode(kvtc_plan* plan) {
     optin = 232448;
   plan->dec_groups.assign(plan->L, {});
   const bool pack = plan->G <= 4;
-  // the epilogue's scratch: the warps' partials and a cluster leader's slots, then the merge
-  const size_t merge_bytes =
-      std::max<size_t>(static_cast<size_t>(kWarps + kCluster) * 8 * kPartStride, kMergeFloats) * sizeof(float);
+  // the epilogue's scratch: the warps' partials, then the merge
+  const size_t merge_bytes = std::max<size_t>(static_cast<size_t>(kWarps) * 8 * kPartStride, kMergeFloats) * sizeof(float);
   for (int layer = 0; layer < plan->L; ++layer) {
     std::vector<DecodeGroup>& gs = plan->dec_groups[layer];
     for (int h = 0; h < plan->H; ++h) {
@@ -135,19 +128,25 @@ kvtc_status prepare_decode(kvtc_plan* plan) {
       // the most CTAs per SM that leave at least one stage per warp (more resident warps
       // beat deeper rings: with one stage a warp waits for its next page, but the other
       // warps of the SM keep the pipes and the memory system busy)
-      int n_stage = 0;
-      for (int target = kMinBlocks; target >= 1 && n_stage < 1; --target) {
+      int n_stage = 0, target = kMinBlocks;
+      for (; target >= 1 && n_stage < 1; --target) {
         const size_t budget = kSmemPerSM / target - kSmemReserved - kReadSlack - kHeadBytes;
         n_stage = static_cast<int>(budget / (static_cast<size_t>(kWarps) * gr.stage_bytes));
+        if (n_stage >= 1) break;
       }
       if (n_stage < 1) return fail(KVTC_EINVAL, "a page of this plan does not fit in shared memory");
       // the ring of each warp takes the whole budget (up to six of the widest stages): the
       // kernel fits as many stages of its own head's pages as the ring holds
       gr.n_stage = std::min(n_stage, 6);
-      // + slack: the kernel reads whole 16-row tiles, up to 2 KB past a page's last row
-      gr.smem = kHeadBytes + std::max<size_t>(static_cast<size_t>(kWarps) * gr.n_stage * gr.stage_bytes, merge_bytes) +
-                kReadSlack;
-      if (gr.smem > static_cast<size_t>(optin)) return fail(KVTC_EINVAL, "a page of this plan does not fit in shared memory");
+      // Every launch with the same CTAs per SM asks for the same shared memory, the whole
+      // share of one CTA: the next layer's CTAs start while this layer's last ones run
+      // (programmatic dependent launch), and a larger request than the one before could
+      // not use the holes the earlier CTAs leave, stranding a few CTAs for a second wave.
+      gr.smem = kSmemPerSM / target - kSmemReserved;
+      const size_t need = kHeadBytes + std::max<size_t>(static_cast<size_t>(kWarps) * gr.n_stage * gr.stage_bytes, merge_bytes) +
+                          kReadSlack;  // + slack: the kernel reads whole 16-row tiles, up to 2 KB past a page's last row
+      if (need > gr.smem || gr.smem > static_cast<size_t>(optin))
+        return fail(KVTC_EINVAL, "a page of this plan does not fit in shared memory");
       // the attribute is per kernel, shared by every group and plan: allow the device's
       // opt-in maximum once (each launch still asks for its own size)
       e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
@@ -155,25 +154,6 @@ kvtc_status prepare_decode(kvtc_plan* plan) {
       int occ = 1;
       if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kThreads, gr.smem) != cudaSuccess || occ < 1) occ = 1;
       gr.per_sm = occ;
-      // clusters are placed whole inside a GPC, so fewer CTAs may be resident in clusters
-      // than alone: the launch sizes its cluster grid by this count
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(kCluster * 64);
-      cfg.blockDim = dim3(kThreads);
-      cfg.dynamicSmemBytes = gr.smem;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = kCluster;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int ncl = 0;
-      if (cudaOccupancyMaxActiveClusters(&ncl, fn, &cfg) != cudaSuccess || ncl < 1) {
-        (void)cudaGetLastError();
-        ncl = 0;
-      }
-      gr.clusters = ncl;
     }
   }
   return KVTC_OK;
@@ -240,16 +220,7 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     const double share = group_cost / layer_cost;
     const int rows = std::max(1, n_hg * n_seq);
     const int wave = static_cast<int>(gr.per_sm * plan->sm_count * share);
-    int columns = std::max(nh, wave / rows);
-    // Splits come in clusters of C = kCluster CTAs that merge their partials among
-    // themselves first, where every head can take two clusters within the resident
-    // clusters' share.
-    int C = 1;
-    const int cl_columns = static_cast<int>(gr.clusters * share) / rows * kCluster;
-    if (cl_columns >= 2 * kCluster * nh && cap >= 2 * kCluster) {
-      C = kCluster;
-      columns = cl_columns;
-    }
+    const int columns = std::max(nh, wave / rows);
     DecodeArgs a;
     a.units = plan->d_units;
     a.layer = layer;
@@ -260,17 +231,17 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     a.part_stride = cap;
     // Splits per head: greedy on the modelled finishing time.  A head with s splits
     // gives each of its 4 s warps at most ceil(P / 4 s) pages, so it ends after about
-    // ceil(P / 4 s) * cost; the next C columns go to the head that ends last, while
-    // columns remain (and the head has at least 8 pages per split).
+    // ceil(P / 4 s) * cost; the column goes to the head that ends last, while columns
+    // remain (and the head has at least 8 pages per split).
     int ns[kMaxHeadsPerLaunch];
-    for (int i = 0; i < nh; ++i) ns[i] = C;
+    for (int i = 0; i < nh; ++i) ns[i] = 1;
     auto ends = [&](int i) { return std::ceil(static_cast<double>(max_pages_seq) / (kWarps * ns[i])) * gr.cost[i]; };
-    for (int used = C * nh; used + C <= columns; used += C) {
+    for (int used = nh; used < columns; ++used) {
       int best = -1;
       for (int i = 0; i < nh; ++i)
-        if (ns[i] + C <= cap && (best < 0 || ends(i) > ends(best))) best = i;
+        if (ns[i] < cap && (best < 0 || ends(i) > ends(best))) best = i;
       if (best < 0) break;
-      ns[best] += C;
+      ++ns[best];
     }
     a.split_prefix[0] = 0;
     for (int i = 0; i < nh; ++i) {
@@ -288,6 +259,7 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     a.pages_per_unit = cache->pages_per_unit;
     a.block_table = cache->block_table;
     a.max_pages = cache->max_pages;
+    a.part_pages = max_pages_seq;
     a.status = cache->status;
     a.scale = scale;
     a.n_stage = gr.n_stage;
@@ -295,7 +267,7 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
     a.tickets = tickets;
     a.ws = parts;
     dim3 grid(a.split_prefix[nh], n_hg, n_seq);
-    cudaError_t e = launch_pdl(reinterpret_cast<SplitFn>(const_cast<void*>(gr.fn)), grid, dim3(kThreads), gr.smem, cs, C, a);
+    cudaError_t e = launch_pdl(reinterpret_cast<SplitFn>(const_cast<void*>(gr.fn)), grid, dim3(kThreads), gr.smem, cs, a);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     first = false;
   }

@@ -27,14 +27,11 @@
 // so the tensor core accumulates signed terms near the size of the result; the 0.5 l left
 // over is folded into z after every page in packed mode (once at the end otherwise).
 // A page's eight 16-token blocks are processed together (their MMA chains interleave).
-// The four warps' (m, l, z) meet in shared memory.  In a launch with clusters, the CTAs
-// of a cluster (consecutive splits of one head) then merge into the leader's shared
-// memory, and each cluster writes one partial per query head (else each CTA does); the
-// CTA that writes the last partial of a (sequence, KV head, head group) (an atomic
-// ticket in the workspace) merges every partial with a log-sum-exp, dequantizes
+// The four warps' (m, l, z) meet in shared memory and each CTA writes one partial per
+// query head; the CTA that completes a (sequence, KV head, head group) last (an atomic
+// ticket in the workspace) merges every split's partial with a log-sum-exp, dequantizes
 // (delta_V) and back-projects o = M_V^T y itself, then re-arms the ticket.
 #pragma once
-#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -48,10 +45,7 @@
 namespace kvtc {
 namespace dec {
 
-namespace cg = cooperative_groups;
-
 constexpr int kWarps = 4;
-constexpr int kCluster = 4;           // CTAs (consecutive splits of one head) per cluster
 constexpr int kThreads = kWarps * 32;
 constexpr int kNT = 8;                // 16-row tiles of a rank (r <= 128)
 constexpr int kIL = 8;                // blocks processed together (one page)
@@ -83,6 +77,7 @@ struct DecodeArgs {
   uint64_t pages_per_unit;
   const int32_t* block_table;
   int max_pages;
+  int part_pages;     // pages the split partition covers: ceil(max_seq_len / 128)
   int32_t* status;
   float scale;
   int n_stage;          // stages per warp of the widest head of the launch
@@ -604,39 +599,53 @@ constexpr size_t kHeadBytes = ((kBarOffset + 8 * kWarps * 8 + 127) / 128) * 128;
 // ---- q~ = M_K q for the CTA's query heads, on the tensor cores -------------------------
 // q of head n (n < ng) is scaled by 2^-Eq[n] and stored as fp16 hi (+ lo for fp32 input);
 // A = M_K's fp16 hi and lo fragments (plan), so q~ = (M_hi + M_lo)(q_hi + q_lo) with the
-// lo x lo product dropped (below 2^-22 relative).  Warp w forms m-tiles w, w + 4; the
+// lo x lo product dropped (below 2^-22 relative).  Warp w forms m-tiles w and w + 4; the
 // result (column n = head n) lands in sh.qt, rows past r_K exactly zero (zero A rows).
+// The first tile's fragments were loaded before the wait for the preceding grid; the
+// second tile's loads go out before the first tile's MMAs, and each tile accumulates in
+// four independent chains (k-step parity x M part), so the MMA latency does not add up
+// along the 8 k-steps.
+__device__ __forceinline__ void qtilde_tile(SmemHead& sh, const uint4 (&fr)[16], int mt, int g, int tq, bool q_lo) {
+  float c[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i][0] = c[i][1] = c[i][2] = c[i][3] = 0.0f;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const uint4 ah = fr[2 * ks], alo = fr[2 * ks + 1];
+    float (&ch)[4] = c[(ks & 1) * 2], (&cl)[4] = c[(ks & 1) * 2 + 1];
+    const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.hi[g][16 * ks + 2 * tq]);
+    const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.hi[g][16 * ks + 8 + 2 * tq]);
+    mma_16816(ch, ah.x, ah.y, ah.z, ah.w, b0, b1);
+    mma_16816(cl, alo.x, alo.y, alo.z, alo.w, b0, b1);
+    if (q_lo) {
+      const uint32_t l0 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.lo[g][16 * ks + 2 * tq]);
+      const uint32_t l1 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.lo[g][16 * ks + 8 + 2 * tq]);
+      mma_16816(cl, ah.x, ah.y, ah.z, ah.w, l0, l1);
+    }
+  }
+  float r[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) r[e] = (c[0][e] + c[2][e]) + (c[1][e] + c[3][e]);
+  const int j = 16 * mt + g;
+  const float s0 = ldexpf(1.0f, sh.Eq[2 * tq]), s1 = ldexpf(1.0f, sh.Eq[2 * tq + 1]);
+  sh.qt[2 * tq][j] = r[0] * s0;
+  sh.qt[2 * tq + 1][j] = r[1] * s1;
+  sh.qt[2 * tq][j + 8] = r[2] * s0;
+  sh.qt[2 * tq + 1][j + 8] = r[3] * s1;
+}
+
 __device__ __forceinline__ void form_qtilde(SmemHead& sh, const uint32_t* mfrag, int nmtK, int warp, int lane,
                                             bool q_lo, const uint4 (&pre)[16]) {
   const int g = lane >> 2, tq = lane & 3;
-  for (int mt = warp; mt < nmtK; mt += kWarps) {
-    // this tile's 16 fragments (hi, lo for 8 k-steps): the first tile's were loaded before
-    // the wait for the preceding grid; a second tile's are loaded here in one batch
-    uint4 fr[16];
-    const uint4* src = reinterpret_cast<const uint4*>(mfrag) + static_cast<size_t>(mt) * 8 * 2 * 32 + lane;
+  const int mt1 = warp + kWarps;
+  uint4 fr1[16];
+  if (mt1 < nmtK) {
+    const uint4* src = reinterpret_cast<const uint4*>(mfrag) + static_cast<size_t>(mt1) * 8 * 2 * 32 + lane;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) fr[k] = mt == warp ? pre[k] : __ldg(src + k * 32);
-    float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint4 ah = fr[2 * ks], alo = fr[2 * ks + 1];
-      const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.hi[g][16 * ks + 2 * tq]);
-      const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.hi[g][16 * ks + 8 + 2 * tq]);
-      mma_16816(c, ah.x, ah.y, ah.z, ah.w, b0, b1);
-      mma_16816(c, alo.x, alo.y, alo.z, alo.w, b0, b1);
-      if (q_lo) {
-        const uint32_t l0 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.lo[g][16 * ks + 2 * tq]);
-        const uint32_t l1 = *reinterpret_cast<const uint32_t*>(&sh.u.q16.lo[g][16 * ks + 8 + 2 * tq]);
-        mma_16816(c, ah.x, ah.y, ah.z, ah.w, l0, l1);
-      }
-    }
-    const int j = 16 * mt + g;
-    const float s0 = ldexpf(1.0f, sh.Eq[2 * tq]), s1 = ldexpf(1.0f, sh.Eq[2 * tq + 1]);
-    sh.qt[2 * tq][j] = c[0] * s0;
-    sh.qt[2 * tq + 1][j] = c[1] * s1;
-    sh.qt[2 * tq][j + 8] = c[2] * s0;
-    sh.qt[2 * tq + 1][j + 8] = c[3] * s1;
+    for (int k = 0; k < 16; ++k) fr1[k] = __ldg(src + k * 32);
   }
+  if (warp < nmtK) qtilde_tile(sh, pre, warp, g, tq, q_lo);
+  if (mt1 < nmtK) qtilde_tile(sh, fr1, mt1, g, tq, q_lo);
 }
 
 // ---- the last CTA of a (sequence, KV head, head group): merge and back-project ------------
@@ -763,21 +772,31 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     return;
   }
   // (4) o = M_V^T y: warp w takes rows w, w + 4, ... (lane: four output columns; M_V was
-  // prefetched into L2 by every CTA of the head)
+  // prefetched into L2 by every CTA of the head), eight rows' loads in flight at a time
   float4 o[8];
 #pragma unroll
   for (int n = 0; n < 8; ++n) o[n] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 2
-  for (int j = warp; j < rV; j += kWarps) {
-    const float4 m4 = __ldg(reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD) + lane);
+  for (int j0 = warp; j0 < rV; j0 += 8 * kWarps) {
+    float4 m4[8];
 #pragma unroll
-    for (int n = 0; n < 8; ++n) {
-      if (n < ng) {
-        const float yj = ybuf[n * 128 + j];
-        o[n].x = fmaf(m4.x, yj, o[n].x);
-        o[n].y = fmaf(m4.y, yj, o[n].y);
-        o[n].z = fmaf(m4.z, yj, o[n].z);
-        o[n].w = fmaf(m4.w, yj, o[n].w);
+    for (int k = 0; k < 8; ++k) {
+      const int j = j0 + k * kWarps;
+      m4[k] = j < rV ? __ldg(reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD) + lane)
+                     : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int j = j0 + k * kWarps;
+      if (j >= rV) break;  // (warp-uniform; y past r_V is not written)
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        if (n < ng) {
+          const float yj = ybuf[n * 128 + j];
+          o[n].x = fmaf(m4[k].x, yj, o[n].x);
+          o[n].y = fmaf(m4[k].y, yj, o[n].y);
+          o[n].z = fmaf(m4[k].z, yj, o[n].z);
+          o[n].w = fmaf(m4[k].w, yj, o[n].w);
+        }
       }
     }
   }
@@ -850,9 +869,20 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   if (a.wait_first) griddep_wait();
   griddep_launch_dependents();
 
-  // the inputs the preceding kernels may have written: the sequence length and the
-  // group's queries (warp w: heads 2w, 2w + 1; lane l: elements 4l .. 4l + 3), all loads
-  // issued together
+  // The head's pages, as many as the call's longest sequence may have, are cut into
+  // n_split * kWarps contiguous runs whose lengths differ by at most one page; warp w of
+  // split c takes run c * kWarps + w, cut short at this sequence's end.  The partition
+  // does not depend on the sequence length, so the block-table window of the run goes
+  // out together with the other inputs the preceding kernels may have written: the
+  // sequence length and the group's queries (warp w: heads 2w, 2w + 1; lane l: elements
+  // 4l .. 4l + 3).
+  const int n_workers = n_split * kWarps;
+  const int worker = split * kWarps + warp;
+  const int p_begin = static_cast<int>(static_cast<long long>(worker) * a.part_pages / n_workers);
+  const int p_run = static_cast<int>(static_cast<long long>(worker + 1) * a.part_pages / n_workers) - p_begin;
+  const int32_t* bt = a.block_table + static_cast<size_t>(s) * a.max_pages;
+  // lane l holds the id of page base + l of the current window of 32 (-1 past the run)
+  int pid_win = lane < p_run ? bt[p_begin + lane] : -1;
   int seq_len = a.seq_lens[s];
   float4 qv[2];
 #pragma unroll
@@ -870,18 +900,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       }
     }
   }
-  if (seq_len < 0 || seq_len > a.max_pages * kPage) {
+  if (seq_len < 0 || seq_len > a.part_pages * kPage) {
     if (tid == 0 && a.status) atomicOr(a.status, KVTC_STATUS_BAD_POS);
-    seq_len = seq_len < 0 ? 0 : a.max_pages * kPage;
+    seq_len = seq_len < 0 ? 0 : a.part_pages * kPage;
   }
   const int n_pages = (seq_len + kPage - 1) / kPage;
-  // The head's pages are cut into n_split * kWarps contiguous runs whose lengths differ
-  // by at most one page; warp w of split c takes run c * kWarps + w.
-  const int n_workers = n_split * kWarps;
-  const int worker = split * kWarps + warp;
-  const int p_begin = static_cast<int>(static_cast<long long>(worker) * n_pages / n_workers);
-  const int n_my = static_cast<int>(static_cast<long long>(worker + 1) * n_pages / n_workers) - p_begin;
-  const int32_t* bt = a.block_table + static_cast<size_t>(s) * a.max_pages;
+  const int n_my = max(0, min(p_run, n_pages - p_begin));
 
   // ---- prologue: first copies (the barriers were set up by lane 0 of each warp, which
   // also issues the copies), then q~ while they are in flight ----
@@ -893,10 +917,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const char* poolV = a.pool + a.pages_per_unit * dV.prefix;
   unsigned char* const warp_stages = stages + static_cast<size_t>(warp) * ring_b;
   auto stage_ptr = [&](int slot) { return warp_stages + static_cast<size_t>(slot) * stage_b; };
-  // Page ids of this warp's pages, 32 at a time: lane l holds the id of page base + l of
-  // the current window (-1 past the end), so no dependent global load is left in the loop.
-  int pid_win = -1;
-  int pid_base = -1;
+  // Page ids of this warp's pages, 32 at a time (the first window was loaded above), so
+  // no dependent global load is left in the loop.
+  int pid_base = 0;
   auto pid_of = [&](int i) {  // warp-uniform i
     const int base = i & ~31;
     if (base != pid_base) {
@@ -1165,24 +1188,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     }
   }
   __syncthreads();
-  // ---- a launch with clusters of C CTAs (C consecutive splits of one head) first merges
-  // inside the cluster: after every CTA of the cluster has left its main loop (the
-  // leader's stage buffers are free), each CTA stores its partial into the leader's
-  // shared memory, and the leader merges the C partials into the one it writes.  The
-  // final merge then reads C times fewer partials. ----
-  cg::cluster_group cluster = cg::this_cluster();
-  const int C = static_cast<int>(cluster.num_blocks());
-  const int rank = C > 1 ? static_cast<int>(cluster.block_rank()) : 0;
-  float* slots = mb + kWarps * 8 * kPartStride;  // leader: [kCluster][8][kPartStride]
-  float* to = nullptr;
-  if (C > 1) {
-    cluster.sync();
-    to = cluster.map_shared_rank(slots, 0) + rank * 8 * kPartStride;
-  } else {
-    to = a.ws + (static_cast<size_t>(s) * Hq + h * a.G + g0) * a.part_stride * kPartStride +
-         static_cast<size_t>(split) * kPartStride;
-  }
-  const size_t to_head = C > 1 ? kPartStride : static_cast<size_t>(a.part_stride) * kPartStride;
+  float* dstb = a.ws + (static_cast<size_t>(s) * Hq + h * a.G + g0) * a.part_stride * kPartStride +
+                static_cast<size_t>(split) * kPartStride;
   for (int idx = tid; idx < ng * (rV + 2); idx += kThreads) {
     const int n = idx / (rV + 2), e = idx - n * (rV + 2);
     float mw[kWarps], M = -INFINITY;
@@ -1192,63 +1199,31 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       M = fmaxf(M, mw[q]);
     }
     float acc = 0.0f;
-    if (M != -INFINITY) {
-      const int src = e == 0 ? 1 : 4 + (e - 1);  // e == 0: l; e >= 1: z[e - 1]
-      if (e <= rV) {
+    const int src = e == 0 ? 1 : 4 + (e - 1);  // e == 0: l; e >= 1: z[e - 1]
+    if (M != -INFINITY && e <= rV) {
 #pragma unroll
-        for (int q = 0; q < kWarps; ++q)
-          if (mw[q] != -INFINITY) acc = fmaf(ex2(mw[q] - M), mb[(q * 8 + n) * kPartStride + src], acc);
-      }
+      for (int q = 0; q < kWarps; ++q)
+        if (mw[q] != -INFINITY) acc = fmaf(ex2(mw[q] - M), mb[(q * 8 + n) * kPartStride + src], acc);
     }
-    float* dst = to + n * to_head;
+    float* dst = dstb + static_cast<size_t>(n) * a.part_stride * kPartStride;
     if (e == 0) {
       dst[0] = M;
       dst[1] = acc;
     } else if (e <= rV) {
-      dst[4 + (e - 1)] = acc;
-    }
-  }
-  if (C > 1) {
-    cluster.sync();  // the partials have landed in the leader's shared memory
-    if (rank != 0) return;  // (the leader's wait below keeps the launch ordered)
-    float* dstb = a.ws + (static_cast<size_t>(s) * Hq + h * a.G + g0) * a.part_stride * kPartStride +
-                  static_cast<size_t>(split / C) * kPartStride;
-    for (int idx = tid; idx < ng * (rV + 2); idx += kThreads) {
-      const int n = idx / (rV + 2), e = idx - n * (rV + 2);
-      float mw[kCluster], M = -INFINITY;
-#pragma unroll
-      for (int r = 0; r < kCluster; ++r) {
-        mw[r] = r < C ? slots[(r * 8 + n) * kPartStride] : -INFINITY;
-        M = fmaxf(M, mw[r]);
-      }
-      const int src = e == 0 ? 1 : 4 + (e - 1);
-      float acc = 0.0f;
-      if (M != -INFINITY && e <= rV) {
-#pragma unroll
-        for (int r = 0; r < kCluster; ++r)
-          if (mw[r] != -INFINITY) acc = fmaf(ex2(mw[r] - M), slots[(r * 8 + n) * kPartStride + src], acc);
-      }
-      float* dst = dstb + static_cast<size_t>(n) * a.part_stride * kPartStride;
-      if (e == 0) {
-        dst[0] = M;
-        dst[1] = acc;
-      } else if (e <= rV) {
-        dst[src] = acc;
-      }
+      dst[src] = acc;
     }
   }
 
-  // ---- arrival ticket: the CTA that writes the last partial of a (sequence, KV head,
-  // head group) merges every partial and writes the output, then re-arms the ticket ----
-  const int n_part = n_split / C;
+  // ---- arrival ticket: the CTA that completes the (sequence, KV head, head group) last
+  // merges every split's partial and writes the output, then re-arms the ticket ----
   __threadfence();
   __syncthreads();
   int* ticket = a.tickets + (static_cast<size_t>(s) * a.H + h) * a.n_hg + hg;
-  if (tid == 0) sh.last = atomicAdd(ticket, 1) == n_part - 1;
+  if (tid == 0) sh.last = atomicAdd(ticket, 1) == n_split - 1;
   __syncthreads();
   if (sh.last) {
     __threadfence();
-    merge_project(a, dV, mb, s, h * a.G + g0, ng, n_part, warp, lane, tid);
+    merge_project(a, dV, mb, s, h * a.G + g0, ng, n_split, warp, lane, tid);
     if (tid == 0) atomicExch(ticket, 0);
   }
   if (!a.wait_first) griddep_wait();

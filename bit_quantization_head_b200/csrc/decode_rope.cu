@@ -661,6 +661,7 @@ extern "C" kvtc_status kvtc_decode_attention_rope(const kvtc_plan* plan, const k
   a.pages_per_unit = cache->pages_per_unit;
   a.block_table = cache->block_table;
   a.max_pages = cache->max_pages;
+  a.part_pages = std::max(1, (max_seq_len + kPage - 1) / kPage);  // (this kernel splits by seq_len)
   a.status = cache->status;
   a.scale = scale;
   a.tickets = static_cast<int*>(workspace);

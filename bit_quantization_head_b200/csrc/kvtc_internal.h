@@ -52,7 +52,6 @@ struct DecodeGroup {
   int n_stage = 0;              // stages per warp
   size_t smem = 0;              // dynamic shared memory per CTA
   int per_sm = 1;               // resident CTAs per SM at that size
-  int clusters = 0;             // resident clusters of 4 CTAs on the device (0: none)
   const void* fn = nullptr;     // the kernel variant
 };
 

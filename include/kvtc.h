@@ -310,8 +310,7 @@ uint64_t kvtc_decode_workspace_bytes(const kvtc_plan* plan, int n_seq, int max_s
  * that fits), but two calls that share a workspace and overlap on the GPU race.
  * Launches one kernel per group of KV heads with the same (b_K, b_V) (each pair has its
  * own kernel variant; one launch per layer when every head has the same widths);
- * nothing is allocated.  Long contexts run their splits in clusters of four CTAs that
- * merge their partials in distributed shared memory before the final merge.
+ * nothing is allocated.
  */
 kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_cache* cache, int layer,
                                   const void* q, kvtc_dtype q_dtype, const int32_t* seq_lens,
