@@ -601,10 +601,9 @@ constexpr size_t kHeadBytes = ((kBarOffset + 8 * kWarps * 8 + 127) / 128) * 128;
 // A = M_K's fp16 hi and lo fragments (plan), so q~ = (M_hi + M_lo)(q_hi + q_lo) with the
 // lo x lo product dropped (below 2^-22 relative).  Warp w forms m-tiles w and w + 4; the
 // result (column n = head n) lands in sh.qt, rows past r_K exactly zero (zero A rows).
-// The first tile's fragments were loaded before the wait for the preceding grid; the
-// second tile's loads go out before the first tile's MMAs, and each tile accumulates in
-// four independent chains (k-step parity x M part), so the MMA latency does not add up
-// along the 8 k-steps.
+// Both tiles' fragments were loaded before the wait for the preceding grid (the plan is
+// constant), and each tile accumulates in four independent chains (k-step parity x M
+// part), so the MMA latency does not add up along the 8 k-steps.
 __device__ __forceinline__ void qtilde_tile(SmemHead& sh, const uint4 (&fr)[16], int mt, int g, int tq, bool q_lo) {
   float c[4][4];
 #pragma unroll
@@ -634,18 +633,11 @@ __device__ __forceinline__ void qtilde_tile(SmemHead& sh, const uint4 (&fr)[16],
   sh.qt[2 * tq + 1][j + 8] = r[3] * s1;
 }
 
-__device__ __forceinline__ void form_qtilde(SmemHead& sh, const uint32_t* mfrag, int nmtK, int warp, int lane,
-                                            bool q_lo, const uint4 (&pre)[16]) {
+__device__ __forceinline__ void form_qtilde(SmemHead& sh, int nmtK, int warp, int lane, bool q_lo,
+                                            const uint4 (&fr0)[16], const uint4 (&fr1)[16]) {
   const int g = lane >> 2, tq = lane & 3;
-  const int mt1 = warp + kWarps;
-  uint4 fr1[16];
-  if (mt1 < nmtK) {
-    const uint4* src = reinterpret_cast<const uint4*>(mfrag) + static_cast<size_t>(mt1) * 8 * 2 * 32 + lane;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) fr1[k] = __ldg(src + k * 32);
-  }
-  if (warp < nmtK) qtilde_tile(sh, pre, warp, g, tq, q_lo);
-  if (mt1 < nmtK) qtilde_tile(sh, fr1, mt1, g, tq, q_lo);
+  if (warp < nmtK) qtilde_tile(sh, fr0, warp, g, tq, q_lo);
+  if (warp + kWarps < nmtK) qtilde_tile(sh, fr1, warp + kWarps, g, tq, q_lo);
 }
 
 // ---- the last CTA of a (sequence, KV head, head group): merge and back-project ------------
@@ -854,17 +846,25 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const int n_stage = min(6, static_cast<int>(ring_b / stage_b));
   if (lane == 0)
     for (int i = 0; i < n_stage; ++i) mbar_init(&bars[warp * 8 + i], 1);
+  fence_mbar_init();
+  __syncwarp();
   if (tid == 0) {
     prefetch_l2(dK.Mfrag, static_cast<uint32_t>(nmtK) * 8 * 2 * 32 * 16);
     if (dV.b != kRawBits) prefetch_l2(dV.M, static_cast<uint32_t>(rV) * kD * 4);
   }
-  // this warp's first m-tile of M_K fragments for q~ (16 x 16 bytes per lane)
-  uint4 mfrag[16];
+  // this warp's m-tiles of M_K fragments for q~ (tiles w and w + 4; 16 x 16 bytes per
+  // lane each; a warp without a tile reads the unit's first tile, in bounds, and never
+  // uses it)
+  uint4 mfrag[16], mfrag1[16];
   {
-    // (a warp without a tile reads the unit's first tile, in bounds, and never uses it)
     const uint4* src = reinterpret_cast<const uint4*>(dK.Mfrag) + static_cast<size_t>(warp < nmtK ? warp : 0) * 8 * 2 * 32 + lane;
+    const uint4* src1 = reinterpret_cast<const uint4*>(dK.Mfrag) +
+                        static_cast<size_t>(warp + kWarps < nmtK ? warp + kWarps : 0) * 8 * 2 * 32 + lane;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) mfrag[k] = __ldg(src + k * 32);
+    for (int k = 0; k < 16; ++k) {
+      mfrag[k] = __ldg(src + k * 32);
+      mfrag1[k] = __ldg(src1 + k * 32);
+    }
   }
   if (a.wait_first) griddep_wait();
   griddep_launch_dependents();
@@ -909,8 +909,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
 
   // ---- prologue: first copies (the barriers were set up by lane 0 of each warp, which
   // also issues the copies), then q~ while they are in flight ----
-  fence_mbar_init();
-  __syncwarp();
 
   const uint32_t bytesK = static_cast<uint32_t>(dK.page_bytes), bytesV = static_cast<uint32_t>(dV.page_bytes);
   const char* poolK = a.pool + a.pages_per_unit * dK.prefix;
@@ -975,7 +973,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   }
   for (int i = tid; i < 8 * 128; i += kThreads) sh.qt[i >> 7][i & 127] = 0.0f;
   __syncthreads();
-  form_qtilde(sh, dK.Mfrag, nmtK, warp, lane, q_lo, mfrag);
+  form_qtilde(sh, nmtK, warp, lane, q_lo, mfrag, mfrag1);
   __syncthreads();
 
   // per head: S = sum_j q~_j and the fp16 normalisation exponent (warp w: heads 2w, 2w+1)
