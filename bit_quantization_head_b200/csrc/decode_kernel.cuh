@@ -649,6 +649,8 @@ __device__ __forceinline__ void form_qtilde(SmemHead& sh, int nmtK, int warp, in
 // lane: four output columns; the four warps' sums meet in shared memory).
 // scratch: 2 * 8 * kMaxSplits (m, l) + 8 * 128 (y) + 4 * 8 * 128 (the reductions of the
 // split shares and of the back-projection) + 8 (l per head) floats.
+constexpr int kZBatch = 24;  // partials' z loads in flight per thread in the merge
+constexpr int kVBatch = 16;  // M_V rows in flight per warp in the back-projection
 __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDesc& dV, float* scratch, int s,
                                               int qh0, int ng, int n_split, int warp, int lane, int tid) {
   const int Hq = a.H * a.G;
@@ -693,7 +695,7 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
   }
   __syncthreads();
   // (3) z: slice p = (head, 4-coordinate group) and split share u; U shares per slice.
-  // The loads go out in explicit batches of sixteen (a register array filled before it is
+  // The loads go out in explicit batches of kZBatch (a register array filled before it is
   // used): measured here, a plain loop over the splits issued one L2 round trip per split.
   const int quads = (rV + 3) >> 2;
   const int P = ng * quads;
@@ -705,11 +707,11 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     const float* zp = base0 + n * head_stride + 4 + 4 * q;
     const float* wn = mbuf + n * n_split;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int i0 = u; i0 < n_split; i0 += 16 * U) {
-      float4 zz[16];
-      float ww[16];
+    for (int i0 = u; i0 < n_split; i0 += kZBatch * U) {
+      float4 zz[kZBatch];
+      float ww[kZBatch];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
+      for (int k = 0; k < kZBatch; ++k) {
         const int i = i0 + k * U;
         const bool in = i < n_split;
         zz[k] = in ? __ldcg(reinterpret_cast<const float4*>(zp + static_cast<size_t>(i) * kPartStride))
@@ -717,7 +719,7 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
         ww[k] = in ? wn[i] : 0.0f;
       }
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
+      for (int k = 0; k < kZBatch; ++k) {
         acc.x = fmaf(ww[k], zz[k].x, acc.x);
         acc.y = fmaf(ww[k], zz[k].y, acc.y);
         acc.z = fmaf(ww[k], zz[k].z, acc.z);
@@ -764,20 +766,20 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
     return;
   }
   // (4) o = M_V^T y: warp w takes rows w, w + 4, ... (lane: four output columns; M_V was
-  // prefetched into L2 by every CTA of the head), eight rows' loads in flight at a time
+  // prefetched into L2 by every CTA of the head), kVBatch rows' loads in flight at a time
   float4 o[8];
 #pragma unroll
   for (int n = 0; n < 8; ++n) o[n] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  for (int j0 = warp; j0 < rV; j0 += 8 * kWarps) {
-    float4 m4[8];
+  for (int j0 = warp; j0 < rV; j0 += kVBatch * kWarps) {
+    float4 m4[kVBatch];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < kVBatch; ++k) {
       const int j = j0 + k * kWarps;
       m4[k] = j < rV ? __ldg(reinterpret_cast<const float4*>(dV.M + static_cast<size_t>(j) * kD) + lane)
                      : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < kVBatch; ++k) {
       const int j = j0 + k * kWarps;
       if (j >= rV) break;  // (warp-uniform; y past r_V is not written)
 #pragma unroll
