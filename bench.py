@@ -52,10 +52,11 @@ DECODE_WORKLOAD = "llama8b-32L-128k-1bpd"
 ENCODE_WORKLOAD = "qwen7b-28L-128k-2bpd"
 
 # DRAM bytes (read + write) of one decode call per layer, from an ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum) of the current decode kernels on layers
-# 0-3 of the workload (the file named beside it); reported as roofline.traffic next to the
-# algorithmic bytes.  None whenever a decode kernel has changed since the capture.
-DECODE_TRAFFIC = {"llama8b-32L-128k-1bpd": (None, None)}
+# (dram__bytes_read.sum + dram__bytes_write.sum) of the current decode kernel: layer 6 of
+# the 8-layer copy of the workload read 32.40 MB against its 32.08 MB of algorithmic
+# bytes (1.010x); scaled by that ratio to this workload's mean layer (the file named
+# beside it).  None whenever a decode kernel has changed since the capture.
+DECODE_TRAFFIC = {"llama8b-32L-128k-1bpd": (34.42e6, "profiles/decode_split_llama8b-8L-128k-1bpd_ncu.md")}
 METRIC = "decode-attn effective HBM GB/s (% of peak) at 128k ctx; encode Mtok/s"
 
 
@@ -215,17 +216,14 @@ def decode_step(st, w, stream=None):
 
 
 def kernels_per_step(plan, w):
-    """Launches of the library's kernels per step: per layer the append, the q~ prep, one
-    split kernel per code-width class pair of the layer's KV heads (2, 4 and 8 have their
-    own kernels, other widths share one) and the combine."""
-    def cls(b):
-        return b if b in (2, 4, 8) else 0
+    """Launches of the library's kernels per step: per layer the append and one split
+    kernel per distinct (b_K, b_V) pair among the layer's KV heads (the merge and the
+    back-projection run inside the split kernel)."""
     n = 0
     H = plan.shape["n_kv_heads"]
     for layer in range(w.n_layers):
-        groups = {(cls(plan.unit((layer * H + h) * 2)["b"]), cls(plan.unit((layer * H + h) * 2 + 1)["b"]))
-                  for h in range(H)}
-        n += 3 + len(groups)
+        groups = {(plan.unit((layer * H + h) * 2)["b"], plan.unit((layer * H + h) * 2 + 1)["b"]) for h in range(H)}
+        n += 1 + len(groups)
     return n
 
 

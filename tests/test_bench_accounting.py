@@ -37,16 +37,14 @@ def test_algorithmic_bytes_count_codes_and_bases():
             assert sum(got) - bases <= n_seq * T * 32 * 128 // 8
 
 
-def test_kernels_per_step_counts_append_prep_splits_and_combine():
+def test_kernels_per_step_counts_append_and_one_split_launch_per_width_pair():
+    # per layer: the append, then one decode launch per distinct (b_K, b_V) of its heads
     w, plan = _plan(False)
     w2 = synth.scaled(w, n_layers=2)
     n = bench.kernels_per_step(plan, w2)
-    classes = []
+    pairs = []
     for layer in range(2):
-        pairs = set()
-        for h in range(8):
-            bk, bv = plan.unit((layer * 8 + h) * 2)["b"], plan.unit((layer * 8 + h) * 2 + 1)["b"]
-            pairs.add((bk if bk in (2, 4, 8) else 0, bv if bv in (2, 4, 8) else 0))
-        classes.append(len(pairs))
-    assert n == sum(3 + c for c in classes)
-    assert np.all(np.array(classes) >= 1)
+        pairs.append({(plan.unit((layer * 8 + h) * 2)["b"], plan.unit((layer * 8 + h) * 2 + 1)["b"])
+                      for h in range(8)})
+    assert n == sum(1 + len(p) for p in pairs)
+    assert all(len(p) >= 1 for p in pairs)
