@@ -198,8 +198,8 @@ struct SmemHead {
     } q16;
     uint32_t frag[2][8][2][32];  // B fragments of q^: [hi, lo][k-step][half][lane]
   } u;
-  float S[8];              // sum_j q~_j
-  int E[8];                // power-of-two normalisation of q~ for fp16
+  float Spart[8][8];       // [m-tile][head]: sum of q~ over the tile's 16 rows
+  int E[8];                // power-of-two normalisation of q~ for fp16 (from a bound on |q~|)
   int Eq[8];               // power-of-two normalisation of q for fp16
   int last;                // this CTA merges the (sequence, KV head, head group)
 };
@@ -609,7 +609,8 @@ constexpr size_t kHeadBytes = ((kBarOffset + 8 * kWarps * 8 + 127) / 128) * 128;
 // q of head n (n < ng) is scaled by 2^-Eq[n] and stored as fp16 hi (+ lo for fp32 input);
 // A = M_K's fp16 hi and lo fragments (plan), so q~ = (M_hi + M_lo)(q_hi + q_lo) with the
 // lo x lo product dropped (below 2^-22 relative).  Warp w forms m-tiles w and w + 4; the
-// result (column n = head n) lands in sh.qt, rows past r_K exactly zero (zero A rows).
+// result (column n = head n) lands in sh.qt, rows past r_K exactly zero (zero A rows),
+// and each tile's sum over its rows in sh.Spart.
 // Both tiles' fragments were loaded before the wait for the preceding grid (the plan is
 // constant), and each tile accumulates in four independent chains (k-step parity x M
 // part), so the MMA latency does not add up along the 8 k-steps.
@@ -640,6 +641,17 @@ __device__ __forceinline__ void qtilde_tile(SmemHead& sh, const uint4 (&fr)[16],
   sh.qt[2 * tq + 1][j] = r[1] * s1;
   sh.qt[2 * tq][j + 8] = r[2] * s0;
   sh.qt[2 * tq + 1][j + 8] = r[3] * s1;
+  // the tile's share of S = sum_j q~_j for heads 2 tq, 2 tq + 1 (summed over g)
+  float sa = (r[0] + r[2]) * s0, sb = (r[1] + r[3]) * s1;
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    sa += __shfl_xor_sync(0xffffffffu, sa, o);
+    sb += __shfl_xor_sync(0xffffffffu, sb, o);
+  }
+  if (g == 0) {
+    sh.Spart[mt][2 * tq] = sa;
+    sh.Spart[mt][2 * tq + 1] = sb;
+  }
 }
 
 __device__ __forceinline__ void form_qtilde(SmemHead& sh, int nmtK, int warp, int lane, bool q_lo,
@@ -961,15 +973,25 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     if (lane == 0) issue(i, pid);  // page i < n_stage uses slot i
   }
 
-  // ---- q of the group into shared memory as fp16, scaled per head; q~ cleared
+  // ---- q of the group into shared memory as fp16, scaled per head, and the fp16
+  // normalisation of q~: |q~_j| <= ||M_K row j|| ||q||_2 <= mnorm ||q||_2 (Cauchy-Schwarz;
+  // mnorm is rounded up, the factor 1.01 covers the rounding of the formed q~), so
+  // q^ = q~ 2^-E with E = ilogb(bound) - 14 stays below 2^15
   const bool q_lo = !a.q_bf16;
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     const int gg = 2 * warp + hh;
     const float4 v = qv[hh];
     float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    float ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, v.w * v.w)));
 #pragma unroll
-    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    for (int o = 16; o; o >>= 1) {
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    }
+    // (||q||_2 from max |q| when the squares leave the fp32 range)
+    const float qn = (ss > 0x1p-100f && ss < 0x1p100f) ? sqrtf(ss) : amax * 11.32f;
+    const float bound = dK.mnorm * qn * 1.01f;
     // max |q| 2^-Eq in [2^14, 2^15): fp16 holds it with headroom
     const int Eq = (amax > 0.0f && amax < INFINITY) ? ilogbf(amax) - 14 : 0;
     const float sc = ldexpf(1.0f, -Eq);
@@ -980,36 +1002,20 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       sh.u.q16.hi[gg][4 * lane + e] = __half_as_ushort(hq);
       sh.u.q16.lo[gg][4 * lane + e] = __half_as_ushort(__float2half_rn(xs[e] - __half2float(hq)));
     }
-    if (lane == 0) sh.Eq[gg] = Eq;
+    if (lane == 0) {
+      sh.Eq[gg] = Eq;
+      sh.E[gg] = (bound > 0.0f && bound < INFINITY) ? ilogbf(bound) - 14 : 0;
+    }
   }
-  for (int i = tid; i < 8 * 128; i += kThreads) sh.qt[i >> 7][i & 127] = 0.0f;
   __syncthreads();
   form_qtilde(sh, nmtK, warp, lane, q_lo, mfrag, mfrag1);
   __syncthreads();
 
-  // per head: S = sum_j q~_j and the fp16 normalisation exponent (warp w: heads 2w, 2w+1)
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int gg = 2 * warp + hh;
-    float S = sh.qt[gg][lane] + sh.qt[gg][lane + 32] + sh.qt[gg][lane + 64] + sh.qt[gg][lane + 96];
-    float amax = fmaxf(fmaxf(fabsf(sh.qt[gg][lane]), fabsf(sh.qt[gg][lane + 32])),
-                       fmaxf(fabsf(sh.qt[gg][lane + 64]), fabsf(sh.qt[gg][lane + 96])));
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      S += __shfl_xor_sync(0xffffffffu, S, o);
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    }
-    if (lane == 0) {
-      sh.S[gg] = S;
-      sh.E[gg] = amax > 0.0f ? ilogbf(amax) - 14 : 0;
-    }
-  }
-  __syncthreads();
-
-  // B fragments of q^ = q~ * 2^-E, shared by the four warps: [hi, lo][k-step][half][lane]
-  // (lane (g, t): rows 16 ks + 8 half + 2t, + 1, column g).  Packed (G <= 4): column n
-  // holds head n / 2, its hi part for even n and its lo part for odd n.
-  for (int idx = tid; idx < 8 * 2 * 32; idx += kThreads) {
+  // B fragments of q^ = q~ * 2^-E of the k-steps below r_K, shared by the four warps:
+  // [hi, lo][k-step][half][lane] (lane (g, t): rows 16 ks + 8 half + 2t, + 1, column g).
+  // Packed (G <= 4): column n holds head n / 2, its hi part for even n and its lo part
+  // for odd n.
+  for (int idx = tid; idx < nmtK * 2 * 32; idx += kThreads) {
     const int ks = idx >> 6, half = (idx >> 5) & 1, ln = idx & 31;
     const int gl = ln >> 2, tql = ln & 3;
     const int hsrc = PACK ? (gl >> 1) : gl;
@@ -1057,7 +1063,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     for (int c = 0; c < 2; ++c) {
       const int n = PACK ? tq : 2 * tq + c;  // packed: one head per lane
       w.alpha[c] = n < ng ? base * ldexpf(1.0f, sh.E[n] + 24) : 0.0f;
-      w.beta[c] = n < ng ? base * mK * sh.S[n] : 0.0f;
+      float S = 0.0f;  // sum_j q~_j of head n, tile by tile in a fixed order
+      for (int mt = 0; mt < nmtK; ++mt) S += n < ng ? sh.Spart[mt][n] : 0.0f;
+      w.beta[c] = n < ng ? base * mK * S : 0.0f;
       w.m_run[c] = -INFINITY;
       w.lcvt[c] = 0.0f;
     }
