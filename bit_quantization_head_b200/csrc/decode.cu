@@ -6,10 +6,11 @@
 // same algebra as NOVA-KV's query-side fold on the pith.science review page) and values
 // are accumulated in their latent basis, back-projected once per query head.
 //
-// One kernel launch per layer and width-class group (decode_split_kernel<BK, BV, PACK>,
+// One kernel launch per layer and (b_K, b_V) group (decode_split_kernel<BK, BV, PACK>,
 // decode_kernel.cuh): every CTA forms q~ for its heads on the tensor cores, streams its
-// share of the context's pages (split-K), and writes a partial (m, l, z); the CTA that
-// completes a (sequence, KV head, head group) last merges the partials and back-projects.
+// share of the context's pages (split-K), and writes a partial (m, l, z); the last CTAs to
+// complete a (sequence, KV head, head group) merge the partials and back-project, each
+// for a share of its query heads.
 // The launches use programmatic dependent launch, so their set-up (plan reads, barrier
 // initialisation, L2 prefetch of M_V) overlaps the tail of the preceding kernel.
 #include <cuda_runtime.h>
@@ -76,7 +77,7 @@ cudaError_t launch_pdl(void (*fn)(KArgs...), dim3 grid, dim3 block, size_t smem,
 }
 
 size_t tickets_bytes(const kvtc_plan* plan, int n_seq) {
-  const size_t n = static_cast<size_t>(n_seq) * plan->H * ((plan->G + 7) / 8);
+  const size_t n = static_cast<size_t>(n_seq) * plan->H * ((plan->G + 7) / 8) * kTicketInts;
   return (n * sizeof(int) + 255) / 256 * 256;
 }
 
@@ -164,8 +165,8 @@ kvtc_status prepare_decode(kvtc_plan* plan) {
 using namespace kvtc;
 using namespace kvtc::dec;
 
-// Workspace: the arrival tickets [n_seq][H][ceil(G/8)] int32 (256-byte rounded), then the
-// partials [n_seq][Hq][cap][kPartStride] floats.
+// Workspace: the arrival tickets [n_seq][H][ceil(G/8)][kTicketInts] int32 (256-byte
+// rounded), then the partials [n_seq][Hq][cap][kPartStride] floats.
 extern "C" uint64_t kvtc_decode_workspace_bytes(const kvtc_plan* plan, int n_seq, int max_seq_len) {
   if (!plan || n_seq < 1 || max_seq_len < 0) return 0;
   const uint64_t heads = static_cast<uint64_t>(n_seq) * plan->H * plan->G;

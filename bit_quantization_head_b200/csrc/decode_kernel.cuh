@@ -29,9 +29,11 @@
 // 2-bit value codes in packed mode skip the shift and fold the whole 1.5 l per page.
 // A page's eight 16-token blocks are processed together (their MMA chains interleave).
 // The four warps' (m, l, z) meet in shared memory and each CTA writes one partial per
-// query head; the CTA that completes a (sequence, KV head, head group) last (an atomic
-// ticket in the workspace) merges every split's partial with a log-sum-exp, dequantizes
-// (delta_V) and back-projects o = M_V^T y itself, then re-arms the ticket.
+// query head; the last min(G, splits) CTAs to complete a (sequence, KV head, head group)
+// (an atomic arrival counter in the workspace) each take a share of its query heads:
+// once every split has written its partial, they merge the partials with a log-sum-exp,
+// dequantize (delta_V) and back-project o = M_V^T y on several SMs at once; the last of
+// them re-arms the counters.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -54,6 +56,9 @@ constexpr int kMinBlocks = 3;         // resident CTAs per SM the registers are 
 constexpr int kPartStride = 132;      // floats per partial: m, l, 2 pad, z[128]
 constexpr int kMaxHeadsPerLaunch = 64;
 constexpr int kMaxSplits = 128;       // context splits per KV head (bounds the merge scratch)
+constexpr int kTicketInts = 2;        // per (sequence, KV head, head group): arrivals, merges done
+constexpr uint32_t kSpinLimit = 1u << 20;  // polls (100 ns apart) before a merge share gives up
+constexpr int kParMerge = 16;         // splits from which the merge is shared among the last CTAs
 // floats of merge scratch the last CTA needs ((m, l) of every split, y, the warps'
 // back-projections)
 constexpr int kMergeFloats = 16 * kMaxSplits + 8 * 128 + 4 * 8 * 128 + 8;
@@ -201,7 +206,7 @@ struct SmemHead {
   float Spart[8][8];       // [m-tile][head]: sum of q~ over the tile's 16 rows
   int E[8];                // power-of-two normalisation of q~ for fp16 (from a bound on |q~|)
   int Eq[8];               // power-of-two normalisation of q for fp16
-  int last;                // this CTA merges the (sequence, KV head, head group)
+  int ticket;              // this CTA's arrival position, then whether its merge share may run
 };
 
 // ------------------------------------------------------------------ per-warp state
@@ -661,7 +666,7 @@ __device__ __forceinline__ void form_qtilde(SmemHead& sh, int nmtK, int warp, in
   if (warp + kWarps < nmtK) qtilde_tile(sh, fr1, warp + kWarps, g, tq, q_lo);
 }
 
-// ---- the last CTA of a (sequence, KV head, head group): merge and back-project ------------
+// ---- the last CTAs of a (sequence, KV head, head group): merge and back-project ----------
 // Partials (m in the log2 domain, l, centred z times 2^-17) of every split.  The merge is
 // the serial tail of the call, so it is written for memory-level parallelism: every
 // (m, l) is fetched at once, then each thread owns one (head, 4-coordinate) slice of z
@@ -672,12 +677,16 @@ __device__ __forceinline__ void form_qtilde(SmemHead& sh, int nmtK, int warp, in
 // split shares and of the back-projection) + 8 (l per head) floats.
 constexpr int kZBatch = 24;  // partials' z loads in flight per thread in the merge
 constexpr int kVBatch = 16;  // M_V rows in flight per warp in the back-projection
+// Merges the query heads n0, n0 + nstep, ... (< ng) of the group starting at query head
+// qh0; nl of them, local index ln.
 __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDesc& dV, float* scratch, int s,
-                                              int qh0, int ng, int n_split, int warp, int lane, int tid) {
+                                              int qh0, int ng, int n0, int nstep, int n_split, int warp, int lane,
+                                              int tid) {
   const int Hq = a.H * a.G;
   const int rV = dV.r;
   const bool raw = dV.b == kRawBits;
-  float* mbuf = scratch;                     // [ng][n_split]: the weights 2^(m - M)
+  const int nl = (ng - n0 + nstep - 1) / nstep;
+  float* mbuf = scratch;                     // [nl][n_split]: the weights 2^(m - M)
   float* ybuf = scratch + 16 * kMaxSplits;   // [8][128]
   float* obuf = ybuf + 8 * 128;              // [4][8][128] (also the split-share reduction)
   float* Lsum = ybuf + 8 * 128 + 4 * 8 * 128;  // [8]
@@ -686,8 +695,8 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
   const float* base0 = a.ws + (static_cast<size_t>(s) * Hq + qh0) * head_stride;
   // (1) per head (warp per head): every split's (m, l) in one batch of loads (lane i,
   // i + 32, ...), the largest m, the weights 2^(m - M) and l
-  for (int n = warp; n < ng; n += kWarps) {
-    const float* hb = base0 + n * head_stride;
+  for (int n = warp; n < nl; n += kWarps) {
+    const float* hb = base0 + (n0 + n * nstep) * head_stride;
     float mi[kMaxSplits / 32], li[kMaxSplits / 32];
 #pragma unroll
     for (int k = 0; k < kMaxSplits / 32; ++k) {
@@ -719,13 +728,13 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
   // The loads go out in explicit batches of kZBatch (a register array filled before it is
   // used): measured here, a plain loop over the splits issued one L2 round trip per split.
   const int quads = (rV + 3) >> 2;
-  const int P = ng * quads;
+  const int P = nl * quads;
   const int U = P >= kThreads ? 1 : kThreads / P;
   float4* red = reinterpret_cast<float4*>(obuf);  // [U][P] when U > 1 (U * P <= 128)
   for (int t = tid; t < P * U; t += kThreads) {
     const int p = t % P, u = t / P;
     const int n = p / quads, q = p - n * quads;
-    const float* zp = base0 + n * head_stride + 4 + 4 * q;
+    const float* zp = base0 + (n0 + n * nstep) * head_stride + 4 + 4 * q;
     const float* wn = mbuf + n * n_split;
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     for (int i0 = u; i0 < n_split; i0 += kZBatch * U) {
@@ -776,9 +785,9 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
   __syncthreads();
   if (raw) {
     // an uncompressed value unit is already in d-space (identity back-projection)
-    for (int i = tid; i < ng * 128; i += kThreads) {
+    for (int i = tid; i < nl * 128; i += kThreads) {
       const int n = i >> 7, k = i & 127;
-      const size_t off = (static_cast<size_t>(s) * Hq + qh0 + n) * kD + k;
+      const size_t off = (static_cast<size_t>(s) * Hq + qh0 + n0 + n * nstep) * kD + k;
       if (a.out_bf16)
         static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(ybuf[n * 128 + k]);
       else
@@ -805,7 +814,7 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
       if (j >= rV) break;  // (warp-uniform; y past r_V is not written)
 #pragma unroll
       for (int n = 0; n < 8; ++n) {
-        if (n < ng) {
+        if (n < nl) {
           const float yj = ybuf[n * 128 + j];
           o[n].x = fmaf(m4[k].x, yj, o[n].x);
           o[n].y = fmaf(m4[k].y, yj, o[n].y);
@@ -817,13 +826,13 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
   }
 #pragma unroll
   for (int n = 0; n < 8; ++n)
-    if (n < ng) reinterpret_cast<float4*>(obuf + (warp * 8 + n) * 128)[lane] = o[n];
+    if (n < nl) reinterpret_cast<float4*>(obuf + (warp * 8 + n) * 128)[lane] = o[n];
   __syncthreads();
-  for (int i = tid; i < ng * 128; i += kThreads) {
+  for (int i = tid; i < nl * 128; i += kThreads) {
     const int n = i >> 7, k = i & 127;
     const float v = (obuf[(0 * 8 + n) * 128 + k] + obuf[(1 * 8 + n) * 128 + k]) +
                     (obuf[(2 * 8 + n) * 128 + k] + obuf[(3 * 8 + n) * 128 + k]);
-    const size_t off = (static_cast<size_t>(s) * Hq + qh0 + n) * kD + k;
+    const size_t off = (static_cast<size_t>(s) * Hq + qh0 + n0 + n * nstep) * kD + k;
     if (a.out_bf16)
       static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(v);
     else
@@ -1231,17 +1240,39 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     }
   }
 
-  // ---- arrival ticket: the CTA that completes the (sequence, KV head, head group) last
-  // merges every split's partial and writes the output, then re-arms the ticket ----
+  // ---- arrival tickets: the last n_par = min(ng, n_split) CTAs to finish a (sequence, KV
+  // head, head group) each merge a share of its query heads (the k-th last takes heads k,
+  // k + n_par, ...) once every split has written its partial, so the merge runs on
+  // several SMs at once; the last of them re-arms the counters.  With few splits the
+  // merge is short and the last CTA does it alone (n_par = 1).  A CTA that takes a
+  // share has finished its own work and waits (bounded) only for CTAs that hold a
+  // ticket position after it, which have all started.
   __threadfence();
   __syncthreads();
-  int* ticket = a.tickets + (static_cast<size_t>(s) * a.H + h) * a.n_hg + hg;
-  if (tid == 0) sh.last = atomicAdd(ticket, 1) == n_split - 1;
+  int* ticket = a.tickets + ((static_cast<size_t>(s) * a.H + h) * a.n_hg + hg) * kTicketInts;
+  if (tid == 0) sh.ticket = atomicAdd(ticket, 1);
   __syncthreads();
-  if (sh.last) {
-    __threadfence();
-    merge_project(a, dV, mb, s, h * a.G + g0, ng, n_split, warp, lane, tid);
-    if (tid == 0) atomicExch(ticket, 0);
+  const int n_par = n_split >= kParMerge ? min(ng, n_split) : 1;
+  const int k_last = n_split - 1 - sh.ticket;  // 0: this CTA finished last
+  if (k_last >= 0 && k_last < n_par) {  // (a counter left non-zero by a broken call gives none)
+    if (tid == 0) {
+      uint32_t it = 0;
+      while (ld_acquire_gpu(ticket) < n_split && it < kSpinLimit) {
+        __nanosleep(100);
+        ++it;
+      }
+      sh.ticket = it < kSpinLimit;
+      if (it >= kSpinLimit && a.status) atomicOr(a.status, KVTC_STATUS_TIMEOUT);
+    }
+    __syncthreads();
+    if (sh.ticket) {
+      __threadfence();
+      merge_project(a, dV, mb, s, h * a.G + g0, ng, k_last, n_par, n_split, warp, lane, tid);
+    }
+    if (tid == 0 && atomicAdd(ticket + 1, 1) == n_par - 1) {
+      atomicExch(ticket, 0);
+      atomicExch(ticket + 1, 0);
+    }
   }
   if (!a.wait_first) griddep_wait();
 }

@@ -555,12 +555,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_rope_kernel(const __grid_c
   }
   __threadfence();
   __syncthreads();
-  int* ticket = a.tickets + (static_cast<size_t>(s) * a.H + h) * a.n_hg + hg;
+  int* ticket = a.tickets + ((static_cast<size_t>(s) * a.H + h) * a.n_hg + hg) * kTicketInts;
   if (tid == 0) sm.last = atomicAdd(ticket, 1) == n_split - 1;
   __syncthreads();
   if (sm.last) {
     __threadfence();
-    merge_project(a, dV, mb, s, h * a.G + g0, ng, n_split, warp, lane, tid);
+    merge_project(a, dV, mb, s, h * a.G + g0, ng, 0, 1, n_split, warp, lane, tid);
     if (tid == 0) atomicExch(ticket, 0);
   }
   if (!a.wait_first) griddep_wait();
@@ -665,7 +665,9 @@ extern "C" kvtc_status kvtc_decode_attention_rope(const kvtc_plan* plan, const k
   a.status = cache->status;
   a.scale = scale;
   a.tickets = static_cast<int*>(workspace);
-  const size_t tb = (static_cast<size_t>(n_seq) * plan->H * n_hg * sizeof(int) + 255) / 256 * 256;
+  // the workspace layout of kvtc_decode_attention: tickets [n_seq][H][n_hg][kTicketInts]
+  // (this kernel counts arrivals in the first), then the partials
+  const size_t tb = (static_cast<size_t>(n_seq) * plan->H * n_hg * kTicketInts * sizeof(int) + 255) / 256 * 256;
   a.ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + tb);
   // one launch per (b_K, b_V) variant class; every KV head of the layer in one of them
   struct Group {

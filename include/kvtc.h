@@ -283,7 +283,7 @@ kvtc_status kvtc_plan_prefill_stats(const kvtc_plan* plan, uint64_t* codes, uint
 /* ------------------------------------------------------------------ decode ------- */
 
 /* Workspace bytes kvtc_decode_attention needs for n_seq sequences of at most
- * max_seq_len tokens: arrival tickets (one int32 per sequence, KV head and group of 8
+ * max_seq_len tokens: arrival counters (two int32 per sequence, KV head and group of 8
  * query heads) followed by the split-K partials. */
 uint64_t kvtc_decode_workspace_bytes(const kvtc_plan* plan, int n_seq, int max_seq_len);
 
@@ -296,8 +296,9 @@ uint64_t kvtc_decode_workspace_bytes(const kvtc_plan* plan, int n_seq, int max_s
  *   o = M_V^T (delta_V * z).
  * Equivalent to softmax(scale * q . k_hat_t) v_hat_t with k_hat = M_K^T delta_K (c - m)
  * (the oracle's d-space form).  Split-K over the context; the G query heads of a KV head
- * share every code tile; the last split of a (sequence, KV head) to finish merges the
- * partials (log-sum-exp) and back-projects, in the same kernel.  An uncompressed value
+ * share every code tile; the last splits of a (sequence, KV head) to finish merge the
+ * partials (log-sum-exp) and back-project, each a share of the query heads, in the same
+ * kernel.  An uncompressed value
  * unit (keys-only plans) enters the value MMAs with its fp16 values as they are stored
  * (c_V = v * 2^24, delta_V = 2^-24, m_V = 0, M_V = identity), so o = sum_t p_t v_t.
  * q: device [n_seq][H_q][d] of q_dtype.  seq_lens: device int32 [n_seq] (0 gives an
@@ -305,9 +306,10 @@ uint64_t kvtc_decode_workspace_bytes(const kvtc_plan* plan, int n_seq, int max_s
  * longer sequences set KVTC_STATUS_BAD_POS).  softmax_scale: 0 means 1/sqrt(d).
  * out: device [n_seq][H_q][d] of out_dtype.  workspace: device, at least
  * kvtc_decode_workspace_bytes(plan, n_seq, max_seq_len) bytes (else ECAPACITY), 16-byte
- * aligned and zero-filled before its first use; every call leaves its tickets at zero
+ * aligned and zero-filled before its first use; every call leaves its counters at zero
  * again, so one workspace serves any number of consecutive calls (of any plan and shape
- * that fits), but two calls that share a workspace and overlap on the GPU race.
+ * that fits), but two calls that share a workspace and overlap on the GPU race.  After a
+ * call that set KVTC_STATUS_TIMEOUT the workspace must be zero-filled again.
  * Launches one kernel per group of KV heads with the same (b_K, b_V) (each pair has its
  * own kernel variant; one launch per layer when every head has the same widths);
  * nothing is allocated.
