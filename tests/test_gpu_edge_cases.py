@@ -183,3 +183,36 @@ def test_tiny_rows_at_a_tiny_step_keep_canonical_codes():
     units = gh.plan_units(plan)
     codes = gh.oracle_codes(K[:, 0], units[0], "bf16")
     assert len(np.unique(codes)) > 4
+
+
+def test_shared_merge_wait_is_bounded_and_reports_a_timeout():
+    # The last CTAs of a head group wait for the group's arrival counter to reach the
+    # split count before each merges its share.  A counter that starts at -2 (a workspace
+    # that was not zero-filled) never gets there: the waits must end on their own, set
+    # KVTC_STATUS_TIMEOUT and leave the context usable; a zero-filled workspace then
+    # gives the oracle's result again.
+    rng = np.random.default_rng(31)
+    H, G = 1, 4
+    plan = gh.random_plan(1, H, G, [((32, 2), (32, 2))], rng)
+    T = 16384                       # 128 pages: 16 splits, the shared merge is on
+    cache = gh.make_cache(plan, [T], rng)
+    kv = [(rng.standard_normal((T, H, 128)).astype(np.float32), rng.standard_normal((T, H, 128)).astype(np.float32))]
+    gh.encode_all(plan, cache, 0, kv, "f32")
+    q = (rng.standard_normal((1, H * G, 128)) * 0.5).astype(np.float32)
+    qd = gh.to_dev(q, "f32")
+    sl = torch.tensor([T], dtype=torch.int32, device="cuda")
+    ws = torch.zeros(kvtc.kvtc_decode_workspace_bytes(plan, 1, T), dtype=torch.uint8, device="cuda")
+    out = torch.zeros((1, H * G, 128), dtype=torch.float32, device="cuda")
+    ws.view(torch.int32)[0] = -2
+    kvtc.kvtc_decode_attention(plan, cache, 0, qd, sl, T, out, ws)
+    torch.cuda.synchronize()
+    assert int(cache.status.item()) & kvtc.STATUS_TIMEOUT
+    cache.status.zero_()
+    ws.zero_()
+    kvtc.kvtc_decode_attention(plan, cache, 0, qd, sl, T, out, ws)
+    torch.cuda.synchronize()
+    assert int(cache.status.item()) == 0
+    assert int(ws.view(torch.int32)[:2].abs().sum().item()) == 0   # counters re-armed
+    ref = gh.oracle_decode(plan, cache, 0, q.astype(np.float64), [T], H, G)
+    ab, rel = gh.decode_errors(out.cpu().numpy(), ref)
+    assert ab <= TOL and rel <= TOL, (ab, rel)
