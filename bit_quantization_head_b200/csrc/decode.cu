@@ -85,7 +85,7 @@ size_t tickets_bytes(const kvtc_plan* plan, int n_seq) {
 }  // namespace dec
 
 // The decode launches of every layer: heads grouped by the kernel variant of their
-// (b_K, b_V) width classes, the stage size of each group, and the stage count and
+// (b_K, b_V) pair, the stage size of each group, and the stage count and
 // occupancy that fit (the most CTAs per SM, up to three, that leave a stage per warp).
 // Sets each variant's shared-memory attribute once, here, so decode calls do no host
 // allocation and no attribute calls.

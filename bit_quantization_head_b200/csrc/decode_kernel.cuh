@@ -59,7 +59,7 @@ constexpr int kMaxSplits = 128;       // context splits per KV head (bounds the 
 constexpr int kTicketInts = 2;        // per (sequence, KV head, head group): arrivals, merges done
 constexpr uint32_t kSpinLimit = 1u << 20;  // polls (100 ns apart) before a merge share gives up
 constexpr int kParMerge = 16;         // splits from which the merge is shared among the last CTAs
-// floats of merge scratch the last CTA needs ((m, l) of every split, y, the warps'
+// floats of merge scratch a merging CTA needs ((m, l) of every split, y, the warps'
 // back-projections)
 constexpr int kMergeFloats = 16 * kMaxSplits + 8 * 128 + 4 * 8 * 128 + 8;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -88,7 +88,7 @@ struct DecodeArgs {
   float scale;
   int n_stage;          // stages per warp of the widest head of the launch
   uint32_t stage_bytes;  // that head's stage (K + V page, 128-byte rounded)
-  int* tickets;       // [n_seq][H][n_hg] arrival counters (zero between calls)
+  int* tickets;       // [n_seq][H][n_hg][kTicketInts] arrival counters (zero between calls)
   float* ws;          // partials [n_seq][Hq][part_stride][kPartStride]
 };
 
