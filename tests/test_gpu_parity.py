@@ -205,6 +205,23 @@ def test_query_groups_larger_than_eight_and_peaked_attention():
     _check_decode(plan, cache, 0, q, lens, H, G, "f32")
 
 
+@pytest.mark.parametrize("G", [6, 12])
+def test_shared_merge_over_long_contexts_and_head_groups(G):
+    # 33k tokens give the launch 33 splits per KV head, so the merge is shared by the last
+    # CTAs of each head group (one query head each; G = 12 has groups of 8 and 4, G = 6
+    # one group of 6, unpacked); the short third sequence leaves most of its splits empty
+    rng = np.random.default_rng(40 + G)
+    H = 2
+    plan = gh.random_plan(1, H, G, [((48, 2), (40, 2)), ((96, 3), (128, 4))], rng)
+    lens = [20000, 33000, 700]
+    cache = gh.make_cache(plan, lens, rng)
+    kv = [(rng.standard_normal((T, H, 128)).astype(np.float32),
+           rng.standard_normal((T, H, 128)).astype(np.float32)) for T in lens]
+    gh.encode_all(plan, cache, 0, kv, "f32", path="prefill")
+    q = (rng.standard_normal((len(lens), H * G, 128)) * 1.5).astype(np.float32)
+    _check_decode(plan, cache, 0, q, lens, H, G, "f32")
+
+
 def test_out_of_range_pages_and_positions_set_status_bits():
     rng = np.random.default_rng(4)
     plan = gh.random_plan(1, 1, 1, [((16, 2), (16, 2))], rng)
