@@ -203,7 +203,7 @@ extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_c
   int* tickets = static_cast<int*>(workspace);
   float* parts = reinterpret_cast<float*>(static_cast<char*>(workspace) + tickets_bytes(plan, n_seq));
 
-  // One launch per width-class group; the launches run side by side, so each gets the
+  // One launch per (b_K, b_V) group; the launches run side by side, so each gets the
   // share of a wave of resident CTAs that its work is of the layer's, and within a group
   // each head gets context splits in proportion to its work per page.  The work of a page
   // is mostly instruction issue, not bytes: the online softmax costs the same for every
