@@ -63,6 +63,8 @@ __device__ __forceinline__ void store_code(uint32_t* page, int kind, int r, int 
 // chains then run in the canonical order from registers and broadcast reads.
 __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constant__ AppendArgs a) {
   __shared__ float xs[kD];
+  __shared__ int s_seq;
+  __shared__ long long s_pos;
   const int tok = blockIdx.x, ul = blockIdx.y, j = threadIdx.x;
   const int u = a.unit0 + ul;
   // The plan (unit descriptor, bf16 row of M) is constant: read it before waiting for
@@ -81,12 +83,47 @@ __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constan
   const int kind = ul & 1;
   const int head = ul >> 1;
   const size_t xoff = (static_cast<size_t>(tok) * a.H + head) * kD;
-  if (a.bf16)
-    xs[j] = __bfloat162float((static_cast<const __nv_bfloat16*>(kind ? a.v : a.k) + xoff)[j]);
-  else
-    xs[j] = (static_cast<const float*>(kind ? a.v : a.k) + xoff)[j];
+  // The inputs go out together: the token's row element, and its sequence and position
+  // (thread i tests whether the token lies in [cu_seqlens[i], cu_seqlens[i + 1]), so one
+  // round of loads finds it; more sequences than threads take a binary search).
+  const float xv = a.bf16 ? __bfloat162float((static_cast<const __nv_bfloat16*>(kind ? a.v : a.k) + xoff)[j])
+                          : (static_cast<const float*>(kind ? a.v : a.k) + xoff)[j];
+  if (j == 0) {  // (a token no interval holds is reported as a bad position)
+    s_seq = 0;
+    s_pos = -1;
+  }
+  __syncthreads();
+  if (a.n_seq <= static_cast<int>(blockDim.x)) {
+    if (j < a.n_seq) {
+      const int c0 = a.cu_seqlens[j], c1 = a.cu_seqlens[j + 1];
+      const int ps = a.pos_start[j];
+      if (c0 <= tok && tok < c1) {
+        s_seq = j;
+        s_pos = static_cast<long long>(ps) + (tok - c0);
+      }
+    }
+  } else if (j == 0) {
+    int lo = 0, hi = a.n_seq - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.cu_seqlens[mid] <= tok)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    s_seq = lo;
+    s_pos = static_cast<long long>(a.pos_start[lo]) + (tok - a.cu_seqlens[lo]);
+  }
+  xs[j] = xv;
   __syncthreads();
   if (j >= ud.r) return;
+  // token -> page: the block-table entry is loaded before the arithmetic below
+  const int s = s_seq;
+  const long long pos = s_pos;
+  const bool pos_ok = pos >= 0 && pos < static_cast<long long>(a.max_pages) * kPage;
+  const int lp = pos_ok ? static_cast<int>(pos / kPage) : 0;
+  const int slot = pos_ok ? static_cast<int>(pos % kPage) : 0;
+  const int32_t pid = pos_ok ? a.block_table[static_cast<size_t>(s) * a.max_pages + lp] : -1;
 
   uint32_t code = 0;
   if (raw) {
@@ -125,24 +162,10 @@ __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constan
     code = quantize_code(acc, ud.inv_delta, ud.b);
   }
 
-  // token -> (sequence, position) -> page
-  int lo = 0, hi = a.n_seq - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.cu_seqlens[mid] <= tok)
-      lo = mid;
-    else
-      hi = mid - 1;
-  }
-  const int s = lo;
-  const long long pos = static_cast<long long>(a.pos_start[s]) + (tok - a.cu_seqlens[s]);
-  if (pos < 0 || pos >= static_cast<long long>(a.max_pages) * kPage) {
+  if (!pos_ok) {
     if (a.status) atomicOr(a.status, KVTC_STATUS_BAD_POS);
     return;
   }
-  const int lp = static_cast<int>(pos / kPage);
-  const int slot = static_cast<int>(pos % kPage);
-  const int32_t pid = a.block_table[static_cast<size_t>(s) * a.max_pages + lp];
   if (pid < 0 || static_cast<uint64_t>(pid) >= a.pages_per_unit) {
     if (a.status) atomicOr(a.status, KVTC_STATUS_BAD_PAGE);
     return;
