@@ -174,13 +174,11 @@ extern "C" uint64_t kvtc_decode_workspace_bytes(const kvtc_plan* plan, int n_seq
          heads * static_cast<uint64_t>(split_cap(max_seq_len)) * kPartStride * sizeof(float);
 }
 
-namespace {
-// kvtc_decode_attention, and with k_new / v_new (kvtc_decode_step) the fused append of one
-// new token per sequence at position seq_lens[s] - 1.
-kvtc_status decode_launch(const kvtc_plan* plan, const kvtc_cache* cache, int layer, const void* q,
-                          kvtc_dtype q_dtype, const int32_t* seq_lens, int max_seq_len, float softmax_scale,
-                          void* out, kvtc_dtype out_dtype, void* workspace, uint64_t workspace_bytes,
-                          const void* k_new, const void* v_new, kvtc_dtype kv_dtype, void* stream) {
+extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_cache* cache, int layer,
+                                             const void* q, kvtc_dtype q_dtype, const int32_t* seq_lens,
+                                             int max_seq_len, float softmax_scale, void* out,
+                                             kvtc_dtype out_dtype, void* workspace, uint64_t workspace_bytes,
+                                             void* stream) {
   kvtc_status st = check_uploaded(plan);
   if (st != KVTC_OK) return st;
   if (!cache || !cache->pool || !cache->block_table) return fail(KVTC_EINVAL, "cache is incomplete");
@@ -267,9 +265,6 @@ kvtc_status decode_launch(const kvtc_plan* plan, const kvtc_cache* cache, int la
     a.scale = scale;
     a.n_stage = gr.n_stage;
     a.stage_bytes = gr.stage_bytes;
-    a.k_new = k_new;
-    a.v_new = v_new;
-    a.kv_bf16 = kv_dtype == KVTC_BF16;
     a.tickets = tickets;
     a.ws = parts;
     dim3 grid(a.split_prefix[nh], n_hg, n_seq);
@@ -278,25 +273,4 @@ kvtc_status decode_launch(const kvtc_plan* plan, const kvtc_cache* cache, int la
     first = false;
   }
   return KVTC_OK;
-}
-}  // namespace
-
-extern "C" kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_cache* cache, int layer,
-                                             const void* q, kvtc_dtype q_dtype, const int32_t* seq_lens,
-                                             int max_seq_len, float softmax_scale, void* out,
-                                             kvtc_dtype out_dtype, void* workspace, uint64_t workspace_bytes,
-                                             void* stream) {
-  return decode_launch(plan, cache, layer, q, q_dtype, seq_lens, max_seq_len, softmax_scale, out, out_dtype,
-                       workspace, workspace_bytes, nullptr, nullptr, KVTC_F32, stream);
-}
-
-extern "C" kvtc_status kvtc_decode_step(const kvtc_plan* plan, const kvtc_cache* cache, int layer, const void* k_new,
-                                        const void* v_new, kvtc_dtype kv_dtype, const void* q, kvtc_dtype q_dtype,
-                                        const int32_t* seq_lens, int max_seq_len, float softmax_scale, void* out,
-                                        kvtc_dtype out_dtype, void* workspace, uint64_t workspace_bytes,
-                                        void* stream) {
-  if (!k_new || !v_new) return fail(KVTC_EINVAL, "null device pointer");
-  if (kv_dtype != KVTC_F32 && kv_dtype != KVTC_BF16) return fail(KVTC_EINVAL, "dtype must be F32 or BF16");
-  return decode_launch(plan, cache, layer, q, q_dtype, seq_lens, max_seq_len, softmax_scale, out, out_dtype,
-                       workspace, workspace_bytes, k_new, v_new, kv_dtype, stream);
 }

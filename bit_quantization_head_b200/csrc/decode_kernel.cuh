@@ -42,7 +42,6 @@
 #include <type_traits>
 #include <utility>
 
-#include "canon.cuh"
 #include "kvtc_internal.h"
 #include "ptx.cuh"
 
@@ -89,11 +88,6 @@ struct DecodeArgs {
   float scale;
   int n_stage;          // stages per warp of the widest head of the launch
   uint32_t stage_bytes;  // that head's stage (K + V page, 128-byte rounded)
-  // fused append (decode step): one new K and V row per sequence, [n_seq][H][128] of
-  // kv_bf16 ? bf16 : fp32, written at position seq_lens[s] - 1 (nullptr: plain decode)
-  const void* k_new;
-  const void* v_new;
-  int kv_bf16;
   int* tickets;       // [n_seq][H][n_hg][kTicketInts] arrival counters (zero between calls)
   float* ws;          // partials [n_seq][Hq][part_stride][kPartStride]
 };
@@ -846,20 +840,6 @@ __device__ __forceinline__ void merge_project(const DecodeArgs& a, const UnitDes
   }
 }
 
-// Sets field (word, mask) of a page in global memory to bits in one atomic step (no state
-// with the field cleared is ever visible), so that several CTAs may write the same
-// code while others copy the page.
-__device__ __forceinline__ void set_field_atomic(uint32_t* word, uint32_t mask, uint32_t bits) {
-  uint32_t old = *reinterpret_cast<volatile uint32_t*>(word);
-  for (int it = 0; it < (1 << 20); ++it) {  // lock-free: a failure means another write landed
-    const uint32_t want = (old & ~mask) | bits;
-    if (want == old) return;
-    const uint32_t seen = atomicCAS(word, old, want);
-    if (seen == old) return;
-    old = seen;
-  }
-}
-
 template <int BK, int BV, bool PACK>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
   // Programmatic dependent launch.  The first split launch of a call waits, once it has
@@ -936,7 +916,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   // lane l holds the id of page base + l of the current window of 32 (-1 past the run)
   int pid_win = lane < p_run ? bt[p_begin + lane] : -1;
   int seq_len = a.seq_lens[s];
-  const bool app_launch = a.k_new != nullptr;
   float4 qv[2];
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
@@ -959,17 +938,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   }
   const int n_pages = (seq_len + kPage - 1) / kPage;
   const int n_my = max(0, min(p_run, n_pages - p_begin));
-  // Fused append: the new token sits at position seq_len - 1, in page lp_new.  The CTAs
-  // whose runs cover that page (one per head group) compute its codes (the same canonical
-  // arithmetic as kvtc_encode_append) and each writes them into the cache with atomic
-  // field updates; the warp that reads the page copies it only after that.
-  const int tpos_new = seq_len - 1;
-  const int lp_new = tpos_new >= 0 ? tpos_new / kPage : -1;
-  const int slot_new = tpos_new >= 0 ? tpos_new % kPage : 0;
-  const bool app_cta =
-      app_launch && lp_new >= 0 &&
-      lp_new >= static_cast<int>(static_cast<long long>(split * kWarps) * a.part_pages / n_workers) &&
-      lp_new < static_cast<int>(static_cast<long long>((split + 1) * kWarps) * a.part_pages / n_workers);
 
   // ---- prologue: first copies (the barriers were set up by lane 0 of each warp, which
   // also issues the copies), then q~ while they are in flight ----
@@ -1009,10 +977,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     bulk_copy_g2s(st + bytesK, poolV + static_cast<uint64_t>(pid) * bytesV, bytesV, bar);
   };
   const int n_first = min(n_stage, n_my);
-  const int i_new = app_cta ? lp_new - p_begin : -1;  // the new token's page in this warp's run
   for (int i = 0; i < n_first; ++i) {
     const int pid = pid_of(i);
-    if (lane == 0 && i != i_new) issue(i, pid);  // page i < n_stage uses slot i
+    if (lane == 0) issue(i, pid);  // page i < n_stage uses slot i
   }
 
   // ---- q of the group into shared memory as fp16, scaled per head, and the fp16
@@ -1076,57 +1043,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     }
   }
   __syncthreads();
-
-  // ---- fused append: the new token's codes (q~'s scratch is free now), written into the
-  // cache before the warp that reads their page copies it ----
-  if (app_cta) {
-    // (loaded here, not with the other inputs: the prologue's registers are full before)
-    float* xs_new = &sh.qt[0][0];  // [K, V][128]
-    const size_t xo = (static_cast<size_t>(s) * a.H + h) * kD + tid;
-    const int32_t pid_new = bt[lp_new];
-    if (a.kv_bf16) {
-      xs_new[tid] = __bfloat162float(static_cast<const __nv_bfloat16*>(a.k_new)[xo]);
-      xs_new[kD + tid] = __bfloat162float(static_cast<const __nv_bfloat16*>(a.v_new)[xo]);
-    } else {
-      xs_new[tid] = static_cast<const float*>(a.k_new)[xo];
-      xs_new[kD + tid] = static_cast<const float*>(a.v_new)[xo];
-    }
-    __syncthreads();
-    const bool page_ok = pid_new >= 0 && static_cast<uint64_t>(pid_new) < a.pages_per_unit;
-#pragma unroll 1
-    for (int kind = 0; kind < 2; ++kind) {
-      const UnitDesc& ud = kind ? dV : dK;
-      if (tid < ud.r && page_ok) {
-        uint32_t* gpage = reinterpret_cast<uint32_t*>(const_cast<char*>(a.pool) + a.pages_per_unit * ud.prefix +
-                                                      static_cast<uint64_t>(pid_new) * ud.page_bytes);
-        if (ud.b == kRawBits) {  // raw value page: row j of 64 words (see encode_append_kernel)
-          const uint32_t code = __half_as_ushort(__float2half_rn(xs_new[kD + tid]));
-          const int word = tid * (kPage / 2) + ((slot_new >> 1) ^ ((tid & 7) << 2));
-          set_field_atomic(gpage + word, 0xFFFFu << (16 * (slot_new & 1)), code << (16 * (slot_new & 1)));
-        } else {
-          const float y = a.kv_bf16 ? canon_dot_bf16_mem(xs_new + kind * kD, reinterpret_cast<const uint4*>(
-                                                                                   ud.Mbf + static_cast<size_t>(tid) * kD))
-                                    : canon_dot_f32(xs_new + kind * kD, ud.M + static_cast<size_t>(tid) * kD);
-          const uint32_t code = quantize_code(y, ud.inv_delta, ud.b);
-          const int np = code_nparts(ud.b);
-          for (int i = 0; i < np; ++i) {
-            int lo, wd;
-            code_part(ud.b, i, lo, wd);
-            const FieldPos f = field_pos(kind, ud.r, lo, wd, slot_new, tid);
-            set_field_atomic(gpage + f.word, ((1u << wd) - 1u) << f.bit, ((code >> lo) & ((1u << wd) - 1u)) << f.bit);
-          }
-        }
-      }
-    }
-    // the writes (generic proxy) before the page's bulk copy (async proxy)
-    __threadfence();
-    asm volatile("fence.proxy.async.global;\n" ::: "memory");
-    __syncthreads();
-    if (i_new >= 0 && i_new < n_first) {  // the copy the first issues skipped
-      const int pid = pid_of(i_new);
-      if (lane == 0) issue(i_new, pid);
-    }
-  }
 
   WS<BK, BV, PACK> w;
   w.fr = &sh.u.frag[0][0][0][lane];

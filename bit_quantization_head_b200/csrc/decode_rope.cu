@@ -664,9 +664,6 @@ extern "C" kvtc_status kvtc_decode_attention_rope(const kvtc_plan* plan, const k
   a.part_pages = std::max(1, (max_seq_len + kPage - 1) / kPage);  // (this kernel splits by seq_len)
   a.status = cache->status;
   a.scale = scale;
-  a.k_new = nullptr;  // (no fused append)
-  a.v_new = nullptr;
-  a.kv_bf16 = 0;
   a.tickets = static_cast<int*>(workspace);
   // the workspace layout of kvtc_decode_attention: tickets [n_seq][H][n_hg][kTicketInts]
   // (this kernel counts arrivals in the first), then the partials

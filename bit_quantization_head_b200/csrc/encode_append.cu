@@ -10,7 +10,6 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
-#include "canon.cuh"
 #include "kvtc_internal.h"
 #include "layout.cuh"
 #include "ptx.cuh"
@@ -35,6 +34,29 @@ struct AppendArgs {
   int max_pages;
   int32_t* status;
 };
+
+__device__ __forceinline__ uint8_t quantize_code(float y, float inv_delta, int b) {
+  const float t = __fmul_rn(y, inv_delta);
+  const float u = __fadd_rn(t, static_cast<float>(1 << (b - 1)));
+  float f = floorf(u);
+  f = fmaxf(f, 0.0f);                                   // NaN -> 0
+  f = fminf(f, static_cast<float>((1 << b) - 1));
+  return static_cast<uint8_t>(f);
+}
+
+// Overwrites the b-bit code (t, j) of a page: clears its bits, then sets them.
+__device__ __forceinline__ void store_code(uint32_t* page, int kind, int r, int b, int t, int j, uint32_t c) {
+  const int np = code_nparts(b);
+  for (int i = 0; i < np; ++i) {
+    int lo, w;
+    code_part(b, i, lo, w);
+    const FieldPos f = field_pos(kind, r, lo, w, t, j);
+    const uint32_t mask = ((1u << w) - 1u) << f.bit;
+    const uint32_t bits = ((c >> lo) & ((1u << w) - 1u)) << f.bit;
+    atomicAnd(page + f.word, ~mask);
+    if (bits) atomicOr(page + f.word, bits);
+  }
+}
 
 // CTA = (token, unit of the layer); thread j computes coordinate j.  The token's row is
 // staged in shared memory once; each thread holds its row of M in registers; the fma
@@ -107,7 +129,36 @@ __global__ void __launch_bounds__(128) encode_append_kernel(const __grid_constan
   if (raw) {
     code = __half_as_ushort(__float2half_rn(xs[j]));
   } else {
-    const float acc = a.bf16 ? canon_dot_bf16(xs, mr) : canon_dot_f32(xs, ud.M + static_cast<size_t>(j) * kD);
+    // canonical projection: eight chains a_e = fma(x_k, M_jk, a_e) over k = e (mod 8)
+    // ascending, then ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7))
+    float ch[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    if (a.bf16) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t w[4] = {mr[c].x, mr[c].y, mr[c].z, mr[c].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          ch[2 * q] = __fmaf_rn(xs[8 * c + 2 * q], __uint_as_float(w[q] << 16), ch[2 * q]);
+          ch[2 * q + 1] = __fmaf_rn(xs[8 * c + 2 * q + 1], __uint_as_float(w[q] & 0xFFFF0000u), ch[2 * q + 1]);
+        }
+      }
+    } else {
+      const float4* m4 = reinterpret_cast<const float4*>(ud.M + static_cast<size_t>(j) * kD);
+#pragma unroll 4
+      for (int c = 0; c < 16; ++c) {
+        const float4 m0 = m4[2 * c], m1 = m4[2 * c + 1];
+        ch[0] = __fmaf_rn(xs[8 * c], m0.x, ch[0]);
+        ch[1] = __fmaf_rn(xs[8 * c + 1], m0.y, ch[1]);
+        ch[2] = __fmaf_rn(xs[8 * c + 2], m0.z, ch[2]);
+        ch[3] = __fmaf_rn(xs[8 * c + 3], m0.w, ch[3]);
+        ch[4] = __fmaf_rn(xs[8 * c + 4], m1.x, ch[4]);
+        ch[5] = __fmaf_rn(xs[8 * c + 5], m1.y, ch[5]);
+        ch[6] = __fmaf_rn(xs[8 * c + 6], m1.z, ch[6]);
+        ch[7] = __fmaf_rn(xs[8 * c + 7], m1.w, ch[7]);
+      }
+    }
+    const float acc = __fadd_rn(__fadd_rn(__fadd_rn(ch[0], ch[1]), __fadd_rn(ch[2], ch[3])),
+                                __fadd_rn(__fadd_rn(ch[4], ch[5]), __fadd_rn(ch[6], ch[7])));
     code = quantize_code(acc, ud.inv_delta, ud.b);
   }
 

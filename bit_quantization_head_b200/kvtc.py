@@ -91,8 +91,6 @@ def lib():
         "kvtc_decode_workspace_bytes": (C.c_uint64, [_P, C.c_int, C.c_int]),
         "kvtc_decode_attention": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, C.c_int, _P, C.c_int, C.c_float,
                                        _P, C.c_int, _P, C.c_uint64, _P]),
-        "kvtc_decode_step": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, _P, C.c_int, _P, C.c_int, _P, C.c_int,
-                                  C.c_float, _P, C.c_int, _P, C.c_uint64, _P]),
         "kvtc_decode_attention_noalloc": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, C.c_int, _P, C.c_int,
                                                C.c_float, _P, C.c_int, _P]),
         "kvtc_decode_attention_rope": (st, [_P, C.POINTER(CacheDesc), C.c_int, _P, C.c_int, _P, C.c_int, C.c_float,
@@ -307,18 +305,6 @@ def kvtc_decode_attention(plan, cache, layer, q, seq_lens, max_seq_len, out, wor
                                        _dev_ptr(seq_lens), max_seq_len, scale, _dev_ptr(out), _dtype_code(out),
                                        _dev_ptr(workspace), workspace.numel() * workspace.element_size(),
                                        _stream(stream)))
-
-
-def kvtc_decode_step(plan, cache, layer, k_new, v_new, q, seq_lens, max_seq_len, out, workspace, scale=0.0,
-                     stream=None):
-    """Append one token per sequence (k_new, v_new [n_seq][H][128], at position
-    seq_lens[s] - 1) and decode over the cache including it, in one call."""
-    if k_new.dtype != v_new.dtype:
-        raise ValueError("k_new and v_new must have the same dtype")
-    _check(lib().kvtc_decode_step(plan.handle, C.byref(cache.desc), layer, _dev_ptr(k_new), _dev_ptr(v_new),
-                                  _dtype_code(k_new), _dev_ptr(q), _dtype_code(q), _dev_ptr(seq_lens), max_seq_len,
-                                  scale, _dev_ptr(out), _dtype_code(out), _dev_ptr(workspace),
-                                  workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def kvtc_decode_attention_noalloc(plan, cache, layer, q, seq_lens, max_seq_len, out, scale=0.0, stream=None):

@@ -321,24 +321,6 @@ kvtc_status kvtc_decode_attention(const kvtc_plan* plan, const kvtc_cache* cache
                                   void* stream);
 
 /*
- * kvtc_decode_step -- one decode step of a layer in one call: appends one new token per
- * sequence and attends over the cache including it.  Equivalent to kvtc_encode_append of
- * k_new / v_new with cu_seqlens = 0, 1, ..., n_seq and pos_start[s] = seq_lens[s] - 1
- * (the same canonical codes, bit for bit), followed by kvtc_decode_attention with the
- * same arguments ("How KV-COBRA Works", Inference: encode the new key and value, then
- * the decode read of "Efficiency").  The CTAs that read the page holding position
- * seq_lens[s] - 1 compute the new token's codes themselves and set them in their copy
- * of the page; one of them writes the codes into the cache.  A sequence with
- * seq_lens[s] = 0 appends nothing.
- * k_new, v_new: device [n_seq][H_kv][d] of kv_dtype (F32 or BF16).  Every other argument
- * and the workspace as kvtc_decode_attention.
- */
-kvtc_status kvtc_decode_step(const kvtc_plan* plan, const kvtc_cache* cache, int layer, const void* k_new,
-                             const void* v_new, kvtc_dtype kv_dtype, const void* q, kvtc_dtype q_dtype,
-                             const int32_t* seq_lens, int max_seq_len, float softmax_scale, void* out,
-                             kvtc_dtype out_dtype, void* workspace, uint64_t workspace_bytes, void* stream);
-
-/*
  * kvtc_decode_attention_rope -- kvtc_decode_attention for caches whose keys were coded
  * before the rotary position embedding (KV-COBRA project page, Results: keys compressed
  * pre-RoPE).  The rotation of a key depends on its position, so q is not moved into the
