@@ -977,9 +977,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     bulk_copy_g2s(st + bytesK, poolV + static_cast<uint64_t>(pid) * bytesV, bytesV, bar);
   };
   const int n_first = min(n_stage, n_my);
-  for (int i = 0; i < n_first; ++i) {
-    const int pid = pid_of(i);
-    if (lane == 0) issue(i, pid);  // page i < n_stage uses slot i
+  // only the first page of each warp now: the rest of the ring is issued after q~ (a burst
+  // of every warp's ring at once keeps the copy engine busy while q~ is formed)
+  if (n_first > 0) {
+    const int pid = pid_of(0);
+    if (lane == 0) issue(0, pid);
   }
 
   // ---- q of the group into shared memory as fp16, scaled per head, and the fp16
@@ -1043,6 +1045,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
     }
   }
   __syncthreads();
+
+  for (int i = 1; i < n_first; ++i) {
+    const int pid = pid_of(i);
+    if (lane == 0) issue(i, pid);  // page i < n_stage uses slot i
+  }
 
   WS<BK, BV, PACK> w;
   w.fr = &sh.u.frag[0][0][0][lane];
