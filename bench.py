@@ -56,7 +56,7 @@ ENCODE_WORKLOAD = "qwen7b-28L-128k-2bpd"
 # the 8-layer copy of the workload read 32.40 MB against its 32.08 MB of algorithmic
 # bytes (1.010x); scaled by that ratio to this workload's mean layer (the file named
 # beside it).  None whenever a decode kernel has changed since the capture.
-DECODE_TRAFFIC = {"llama8b-32L-128k-1bpd": (None, None)}
+DECODE_TRAFFIC = {"llama8b-32L-128k-1bpd": (34.42e6, "profiles/decode_split_llama8b-8L-128k-1bpd_ncu.md")}
 METRIC = "decode-attn effective HBM GB/s (% of peak) at 128k ctx; encode Mtok/s"
 
 
