@@ -601,6 +601,58 @@ cudaError_t launch_pdl_rope(void (*fn)(KArgs...), dim3 grid, dim3 block, size_t 
 
 }  // namespace rope
 }  // namespace dec
+
+// The pre-RoPE launches of every layer: heads grouped by kernel variant, the stage size
+// of each group and the stage count and occupancy that fit (two CTAs per SM, the register
+// limit, when the ring allows it).  A group whose page does not fit in shared memory is
+// kept with no kernel; a pre-RoPE decode of its layer then fails with EINVAL (the plan
+// stays usable for every other call).  Sets each variant's shared-memory attribute once.
+kvtc_status prepare_rope(kvtc_plan* plan) {
+  using namespace dec;
+  using namespace dec::rope;
+  plan->rope_groups.assign(plan->L, {});
+  const size_t merge_bytes = std::max<size_t>(static_cast<size_t>(kWarps) * 8 * kPartStride, kMergeFloats) * sizeof(float);
+  for (int layer = 0; layer < plan->L; ++layer) {
+    std::vector<RopeGroup>& gs = plan->rope_groups[layer];
+    for (int h = 0; h < plan->H; ++h) {
+      const int uK = (layer * plan->H + h) * 2;
+      const void* fn = reinterpret_cast<const void*>(rope_fn(plan->b[uK], plan->b[uK + 1]));
+      auto it = std::find_if(gs.begin(), gs.end(), [&](const RopeGroup& x) { return x.fn == fn; });
+      if (it == gs.end()) {
+        gs.emplace_back();
+        it = gs.end() - 1;
+        it->fn = fn;
+      }
+      it->heads.push_back(h);
+      const uint32_t pb = static_cast<uint32_t>(16 * (plan->r[uK] * plan->b[uK] + plan->r[uK + 1] * plan->b[uK + 1]));
+      it->stage_bytes = std::max(it->stage_bytes, (pb + 127u) / 128u * 128u);
+    }
+    for (RopeGroup& gr : gs) {
+      int n_stage = kRopeStages;
+      size_t smem = 0;
+      for (; n_stage >= 1; --n_stage) {
+        smem = head_bytes() + std::max<size_t>(static_cast<size_t>(kWarps) * n_stage * gr.stage_bytes, merge_bytes) +
+               kReadSlack;
+        // two CTAs per SM (the register limit) when the ring allows it
+        if (smem <= kSmemPerSM / 2 - 1024 || (n_stage == 1 && smem <= kSmemPerSM - 1024)) break;
+      }
+      if (n_stage < 1) {
+        gr.fn = nullptr;
+        continue;
+      }
+      gr.n_stage = n_stage;
+      gr.smem = smem;
+      // the attribute is per kernel (shared with other plans): the largest size
+      cudaError_t e = cudaFuncSetAttribute(gr.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kSmemPerSM - 1024));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (rope decode)");
+      int occ = 1;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gr.fn, kThreads, smem) != cudaSuccess || occ < 1) occ = 1;
+      gr.per_sm = occ;
+    }
+  }
+  return KVTC_OK;
+}
 }  // namespace kvtc
 
 using namespace kvtc;
@@ -669,43 +721,14 @@ extern "C" kvtc_status kvtc_decode_attention_rope(const kvtc_plan* plan, const k
   // (this kernel counts arrivals in the first), then the partials
   const size_t tb = (static_cast<size_t>(n_seq) * plan->H * n_hg * kTicketInts * sizeof(int) + 255) / 256 * 256;
   a.ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + tb);
-  // one launch per (b_K, b_V) variant class; every KV head of the layer in one of them
-  struct Group {
-    RopeFn fn;
-    std::vector<int> heads;
-    uint32_t stage_bytes = 0;
-  };
-  std::vector<Group> groups;
-  for (int h = 0; h < plan->H; ++h) {
-    const int uK = (layer * plan->H + h) * 2;
-    RopeFn fn = rope_fn(plan->b[uK], plan->b[uK + 1]);
-    auto it = std::find_if(groups.begin(), groups.end(), [&](const Group& x) { return x.fn == fn; });
-    if (it == groups.end()) {
-      groups.push_back(Group{fn, {}, 0});
-      it = groups.end() - 1;
-    }
-    it->heads.push_back(h);
-    const uint32_t pb = static_cast<uint32_t>(16 * (plan->r[uK] * plan->b[uK] + plan->r[uK + 1] * plan->b[uK + 1]));
-    it->stage_bytes = std::max(it->stage_bytes, (pb + 127u) / 128u * 128u);
-  }
-  const size_t merge_bytes = std::max<size_t>(static_cast<size_t>(kWarps) * 8 * kPartStride, kMergeFloats) * sizeof(float);
+  // one launch per (b_K, b_V) variant class (decided at plan upload); every KV head of
+  // the layer in one of them
   bool first = true;
-  for (const Group& gr : groups) {
-    int n_stage = kRopeStages;
-    size_t smem = 0;
-    for (; n_stage >= 1; --n_stage) {
-      smem = head_bytes() + std::max<size_t>(static_cast<size_t>(kWarps) * n_stage * gr.stage_bytes, merge_bytes) +
-             kReadSlack;
-      // two CTAs per SM (the register limit) when the ring allows it
-      if (smem <= kSmemPerSM / 2 - 1024 || (n_stage == 1 && smem <= kSmemPerSM - 1024)) break;
-    }
-    if (n_stage < 1) return fail(KVTC_EINVAL, "a page of this plan does not fit in shared memory");
-    // the attribute is per kernel (shared with other plans and calls): the largest size
-    cudaError_t e = cudaFuncSetAttribute(gr.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemPerSM - 1024));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (rope decode)");
-    int occ = 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gr.fn, kThreads, smem) != cudaSuccess || occ < 1) occ = 1;
+  for (const RopeGroup& gr : plan->rope_groups[layer]) {
+    if (!gr.fn) return fail(KVTC_EINVAL, "a page of this plan does not fit in shared memory");
+    const int n_stage = gr.n_stage;
+    const size_t smem = gr.smem;
+    const int occ = gr.per_sm;
     const int nh = static_cast<int>(gr.heads.size());
     if (nh > kMaxHeadsPerLaunch) return fail(KVTC_EINVAL, "at most 64 KV heads per layer");
     const int wave = std::max(nh, static_cast<int>(static_cast<double>(occ) * plan->sm_count * nh / plan->H));
@@ -720,7 +743,7 @@ extern "C" kvtc_status kvtc_decode_attention_rope(const kvtc_plan* plan, const k
     a.n_stage = n_stage;
     a.stage_bytes = gr.stage_bytes;
     dim3 grid(a.split_prefix[nh], n_hg, n_seq);
-    e = launch_pdl_rope(gr.fn, grid, dim3(kThreads), smem, cs, ra);
+    const cudaError_t e = launch_pdl_rope(reinterpret_cast<RopeFn>(const_cast<void*>(gr.fn)), grid, dim3(kThreads), smem, cs, ra);
     if (e != cudaSuccess) return cuda_fail(e, "rope decode launch");
     first = false;
   }

@@ -439,7 +439,8 @@ kvtc_status kvtc_plan_upload(kvtc_plan* plan, void* stream) {
     return cuda_fail(e, "plan upload copy");
   }
   plan->device = dev;
-  const kvtc_status ds = prepare_decode(plan);
+  kvtc_status ds = prepare_decode(plan);
+  if (ds == KVTC_OK) ds = prepare_rope(plan);
   if (ds != KVTC_OK) {
     free_device(plan);
     return ds;

@@ -55,6 +55,17 @@ struct DecodeGroup {
   const void* fn = nullptr;     // the kernel variant
 };
 
+// One pre-RoPE decode launch of a layer: the KV heads whose (b_K, b_V) share a kernel
+// variant, with its shared-memory plan and occupancy (decided once, at plan upload).
+struct RopeGroup {
+  const void* fn = nullptr;     // the kernel variant
+  std::vector<int> heads;       // KV heads of the layer in this launch
+  uint32_t stage_bytes = 0;     // one K + V page of the widest head, 128-byte rounded
+  int n_stage = 0;              // stages per warp
+  size_t smem = 0;              // dynamic shared memory per CTA
+  int per_sm = 1;               // resident CTAs per SM at that size
+};
+
 // Sets the thread-local error message and returns the status.
 kvtc_status fail(kvtc_status s, const std::string& msg);
 kvtc_status cuda_fail(int err, const char* what);
@@ -81,6 +92,7 @@ struct kvtc_plan {
   std::vector<kvtc::UnitDesc> h_units;      // descriptors with device pointers
   // decode launch plan, per layer (set at upload): the launches and the device's SM count
   std::vector<std::vector<kvtc::DecodeGroup>> dec_groups;
+  std::vector<std::vector<kvtc::RopeGroup>> rope_groups;  // the same for the pre-RoPE decode
   int sm_count = 0;
 };
 
@@ -90,4 +102,7 @@ kvtc_status check_uploaded(const kvtc_plan* plan);
 // Fills plan->dec_groups and plan->sm_count for the current device and sets the kernel
 // attributes the decode launches need (decode.cu; called by kvtc_plan_upload).
 kvtc_status prepare_decode(kvtc_plan* plan);
+// Fills plan->rope_groups and sets the pre-RoPE kernels' attributes (decode_rope.cu;
+// called by kvtc_plan_upload after prepare_decode).
+kvtc_status prepare_rope(kvtc_plan* plan);
 }  // namespace kvtc
