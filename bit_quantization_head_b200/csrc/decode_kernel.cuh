@@ -939,8 +939,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
   const int n_pages = (seq_len + kPage - 1) / kPage;
   const int n_my = max(0, min(p_run, n_pages - p_begin));
 
-  // ---- prologue: first copies (the barriers were set up by lane 0 of each warp, which
-  // also issues the copies), then q~ while they are in flight ----
+  // ---- prologue: each warp's first copy (the barriers were set up by lane 0 of each warp,
+  // which also issues the copies), then q~ while it is in flight ----
 
   const uint32_t bytesK = static_cast<uint32_t>(dK.page_bytes), bytesV = static_cast<uint32_t>(dV.page_bytes);
   const char* poolK = a.pool + a.pages_per_unit * dK.prefix;
