@@ -26,7 +26,7 @@
 // The value codes enter their MMAs shifted by floor(m_V) (an exact fp16x2 subtraction),
 // so the tensor core accumulates signed terms near the size of the result; the 0.5 l left
 // over is folded into z after every page in packed mode (once at the end otherwise).
-// 2-bit value codes in packed mode skip the shift and fold the whole 1.5 l per page.
+// 2- and 3-bit value codes in packed mode skip the shift and fold the whole m_V l per page.
 // A page's eight 16-token blocks are processed together (their MMA chains interleave).
 // The four warps' (m, l, z) meet in shared memory and each CTA writes one partial per
 // query head; the last min(G, splits) CTAs to complete a (sequence, KV head, head group)
@@ -230,7 +230,7 @@ struct WS {
   int rsw;  // uncompressed value pages: swizzle of this lane's word positions (tq ^ 4 g)
   // Centring of the value sums: the operands are c - floor(m_V), so z accumulates
   // p * (c - m_V + 0.5); the 0.5 l left over is folded into z after every page (packed
-  // mode) or once at the end.  mV = 0.5 (1.5 for unshifted 2-bit codes, 0 for raw
+  // mode) or once at the end.  mV = 0.5 (m_V for unshifted 2- and 3-bit codes, 0 for raw
   // values); lfold = the part of l
   // (times 2^-17) already folded.
   float mV;
@@ -346,9 +346,10 @@ __device__ __forceinline__ void p_block(WS<BK, BV, PACK>& w, const float (&x)[4]
   bp[1] = movmatrix_trans(P1);
 }
 
-// Value codes centred by the per-page fold alone (no operand shift): 2-bit packed mode.
+// Value codes centred by the per-page fold alone (no operand shift): 2- and 3-bit codes in
+// packed mode.
 template <int BV, bool PACK>
-constexpr bool kFoldOnly = PACK && BV == 2;
+constexpr bool kFoldOnly = PACK && (BV == 2 || BV == 3);
 
 // Value MMA of one block for m-tile mt (words as in k_block, of rows j0 and j0 + 8).
 // Rows past r_V hold whatever follows the page in shared memory: their z rows are never
@@ -364,10 +365,10 @@ __device__ __forceinline__ void v_block(const WS<BK, BV, PACK>& w, uint32_t W0, 
   // Signed operands: the codes enter the MMA as c - floor(m_V), so the tensor core sums
   // terms of both signs near the size of the result (an unsigned sum of p c, about
   // m_V l, loses the centred result in the accumulation).  The remaining 0.5 l is
-  // folded into z separately.  2-bit values in packed mode skip the shift: m_V = 1.5 l
-  // is folded into z after every page, which bounds the unsigned part of the sums by
-  // one page's 3 l (measured within the tolerance at every budget; wider codes need the
-  // shift).
+  // folded into z separately.  2- and 3-bit values in packed mode skip the shift: m_V l
+  // is folded into z after every page, which bounds the unsigned part of the sums by one
+  // page's (2^b - 1) l (measured: the same errors against the oracle at every budget;
+  // wider codes need the shift).
   if constexpr (!kFoldOnly<BV, PACK>) {
     constexpr uint32_t c0 = centre_bits<BV, BLK, 0>(), c1 = centre_bits<BV, BLK, 1>();
     A0 = hsub2_bits(A0, c0);
@@ -1096,7 +1097,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_split_kernel(cons
       }
     }
     w.zl[0] = w.zl[1] = w.zl[2] = w.zl[3] = 0.0f;
-    w.mV = dV.b == kRawBits ? 0.0f : (kFoldOnly<BV, PACK> ? 1.5f : 0.5f);
+    w.mV = dV.b == kRawBits ? 0.0f : (kFoldOnly<BV, PACK> ? 0.5f * static_cast<float>((1 << dV.b) - 1) : 0.5f);
     w.lfold = 0.0f;
   }
 #pragma unroll
