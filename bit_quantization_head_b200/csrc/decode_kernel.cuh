@@ -11,9 +11,9 @@
 //     comes straight from the packed words: one AND leaves each code in the low mantissa
 //     bits of an fp16 half, the exact subnormal c * 2^(e-24), e the field's bit offset
 //     (undone in fp32), and widths 3, 5, 6 and 7 add their one or two minor parts with a
-//     shift and an AND-OR each; for G <= 4 (packed mode) head n's hi and lo parts sit in columns
-//     2n and 2n + 1 of one MMA, so each lane adds its own two columns and holds one head's
-//     scores for two token rows;
+//     shift and an AND-OR each; for G <= 4 (packed mode) head n's hi and lo parts sit in
+//     columns 2n and 2n + 1 of one MMA, so each lane adds its own two columns and holds one
+//     head's scores for two token rows;
 //   * runs an online softmax whose rescale is lazy: it happens only when a score exceeds
 //     the running max by more than 2^8 (a warp vote), so the common block costs one FFMA
 //     and one ex2 per score;
@@ -30,7 +30,8 @@
 // A page's eight 16-token blocks are processed together (their MMA chains interleave).
 // The four warps' (m, l, z) meet in shared memory and each CTA writes one partial per
 // query head; the last min(G, splits) CTAs to complete a (sequence, KV head, head group)
-// (an atomic arrival counter in the workspace) each take a share of its query heads:
+// (an atomic arrival counter in the workspace; from 16 splits up, else the last CTA
+// alone) each take a share of its query heads:
 // once every split has written its partial, they merge the partials with a log-sum-exp,
 // dequantize (delta_V) and back-project o = M_V^T y on several SMs at once; the last of
 // them re-arms the counters.
